@@ -1,0 +1,9 @@
+"""The CPU oracle against facts fixed by the pages and by mathematics."""
+import pytest
+
+import oracle_pins as P
+
+
+@pytest.mark.parametrize("pin", P.ALL_PINS, ids=lambda f: f.__name__)
+def test_pin(pin):
+    pin()
