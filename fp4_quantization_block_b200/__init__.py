@@ -1,0 +1,293 @@
+"""FP4 quantization producers + block-scaled FP4 GEMM for B200 (sm_100a).
+
+A thin ctypes binding of ``libfa4.so`` (C ABI in ``include/fa4.h``).  This
+module only allocates tensors with PyTorch, picks the current CUDA stream and
+marshals arguments; every step of the computation runs in the library's CUDA
+kernels.  There is no CPU or PyTorch fallback: if the library is missing or a
+call fails, an exception is raised.
+
+Names follow the pages on format-aware fusion for FP4: the scale domains
+MXFP4 (native mxfp), NVFP4_GLOBAL (global nvfp) and NVFP4_CTA (CTA-local nvfp)
+of "Format-Aware Fusion: The Engineering Practice That Doubles FP4
+Pretraining Throughput", section "The Design Philosophy of Format-Aware
+Fusion"; row-gradient stochastic rounding and the fixed-sign 32-value
+Hadamard of its section "Two Key Numerical Techniques".
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from dataclasses import dataclass
+
+import torch
+
+__all__ = [
+    "MXFP4", "NVFP4_GLOBAL", "NVFP4_CTA", "RNE", "SR", "ROWWISE", "COLWISE",
+    "QTensor", "FA4Error", "lib", "library_path", "quant_sizes", "empty_qtensor", "quantize",
+    "hadamard32_quantize", "gemm", "linear_ws_bytes", "linear_fwd", "linear_dgrad",
+    "linear_wgrad", "workspace", "check_device_status",
+]
+
+MXFP4, NVFP4_GLOBAL, NVFP4_CTA = 0, 1, 2
+RNE, SR = 0, 1
+ROWWISE, COLWISE = 0, 1
+OUT_BF16, OUT_FP32 = 0, 1
+WS_HEADER_BYTES = 256
+BLOCK = {MXFP4: 32, NVFP4_GLOBAL: 16, NVFP4_CTA: 16}
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+library_path = os.path.join(_HERE, "libfa4.so")
+
+STATUS = {0: "ok", 1: "invalid argument", 2: "unsupported shape", 3: "misaligned pointer",
+          4: "unsupported combination", 5: "workspace too small", 6: "CUDA error",
+          7: "bounded device wait timed out"}
+
+
+class FA4Error(RuntimeError):
+    def __init__(self, status: int, what: str):
+        super().__init__(f"{what}: {STATUS.get(status, status)} (status {status})")
+        self.status = status
+
+
+class _QT(ctypes.Structure):
+    _fields_ = [("payload", ctypes.c_void_p), ("scales", ctypes.c_void_p),
+                ("tensor_scale", ctypes.c_void_p)]
+
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded libfa4.so.  Raises if it has not been built."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(library_path):
+            raise ImportError(f"{library_path} is missing: build it with "
+                              "`python -m fp4_quantization_block_b200.build`")
+        _lib = _declare(ctypes.CDLL(library_path))
+    return _lib
+
+
+def _declare(L: ctypes.CDLL) -> ctypes.CDLL:
+    P, i64, u64, u32, sz, ci, f32 = (ctypes.c_void_p, ctypes.c_int64, ctypes.c_uint64,
+                                     ctypes.c_uint32, ctypes.c_size_t, ctypes.c_int,
+                                     ctypes.c_float)
+    PSZ = ctypes.POINTER(ctypes.c_size_t)
+    sig = {
+        "fa4_quant_sizes": [i64, i64, ci, ci, PSZ, PSZ, PSZ, PSZ],
+        "fa4_quantize": [P, i64, i64, i64, ci, ci, ci, u64, _QT, P, sz, P],
+        "fa4_hadamard32_quantize": [P, i64, i64, i64, u32, ci, u64, _QT, P, sz, P],
+        "fa4_gemm_blockscaled": [_QT, _QT, i64, i64, i64, ci, f32, P, i64, ci, P, sz, P],
+        "fa4_linear_ws_bytes": [ci, i64, i64, i64, ci, PSZ],
+        "fa4_linear_fwd": [P, _QT, i64, i64, i64, ci, P, P, sz, P],
+        "fa4_linear_dgrad": [P, _QT, i64, i64, i64, ci, ci, u64, P, P, sz, P],
+        "fa4_linear_wgrad": [P, P, i64, i64, i64, u32, ci, u64, P, ci, P, sz, P],
+        "fa4_workspace_init": [P, sz, P],
+        "fa4_check_device_status": [P, P],
+        "fa4_debug_convert": [P, P, i64, P, P, P, P],
+        "fa4_debug_sr_bits": [u64, P, i64, P, P],
+        "fa4_debug_gemm_timeout": [_QT, _QT, i64, i64, i64, ci, P, i64, ci, u64, P, sz, P],
+    }
+    for name, args in sig.items():
+        fn = getattr(L, name)
+        fn.argtypes = args
+        fn.restype = ci
+    L.fa4_status_string.argtypes = [ci]
+    L.fa4_status_string.restype = ctypes.c_char_p
+    L.fa4_version.argtypes = []
+    L.fa4_version.restype = ci
+    return L
+
+
+def _check(status: int, what: str):
+    if status != 0:
+        raise FA4Error(status, what)
+
+
+def _ptr(t: torch.Tensor | None):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(device: torch.device):
+    return ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
+
+
+@dataclass
+class QTensor:
+    """Quantized operand Q[R, K]: ``payload`` uint8 [R, K/2] (K-major, element
+    2j in the low nibble of byte j), ``scales`` uint8 [R*K/block] in the 128x4
+    atom layout the block-scaled MMA reads, ``ts`` float32 second-level decode
+    scales (NVFP4) or None (MXFP4)."""
+    payload: torch.Tensor
+    scales: torch.Tensor
+    ts: torch.Tensor | None
+    R: int
+    K: int
+    fmt: int
+
+    def c(self) -> _QT:
+        return _QT(self.payload.data_ptr(), self.scales.data_ptr(),
+                   None if self.ts is None else self.ts.data_ptr())
+
+
+def quant_sizes(rows: int, cols: int, fmt: int, orient: int = ROWWISE) -> tuple[int, int, int, int]:
+    a, b, c, d = (ctypes.c_size_t() for _ in range(4))
+    _check(lib().fa4_quant_sizes(rows, cols, fmt, orient, ctypes.byref(a), ctypes.byref(b),
+                                 ctypes.byref(c), ctypes.byref(d)), "fa4_quant_sizes")
+    return a.value, b.value, c.value, d.value
+
+
+def empty_qtensor(rows: int, cols: int, fmt: int, orient: int = ROWWISE, device="cuda") -> QTensor:
+    pb, sb, tc, _ = quant_sizes(rows, cols, fmt, orient)
+    R, K = (rows, cols) if orient == ROWWISE else (cols, rows)
+    payload = torch.empty((R, K // 2), dtype=torch.uint8, device=device)
+    scales = torch.empty(sb, dtype=torch.uint8, device=device)
+    ts = torch.empty(tc, dtype=torch.float32, device=device) if tc else None
+    assert payload.numel() == pb
+    return QTensor(payload, scales, ts, R, K, fmt)
+
+
+def workspace(nbytes: int, device="cuda") -> torch.Tensor:
+    """A zero-filled workspace (the status header must start at zero)."""
+    return torch.zeros(max(int(nbytes), WS_HEADER_BYTES), dtype=torch.uint8, device=device)
+
+
+def _ws(ws, need, device):
+    if ws is None:
+        ws = workspace(need, device)
+    return ws
+
+
+def _as_bf16_2d(x: torch.Tensor, name: str):
+    if x.dtype != torch.bfloat16 or x.dim() != 2 or not x.is_cuda:
+        raise ValueError(f"{name} must be a 2-D bf16 CUDA tensor")
+    if x.stride(1) != 1:
+        raise ValueError(f"{name} must have unit column stride")
+    return x.stride(0)
+
+
+def quantize(x: torch.Tensor, fmt: int, rnd: int = RNE, orient: int = ROWWISE, seed: int = 0,
+             out: QTensor | None = None, ws: torch.Tensor | None = None) -> QTensor:
+    ld = _as_bf16_2d(x, "x")
+    rows, cols = x.shape
+    out = out or empty_qtensor(rows, cols, fmt, orient, x.device)
+    need = quant_sizes(rows, cols, fmt, orient)[3]
+    ws = _ws(ws, need, x.device)
+    _check(lib().fa4_quantize(_ptr(x), rows, cols, ld, fmt, rnd, orient, seed, out.c(), _ptr(ws),
+                              ws.numel(), _stream(x.device)), "fa4_quantize")
+    return out
+
+
+def hadamard32_quantize(x: torch.Tensor, sign_mask: int, rnd: int = RNE, seed: int = 0,
+                        out: QTensor | None = None, ws: torch.Tensor | None = None) -> QTensor:
+    ld = _as_bf16_2d(x, "x")
+    rows, cols = x.shape
+    out = out or empty_qtensor(rows, cols, MXFP4, COLWISE, x.device)
+    ws = _ws(ws, WS_HEADER_BYTES, x.device)
+    _check(lib().fa4_hadamard32_quantize(_ptr(x), rows, cols, ld, sign_mask & 0xFFFFFFFF, rnd, seed,
+                                         out.c(), _ptr(ws), ws.numel(), _stream(x.device)),
+           "fa4_hadamard32_quantize")
+    return out
+
+
+def gemm(A: QTensor, B: QTensor, alpha: float = 1.0, out_dtype=torch.float32,
+         out: torch.Tensor | None = None, ws: torch.Tensor | None = None) -> torch.Tensor:
+    """D[M, N] = alpha * A B^T on the block-scaled FP4 tensor cores."""
+    if A.K != B.K or A.fmt != B.fmt:
+        raise ValueError("A and B must share K and format")
+    dev = A.payload.device
+    if out is None:
+        out = torch.empty((A.R, B.R), dtype=out_dtype, device=dev)
+    od = OUT_FP32 if out.dtype == torch.float32 else OUT_BF16
+    ws = _ws(ws, WS_HEADER_BYTES, dev)
+    _check(lib().fa4_gemm_blockscaled(A.c(), B.c(), A.R, B.R, A.K, A.fmt, float(alpha), _ptr(out),
+                                      out.stride(0), od, _ptr(ws), ws.numel(), _stream(dev)),
+           "fa4_gemm_blockscaled")
+    return out
+
+
+def linear_ws_bytes(kind: int, T: int, Cin: int, Cout: int, fmt: int) -> int:
+    n = ctypes.c_size_t()
+    _check(lib().fa4_linear_ws_bytes(kind, T, Cin, Cout, fmt, ctypes.byref(n)), "fa4_linear_ws_bytes")
+    return n.value
+
+
+def linear_fwd(X: torch.Tensor, Wq: QTensor, fmt: int, out: torch.Tensor | None = None,
+               ws: torch.Tensor | None = None) -> torch.Tensor:
+    """Y = X W^T; Wq is W[Cout, Cin] quantized row-wise."""
+    T, Cin = X.shape
+    Cout = Wq.R
+    _as_bf16_2d(X, "X")
+    out = out if out is not None else torch.empty((T, Cout), dtype=torch.bfloat16, device=X.device)
+    ws = _ws(ws, linear_ws_bytes(0, T, Cin, Cout, fmt), X.device)
+    _check(lib().fa4_linear_fwd(_ptr(X.contiguous()), Wq.c(), T, Cin, Cout, fmt, _ptr(out), _ptr(ws),
+                                ws.numel(), _stream(X.device)), "fa4_linear_fwd")
+    return out
+
+
+def linear_dgrad(dY: torch.Tensor, Wq_col: QTensor, fmt: int, rnd: int = SR, seed: int = 0,
+                 out: torch.Tensor | None = None, ws: torch.Tensor | None = None) -> torch.Tensor:
+    """dX = dY W; Wq_col is W[Cout, Cin] quantized column-wise ([Cin, Cout])."""
+    T, Cout = dY.shape
+    Cin = Wq_col.R
+    _as_bf16_2d(dY, "dY")
+    out = out if out is not None else torch.empty((T, Cin), dtype=torch.bfloat16, device=dY.device)
+    ws = _ws(ws, linear_ws_bytes(1, T, Cin, Cout, fmt), dY.device)
+    _check(lib().fa4_linear_dgrad(_ptr(dY.contiguous()), Wq_col.c(), T, Cin, Cout, fmt, rnd, seed,
+                                  _ptr(out), _ptr(ws), ws.numel(), _stream(dY.device)),
+           "fa4_linear_dgrad")
+    return out
+
+
+def linear_wgrad(dY: torch.Tensor, X: torch.Tensor, sign_mask: int, rnd: int = RNE, seed: int = 0,
+                 out_dtype=torch.float32, out: torch.Tensor | None = None,
+                 ws: torch.Tensor | None = None) -> torch.Tensor:
+    """dW = dY^T X through column-wise fixed-sign Hadamard MXFP4 operands."""
+    T, Cout = dY.shape
+    _, Cin = X.shape
+    _as_bf16_2d(dY, "dY")
+    _as_bf16_2d(X, "X")
+    if out is None:
+        out = torch.empty((Cout, Cin), dtype=out_dtype, device=dY.device)
+    od = OUT_FP32 if out.dtype == torch.float32 else OUT_BF16
+    ws = _ws(ws, linear_ws_bytes(2, T, Cin, Cout, MXFP4), dY.device)
+    _check(lib().fa4_linear_wgrad(_ptr(dY.contiguous()), _ptr(X.contiguous()), T, Cin, Cout,
+                                  sign_mask & 0xFFFFFFFF, rnd, seed, _ptr(out), od, _ptr(ws),
+                                  ws.numel(), _stream(dY.device)), "fa4_linear_wgrad")
+    return out
+
+
+def check_device_status(ws: torch.Tensor) -> int:
+    """Synchronize and return (and clear) the workspace's device status."""
+    return lib().fa4_check_device_status(_ptr(ws), _stream(ws.device))
+
+
+# ------------------------------------------------------------ diagnostics ---
+
+def debug_convert(y: torch.Tensor, u16: torch.Tensor | None = None, e4m3: bool = False):
+    """Device E2M1 RNE / SR and E4M3 conversions of fp32 values (as the
+    quantizers use them)."""
+    n = y.numel()
+    rne = torch.empty(n, dtype=torch.uint8, device=y.device)
+    sr = torch.empty(n, dtype=torch.uint8, device=y.device) if u16 is not None else None
+    e4 = torch.empty(n, dtype=torch.uint8, device=y.device) if e4m3 else None
+    _check(lib().fa4_debug_convert(_ptr(y), _ptr(u16), n, _ptr(rne), _ptr(sr), _ptr(e4),
+                                   _stream(y.device)), "fa4_debug_convert")
+    return rne, sr, e4
+
+
+def debug_sr_bits(seed: int, idx: torch.Tensor) -> torch.Tensor:
+    bits = torch.empty(idx.numel(), dtype=torch.int32, device=idx.device)
+    _check(lib().fa4_debug_sr_bits(seed, _ptr(idx), idx.numel(), _ptr(bits), _stream(idx.device)),
+           "fa4_debug_sr_bits")
+    return bits
+
+
+def debug_gemm_timeout(A: QTensor, B: QTensor, skip_k_tile: int, timeout_ns: int,
+                       ws: torch.Tensor) -> torch.Tensor:
+    dev = A.payload.device
+    out = torch.zeros((A.R, B.R), dtype=torch.float32, device=dev)
+    _check(lib().fa4_debug_gemm_timeout(A.c(), B.c(), A.R, B.R, A.K, A.fmt, _ptr(out), out.stride(0),
+                                        skip_k_tile, timeout_ns, _ptr(ws), ws.numel(), _stream(dev)),
+           "fa4_debug_gemm_timeout")
+    return out

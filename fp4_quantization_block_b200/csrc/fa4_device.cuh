@@ -1,0 +1,193 @@
+// fa4_device.cuh -- device helpers for the FP4 quantizers (sm_100a).
+//
+// Element format E2M1 and the block scales follow the pages on FP4:
+//   "FP4 Is No Longer Just a Hardware Feature -- The NVFP4 Software Stack Is
+//    Taking Shape", section "NVFP4 is more than a 4-bit value" (E2M1 payload,
+//    E4M3 block scale per 16 values, FP32 tensor-level scale), section "The
+//    first change" (amax -> scale -> divide -> E2M1 -> pack), section "The
+//    third change" (scale clamp to the scale type's range);
+//   "Format-Aware Fusion: The Engineering Practice That Doubles FP4
+//    Pretraining Throughput", sections "The Design Philosophy of Format-Aware
+//    Fusion" (native mxfp / global nvfp / CTA-local nvfp) and "Two Key
+//    Numerical Techniques" (row-gradient stochastic rounding, fixed-sign
+//    32-value Hadamard).
+// Every floating-point step that decides a stored byte is one binary32
+// operation with round-to-nearest-even (__fmul_rn / __fdiv_rn / __fsub_rn, so
+// nothing is contracted into an FMA); the library is built without fast-math,
+// so subnormals are kept.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <stdint.h>
+
+namespace fa4 {
+
+enum : int { kMX = 0, kNVG = 1, kNVC = 2 };
+enum : int { kRNE = 0, kSR = 1 };
+
+// ---------------------------------------------------------------- bf16 ---
+// A bf16 value is the top half of a binary32.
+__device__ __forceinline__ float bf16lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
+
+// ---------------------------------------------------------------- E2M1 ---
+// Round-to-nearest-even conversion of two binary32 values by the hardware
+// conversion instruction, saturating to +-6: returns (code(lo) | code(hi)<<4).
+__device__ __forceinline__ uint32_t e2m1x2_rne(float lo, float hi) {
+  uint32_t out;
+  asm("{\n\t.reg .b8 t;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 t, %2, %1;\n\t"
+      "cvt.u32.u8 %0, t;\n\t}"
+      : "=r"(out)
+      : "f"(lo), "f"(hi));
+  return out;
+}
+
+// Eight values -> eight codes packed little-endian by nibble (element 0 in
+// the low nibble of byte 0).
+__device__ __forceinline__ uint32_t e2m1x8_rne(const float *v) {
+  uint32_t out;
+  asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b0, %2, %1;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b1, %4, %3;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b2, %6, %5;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b3, %8, %7;\n\t"
+      "mov.b32 %0, {b0, b1, b2, b3};\n\t}"
+      : "=r"(out)
+      : "f"(v[0]), "f"(v[1]), "f"(v[2]), "f"(v[3]), "f"(v[4]), "f"(v[5]), "f"(v[6]), "f"(v[7]));
+  return out;
+}
+
+// Stochastic rounding of y to a neighbouring E2M1 value with 16 random bits
+// u: with lo <= |y| < hi the neighbouring grid magnitudes and g = hi - lo,
+// round up iff u < (|y| - lo) * 65536 / g.  Both factors are exact (lo and
+// |y| share a binade, g is a power of two), so this equals the definition
+// with f = (|y| - lo) / g computed first.  |y| >= 6 gives 6; the sign of y is
+// kept.  Grid magnitudes 0, .5, 1, 1.5, 2, 3, 4, 6.
+__device__ __forceinline__ uint32_t e2m1_sr(float y, uint32_t u) {
+  const uint32_t s = (__float_as_uint(y) >> 28) & 8u;
+  const float a = fabsf(y);
+  if (a >= 6.0f) return s | 7u;
+  uint32_t c = (a >= 0.5f) + (a >= 1.0f) + (a >= 1.5f) + (a >= 2.0f) + (a >= 3.0f) + (a >= 4.0f);
+  const float lo = (c < 4) ? 0.5f * (float)c : (float)(c - 2);  // exact
+  const float k = (c < 4) ? 131072.0f : ((c < 6) ? 65536.0f : 32768.0f);
+  const float t = __fmul_rn(__fsub_rn(a, lo), k);
+  c += ((float)u < t) ? 1u : 0u;
+  return s | c;
+}
+
+// ---------------------------------------------------------------- E4M3 ---
+// Round-to-nearest-even to E4M3 (bias 7, max 448), saturating; one value.
+__device__ __forceinline__ uint32_t e4m3_rne(float v) {
+  uint16_t out;
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(out) : "f"(0.0f), "f"(v));
+  return (uint32_t)(out & 0xFF);
+}
+
+// Exact E4M3 -> binary32 through the hardware widening conversion.
+__device__ __forceinline__ float e4m3_to_float(uint32_t code) {
+  uint32_t h2;
+  uint16_t in = (uint16_t)(code & 0xFF);
+  asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h2) : "h"(in));
+  return __half2float(__ushort_as_half((unsigned short)(h2 & 0xFFFF)));
+}
+
+// --------------------------------------------------------- scale rules ---
+// MXFP4 (32-value blocks, E8M0): shared exponent e = floor(log2 amax) - 2
+// (2 = exponent of the largest E2M1 value), clamped to [-127, 127], amax = 0
+// giving -127.  From the binary32 exponent field E of amax: E = 0 (zero or
+// subnormal, floor(log2) <= -127) gives -127, otherwise e = E - 129.  The
+// stored byte is e + 127 = max(E - 2, 0); the element multiplier 2^-e has
+// exponent field 127 - e = 254 - byte (always normal for byte <= 252).
+__device__ __forceinline__ uint32_t mx_scale_byte(float amax) {
+  const int E = (int)(__float_as_uint(amax) >> 23) & 0xFF;
+  return (uint32_t)max(E - 2, 0);
+}
+__device__ __forceinline__ float mx_multiplier(uint32_t byte) {
+  return __uint_as_float((254u - byte) << 23);
+}
+
+// NVFP4 second level: encode scale s_enc = 2688 / amax_t (2688 = 6 * 448, the
+// largest E2M1 times the largest E4M3), 1 when amax_t is 0 or the quotient is
+// not finite; the stored decode scale is 1 / s_enc.
+__device__ __forceinline__ float nv_encode_scale(float amax_t) {
+  float s = __fdiv_rn(2688.0f, amax_t);
+  if (amax_t == 0.0f || !isfinite(s)) s = 1.0f;
+  return s;
+}
+__device__ __forceinline__ float nv_decode_scale(float s_enc) { return __fdiv_rn(1.0f, s_enc); }
+
+// NVFP4 block scale: (amax_b / 6) * s_enc, clamped to [2^-9, 448] (the
+// smallest positive and largest E4M3 values), rounded to E4M3.  Returns the
+// code; *mult receives the element multiplier s_enc / decode(code).
+__device__ __forceinline__ uint32_t nv_block_scale(float amax_b, float s_enc, float *mult) {
+  float sb = __fmul_rn(__fdiv_rn(amax_b, 6.0f), s_enc);
+  sb = fminf(fmaxf(sb, 0.001953125f), 448.0f);  // fmaxf maps NaN to the bound
+  const uint32_t code = e4m3_rne(sb);
+  *mult = __fdiv_rn(s_enc, e4m3_to_float(code));
+  return code;
+}
+
+// ------------------------------------------------------------- Philox ---
+// Philox4x32 with 10 rounds (Salmon, Moraes, Dror, Shaw, "Parallel random
+// numbers: as easy as 1, 2, 3", SC'11).  Each round multiplies words 0 and 2
+// by the two round constants, XORs the high halves with the other words and
+// the key; the key advances by the Weyl increments between rounds.
+struct u32x4 {
+  uint32_t x, y, z, w;
+};
+
+__device__ __forceinline__ u32x4 philox10(uint32_t c0, uint32_t c1, uint32_t c2, uint32_t c3,
+                                          uint32_t k0, uint32_t k1) {
+#pragma unroll
+  for (int r = 0; r < 10; ++r) {
+    const uint32_t lo0 = 0xD2511F53u * c0, hi0 = __umulhi(0xD2511F53u, c0);
+    const uint32_t lo1 = 0xCD9E8D57u * c2, hi1 = __umulhi(0xCD9E8D57u, c2);
+    const uint32_t n0 = hi1 ^ c1 ^ k0, n2 = hi0 ^ c3 ^ k1;
+    c0 = n0;
+    c1 = lo1;
+    c2 = n2;
+    c3 = lo0;
+    k0 += 0x9E3779B9u;
+    k1 += 0xBB67AE85u;
+  }
+  return {c0, c1, c2, c3};
+}
+
+// The 128 random bits for the eight elements (8j .. 8j+7) of the quantized
+// operand whose linear index is i = 8j: counter j (64-bit, words 0-1), key =
+// the 64-bit seed.  Element 8j+e uses 16-bit half (e & 1) of word e >> 1.
+__device__ __forceinline__ u32x4 sr_block_bits(uint64_t seed, uint64_t i8) {
+  return philox10((uint32_t)i8, (uint32_t)(i8 >> 32), 0u, 0u, (uint32_t)seed,
+                  (uint32_t)(seed >> 32));
+}
+__device__ __forceinline__ uint32_t sr_half(const u32x4 &b, int e) {
+  const uint32_t w = (e >> 1) == 0 ? b.x : (e >> 1) == 1 ? b.y : (e >> 1) == 2 ? b.z : b.w;
+  return (e & 1) ? (w >> 16) : (w & 0xFFFFu);
+}
+
+// Eight values -> eight SR codes packed like e2m1x8_rne.
+__device__ __forceinline__ uint32_t e2m1x8_sr(const float *v, const u32x4 &b) {
+  uint32_t out = 0;
+#pragma unroll
+  for (int e = 0; e < 8; ++e) out |= e2m1_sr(v[e], sr_half(b, e)) << (4 * e);
+  return out;
+}
+
+// ------------------------------------------------ scale-factor layout ---
+// Byte offset of the scale of (row r, block kb) for kbt blocks per row, in
+// the 128-row x 4-block atoms (512 bytes) the block-scaled tensor-core MMA
+// reads; atoms run along kb first.  kb % 4 == 0 gives a 4-byte aligned word
+// holding blocks kb .. kb+3 of row r.
+__device__ __forceinline__ int64_t sf_offset(int64_t r, int64_t kb, int64_t kbt) {
+  return ((r >> 7) * (kbt >> 2) + (kb >> 2)) * 512 + (r & 31) * 16 + ((r >> 5) & 3) * 4 + (kb & 3);
+}
+
+// ---------------------------------------------------------- reductions ---
+__device__ __forceinline__ float warp_max(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xFFFFFFFFu, v, o));
+  return v;
+}
+
+}  // namespace fa4

@@ -1,0 +1,48 @@
+// fa4_kernels.h -- internal launch interface between the C ABI (fa4_api.cu)
+// and the kernels.  Not installed; not part of the public ABI.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace fa4 {
+
+// Upper bound on the per-CTA partial maxima of the NVFP4-global amax pass.
+constexpr int kMaxAmaxPartials = 1184;  // 8 CTAs x 148 SMs
+
+int amax_partials_count(int64_t rows, int64_t cols);
+cudaError_t launch_tensor_amax(const uint16_t *x, int64_t rows, int64_t cols, int64_t ld,
+                               float *partials, int n_partials, cudaStream_t st);
+cudaError_t launch_quant_rowwise(int fmt, int rnd, const uint16_t *x, int64_t R, int64_t K,
+                                 int64_t ld, uint8_t *payload, uint8_t *scales, float *ts,
+                                 const float *partials, int n_partials, uint64_t seed,
+                                 cudaStream_t st);
+cudaError_t launch_quant_colwise(int fmt, int rnd, bool hadamard, uint32_t sign_mask,
+                                 const uint16_t *x, int64_t T, int64_t C, int64_t ld,
+                                 uint8_t *payload, uint8_t *scales, float *ts,
+                                 const float *partials, int n_partials, uint64_t seed,
+                                 cudaStream_t st);
+cudaError_t launch_debug_convert(const float *y, const uint32_t *u16, int64_t n, uint8_t *rne,
+                                 uint8_t *sr, uint8_t *e4m3, cudaStream_t st);
+cudaError_t launch_debug_sr_bits(uint64_t seed, const uint64_t *idx, int64_t n, uint32_t *bits,
+                                 cudaStream_t st);
+
+// Block-scaled GEMM.  status: device word for bounded-wait timeouts.
+struct GemmArgs {
+  const uint8_t *a_payload, *a_scales;
+  const float *a_ts;
+  const uint8_t *b_payload, *b_scales;
+  const float *b_ts;
+  int64_t M, N, K;
+  int fmt;
+  float alpha;
+  void *D;
+  int64_t ldd;
+  int out_fp32;
+  uint32_t *status;
+  int debug_skip_stage;     // < 0 normally; >= 0: the producer never loads that k-tile (test hook)
+  uint64_t timeout_ns;      // bounded-wait limit
+};
+cudaError_t launch_gemm_blockscaled(const GemmArgs &a, cudaStream_t st);
+
+}  // namespace fa4

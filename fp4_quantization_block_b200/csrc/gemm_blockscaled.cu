@@ -1,0 +1,607 @@
+// gemm_blockscaled.cu -- block-scaled FP4 GEMM on the sm_100a tensor cores.
+//
+//   D[m][n] = alpha * sum_k A[m][k] * B[n][k]
+//
+// A and B are FP4 operands as the quantizers emit them: packed E2M1 payload
+// (K-major, two values per byte) plus one scale byte per block in 128x4
+// atoms ("FP4 Is No Longer Just a Hardware Feature -- The NVFP4 Software
+// Stack Is Taking Shape", section "NVFP4 is more than a 4-bit value": the
+// contract is payload + block scales + tensor scale + a defined layout; the
+// GEMM is the consumer whose layout the producer matches, "Format-Aware
+// Fusion: The Engineering Practice That Doubles FP4 Pretraining Throughput",
+// section "The Design Philosophy of Format-Aware Fusion").
+//
+// Structure (one CTA per SM, persistent over output tiles, 10 warps):
+//   warp 0      TMA producer: per k-tile of 256 elements, the A tile
+//               (128 rows x 128 B) and B tile (BN rows x 128 B) by
+//               cp.async.bulk.tensor with 128-byte swizzle, and the scale
+//               atoms (contiguous 512-byte runs) by cp.async.bulk, into a
+//               4-stage shared-memory ring guarded by mbarriers.
+//   warp 1      MMA issuer: tcgen05.cp moves the scale atoms into tensor
+//               memory, tcgen05.mma kind::mxf4 (MX, 32-blocks, E8M0) or
+//               kind::mxf4nvf4 (NV, 16-blocks, E4M3) accumulates a 128 x BN
+//               FP32 tile in tensor memory; tcgen05.commit frees each stage.
+//   warps 2..9  epilogue: tcgen05.ld of the accumulator, alpha (and the
+//               NVFP4 second-level scales), conversion, global stores.
+// NVFP4-CTA-local: the second-level scale differs per 128-wide K chunk, so
+// each chunk accumulates into one of two tensor-memory partials and the
+// epilogue warps fold tsA[m/128][kc] * tsB[n/128][kc] * partial into FP32
+// registers.
+//
+// Every mbarrier wait is bounded: past `timeout_ns` the waiting thread sets
+// the device status word, raises a CTA-wide abort flag and leaves its loop;
+// the CTA then waits (bounded) for its own copies in flight, frees its
+// tensor memory and returns.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include <cuda_bf16.h>
+
+#include "fa4_device.cuh"
+#include "fa4_kernels.h"
+
+namespace fa4 {
+namespace gemm {
+
+constexpr int BM = 128;
+constexpr int BK = 256;            // elements per k-tile (128 bytes per row)
+constexpr int BKB = BK / 2;        // bytes per row per k-tile
+constexpr int STAGES = 4;
+constexpr int NUM_THREADS = 320;   // 10 warps
+constexpr int TMEM_COLS = 512;
+constexpr int SFA_COL = 256;       // tensor-memory column of the A scale atoms
+constexpr int SFB_COL = 288;       // ... of the B scale atoms
+constexpr uint32_t kStatusTimeout = 7;
+
+// ------------------------------------------------------------ PTX wrappers
+__device__ __forceinline__ uint32_t smem_u32(const void *p) {
+  return (uint32_t)__cvta_generic_to_shared(p);
+}
+__device__ __forceinline__ uint64_t globaltimer() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
+}
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
+               : "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap *map, int x, int y,
+                                            uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar)
+      : "memory");
+}
+__device__ __forceinline__ void bulk_load(uint32_t dst, const void *src, uint32_t bytes,
+                                          uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+          dst),
+      "l"(src), "r"(bytes), "r"(bar)
+      : "memory");
+}
+__device__ __forceinline__ void tc_fence_before() {
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_commit(uint32_t bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                   bar)
+               : "memory");
+}
+__device__ __forceinline__ void tc_cp_32x128b_warpx4(uint32_t taddr, uint64_t sdesc) {
+  asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc)
+               : "memory");
+}
+template <int KIND>
+__device__ __forceinline__ void tc_mma(uint32_t d, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                       uint32_t sfa, uint32_t sfb, uint32_t accumulate) {
+  if constexpr (KIND == kMX) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %6, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::mxf4.block_scale.scale_vec::2X [%0], %1, %2, %3, [%4], [%5], p;\n\t}" ::"r"(d),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(sfa), "r"(sfb), "r"(accumulate)
+        : "memory");
+  } else {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %6, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::mxf4nvf4.block_scale.scale_vec::4X [%0], %1, %2, %3, [%4], [%5], p;\n\t}" ::"r"(d),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(sfa), "r"(sfb), "r"(accumulate)
+        : "memory");
+  }
+}
+// 32 lanes x 32 consecutive 32-bit columns -> 32 registers per thread.
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t *r) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,"
+      "%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+        "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]),
+        "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]),
+        "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr));
+}
+__device__ __forceinline__ void tmem_wait_ld() {
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
+// Shared-memory matrix descriptor (sm_100 layout): start address >> 4 in
+// bits 0-13, leading byte offset >> 4 in 16-29, stride byte offset >> 4 in
+// 32-45, version 1 in bits 46-47, layout type in 61-63.
+__device__ __forceinline__ uint64_t smem_desc(uint32_t addr, uint32_t lbo, uint32_t sbo,
+                                              uint32_t layout) {
+  return (uint64_t)((addr & 0x3FFFFu) >> 4) | ((uint64_t)(lbo >> 4) << 16) |
+         ((uint64_t)(sbo >> 4) << 32) | (1ull << 46) | ((uint64_t)layout << 61);
+}
+// K-major operand tile, rows of 128 bytes, 128-byte swizzle, 8-row groups
+// 1024 bytes apart.
+__device__ __forceinline__ uint64_t operand_desc(uint32_t addr) {
+  return smem_desc(addr, 16, 1024, 2);
+}
+// One 512-byte scale atom: 32 rows of 16 bytes, 8-row core matrices 128
+// bytes apart, no swizzle.
+__device__ __forceinline__ uint64_t scale_desc(uint32_t addr) { return smem_desc(addr, 0, 128, 0); }
+
+// Block-scaled instruction descriptor: E2M1 A and B (format 1), K-major,
+// N >> 3 in bits 17-22, scale type in bit 23 (1 = E8M0, 0 = E4M3), M >> 4
+// in bits 24-28, scale-factor byte ids in bits 4-5 (B) and 29-30 (A).
+template <int KIND, int N>
+__device__ __forceinline__ uint32_t instr_desc(uint32_t sf_id) {
+  return (1u << 7) | (1u << 10) | ((uint32_t)(N >> 3) << 17) |
+         ((KIND == kMX ? 1u : 0u) << 23) | ((uint32_t)(BM >> 4) << 24) | (sf_id << 4) |
+         (sf_id << 29);
+}
+
+template <int KIND>
+struct Cfg {  // KIND kMX: 32-blocks; kNVG / kNVC: 16-blocks
+  static constexpr int BS = (KIND == kMX) ? 32 : 16;   // block size
+  static constexpr int SF_PER_ROW = BK / BS;           // scale bytes per row per k-tile
+  static constexpr int ATOMS_K = SF_PER_ROW / 4;       // 128x4 atoms along K per k-tile
+  static constexpr int SFA_BYTES = ATOMS_K * 512;      // per 128 rows
+};
+
+struct Smem {
+  uint64_t full[STAGES], empty[STAGES];
+  uint64_t acc_full, acc_empty, part_full[2], part_empty[2], mma_done;
+  uint32_t tmem_base;
+  int abort;
+};
+
+template <int KIND, int BN>
+struct Layout {
+  static constexpr int A_BYTES = BM * BKB;                       // 16 KB
+  static constexpr int B_BYTES = BN * BKB;                       // 16 or 32 KB
+  static constexpr int SFA_BYTES = Cfg<KIND>::SFA_BYTES;
+  static constexpr int SFB_BYTES = Cfg<KIND>::SFA_BYTES * (BN / 128);
+  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES;
+  static constexpr int OFF_A = 0;
+  static constexpr int OFF_B = OFF_A + STAGES * A_BYTES;
+  static constexpr int OFF_SFA = OFF_B + STAGES * B_BYTES;
+  static constexpr int OFF_SFB = OFF_SFA + STAGES * SFA_BYTES;
+  static constexpr int OFF_CTRL = OFF_SFB + STAGES * SFB_BYTES;
+  static constexpr int TOTAL = OFF_CTRL + (int)sizeof(Smem) + 1024;  // + alignment slack
+};
+
+struct Params {
+  const uint8_t *a_scales, *b_scales;
+  const float *a_ts, *b_ts;
+  int64_t M, N, K;
+  float alpha;
+  void *D;
+  int64_t ldd;
+  int out_fp32;
+  uint32_t *status;
+  int debug_skip_stage;
+  uint64_t timeout_ns;
+};
+
+// Bounded wait.  Returns false on timeout (status set, abort raised) or when
+// another role already aborted.
+__device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, Smem *sm, const Params &p,
+                                         uint32_t where) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = globaltimer();
+  while (true) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if (*(volatile int *)&sm->abort) return false;
+    if (globaltimer() - t0 > p.timeout_ns) {
+      *(volatile int *)&sm->abort = 1;
+      if (atomicCAS(p.status, 0u, kStatusTimeout) == 0u) atomicExch(p.status + 1, where);
+      return false;
+    }
+  }
+}
+
+// Warp-uniform bounded wait: lane 0 waits, every lane gets the result, and
+// the warp is converged afterwards (the .sync.aligned tcgen05 loads that
+// follow need all 32 lanes together).
+__device__ __forceinline__ bool warp_wait_bar(uint32_t bar, uint32_t parity, Smem *sm,
+                                              const Params &p, uint32_t where) {
+  int ok = 0;
+  if ((threadIdx.x & 31) == 0) ok = wait_bar(bar, parity, sm, p, where) ? 1 : 0;
+  ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
+  return ok != 0;
+}
+
+// KIND: kMX, kNVG or kNVC (CTA-local second-level scales).
+template <int KIND, int BN>
+__global__ void __launch_bounds__(NUM_THREADS, 1)
+    gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_b,
+                const Params p) {
+  constexpr bool CTA = (KIND == kNVC);
+  using L = Layout<KIND, BN>;
+  using C = Cfg<KIND>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                              ~uintptr_t(1023));
+  Smem *sm = reinterpret_cast<Smem *>(smem + L::OFF_CTRL);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  const int num_m = (int)(p.M / BM), num_n = (int)(p.N / BN);
+  const int num_tiles = num_m * num_n;
+  const int KT = (int)(p.K / BK);
+  const int64_t kbt4 = (p.K / C::BS) / 4;  // scale atoms per 128 rows
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(smem_u32(&sm->full[s]), 1);
+      mbar_init(smem_u32(&sm->empty[s]), 1);
+    }
+    mbar_init(smem_u32(&sm->acc_full), 1);
+    mbar_init(smem_u32(&sm->acc_empty), 8);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(smem_u32(&sm->part_full[i]), 1);
+      mbar_init(smem_u32(&sm->part_empty[i]), 8);
+    }
+    mbar_init(smem_u32(&sm->mma_done), 1);
+    sm->abort = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     smem_u32(&sm->tmem_base)),
+                 "r"(TMEM_COLS)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = sm->tmem_base;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      uint32_t issued = 0;       // stages with a load in flight or landed
+      uint32_t last_parity = 0;  // parity bit of the last load issued per stage
+      bool ok = true;
+      int k_global = 0;
+      for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
+        const int mt = tile % num_m, nt = tile / num_m;
+        for (int kt = 0; kt < KT; ++kt, ++k_global) {
+          if (!wait_bar(smem_u32(&sm->empty[stage]), phase ^ 1u, sm, p, 0x100u | stage)) {
+            ok = false;
+            break;
+          }
+          if (k_global != p.debug_skip_stage) {
+            const uint32_t fb = smem_u32(&sm->full[stage]);
+            mbar_arrive_expect_tx(fb, L::STAGE_BYTES);
+            tma_load_2d(smem_u32(smem + L::OFF_A + stage * L::A_BYTES), &map_a, kt * BKB, mt * BM, fb);
+            tma_load_2d(smem_u32(smem + L::OFF_B + stage * L::B_BYTES), &map_b, kt * BKB, nt * BN, fb);
+            const uint8_t *sa = p.a_scales + ((int64_t)mt * kbt4 + (int64_t)kt * C::ATOMS_K) * 512;
+            bulk_load(smem_u32(smem + L::OFF_SFA + stage * L::SFA_BYTES), sa, L::SFA_BYTES, fb);
+#pragma unroll
+            for (int nb = 0; nb < BN / 128; ++nb) {
+              const uint8_t *sb =
+                  p.b_scales + ((int64_t)(nt * (BN / 128) + nb) * kbt4 + (int64_t)kt * C::ATOMS_K) * 512;
+              bulk_load(smem_u32(smem + L::OFF_SFB + stage * L::SFB_BYTES + nb * C::SFA_BYTES), sb,
+                        C::SFA_BYTES, fb);
+            }
+            issued |= 1u << stage;
+            last_parity = (last_parity & ~(1u << stage)) | (phase << stage);
+          }
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+      }
+      // never leave with a copy in flight into this CTA's shared memory
+      for (int s = 0; s < STAGES; ++s) {
+        if (!((issued >> s) & 1u)) continue;
+        const uint32_t par = (last_parity >> s) & 1u;
+        const uint64_t t0 = globaltimer();
+        while (!mbar_try_wait(smem_u32(&sm->full[s]), par)) {
+          if (globaltimer() - t0 > p.timeout_ns) {
+            if (atomicCAS(p.status, 0u, kStatusTimeout) == 0u) atomicExch(p.status + 1, 0x400u | s);
+            break;
+          }
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ----------------------------------------------------------- MMA issue
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0, acc_phase = 0;
+      uint32_t chunk = 0;  // CTA-local: global 128-K chunk counter
+      bool ok = true;
+      for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
+        if constexpr (!CTA) {
+          if (!wait_bar(smem_u32(&sm->acc_empty), acc_phase ^ 1u, sm, p, 0x200u)) break;
+          tc_fence_after();
+        }
+        for (int kt = 0; kt < KT; ++kt) {
+          if (!wait_bar(smem_u32(&sm->full[stage]), phase, sm, p, 0x210u | stage)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a_base = smem_u32(smem + L::OFF_A + stage * L::A_BYTES);
+          const uint32_t b_base = smem_u32(smem + L::OFF_B + stage * L::B_BYTES);
+          const uint32_t sfa_base = smem_u32(smem + L::OFF_SFA + stage * L::SFA_BYTES);
+          const uint32_t sfb_base = smem_u32(smem + L::OFF_SFB + stage * L::SFB_BYTES);
+          // scale atoms -> tensor memory: A atom a at column SFA_COL + 4a; B
+          // atom (row block nb, a) at SFB_COL + (BN/32)*a + 4*nb
+#pragma unroll
+          for (int a = 0; a < C::ATOMS_K; ++a) {
+            tc_cp_32x128b_warpx4(tmem + SFA_COL + 4 * a, scale_desc(sfa_base + a * 512));
+#pragma unroll
+            for (int nb = 0; nb < BN / 128; ++nb)
+              tc_cp_32x128b_warpx4(tmem + SFB_COL + (BN / 32) * a + 4 * nb,
+                                   scale_desc(sfb_base + nb * C::SFA_BYTES + a * 512));
+          }
+#pragma unroll
+          for (int j = 0; j < BK / 64; ++j) {
+            // MX: two MMAs share one atom (scale bytes 0-1 and 2-3 of the
+            // word); NV: one atom per MMA
+            const int a = (KIND == kMX) ? (j >> 1) : j;
+            const uint32_t sf_id = (KIND == kMX) ? (uint32_t)(2 * (j & 1)) : 0u;
+            const uint32_t sfa = (tmem + SFA_COL + 4 * a) | (sf_id << 30);
+            const uint32_t sfb = (tmem + SFB_COL + (BN / 32) * a) | (sf_id << 30);
+            const uint64_t ad = operand_desc(a_base + j * 32);
+            const uint64_t bd = operand_desc(b_base + j * 32);
+            if constexpr (CTA) {
+              const int c = j >> 1;  // 128-K chunk within the k-tile
+              const uint32_t pb = (chunk + c) & 1u;
+              if ((j & 1) == 0) {
+                if (!wait_bar(smem_u32(&sm->part_empty[pb]), (((chunk + c) >> 1) & 1u) ^ 1u, sm, p,
+                              0x220u | pb)) {
+                  ok = false;
+                  break;
+                }
+                tc_fence_after();
+              }
+              tc_mma<KIND>(tmem + pb * 128, ad, bd, instr_desc<KIND, BN>(sf_id), sfa, sfb,
+                           (uint32_t)(j & 1));
+              if (j & 1) tc_commit(smem_u32(&sm->part_full[pb]));
+            } else {
+              tc_mma<KIND>(tmem, ad, bd, instr_desc<KIND, BN>(sf_id), sfa, sfb,
+                           (kt > 0 || j > 0) ? 1u : 0u);
+            }
+          }
+          if constexpr (CTA) chunk += BK / 128;
+          tc_commit(smem_u32(&sm->empty[stage]));
+          if (!ok) break;
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+        if constexpr (!CTA) {
+          if (ok) tc_commit(smem_u32(&sm->acc_full));
+          acc_phase ^= 1u;
+        }
+      }
+      // all MMAs issued by this thread have completed before tensor memory
+      // is released
+      tc_commit(smem_u32(&sm->mma_done));
+      const uint64_t t0 = globaltimer();
+      while (!mbar_try_wait(smem_u32(&sm->mma_done), 0)) {
+        if (globaltimer() - t0 > p.timeout_ns) {
+          if (atomicCAS(p.status, 0u, kStatusTimeout) == 0u) atomicExch(p.status + 1, 0x500u);
+          break;
+        }
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const int q = warp & 3;          // tensor-memory lane quadrant this warp may access
+    const int h = (warp - 2) >> 2;   // column half
+    constexpr int COLS = BN / 2;     // columns per warp
+    constexpr int NCH = COLS / 32;   // 32-column loads
+    const int nk = (int)(p.K / 128);
+    uint32_t acc_phase = 0, chunk = 0;
+    float alpha_g = p.alpha;
+    if constexpr (KIND == kNVG && !CTA) alpha_g = p.alpha * p.a_ts[0] * p.b_ts[0];
+    for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
+      const int mt = tile % num_m, nt = tile / num_m;
+      float v[COLS];
+      bool ok = true;
+      if constexpr (CTA) {
+#pragma unroll
+        for (int i = 0; i < COLS; ++i) v[i] = 0.0f;
+        for (int kc = 0; kc < nk; ++kc, ++chunk) {
+          const uint32_t pb = chunk & 1u;
+          if (!warp_wait_bar(smem_u32(&sm->part_full[pb]), (chunk >> 1) & 1u, sm, p, 0x300u | pb)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          uint32_t r[COLS];
+#pragma unroll
+          for (int c = 0; c < NCH; ++c)
+            tmem_ld32(tmem + ((uint32_t)(32 * q) << 16) + pb * 128 + h * COLS + 32 * c, &r[32 * c]);
+          tmem_wait_ld();
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(smem_u32(&sm->part_empty[pb]));
+          const float s = p.a_ts[(int64_t)mt * nk + kc] * p.b_ts[(int64_t)nt * nk + kc];
+#pragma unroll
+          for (int i = 0; i < COLS; ++i) v[i] = fmaf(s, __uint_as_float(r[i]), v[i]);
+        }
+        if (!ok) break;
+#pragma unroll
+        for (int i = 0; i < COLS; ++i) v[i] *= p.alpha;
+      } else {
+        if (!warp_wait_bar(smem_u32(&sm->acc_full), acc_phase, sm, p, 0x310u)) break;
+        tc_fence_after();
+        uint32_t r[COLS];
+#pragma unroll
+        for (int c = 0; c < NCH; ++c)
+          tmem_ld32(tmem + ((uint32_t)(32 * q) << 16) + h * COLS + 32 * c, &r[32 * c]);
+        tmem_wait_ld();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(smem_u32(&sm->acc_empty));
+        acc_phase ^= 1u;
+#pragma unroll
+        for (int i = 0; i < COLS; ++i) v[i] = __uint_as_float(r[i]) * alpha_g;
+      }
+      // each thread owns one output row segment of COLS columns
+      const int64_t row = (int64_t)mt * BM + 32 * q + lane;
+      const int64_t col = (int64_t)nt * BN + h * COLS;
+      if (p.out_fp32) {
+        float *dst = reinterpret_cast<float *>(p.D) + row * p.ldd + col;
+#pragma unroll
+        for (int i = 0; i < COLS; i += 4)
+          *reinterpret_cast<float4 *>(dst + i) = make_float4(v[i], v[i + 1], v[i + 2], v[i + 3]);
+      } else {
+        uint16_t *dst = reinterpret_cast<uint16_t *>(p.D) + row * p.ldd + col;
+#pragma unroll
+        for (int i = 0; i < COLS; i += 8) {
+          uint32_t w[4];
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            __nv_bfloat162 b2 = __floats2bfloat162_rn(v[i + 2 * u], v[i + 2 * u + 1]);
+            w[u] = *reinterpret_cast<uint32_t *>(&b2);
+          }
+          *reinterpret_cast<uint4 *>(dst + i) = make_uint4(w[0], w[1], w[2], w[3]);
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) {
+    __syncwarp();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(TMEM_COLS)
+                 : "memory");
+  }
+}
+
+}  // namespace gemm
+}  // namespace fa4
+
+namespace fa4 {
+
+using PFN_encodeTiled = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
+                                     const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
+                                     const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                     CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+static PFN_encodeTiled get_encode() {
+  static PFN_encodeTiled fn = nullptr;
+  if (!fn) {
+    void *ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_encodeTiled>(ptr);
+  }
+  return fn;
+}
+
+// Payload tile map: uint8 [rows, K/2] row-major, box 128 bytes x box_rows,
+// 128-byte swizzle (the layout the MMA's operand descriptors describe).
+static bool make_payload_map(CUtensorMap *m, const void *base, int64_t rows, int64_t K,
+                             int box_rows) {
+  PFN_encodeTiled enc = get_encode();
+  if (!enc) return false;
+  cuuint64_t dims[2] = {(cuuint64_t)(K / 2), (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)(K / 2)};
+  cuuint32_t box[2] = {(cuuint32_t)gemm::BKB, (cuuint32_t)box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void *>(base), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int KIND, int BN>
+static cudaError_t launch_t(const GemmArgs &a, cudaStream_t st) {
+  using L = gemm::Layout<KIND, BN>;
+  CUtensorMap ma, mb;
+  if (!make_payload_map(&ma, a.a_payload, a.M, a.K, gemm::BM)) return cudaErrorInvalidValue;
+  if (!make_payload_map(&mb, a.b_payload, a.N, a.K, BN)) return cudaErrorInvalidValue;
+  gemm::Params p;
+  p.a_scales = a.a_scales;
+  p.b_scales = a.b_scales;
+  p.a_ts = a.a_ts;
+  p.b_ts = a.b_ts;
+  p.M = a.M;
+  p.N = a.N;
+  p.K = a.K;
+  p.alpha = a.alpha;
+  p.D = a.D;
+  p.ldd = a.ldd;
+  p.out_fp32 = a.out_fp32;
+  p.status = a.status;
+  p.debug_skip_stage = a.debug_skip_stage;
+  p.timeout_ns = a.timeout_ns;
+  auto kern = gemm::gemm_kernel<KIND, BN>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::TOTAL);
+  if (e != cudaSuccess) return e;
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int64_t tiles = (a.M / gemm::BM) * (a.N / BN);
+  const int grid = (int)(tiles < sms ? tiles : sms);
+  kern<<<grid, gemm::NUM_THREADS, L::TOTAL, st>>>(ma, mb, p);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_gemm_blockscaled(const GemmArgs &a, cudaStream_t st) {
+  const bool wide = (a.N % 256) == 0;
+  switch (a.fmt) {
+    case kMX:
+      return wide ? launch_t<kMX, 256>(a, st) : launch_t<kMX, 128>(a, st);
+    case kNVG:
+      return wide ? launch_t<kNVG, 256>(a, st) : launch_t<kNVG, 128>(a, st);
+    case kNVC:
+      return launch_t<kNVC, 128>(a, st);
+    default:
+      return cudaErrorInvalidValue;
+  }
+}
+
+}  // namespace fa4

@@ -1,0 +1,416 @@
+// quantize.cu -- fused FP4 quantization producers for sm_100a.
+//
+// One kernel per orientation does the whole producer of "FP4 Is No Longer
+// Just a Hardware Feature -- The NVFP4 Software Stack Is Taking Shape",
+// section "The first change" (block amax -> scale -> divide -> E2M1 -> pack
+// two values per byte) in registers, and writes the scale bytes straight into
+// the 128x4 atoms the block-scaled MMA reads, so nothing intermediate goes to
+// memory (the unfused pipeline that section warns about writes amax and
+// scales and re-reads the tensor).  The scale domain is a template parameter
+// ("Format-Aware Fusion: The Engineering Practice That Doubles FP4
+// Pretraining Throughput", section "The Design Philosophy of Format-Aware
+// Fusion"): native MX, global NV (second pass after tensor_amax_kernel) or
+// CTA-local NV (the 128x128 tile amax is reduced inside the CTA that
+// quantizes the tile, so the tensor is read once).
+//
+// Work unit: one CTA of 256 threads per 128x128 tile of the quantized
+// operand Q.  The tile (32 KB of bf16) is loaded with 16-byte coalesced
+// loads, all issued before any arithmetic.
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "fa4_device.cuh"
+#include "fa4_kernels.h"
+
+namespace fa4 {
+
+__device__ __forceinline__ uint4 ld_stream(const void *p) {
+  uint4 v;
+  asm volatile("ld.global.nc.L1::no_allocate.L2::256B.v4.u32 {%0,%1,%2,%3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "l"(p));
+  return v;
+}
+
+__device__ __forceinline__ void unpack8(const uint4 &w, float *f) {
+  f[0] = bf16lo(w.x); f[1] = bf16hi(w.x);
+  f[2] = bf16lo(w.y); f[3] = bf16hi(w.y);
+  f[4] = bf16lo(w.z); f[5] = bf16hi(w.z);
+  f[6] = bf16lo(w.w); f[7] = bf16hi(w.w);
+}
+
+__device__ __forceinline__ float absmax8(const uint4 &w) {
+  // |bf16| max on the packed pairs: clear sign bits, max of the magnitudes
+  // as unsigned integers orders non-negative floats correctly
+  const uint32_t m = 0x7FFF7FFFu;
+  uint32_t a = __vmaxu2(w.x & m, w.y & m);
+  uint32_t b = __vmaxu2(w.z & m, w.w & m);
+  a = __vmaxu2(a, b);
+  const uint32_t hi = a >> 16, lo = a & 0xFFFFu;
+  return __uint_as_float((hi > lo ? hi : lo) << 16);
+}
+
+// CTA-wide max of one value per thread (256 threads).
+__device__ __forceinline__ float cta_max256(float v, float *red) {
+  v = warp_max(v);
+  const int w = threadIdx.x >> 5, l = threadIdx.x & 31;
+  __syncthreads();
+  if (l == 0) red[w] = v;
+  __syncthreads();
+  float r = red[0];
+#pragma unroll
+  for (int i = 1; i < 8; ++i) r = fmaxf(r, red[i]);
+  return r;
+}
+
+// Largest of the NV-global amax partials, read by every CTA.
+__device__ __forceinline__ float reduce_partials(const float *partials, int n, float *red) {
+  float m = 0.0f;
+  for (int i = threadIdx.x; i < n; i += blockDim.x) m = fmaxf(m, partials[i]);
+  return cta_max256(m, red);
+}
+
+// --------------------------------------------------------------------------
+// Tensor amax (NVFP4-global, pass 1): grid-stride over x[rows, cols] in
+// 8-element chunks; one partial maximum per CTA.
+// --------------------------------------------------------------------------
+__global__ void __launch_bounds__(256) tensor_amax_kernel(const uint16_t *__restrict__ x,
+                                                          int64_t rows, int64_t cols, int64_t ld,
+                                                          float *__restrict__ partials) {
+  __shared__ float red[8];
+  const int64_t cpr = cols >> 3;  // chunks per row
+  const int64_t n = rows * cpr;
+  float m = 0.0f;
+  int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+  for (; i + 3 * stride < n; i += 4 * stride) {
+    uint4 v[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int64_t c = i + u * stride;
+      v[u] = ld_stream(x + (c / cpr) * ld + (c % cpr) * 8);
+    }
+#pragma unroll
+    for (int u = 0; u < 4; ++u) m = fmaxf(m, absmax8(v[u]));
+  }
+  for (; i < n; i += stride) m = fmaxf(m, absmax8(ld_stream(x + (i / cpr) * ld + (i % cpr) * 8)));
+  m = cta_max256(m, red);
+  if (threadIdx.x == 0) partials[blockIdx.x] = m;
+}
+
+// --------------------------------------------------------------------------
+// Row-wise quantizer: Q = x[R, K], blocks along a row.
+// Thread layout in a 128x128 tile: warp w, lane l -> rows 16*s + 2*w + (l>>4)
+// for steps s = 0..7, columns 8*(l&15) .. +8.  A half-warp covers one row;
+// NV blocks (16) are lane pairs, MX blocks (32) lane quads.
+// --------------------------------------------------------------------------
+template <int FMT, int RND>
+__global__ void __launch_bounds__(256) quant_rowwise_kernel(
+    const uint16_t *__restrict__ x, int64_t R, int64_t K, int64_t ld, uint8_t *__restrict__ payload,
+    uint8_t *__restrict__ scales, float *__restrict__ ts, const float *__restrict__ partials,
+    int n_partials, uint64_t seed) {
+  __shared__ float red[8];
+  const int w = threadIdx.x >> 5, l = threadIdx.x & 31;
+  const int64_t k0 = (int64_t)blockIdx.x * 128, r0 = (int64_t)blockIdx.y * 128;
+  const int c = l & 15;          // 8-element chunk within the 128-wide row
+  const int64_t kc = k0 + 8 * c;  // first column of the chunk
+
+  uint4 v[8];
+#pragma unroll
+  for (int s = 0; s < 8; ++s) {
+    const int64_t r = r0 + 16 * s + 2 * w + (l >> 4);
+    v[s] = ld_stream(x + r * ld + kc);
+  }
+
+  float s_enc = 1.0f;
+  if constexpr (FMT == kNVC) {
+    float m = 0.0f;
+#pragma unroll
+    for (int s = 0; s < 8; ++s) m = fmaxf(m, absmax8(v[s]));
+    s_enc = nv_encode_scale(cta_max256(m, red));
+    if (threadIdx.x == 0) ts[blockIdx.y * gridDim.x + blockIdx.x] = nv_decode_scale(s_enc);
+  } else if constexpr (FMT == kNVG) {
+    s_enc = nv_encode_scale(reduce_partials(partials, n_partials, red));
+    if (threadIdx.x == 0 && blockIdx.x == 0 && blockIdx.y == 0) ts[0] = nv_decode_scale(s_enc);
+  }
+
+  const int64_t kbt = (FMT == kMX) ? (K >> 5) : (K >> 4);
+#pragma unroll
+  for (int s = 0; s < 8; ++s) {
+    const int64_t r = r0 + 16 * s + 2 * w + (l >> 4);
+    float f[8];
+    unpack8(v[s], f);
+    float amax = absmax8(v[s]);
+    amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, 1));
+    if constexpr (FMT == kMX) amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, 2));
+    uint32_t sbyte;
+    if constexpr (FMT == kMX) {
+      sbyte = mx_scale_byte(amax);
+      const float mult = mx_multiplier(sbyte);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) f[e] = __fmul_rn(f[e], mult);
+    } else {
+      float mult;
+      sbyte = nv_block_scale(amax, s_enc, &mult);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) f[e] = __fmul_rn(f[e], mult);
+    }
+    uint32_t codes;
+    if constexpr (RND == kSR) {
+      codes = e2m1x8_sr(f, sr_block_bits(seed, (uint64_t)(r * K + kc) >> 3));
+    } else {
+      codes = e2m1x8_rne(f);
+    }
+    *reinterpret_cast<uint32_t *>(payload + r * (K >> 1) + (kc >> 1)) = codes;
+
+    // gather four consecutive block scales of the row into one word
+    uint32_t word;
+    if constexpr (FMT == kMX) {
+      word = sbyte << (8 * (c >> 2));
+      word |= __shfl_xor_sync(0xFFFFFFFFu, word, 4);
+      word |= __shfl_xor_sync(0xFFFFFFFFu, word, 8);
+      if (c == 0) *reinterpret_cast<uint32_t *>(scales + sf_offset(r, k0 >> 5, kbt)) = word;
+    } else {
+      word = sbyte << (8 * ((c >> 1) & 3));
+      word |= __shfl_xor_sync(0xFFFFFFFFu, word, 2);
+      word |= __shfl_xor_sync(0xFFFFFFFFu, word, 4);
+      if ((c & 7) == 0)
+        *reinterpret_cast<uint32_t *>(scales + sf_offset(r, (k0 >> 4) + 4 * (c >> 3), kbt)) = word;
+    }
+  }
+}
+
+// --------------------------------------------------------------------------
+// Column-wise quantizer: Q = x^T, x[T, C] row-major; Q[R = C, K = T].
+// The 128(tokens) x 128(channels) tile is staged in shared memory; each
+// thread then owns two adjacent channels and one 32-token block, reading
+// down the columns (a warp reads 128 contiguous bytes per token: no bank
+// conflicts) and keeping all 64 values in registers, so the optional
+// Hadamard-32 is an in-register butterfly.
+// --------------------------------------------------------------------------
+__device__ __forceinline__ void fwht32(float *v) {
+#pragma unroll
+  for (int h = 1; h < 32; h <<= 1) {
+#pragma unroll
+    for (int i = 0; i < 32; ++i) {
+      if ((i & h) == 0) {
+        const float a = v[i], b = v[i + h];
+        v[i] = __fadd_rn(a, b);
+        v[i + h] = __fsub_rn(a, b);
+      }
+    }
+  }
+}
+
+template <int FMT, int RND, bool HAD>
+__global__ void __launch_bounds__(256) quant_colwise_kernel(
+    const uint16_t *__restrict__ x, int64_t T, int64_t C, int64_t ld, uint8_t *__restrict__ payload,
+    uint8_t *__restrict__ scales, float *__restrict__ ts, const float *__restrict__ partials,
+    int n_partials, uint64_t seed, uint32_t sign_mask) {
+  __shared__ __align__(16) uint16_t tile[128 * 128];  // [token][channel]
+  __shared__ __align__(16) uint8_t sbuf[128 * 8];     // [channel][block in tile]
+  __shared__ float red[8];
+  const int w = threadIdx.x >> 5, l = threadIdx.x & 31;
+  const int64_t c0 = (int64_t)blockIdx.x * 128;  // channel = row of Q
+  const int64_t t0 = (int64_t)blockIdx.y * 128;  // token = K of Q
+
+  // stage the tile: half-warp per token row, 16 bytes per lane
+  float s_enc_tile = 1.0f;
+  {
+    uint4 v[8];
+#pragma unroll
+    for (int s = 0; s < 8; ++s) {
+      const int64_t t = t0 + 16 * s + 2 * w + (l >> 4);
+      v[s] = ld_stream(x + t * ld + c0 + 8 * (l & 15));
+    }
+    float m = 0.0f;
+#pragma unroll
+    for (int s = 0; s < 8; ++s) {
+      const int tt = 16 * s + 2 * w + (l >> 4);
+      *reinterpret_cast<uint4 *>(&tile[tt * 128 + 8 * (l & 15)]) = v[s];
+      if constexpr (FMT == kNVC) m = fmaxf(m, absmax8(v[s]));
+    }
+    if constexpr (FMT == kNVC) {
+      // every thread receives the same tile maximum
+      s_enc_tile = nv_encode_scale(cta_max256(m, red));
+      if (threadIdx.x == 0) ts[blockIdx.x * gridDim.y + blockIdx.y] = nv_decode_scale(s_enc_tile);
+    }
+  }
+  float s_enc = s_enc_tile;
+  if constexpr (FMT == kNVG) {
+    s_enc = nv_encode_scale(reduce_partials(partials, n_partials, red));
+    if (threadIdx.x == 0 && blockIdx.x == 0 && blockIdx.y == 0) ts[0] = nv_decode_scale(s_enc);
+  }
+  __syncthreads();
+
+  const int p = (w & 1) * 32 + l;  // channel pair within the tile: 2p, 2p+1
+  const int j = w >> 1;            // 32-token block within the tile
+  float v0[32], v1[32];
+#pragma unroll
+  for (int t = 0; t < 32; ++t) {
+    const uint32_t pair = *reinterpret_cast<const uint32_t *>(&tile[(32 * j + t) * 128 + 2 * p]);
+    v0[t] = bf16lo(pair);
+    v1[t] = bf16hi(pair);
+  }
+  const int64_t kbt = (FMT == kMX) ? (T >> 5) : (T >> 4);
+
+#pragma unroll
+  for (int half = 0; half < 2; ++half) {
+    float *v = half ? v1 : v0;
+    const int cl = 2 * p + half;  // channel within the tile
+    const int64_t r = c0 + cl;
+    if constexpr (HAD) {
+#pragma unroll
+      for (int t = 0; t < 32; ++t)
+        if ((sign_mask >> t) & 1u) v[t] = -v[t];
+      fwht32(v);
+    }
+    uint32_t codes[4];
+    const int64_t kfirst = t0 + 32 * j;  // first K index of this 32-block
+    if constexpr (FMT == kMX) {
+      float amax = 0.0f;
+#pragma unroll
+      for (int t = 0; t < 32; ++t) amax = fmaxf(amax, fabsf(v[t]));
+      const uint32_t sbyte = mx_scale_byte(amax);
+      const float mult = mx_multiplier(sbyte);
+#pragma unroll
+      for (int t = 0; t < 32; ++t) v[t] = __fmul_rn(v[t], mult);
+      sbuf[cl * 8 + j] = (uint8_t)sbyte;
+    } else {
+#pragma unroll
+      for (int hb = 0; hb < 2; ++hb) {
+        float amax = 0.0f;
+#pragma unroll
+        for (int t = 0; t < 16; ++t) amax = fmaxf(amax, fabsf(v[16 * hb + t]));
+        float mult;
+        const uint32_t sbyte = nv_block_scale(amax, s_enc, &mult);
+#pragma unroll
+        for (int t = 0; t < 16; ++t) v[16 * hb + t] = __fmul_rn(v[16 * hb + t], mult);
+        sbuf[cl * 8 + 2 * j + hb] = (uint8_t)sbyte;
+      }
+    }
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      if constexpr (RND == kSR) {
+        codes[q] = e2m1x8_sr(&v[8 * q], sr_block_bits(seed, (uint64_t)(r * T + kfirst + 8 * q) >> 3));
+      } else {
+        codes[q] = e2m1x8_rne(&v[8 * q]);
+      }
+    }
+    *reinterpret_cast<uint4 *>(payload + r * (T >> 1) + (kfirst >> 1)) =
+        make_uint4(codes[0], codes[1], codes[2], codes[3]);
+  }
+  __syncthreads();
+  // scale words: MX 4 blocks (one word) per channel, NV 8 blocks (two words)
+  if constexpr (FMT == kMX) {
+    if (threadIdx.x < 128) {
+      const int cl = threadIdx.x;
+      const uint32_t word = *reinterpret_cast<const uint32_t *>(&sbuf[cl * 8]);
+      *reinterpret_cast<uint32_t *>(scales + sf_offset(c0 + cl, t0 >> 5, kbt)) = word;
+    }
+  } else {
+    const int cl = threadIdx.x >> 1, h = threadIdx.x & 1;
+    const uint32_t word = *reinterpret_cast<const uint32_t *>(&sbuf[cl * 8 + 4 * h]);
+    *reinterpret_cast<uint32_t *>(scales + sf_offset(c0 + cl, (t0 >> 4) + 4 * h, kbt)) = word;
+  }
+}
+
+// --------------------------------------------------------------------------
+// Diagnostics kernels (element conversions and SR bits, as the quantizers
+// use them).
+// --------------------------------------------------------------------------
+__global__ void debug_convert_kernel(const float *y, const uint32_t *u16, int64_t n, uint8_t *rne,
+                                     uint8_t *sr, uint8_t *e4m3) {
+  const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= n) return;
+  const float v = y[i];
+  rne[i] = (uint8_t)(e2m1x2_rne(v, 0.0f) & 0xF);
+  if (sr) sr[i] = (uint8_t)e2m1_sr(v, u16[i] & 0xFFFFu);
+  if (e4m3) {
+    const float sb = fminf(fmaxf(v, 0.001953125f), 448.0f);
+    e4m3[i] = (uint8_t)e4m3_rne(sb);
+  }
+}
+
+__global__ void debug_sr_bits_kernel(uint64_t seed, const uint64_t *idx, int64_t n, uint32_t *bits) {
+  const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= n) return;
+  const uint64_t e = idx[i];
+  bits[i] = sr_half(sr_block_bits(seed, e >> 3), (int)(e & 7));
+}
+
+// --------------------------------------------------------------------------
+// Host-side launchers (called by the C ABI after validation).
+// --------------------------------------------------------------------------
+int amax_partials_count(int64_t rows, int64_t cols) {
+  const int64_t chunks = rows * (cols >> 3);
+  int64_t blocks = (chunks + 256 * 8 - 1) / (256 * 8);
+  if (blocks > kMaxAmaxPartials) blocks = kMaxAmaxPartials;
+  if (blocks < 1) blocks = 1;
+  return (int)blocks;
+}
+
+cudaError_t launch_tensor_amax(const uint16_t *x, int64_t rows, int64_t cols, int64_t ld,
+                               float *partials, int n_partials, cudaStream_t st) {
+  tensor_amax_kernel<<<n_partials, 256, 0, st>>>(x, rows, cols, ld, partials);
+  return cudaGetLastError();
+}
+
+template <int FMT, int RND>
+static void launch_row(dim3 g, cudaStream_t st, const uint16_t *x, int64_t R, int64_t K, int64_t ld,
+                       uint8_t *p, uint8_t *s, float *ts, const float *part, int np, uint64_t seed) {
+  quant_rowwise_kernel<FMT, RND><<<g, 256, 0, st>>>(x, R, K, ld, p, s, ts, part, np, seed);
+}
+
+cudaError_t launch_quant_rowwise(int fmt, int rnd, const uint16_t *x, int64_t R, int64_t K,
+                                 int64_t ld, uint8_t *payload, uint8_t *scales, float *ts,
+                                 const float *partials, int n_partials, uint64_t seed,
+                                 cudaStream_t st) {
+  dim3 g((unsigned)(K / 128), (unsigned)(R / 128));
+#define FA4_ROW(F, Q) \
+  if (fmt == F && rnd == Q) launch_row<F, Q>(g, st, x, R, K, ld, payload, scales, ts, partials, n_partials, seed);
+  FA4_ROW(kMX, kRNE) FA4_ROW(kMX, kSR) FA4_ROW(kNVG, kRNE) FA4_ROW(kNVG, kSR) FA4_ROW(kNVC, kRNE)
+  FA4_ROW(kNVC, kSR)
+#undef FA4_ROW
+  return cudaGetLastError();
+}
+
+template <int FMT, int RND, bool HAD>
+static void launch_col(dim3 g, cudaStream_t st, const uint16_t *x, int64_t T, int64_t C, int64_t ld,
+                       uint8_t *p, uint8_t *s, float *ts, const float *part, int np, uint64_t seed,
+                       uint32_t mask) {
+  quant_colwise_kernel<FMT, RND, HAD><<<g, 256, 0, st>>>(x, T, C, ld, p, s, ts, part, np, seed, mask);
+}
+
+cudaError_t launch_quant_colwise(int fmt, int rnd, bool hadamard, uint32_t sign_mask,
+                                 const uint16_t *x, int64_t T, int64_t C, int64_t ld,
+                                 uint8_t *payload, uint8_t *scales, float *ts,
+                                 const float *partials, int n_partials, uint64_t seed,
+                                 cudaStream_t st) {
+  dim3 g((unsigned)(C / 128), (unsigned)(T / 128));
+#define FA4_COL(F, Q, H)                                                                      \
+  if (fmt == F && rnd == Q && hadamard == H)                                                  \
+    launch_col<F, Q, H>(g, st, x, T, C, ld, payload, scales, ts, partials, n_partials, seed, \
+                        sign_mask);
+  FA4_COL(kMX, kRNE, false) FA4_COL(kMX, kSR, false) FA4_COL(kMX, kRNE, true)
+  FA4_COL(kMX, kSR, true) FA4_COL(kNVG, kRNE, false) FA4_COL(kNVG, kSR, false)
+  FA4_COL(kNVC, kRNE, false) FA4_COL(kNVC, kSR, false)
+#undef FA4_COL
+  return cudaGetLastError();
+}
+
+cudaError_t launch_debug_convert(const float *y, const uint32_t *u16, int64_t n, uint8_t *rne,
+                                 uint8_t *sr, uint8_t *e4m3, cudaStream_t st) {
+  const unsigned blocks = (unsigned)((n + 255) / 256);
+  if (n > 0) debug_convert_kernel<<<blocks, 256, 0, st>>>(y, u16, n, rne, sr, e4m3);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_debug_sr_bits(uint64_t seed, const uint64_t *idx, int64_t n, uint32_t *bits,
+                                 cudaStream_t st) {
+  const unsigned blocks = (unsigned)((n + 255) / 256);
+  if (n > 0) debug_sr_bits_kernel<<<blocks, 256, 0, st>>>(seed, idx, n, bits);
+  return cudaGetLastError();
+}
+
+}  // namespace fa4

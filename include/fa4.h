@@ -1,0 +1,234 @@
+/*
+ * fa4.h -- C ABI of the B200 (sm_100a) FP4 quantization + block-scaled GEMM
+ * library (libfa4.so).
+ *
+ * The operation is the one the pages on format-aware fusion for FP4 describe:
+ * a quantization producer bound to its scale domain and its consumer layout
+ * ("Format-Aware Fusion: The Engineering Practice That Doubles FP4
+ * Pretraining Throughput", section "The Design Philosophy of Format-Aware
+ * Fusion"), i.e. block amax -> scale -> divide -> E2M1 -> two values per byte
+ * ("FP4 Is No Longer Just a Hardware Feature -- The NVFP4 Software Stack Is
+ * Taking Shape", section "The first change: PyTorch is bringing FP4 packing
+ * into compiler fusion"), with the scales written in the storage the tensor
+ * cores read, followed by the FP4 tensor-core matmul.
+ *
+ * Conventions for every entry point:
+ *  - Pointers named x/X/dY/D/workspace and the members of fa4_qtensor are
+ *    DEVICE pointers, allocated and owned by the caller.  The library never
+ *    allocates device memory and never synchronizes, except
+ *    fa4_check_device_status.
+ *  - `stream` is a cudaStream_t passed as void* (NULL = the legacy default
+ *    stream).  All work is enqueued asynchronously on it.
+ *  - Every function returns an fa4_status; nothing throws across the ABI.
+ *    Argument errors are detected on the host before anything is launched.
+ *    A launch failure returns FA4_ERR_CUDA (cudaGetLastError).
+ *  - Shapes: rows and cols multiples of 128 (GEMM K a multiple of 256);
+ *    leading dimensions in elements,
+ *    multiples of 8 and >= the row length; every pointer 16-byte aligned.
+ *    Anything else returns FA4_ERR_SHAPE / FA4_ERR_ALIGN.
+ *  - Inputs must be finite; with a non-finite input the output bytes are
+ *    unspecified (no error is raised).
+ *  - Workspace: the first FA4_WS_HEADER_BYTES bytes hold a sticky device
+ *    status word that bounded waits inside the kernels set on timeout.  The
+ *    caller zero-fills the workspace (or calls fa4_workspace_init) once
+ *    before first use; fa4_check_device_status reads and clears the word.
+ *  - Thread-safe: no global mutable state except a mutex-guarded cache of
+ *    TMA descriptors keyed by pointer and shape.
+ */
+#ifndef FA4_H
+#define FA4_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define FA4_WS_HEADER_BYTES 256
+
+/* Exported symbols (the library is built with hidden default visibility). */
+#if defined(__GNUC__)
+#define FA4_API __attribute__((visibility("default")))
+#else
+#define FA4_API
+#endif
+
+/* Scale domains ("Format-Aware Fusion...", section "The Design Philosophy of
+ * Format-Aware Fusion": native mxfp, global nvfp, CTA-local nvfp).
+ *  FA4_MXFP4        32-value blocks, power-of-two E8M0 scale byte.
+ *  FA4_NVFP4_GLOBAL 16-value blocks, E4M3 scale byte, one FP32 decode scale
+ *                   for the tensor ("FP4 Is No Longer Just a Hardware
+ *                   Feature...", section "NVFP4 is more than a 4-bit value").
+ *  FA4_NVFP4_CTA    as NVFP4_GLOBAL but one FP32 decode scale per 128x128
+ *                   tile of the quantized operand, [R/128][K/128]. */
+typedef enum { FA4_MXFP4 = 0, FA4_NVFP4_GLOBAL = 1, FA4_NVFP4_CTA = 2 } fa4_format;
+
+/* E2M1 rounding: round-to-nearest-even, or stochastic rounding with 16
+ * Philox4x32-10 bits per element keyed by `seed` ("Format-Aware Fusion...",
+ * section "Two Key Numerical Techniques": row-gradient stochastic rounding). */
+typedef enum { FA4_RNE = 0, FA4_SR = 1 } fa4_round;
+
+/* Orientation of the quantized operand Q[R, K] relative to the bf16 input
+ * x[rows, cols] (row-major, leading dimension ld):
+ *   FA4_ROWWISE: Q = x,   R = rows, K = cols (blocks run along a row of x)
+ *   FA4_COLWISE: Q = x^T, R = cols, K = rows (blocks run down a column of x;
+ *                x^T is never materialized). */
+typedef enum { FA4_ROWWISE = 0, FA4_COLWISE = 1 } fa4_orient;
+
+typedef enum { FA4_OUT_BF16 = 0, FA4_OUT_FP32 = 1 } fa4_out_dtype;
+
+typedef enum {
+  FA4_OK = 0,
+  FA4_ERR_INVALID_ARG = 1, /* null pointer, bad enum value */
+  FA4_ERR_SHAPE = 2,       /* size not a multiple of 128, bad ld, K mismatch */
+  FA4_ERR_ALIGN = 3,       /* pointer not 16-byte aligned */
+  FA4_ERR_UNSUPPORTED = 4, /* e.g. Hadamard with NVFP4, mixed GEMM formats */
+  FA4_ERR_WORKSPACE = 5,   /* workspace missing or smaller than required */
+  FA4_ERR_CUDA = 6,        /* a CUDA runtime call or launch failed */
+  FA4_ERR_TIMEOUT = 7      /* a bounded device wait gave up (device status) */
+} fa4_status;
+
+/* A quantized operand Q[R, K] (all device pointers, caller-owned):
+ *  payload      R*K/2 bytes, K-major: byte j of row r holds element 2j in its
+ *               low nibble and element 2j+1 in its high nibble (E2M1 code =
+ *               sign<<3 | exponent<<1 | mantissa).
+ *  scales       one byte per block (E8M0 for MXFP4, E4M3 for NVFP4) in the
+ *               128-row x 4-block atom layout the block-scaled tensor-core
+ *               MMA reads: byte offset of (row r, block kb), Kb = K/block,
+ *               ((r/128)*(Kb/4) + kb/4)*512 + (r%32)*16 + ((r%128)/32)*4
+ *               + kb%4.  R*Kb bytes.
+ *  tensor_scale FP32 decode scales: NVFP4_GLOBAL 1 value, NVFP4_CTA
+ *               (R/128)*(K/128) values, row-major; unused (may be NULL) for
+ *               MXFP4.  value = e2m1 * block scale * tensor_scale. */
+typedef struct {
+  void *payload;
+  void *scales;
+  float *tensor_scale;
+} fa4_qtensor;
+
+/* Sizes of a quantized operand of the bf16 input x[rows, cols] and the
+ * workspace fa4_quantize needs.  Host only; any output pointer may be NULL.
+ * Errors: FA4_ERR_SHAPE, FA4_ERR_INVALID_ARG. */
+FA4_API fa4_status fa4_quant_sizes(int64_t rows, int64_t cols, fa4_format fmt, fa4_orient orient,
+                           size_t *payload_bytes, size_t *scale_bytes, size_t *tscale_count,
+                           size_t *workspace_bytes);
+
+/* Quantize bf16 x[rows, cols] (leading dimension ld elements) into `out`
+ * ("FP4 Is No Longer Just a Hardware Feature...", section "The first change":
+ * block amax, scale, divide, convert to E2M1, pack two values per byte).
+ * MXFP4 and NVFP4_CTA read x once; NVFP4_GLOBAL reads it twice (tensor amax,
+ * then quantize).  The scale rules:
+ *  MXFP4: e = floor(log2 amax_b) - 2 clamped to [-127, 127] (amax_b = 0 gives
+ *         -127); scale byte e + 127; y = x * 2^-e.
+ *  NVFP4: s_enc = 2688 / amax_t (1 when amax_t is 0 or the quotient is not
+ *         finite), decode scale 1/s_enc; block scale (amax_b / 6) * s_enc
+ *         clamped to [2^-9, 448] and rounded to E4M3; y = x * (s_enc / that
+ *         E4M3 value).  amax_t is the tensor amax (GLOBAL) or the 128x128
+ *         tile amax of Q (CTA).  All binary32, round-to-nearest-even.
+ * Then y -> E2M1 by RNE (|y| >= 6 gives 6, the sign is kept) or SR.  SR bits
+ * for element Q[r][k] come from counter (r*K + k) >> 3 of Philox4x32-10 keyed
+ * by `seed`.  Errors: SHAPE, ALIGN, INVALID_ARG, WORKSPACE, CUDA. */
+FA4_API fa4_status fa4_quantize(const void *x, int64_t rows, int64_t cols, int64_t ld, fa4_format fmt,
+                        fa4_round rnd, fa4_orient orient, uint64_t seed, fa4_qtensor out,
+                        void *workspace, size_t workspace_bytes, void *stream);
+
+/* Column-wise MXFP4 quantization of x[rows, cols] with a fixed-sign 32-point
+ * Hadamard applied to each 32-value block first ("Format-Aware Fusion...",
+ * section "Two Key Numerical Techniques": fixed-sign 32-value Hadamard
+ * weight-gradient preconditioning).  For each block v of 32 consecutive
+ * elements down a column: y = H32 (s .* v), H32 the unnormalised Sylvester
+ * matrix (H H^T = 32 I), s_j = -1 iff bit j of sign_mask, computed by the
+ * butterfly with strides 1,2,4,8,16; then MXFP4 as in fa4_quantize.  A GEMM
+ * of two such operands carries a factor 32: pass alpha = 1/32.
+ * Errors: as fa4_quantize. */
+FA4_API fa4_status fa4_hadamard32_quantize(const void *x, int64_t rows, int64_t cols, int64_t ld,
+                                   uint32_t sign_mask, fa4_round rnd, uint64_t seed,
+                                   fa4_qtensor out, void *workspace, size_t workspace_bytes,
+                                   void *stream);
+
+/* Block-scaled FP4 GEMM on the tcgen05 tensor cores:
+ *   D[m][n] = alpha * sum_k A[m][k] * B[n][k]       (D = alpha A B^T)
+ * with A[M, K] and B[N, K] quantized operands in the same format (both
+ * K-major).  NVFP4_GLOBAL multiplies by the two tensor decode scales;
+ * NVFP4_CTA multiplies every 128-wide K chunk by tsA[m/128][kc] *
+ * tsB[n/128][kc].  FP32 accumulation.  D is row-major [M, N] with leading
+ * dimension ldd elements, bf16 or fp32.  M, N, K multiples of 128.
+ * Errors: SHAPE, ALIGN, INVALID_ARG, UNSUPPORTED, WORKSPACE, CUDA. */
+FA4_API fa4_status fa4_gemm_blockscaled(fa4_qtensor A, fa4_qtensor B, int64_t M, int64_t N, int64_t K,
+                                fa4_format fmt, float alpha, void *D, int64_t ldd,
+                                fa4_out_dtype out_dtype, void *workspace, size_t workspace_bytes,
+                                void *stream);
+
+/* Linear layer compositions for T tokens, Cin inputs, Cout outputs (the
+ * configurations the pages' Llama-3-8B results train: "Format-Aware
+ * Fusion...", section "Empirical Results").  bf16 activations row-major.
+ *
+ * fa4_linear_fwd:   Y[T, Cout] (bf16) = X[T, Cin] W^T.  X is quantized
+ *                   row-wise (RNE) in `fmt` into the workspace; Wq is W[Cout,
+ *                   Cin] quantized row-wise in the same format.
+ * fa4_linear_dgrad: dX[T, Cin] (bf16) = dY[T, Cout] W.  dY is quantized
+ *                   row-wise with `rnd` (SR = row-gradient stochastic
+ *                   rounding) into the workspace; Wq_col is W quantized
+ *                   column-wise ([Cin, Cout] operand) in the same format.
+ * fa4_linear_wgrad: dW[Cout, Cin] = dY^T X, MXFP4: dY and X are quantized
+ *                   column-wise with the fixed-sign Hadamard (sign_mask) and
+ *                   `rnd`, then multiplied with alpha = 1/32.
+ * fa4_linear_ws_bytes gives the workspace each needs (kind 0 fwd, 1 dgrad,
+ * 2 wgrad).  Errors: as the calls they are made of. */
+FA4_API fa4_status fa4_linear_ws_bytes(int kind, int64_t T, int64_t Cin, int64_t Cout, fa4_format fmt,
+                               size_t *workspace_bytes);
+FA4_API fa4_status fa4_linear_fwd(const void *X, fa4_qtensor Wq, int64_t T, int64_t Cin, int64_t Cout,
+                          fa4_format fmt, void *Y, void *workspace, size_t workspace_bytes,
+                          void *stream);
+FA4_API fa4_status fa4_linear_dgrad(const void *dY, fa4_qtensor Wq_col, int64_t T, int64_t Cin,
+                            int64_t Cout, fa4_format fmt, fa4_round rnd, uint64_t seed, void *dX,
+                            void *workspace, size_t workspace_bytes, void *stream);
+FA4_API fa4_status fa4_linear_wgrad(const void *dY, const void *X, int64_t T, int64_t Cin, int64_t Cout,
+                            uint32_t sign_mask, fa4_round rnd, uint64_t seed, void *dW,
+                            fa4_out_dtype out_dtype, void *workspace, size_t workspace_bytes,
+                            void *stream);
+
+/* Zero the workspace header (stream-ordered memset of FA4_WS_HEADER_BYTES). */
+FA4_API fa4_status fa4_workspace_init(void *workspace, size_t workspace_bytes, void *stream);
+
+/* Synchronize `stream`, read the sticky device status word of `workspace`
+ * and clear it.  Returns FA4_OK, FA4_ERR_TIMEOUT (a bounded wait in a kernel
+ * gave up; the kernel returned early and its output is incomplete) or
+ * FA4_ERR_CUDA. */
+FA4_API fa4_status fa4_check_device_status(void *workspace, void *stream);
+
+/* Static description of a status code; never NULL. */
+FA4_API const char *fa4_status_string(fa4_status s);
+
+/* Library version as major*10000 + minor*100 + patch. */
+FA4_API int fa4_version(void);
+
+/* Diagnostics: run the device element conversions the quantizers use on n
+ * fp32 inputs (device pointers).  rne_codes[i] = E2M1 RNE code of y[i];
+ * sr_codes[i] = E2M1 SR code of y[i] with the 16 random bits u16[i] (may be
+ * NULL to skip); e4m3_codes[i] = E4M3 RNE code of the clamped block scale
+ * y[i] (may be NULL to skip).  sr_bits[i] (may be NULL) = the 16 Philox bits
+ * of element index idx[i] under `seed`. */
+FA4_API fa4_status fa4_debug_convert(const float *y, const uint32_t *u16, int64_t n, uint8_t *rne_codes,
+                             uint8_t *sr_codes, uint8_t *e4m3_codes, void *stream);
+FA4_API fa4_status fa4_debug_sr_bits(uint64_t seed, const uint64_t *idx, int64_t n, uint32_t *bits,
+                             void *stream);
+
+/* Diagnostics for the bounded waits: fa4_gemm_blockscaled (fp32 output,
+ * alpha 1) with every wait limited to timeout_ns (0 < timeout_ns <= 2 s)
+ * and, when skip_k_tile >= 0, a producer that never loads the skip_k_tile-th
+ * k-tile it owns, so the consumer's wait must run out.  The kernel then sets
+ * the workspace status word, waits for its own copies in flight, releases
+ * its tensor memory and returns; fa4_check_device_status reports
+ * FA4_ERR_TIMEOUT and the context stays usable. */
+FA4_API fa4_status fa4_debug_gemm_timeout(fa4_qtensor A, fa4_qtensor B, int64_t M, int64_t N, int64_t K,
+                                  fa4_format fmt, void *D, int64_t ldd, int skip_k_tile,
+                                  uint64_t timeout_ns, void *workspace, size_t workspace_bytes,
+                                  void *stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FA4_H */

@@ -84,7 +84,7 @@ def _setup(lib: ctypes.CDLL) -> ctypes.CDLL:
         "orc_sf_offset": (i64, [i64, i64, i64]),
         "orc_sf_bytes": (i64, [i64, i64]),
         "orc_hadamard32": (None, [P, u32, P]),
-        "orc_quantize": (ci, [P, i64, i64, i64, ci, ci, ci, u64, ci, u32, P, P, P]),
+        "orc_quantize": (ci, [P, i64, i64, i64, ci, ci, ci, u64, ci, u32, P, P, P, i64, i64]),
         "orc_dequantize_blocks": (ci, [P, P, i64, i64, ci, P, i64, P]),
         "orc_gemm": (ci, [P, P, P, P, P, P, i64, i64, i64, ci, f64, P, i64, P, i64, P]),
         "orc_e2m1_rne_batch": (None, [P, i64, P]),
@@ -224,7 +224,10 @@ def ts_count(R: int, K: int, fmt: int) -> int:
 
 
 def quantize(x, fmt: int, rnd: int = RNE, orient: int = ROWWISE, seed: int = 0,
-             hadamard_mask: int | None = None) -> QTensor:
+             hadamard_mask: int | None = None, row_range: tuple[int, int] | None = None) -> QTensor:
+    """Quantize bf16 x.  ``row_range=(r0, r1)`` produces only rows r0..r1-1 of the
+    quantized operand (the rest stay zero); second-level scales always cover
+    the whole operand."""
     bits = _bf16_bits(x)
     rows, cols = bits.shape
     R, K = (rows, cols) if orient == ROWWISE else (cols, rows)
@@ -235,7 +238,9 @@ def quantize(x, fmt: int, rnd: int = RNE, orient: int = ROWWISE, seed: int = 0,
     rc = load().orc_quantize(_ptr(bits), rows, cols, cols, fmt, rnd, orient, int(seed),
                              0 if hadamard_mask is None else 1,
                              0 if hadamard_mask is None else int(hadamard_mask) & 0xFFFFFFFF,
-                             _ptr(payload), _ptr(scales), _ptr(ts))
+                             _ptr(payload), _ptr(scales), _ptr(ts),
+                             0 if row_range is None else int(row_range[0]),
+                             0 if row_range is None else int(row_range[1]))
     if rc != 0:
         raise ValueError(f"oracle quantize rejected the arguments (rc={rc})")
     if fmt == MXFP4:

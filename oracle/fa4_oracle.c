@@ -354,7 +354,8 @@ void orc_hadamard32(const float *x, uint32_t sign_mask, float *y) {
 /* amax over the 128x128 tile of Q that holds the block (reading; the pages  */
 /* name only "CTA-local nvfp").                                             */
 /* hadamard: apply orc_hadamard32 to each 32-value block before the scale    */
-/* (MXFP4 only).  SR bits use i = r*K + k.                                   */
+/* (MXFP4 only).  SR bits use i = r*K + k.  Only rows [r_begin, r_end) of Q  */
+/* are produced (all when r_end <= 0), for sampled checks of large tensors.  */
 /* Returns 0 on success, -1 on an unsupported combination.                   */
 /* ------------------------------------------------------------------------ */
 
@@ -373,7 +374,7 @@ static void put_code(uint8_t *payload, int64_t K, int64_t r, int64_t k, int code
 
 int orc_quantize(const uint16_t *x, int64_t rows, int64_t cols, int64_t ld, int fmt, int rnd,
                  int orient, uint64_t seed, int hadamard, uint32_t sign_mask, uint8_t *payload,
-                 uint8_t *scales, float *ts) {
+                 uint8_t *scales, float *ts, int64_t r_begin, int64_t r_end) {
   int64_t R = orient == 0 ? rows : cols;
   int64_t K = orient == 0 ? cols : rows;
   int bs = (fmt == ORC_MXFP4) ? 32 : 16;
@@ -415,8 +416,12 @@ int orc_quantize(const uint16_t *x, int64_t rows, int64_t cols, int64_t ld, int 
       }
   }
 
+  /* rows of Q to produce: [r_begin, r_end) (all rows when r_end <= 0); the
+     second-level scales above always cover the whole operand */
+  if (r_end <= 0 || r_end > R) r_end = R;
+  if (r_begin < 0) r_begin = 0;
   float v[32];
-  for (int64_t r = 0; r < R; ++r) {
+  for (int64_t r = r_begin; r < r_end; ++r) {
     for (int64_t kb = 0; kb < kb_total; ++kb) {
       for (int j = 0; j < bs; ++j) v[j] = q_elem(x, ld, orient, r, kb * bs + j);
       if (hadamard) {

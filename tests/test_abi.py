@@ -1,0 +1,157 @@
+"""Host-only checks of the C ABI: the library loads, exports every function
+include/fa4.h declares, and rejects bad arguments before launching anything.
+No call here reaches a kernel launch, so no GPU is needed."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import fp4_quantization_block_b200 as fa
+import oracle as O
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def declared_functions():
+    src = open(os.path.join(ROOT, "include", "fa4.h")).read()
+    return sorted(set(re.findall(r"^FA4_API[^(]*?\b(fa4_\w+)\s*\(", src, flags=re.M)))
+
+
+def test_header_declares_the_boundary():
+    names = declared_functions()
+    for required in ("fa4_quantize", "fa4_hadamard32_quantize", "fa4_gemm_blockscaled",
+                     "fa4_linear_fwd", "fa4_linear_dgrad", "fa4_linear_wgrad"):
+        assert required in names
+
+
+def test_library_exports_every_declared_symbol():
+    lib = ctypes.CDLL(fa.library_path)
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+
+
+def test_version_and_status_strings():
+    L = fa.lib()
+    assert L.fa4_version() >= 100
+    for s in range(8):
+        assert L.fa4_status_string(s)
+    assert L.fa4_status_string(99) == b"unknown status"
+
+
+@pytest.mark.parametrize("fmt", [fa.MXFP4, fa.NVFP4_GLOBAL, fa.NVFP4_CTA])
+@pytest.mark.parametrize("orient", [fa.ROWWISE, fa.COLWISE])
+def test_quant_sizes_match_the_layout(fmt, orient):
+    rows, cols = 384, 640
+    pb, sb, tc, ws = fa.quant_sizes(rows, cols, fmt, orient)
+    R, K = (rows, cols) if orient == fa.ROWWISE else (cols, rows)
+    assert pb == R * K // 2
+    assert sb == O.sf_bytes(R, K // fa.BLOCK[fmt])
+    assert tc == O.ts_count(R, K, fmt)
+    assert ws >= fa.WS_HEADER_BYTES
+
+
+def _qt(p=0x10000, s=0x20000, t=0x30000):
+    return fa._QT(p, s, t)
+
+
+DEV = 0x7F0000000000  # never dereferenced: every call below fails validation first
+
+
+@pytest.mark.parametrize("case,expect", [
+    (dict(x=None), 1),
+    (dict(rows=100), 2),
+    (dict(cols=200), 2),
+    (dict(ld=120), 2),
+    (dict(ld=132), 2),
+    (dict(x=DEV + 8), 3),
+    (dict(fmt=7), 1),
+    (dict(rnd=5), 1),
+    (dict(orient=3), 1),
+    (dict(ws=None), 5),
+    (dict(ws_bytes=16), 5),
+    (dict(out=fa._QT(0, 0x20000, 0x30000)), 1),
+    (dict(out=fa._QT(0x10008, 0x20000, 0x30000)), 3),
+    (dict(fmt=fa.NVFP4_GLOBAL, out=fa._QT(0x10000, 0x20000, 0)), 1),
+    (dict(fmt=fa.NVFP4_GLOBAL, ws_bytes=256), 5),
+])
+def test_quantize_rejects_bad_arguments(case, expect):
+    a = dict(x=DEV, rows=256, cols=512, ld=512, fmt=fa.MXFP4, rnd=fa.RNE, orient=fa.ROWWISE,
+             out=_qt(), ws=DEV + 4096, ws_bytes=1 << 20)
+    a.update(case)
+    st = fa.lib().fa4_quantize(a["x"], a["rows"], a["cols"], a["ld"], a["fmt"], a["rnd"],
+                               a["orient"], 0, a["out"], a["ws"], a["ws_bytes"], None)
+    assert st == expect
+
+
+def test_hadamard_quantize_rejects_bad_arguments():
+    L = fa.lib()
+    assert L.fa4_hadamard32_quantize(None, 256, 256, 256, 1, 0, 0, _qt(), DEV, 4096, None) == 1
+    assert L.fa4_hadamard32_quantize(DEV, 250, 256, 256, 1, 0, 0, _qt(), DEV, 4096, None) == 2
+    assert L.fa4_hadamard32_quantize(DEV, 256, 256, 256, 1, 9, 0, _qt(), DEV, 4096, None) == 1
+    assert L.fa4_hadamard32_quantize(DEV, 256, 256, 256, 1, 0, 0, _qt(), DEV, 8, None) == 5
+
+
+@pytest.mark.parametrize("case,expect", [
+    (dict(M=100), 2),
+    (dict(K=384), 2),          # K must be a multiple of 256
+    (dict(ldd=100), 2),
+    (dict(D=None), 1),
+    (dict(D=DEV + 4), 3),
+    (dict(fmt=9), 1),
+    (dict(od=3), 1),
+    (dict(ws=None), 5),
+    (dict(ws_bytes=100), 5),
+    (dict(A=fa._QT(0, 0x20000, 0)), 1),
+    (dict(fmt=fa.NVFP4_CTA, B=fa._QT(0x10000, 0x20000, 0)), 1),
+])
+def test_gemm_rejects_bad_arguments(case, expect):
+    a = dict(A=_qt(), B=_qt(), M=256, N=256, K=512, fmt=fa.MXFP4, D=DEV, ldd=256, od=1,
+             ws=DEV + 65536, ws_bytes=4096)
+    a.update(case)
+    st = fa.lib().fa4_gemm_blockscaled(a["A"], a["B"], a["M"], a["N"], a["K"], a["fmt"], 1.0,
+                                       a["D"], a["ldd"], a["od"], a["ws"], a["ws_bytes"], None)
+    assert st == expect
+
+
+def test_linear_workspace_sizes_and_checks():
+    L = fa.lib()
+    n = ctypes.c_size_t()
+    assert L.fa4_linear_ws_bytes(0, 8192, 4096, 6144, fa.NVFP4_GLOBAL, ctypes.byref(n)) == 0
+    assert n.value >= 8192 * 4096 // 2 + 8192 * 4096 // 16
+    assert L.fa4_linear_ws_bytes(2, 8192, 4096, 6144, fa.MXFP4, ctypes.byref(n)) == 0
+    assert n.value >= (4096 + 6144) * 8192 // 2
+    assert L.fa4_linear_ws_bytes(5, 128, 128, 128, 0, ctypes.byref(n)) == 1
+    assert L.fa4_linear_ws_bytes(0, 100, 128, 128, 0, ctypes.byref(n)) == 2
+    assert L.fa4_linear_fwd(DEV, _qt(), 256, 256, 256, fa.MXFP4, DEV, DEV, 64, None) == 5
+    assert L.fa4_linear_dgrad(DEV, _qt(), 256, 256, 256, fa.MXFP4, 4, 0, DEV, DEV, 1 << 20, None) == 1
+    assert L.fa4_linear_wgrad(DEV, None, 256, 256, 256, 1, 0, 0, DEV, 1, DEV, 1 << 24, None) == 1
+
+
+def test_debug_entry_points_reject_bad_arguments():
+    L = fa.lib()
+    assert L.fa4_debug_convert(None, None, 10, DEV, None, None, None) == 1
+    assert L.fa4_debug_convert(DEV, None, 10, DEV, DEV, None, None) == 1
+    assert L.fa4_debug_sr_bits(0, None, 10, DEV, None) == 1
+    assert L.fa4_debug_gemm_timeout(_qt(), _qt(), 256, 256, 512, 0, DEV, 256, 0, 0, DEV, 4096,
+                                    None) == 1
+    assert L.fa4_check_device_status(None, None) == 5
+    assert L.fa4_workspace_init(None, 0, None) == 5
+
+
+def test_product_package_does_not_import_the_oracle():
+    import ast
+    pkg = os.path.join(ROOT, "fp4_quantization_block_b200")
+    for dirpath, _, files in os.walk(pkg):
+        for f in files:
+            path = os.path.join(dirpath, f)
+            if f.endswith(".py"):
+                tree = ast.parse(open(path).read())
+                for node in ast.walk(tree):
+                    if isinstance(node, ast.Import):
+                        assert all(not a.name.startswith("oracle") for a in node.names), path
+                    if isinstance(node, ast.ImportFrom):
+                        assert not (node.module or "").startswith("oracle"), path
+            if f.endswith((".cu", ".cuh", ".h", ".cpp")):
+                assert "fa4_oracle" not in open(path).read(), path
+                assert "orc_" not in open(path).read(), path
