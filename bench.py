@@ -1,0 +1,561 @@
+"""Benchmark of the FP4 hot path on B200.
+
+One step = the linear layers of one Llama-3-8B-shaped transformer block
+(QKV 4096->6144, O 4096->4096, gate+up 4096->28672, down 14336->4096) at 8192
+tokens, forward and backward:
+  fwd    Y  = X W^T     X quantized row-wise NVFP4-global (RNE), block-scaled GEMM
+  dgrad  dX = dY W      dY quantized row-wise MXFP4 with stochastic rounding
+  wgrad  dW = dY^T X    dY and X quantized column-wise MXFP4 with the
+                        fixed-sign 32-point Hadamard (RNE), GEMM with alpha 1/32
+Weights are quantized once before timing (row-wise NVFP4-global for fwd,
+column-wise MXFP4 for dgrad).  Inputs are synthetic (seeded generators in
+workloads.py).  Each step reads ~1.1 GB of bf16 inputs, more than the 126 MB
+L2, so no timed iteration finds its inputs in L2.
+
+Prints one JSON line (rank 0).  `value` is whole-job tokens/s; the three
+metrics the FP4 path is judged on (fused-quantize GB/s, block-scaled GEMM
+TFLOP/s, linear tokens/s) are under "metrics".
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl fa4|reference]
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import workloads  # noqa: E402
+
+METRIC = "fused quantize GB/s; block-scaled FP4 GEMM TFLOPS; 8B-shaped linear tokens/s"
+SIGN_MASK = 0x2545F491
+T = workloads.LLAMA8B_TOKENS
+LAYERS = workloads.LLAMA8B_LINEARS
+BYTES_PER_ELEM = {"mx": 2.0 + 0.5 + 1.0 / 32, "nvg": 2.0 + 2.0 + 0.5 + 1.0 / 16,
+                  "nvc": 2.0 + 0.5 + 1.0 / 16 + 4.0 / (128 * 128)}
+
+
+def _peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            p = json.load(f)
+        return float(p["hbm_gbs"]), float(p["bf16_tflops"]), float(p["bf16_tflops_sustained"]), "measured"
+    except Exception:
+        return 6650.0, 1590.0, 1400.0, "fallback"
+
+
+# --------------------------------------------------------------- clocks ---
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+            time.sleep(0.3)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+        return False
+
+    def summary(self) -> dict:
+        rows = []
+        try:
+            for line in open(self.path):
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) >= 9:
+                    rows.append(parts)
+        except Exception:
+            pass
+        finally:
+            if self.path and os.path.exists(self.path):
+                os.remove(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        smax = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        loaded = [s for s, r in zip(sm, rows) if r[3] and _f(r[3]) > 250.0] or sm
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({n for r in rows for n, v in zip(names, r[5:9]) if v.lower().startswith("active")})
+        return {"sm_mhz": statistics.median(loaded) if loaded else None,
+                "sm_max_mhz": max(smax) if smax else None, "reasons": reasons,
+                "samples": len(rows), "power_w_max": max(_f(r[3]) for r in rows)}
+
+
+def _f(s):
+    try:
+        return float(s)
+    except ValueError:
+        return 0.0
+
+
+# ------------------------------------------------------------ fa4 arm ---
+
+class Block:
+    """Inputs, quantized weights and output buffers of one block's linears."""
+
+    def __init__(self, fa, seed: int, device):
+        self.layers = {}
+        for i, (name, (cin, cout)) in enumerate(LAYERS.items()):
+            s = seed * 1000 + 10 * i
+            x = workloads.act(T, cin, seed=s, device=device)
+            dy = workloads.grad(T, cout, seed=s + 1, device=device)
+            w = workloads.weight(cout, cin, seed=s + 2, device=device)
+            L = dict(cin=cin, cout=cout, x=x, dy=dy, w=w)
+            L["xq"] = fa.empty_qtensor(T, cin, fa.NVFP4_GLOBAL, fa.ROWWISE, device)
+            L["gq"] = fa.empty_qtensor(T, cout, fa.MXFP4, fa.ROWWISE, device)
+            L["gc"] = fa.empty_qtensor(T, cout, fa.MXFP4, fa.COLWISE, device)
+            L["xc"] = fa.empty_qtensor(T, cin, fa.MXFP4, fa.COLWISE, device)
+            L["y"] = torch.empty(T, cout, dtype=torch.bfloat16, device=device)
+            L["dx"] = torch.empty(T, cin, dtype=torch.bfloat16, device=device)
+            L["dw"] = torch.empty(cout, cin, dtype=torch.float32, device=device)
+            self.layers[name] = L
+        self.ws = fa.workspace(1 << 16, device)
+
+    def quantize_weights(self, fa):
+        for L in self.layers.values():
+            L["wq"] = fa.quantize(L["w"], fa.NVFP4_GLOBAL, fa.RNE, fa.ROWWISE, ws=self.ws)
+            L["wc"] = fa.quantize(L["w"], fa.MXFP4, fa.RNE, fa.COLWISE, ws=self.ws)
+
+
+KINDS = ["quant_fwd_nvg", "gemm_fwd", "quant_dgrad_mx_sr", "gemm_dgrad", "quant_wgrad_had",
+         "gemm_wgrad"]
+
+
+def run_step(fa, blk: Block, step: int, events=None):
+    """One fwd+bwd pass over the block's four linears.  With `events`, a CUDA
+    event is recorded after each call (list of (kind, layer, event))."""
+    stream = torch.cuda.current_stream()
+    seed = 1000003 * (step + 1)
+
+    def mark(kind, name):
+        if events is not None:
+            e = torch.cuda.Event(enable_timing=True)
+            e.record(stream)
+            events.append((kind, name, e))
+
+    for name, L in blk.layers.items():
+        fa.quantize(L["x"], fa.NVFP4_GLOBAL, fa.RNE, fa.ROWWISE, out=L["xq"], ws=blk.ws)
+        mark("quant_fwd_nvg", name)
+        fa.gemm(L["xq"], L["wq"], 1.0, out=L["y"], ws=blk.ws)
+        mark("gemm_fwd", name)
+        fa.quantize(L["dy"], fa.MXFP4, fa.SR, fa.ROWWISE, seed=seed, out=L["gq"], ws=blk.ws)
+        mark("quant_dgrad_mx_sr", name)
+        fa.gemm(L["gq"], L["wc"], 1.0, out=L["dx"], ws=blk.ws)
+        mark("gemm_dgrad", name)
+        fa.hadamard32_quantize(L["dy"], SIGN_MASK, fa.RNE, out=L["gc"], ws=blk.ws)
+        fa.hadamard32_quantize(L["x"], SIGN_MASK, fa.RNE, out=L["xc"], ws=blk.ws)
+        mark("quant_wgrad_had", name)
+        fa.gemm(L["gc"], L["xc"], 1.0 / 32, out=L["dw"], ws=blk.ws)
+        mark("gemm_wgrad", name)
+
+
+def kernel_work(kind: str, cin: int, cout: int) -> tuple[float, str]:
+    """Algorithmic work of one call: bytes (quantizers) or FLOPs (GEMMs)."""
+    if kind.startswith("gemm"):
+        return 2.0 * T * cin * cout, "flop"
+    if kind == "quant_fwd_nvg":
+        return BYTES_PER_ELEM["nvg"] * T * cin, "byte"
+    if kind == "quant_dgrad_mx_sr":
+        return BYTES_PER_ELEM["mx"] * T * cout, "byte"
+    return BYTES_PER_ELEM["mx"] * T * (cin + cout), "byte"  # two Hadamard quantizations
+
+
+def launches_per_step() -> int:
+    # per layer: amax + quant (NVG), gemm, quant (SR), gemm, 2 Hadamard quants, gemm
+    return len(LAYERS) * 8
+
+
+def quantize_sweep(fa, device, reps: int = 20) -> list[dict]:
+    """Quantizer sweep shapes (0.5*t_3 with outlier columns), row-wise RNE,
+    rotating over enough input copies that the working set exceeds L2."""
+    out = []
+    for rows, cols in workloads.SWEEP_SHAPES:
+        nbuf = max(1, (512 << 20) // (rows * cols * 2))
+        xs = [workloads.sweep(rows, cols, seed=i, device=device) for i in range(min(nbuf, 8))]
+        for fmt, key in ((fa.MXFP4, "mx"), (fa.NVFP4_GLOBAL, "nvg"), (fa.NVFP4_CTA, "nvc")):
+            for rnd in (fa.RNE, fa.SR):
+                qs = [fa.empty_qtensor(rows, cols, fmt, fa.ROWWISE, device) for _ in xs]
+                ws = fa.workspace(1 << 16, device)
+                for i in range(3):
+                    fa.quantize(xs[i % len(xs)], fmt, rnd, fa.ROWWISE, 1, out=qs[i % len(xs)], ws=ws)
+                torch.cuda.synchronize()
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                e0.record()
+                for i in range(reps):
+                    fa.quantize(xs[i % len(xs)], fmt, rnd, fa.ROWWISE, 1, out=qs[i % len(xs)], ws=ws)
+                e1.record()
+                torch.cuda.synchronize()
+                us = e0.elapsed_time(e1) * 1000.0 / reps
+                gbs = BYTES_PER_ELEM[key] * rows * cols / (us * 1e-6) / 1e9
+                out.append({"shape": [rows, cols], "fmt": key, "rnd": "sr" if rnd else "rne",
+                            "us": round(us, 2), "GBps": round(gbs, 1)})
+                del qs
+        del xs
+        torch.cuda.empty_cache()
+    return out
+
+
+def e2e_run(fa, blk: Block, steps: int, device) -> dict:
+    """Same step through the public linear_* calls with host (pinned) inputs
+    and outputs: the H2D copy of X and dY and the D2H copy of Y, dX and dW of
+    every layer are inside the timed region."""
+    host = {}
+    h2d = d2h = 0
+    for name, L in blk.layers.items():
+        host[name] = dict(x=L["x"].cpu().pin_memory(), dy=L["dy"].cpu().pin_memory(),
+                          y=torch.empty_like(L["y"], device="cpu").pin_memory(),
+                          dx=torch.empty_like(L["dx"], device="cpu").pin_memory(),
+                          dw=torch.empty_like(L["dw"], device="cpu").pin_memory())
+        h2d += L["x"].numel() * 2 + L["dy"].numel() * 2
+        d2h += L["y"].numel() * 2 + L["dx"].numel() * 2 + L["dw"].numel() * 4
+    wsz = max(fa.linear_ws_bytes(k, T, cin, cout, fa.NVFP4_GLOBAL if k == 0 else fa.MXFP4)
+              for k in range(3) for cin, cout in LAYERS.values())
+    ws = fa.workspace(wsz, device)
+
+    def one(step):
+        for name, L in blk.layers.items():
+            H = host[name]
+            L["x"].copy_(H["x"], non_blocking=True)
+            L["dy"].copy_(H["dy"], non_blocking=True)
+            fa.linear_fwd(L["x"], L["wq"], fa.NVFP4_GLOBAL, out=L["y"], ws=ws)
+            fa.linear_dgrad(L["dy"], L["wc"], fa.MXFP4, fa.SR, seed=step, out=L["dx"], ws=ws)
+            fa.linear_wgrad(L["dy"], L["x"], SIGN_MASK, fa.RNE, seed=step, out=L["dw"], ws=ws)
+            H["y"].copy_(L["y"], non_blocking=True)
+            H["dx"].copy_(L["dx"], non_blocking=True)
+            H["dw"].copy_(L["dw"], non_blocking=True)
+
+    one(0)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for s in range(steps):
+        one(s + 1)
+    e1.record()
+    torch.cuda.synchronize()
+    if fa.check_device_status(ws) != 0:
+        raise RuntimeError("device status set during the e2e run")
+    ms = e0.elapsed_time(e1) / steps
+    return {"ms_per_step": ms, "tokens_per_s": T / (ms * 1e-3), "h2d_bytes_per_step": h2d,
+            "d2h_bytes_per_step": d2h}
+
+
+_ORACLE_WEIGHTS = None
+
+
+def _oracle_weights():
+    """Weights quantized by the oracle and expanded to binary64 block values,
+    once (the GPU arm also quantizes weights before timing)."""
+    global _ORACLE_WEIGHTS
+    if _ORACLE_WEIGHTS is None:
+        import oracle as O
+        _ORACLE_WEIGHTS = {}
+        for i, (name, (cin, cout)) in enumerate(LAYERS.items()):
+            w = workloads.weight(cout, cin, seed=10 * i + 2)
+            wq = O.quantize(w, O.NVFP4_GLOBAL)
+            wc = O.quantize(w, O.MXFP4, orient=O.COLWISE)
+            _ORACLE_WEIGHTS[name] = (wq, O.dequantize_blocks(wq), O.dequantize_blocks(wc))
+    return _ORACLE_WEIGHTS
+
+
+def cpu_baseline(sample_tokens: int = 128) -> dict:
+    """The oracle as it stands on a bounded sample of the same step:
+    `sample_tokens` tokens through the four linears, fwd + dgrad + wgrad.
+    Quantization by the C oracle; each GEMM is the oracle's binary64 block
+    values summed by a numpy binary64 matmul (its large-shape path), with the
+    weight operands prepared once outside the timed part."""
+    import oracle as O
+    try:
+        from threadpoolctl import threadpool_info
+        threads = max([d.get("num_threads", 1) for d in threadpool_info()] + [1])
+    except Exception:
+        threads = os.cpu_count() or 1
+    S = sample_tokens
+    prepared = _oracle_weights()
+    inputs = {name: (workloads.act(S, cin, seed=10 * i), workloads.grad(S, cout, seed=10 * i + 1))
+              for i, (name, (cin, cout)) in enumerate(LAYERS.items())}
+    t0 = time.perf_counter()
+    for name in LAYERS:
+        x, dy = inputs[name]
+        wq, wq_blocks, wc_blocks = prepared[name]
+        xq = O.quantize(x, O.NVFP4_GLOBAL)                                       # fwd
+        _ = (O.dequantize_blocks(xq) @ wq_blocks.T) * (float(xq.ts[0]) * float(wq.ts[0]))
+        gq = O.quantize(dy, O.MXFP4, O.SR, seed=1)                               # dgrad
+        _ = O.dequantize_blocks(gq) @ wc_blocks.T
+        gc = O.quantize(dy, O.MXFP4, O.RNE, O.COLWISE, hadamard_mask=SIGN_MASK)  # wgrad
+        xc = O.quantize(x, O.MXFP4, O.RNE, O.COLWISE, hadamard_mask=SIGN_MASK)
+        _ = O.gemm_sampled(gc, xc, 1.0 / 32)
+    dt = time.perf_counter() - t0
+    return {"value": round(S / dt, 3), "unit": "tokens/s", "cores": threads, "kind": "oracle",
+            "sample": f"{S} tokens through the block's 4 linears fwd+dgrad+wgrad, {dt:.2f} s "
+                      f"(weights prepared by the oracle before timing)"}
+
+
+def fa4_arm(args, rank, world, device) -> dict | None:
+    import fp4_quantization_block_b200 as fa
+    fa.lib()
+    hbm, bf16, bf16s, peak_src = _peaks()
+    blk = Block(fa, seed=rank, device=device)
+    t_wq = time.perf_counter()
+    blk.quantize_weights(fa)
+    torch.cuda.synchronize()
+    t_wq = time.perf_counter() - t_wq
+
+    for s in range(args.warmup):
+        run_step(fa, blk, s)
+    torch.cuda.synchronize()
+    if fa.check_device_status(blk.ws) != 0:
+        raise RuntimeError("device status set during warm-up")
+
+    events = []
+    stream = torch.cuda.current_stream()
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(device.index if device.index is not None else 0) as clk:
+        start.record(stream)
+        for s in range(args.steps):
+            events.append(("step_begin", None, None))
+            run_step(fa, blk, args.warmup + s, events)
+        end.record(stream)
+        torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    if fa.check_device_status(blk.ws) != 0:
+        raise RuntimeError("device status set during the timed region")
+    ms_total = start.elapsed_time(end)
+    if world > 1:
+        t = torch.tensor([ms_total], dtype=torch.float64, device=device)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        ms_total = float(t.item())
+    ms_step = ms_total / args.steps
+
+    # per-kind durations from consecutive events (previous event = start of call)
+    per_kind = {k: [0.0, 0.0] for k in KINDS}  # ms, work
+    prev = start
+    for kind, name, ev in events:
+        if kind == "step_begin":
+            continue
+        dt = prev.elapsed_time(ev)
+        cin, cout = LAYERS[name]
+        work, _ = kernel_work(kind, cin, cout)
+        per_kind[kind][0] += dt
+        per_kind[kind][1] += work
+        prev = ev
+    gemm_ms = sum(per_kind[k][0] for k in KINDS if k.startswith("gemm"))
+    gemm_flop = sum(per_kind[k][1] for k in KINDS if k.startswith("gemm"))
+    q_ms = sum(per_kind[k][0] for k in KINDS if k.startswith("quant"))
+    q_bytes = sum(per_kind[k][1] for k in KINDS if k.startswith("quant"))
+    gemm_tflops = gemm_flop / (gemm_ms * 1e-3) / 1e12
+    q_gbs = q_bytes / (q_ms * 1e-3) / 1e9
+    fp4_peak = 4.0 * bf16  # dense FP4 = 4 x dense bf16 (nominal ratio 9 / 2.25 PFLOP/s)
+    breakdown = {k: {"ms_per_step": round(v[0] / args.steps, 4),
+                     ("TFLOPS" if k.startswith("gemm") else "GBps"):
+                         round(v[1] / (v[0] * 1e-3) / (1e12 if k.startswith("gemm") else 1e9), 1)}
+                 for k, v in per_kind.items()}
+    clocks = clk.summary()
+
+    result = None
+    if rank == 0:
+        sweep = quantize_sweep(fa, device) if not args.quick else []
+        e2e = e2e_run(fa, blk, max(2, min(args.steps, 5)), device)
+        cpu = cpu_baseline() if (world == 1 and not args.no_cpu_baseline) else None
+        tok_s = world * T / (ms_step * 1e-3)
+        result = {
+            "metric": METRIC,
+            "value": round(tok_s, 1),
+            "unit": "tokens/s",
+            "n_gpus": world,
+            "steps": args.steps,
+            "warmup": args.warmup,
+            "ms_per_step": round(ms_step, 4),
+            "higher_is_better": True,
+            "scaling": "weak",
+            "vs_baseline": None,
+            "dtype": "e2m1",
+            "data": "synthetic (seeded generators: act N(0,1)+0.5% channels x20, W N(0,0.02), "
+                    "dY N(0,1e-3) x lognormal rows)",
+            "config": {"workload": "llama3-8b-block-linears-fwd-bwd", "tokens": T,
+                       "layers": {k: list(v) for k, v in LAYERS.items()},
+                       "fwd": "NVFP4-global RNE", "dgrad": "MXFP4 row-wise SR",
+                       "wgrad": "MXFP4 column-wise fixed-sign Hadamard-32 RNE, alpha 1/32",
+                       "parallelism": f"replicas x{world}", "l2": "inputs > L2 (1.1 GB bf16 read per step)"},
+            "metrics": {"linear_tokens_per_s": round(tok_s, 1),
+                        "fp4_gemm_TFLOPS": round(gemm_tflops, 1),
+                        "fused_quantize_GBps": round(q_gbs, 1),
+                        "breakdown": breakdown,
+                        "weight_quantize_s": round(t_wq, 4),
+                        "quantize_sweep": sweep},
+            "roofline": {"bound": "tensor", "achieved": round(gemm_tflops, 1),
+                         "peak": round(fp4_peak, 1), "unit": "TFLOP/s",
+                         "frac": round(gemm_tflops / fp4_peak, 4), "traffic": None,
+                         "kernel": "gemm_blockscaled (all 12 GEMMs of the step, flop-weighted)",
+                         "peak_src": f"{peak_src} bf16 burst {bf16} x 4 (nominal FP4/bf16 ratio)"},
+            "roofline_quantize": {"bound": "hbm", "achieved": round(q_gbs, 1), "peak": hbm,
+                                  "unit": "GB/s", "frac": round(q_gbs / hbm, 4),
+                                  "peak_src": f"{peak_src} HBM copy"},
+            "e2e": {"value": round(e2e["tokens_per_s"], 1), "unit": "tokens/s",
+                    "h2d_bytes_per_step": e2e["h2d_bytes_per_step"],
+                    "d2h_bytes_per_step": e2e["d2h_bytes_per_step"],
+                    "ms_per_step": round(e2e["ms_per_step"], 3)},
+            "gpu_launches": launches_per_step() * args.steps,
+            "clocks": clocks,
+            "cpu_baseline": cpu,
+        }
+        del bf16s
+    return result
+
+
+def profile_arm(args, device) -> dict:
+    """Run one call kind on one layer only (warm-up + steps launches), for a
+    profiler capture of a single kernel: --profile KIND:LAYER, KIND one of
+    gemm_fwd, gemm_dgrad, gemm_wgrad, quant_fwd_nvg, quant_dgrad_mx_sr,
+    quant_wgrad_had."""
+    import fp4_quantization_block_b200 as fa
+    kind, layer = args.profile.split(":")
+    cin, cout = LAYERS[layer]
+    x = workloads.act(T, cin, seed=1, device=device)
+    dy = workloads.grad(T, cout, seed=2, device=device)
+    w = workloads.weight(cout, cin, seed=3, device=device)
+    ws = fa.workspace(1 << 16, device)
+    if kind == "gemm_fwd":
+        a, b = fa.quantize(x, fa.NVFP4_GLOBAL, ws=ws), fa.quantize(w, fa.NVFP4_GLOBAL, ws=ws)
+        out = torch.empty(T, cout, dtype=torch.bfloat16, device=device)
+        call = lambda: fa.gemm(a, b, 1.0, out=out, ws=ws)
+    elif kind == "gemm_dgrad":
+        a = fa.quantize(dy, fa.MXFP4, fa.SR, seed=1, ws=ws)
+        b = fa.quantize(w, fa.MXFP4, orient=fa.COLWISE, ws=ws)
+        out = torch.empty(T, cin, dtype=torch.bfloat16, device=device)
+        call = lambda: fa.gemm(a, b, 1.0, out=out, ws=ws)
+    elif kind == "gemm_wgrad":
+        a = fa.hadamard32_quantize(dy, SIGN_MASK, ws=ws)
+        b = fa.hadamard32_quantize(x, SIGN_MASK, ws=ws)
+        out = torch.empty(cout, cin, dtype=torch.float32, device=device)
+        call = lambda: fa.gemm(a, b, 1.0 / 32, out=out, ws=ws)
+    elif kind == "quant_fwd_nvg":
+        q = fa.empty_qtensor(T, cin, fa.NVFP4_GLOBAL, fa.ROWWISE, device)
+        call = lambda: fa.quantize(x, fa.NVFP4_GLOBAL, out=q, ws=ws)
+    elif kind == "quant_dgrad_mx_sr":
+        q = fa.empty_qtensor(T, cout, fa.MXFP4, fa.ROWWISE, device)
+        call = lambda: fa.quantize(dy, fa.MXFP4, fa.SR, seed=1, out=q, ws=ws)
+    elif kind == "quant_wgrad_had":
+        q = fa.empty_qtensor(T, cout, fa.MXFP4, fa.COLWISE, device)
+        call = lambda: fa.hadamard32_quantize(dy, SIGN_MASK, out=q, ws=ws)
+    else:
+        raise SystemExit(f"unknown kind {kind}")
+    for _ in range(args.warmup):
+        call()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(args.steps):
+        call()
+    e1.record()
+    torch.cuda.synchronize()
+    if fa.check_device_status(ws) != 0:
+        raise RuntimeError("device status set")
+    us = e0.elapsed_time(e1) * 1000 / args.steps
+    work, unit = kernel_work(kind, cin, cout)
+    rate = work / (us * 1e-6) / (1e12 if unit == "flop" else 1e9)
+    return {"profile": args.profile, "us_per_call": round(us, 2),
+            ("TFLOPS" if unit == "flop" else "GBps"): round(rate, 1)}
+
+
+# ------------------------------------------------------ reference arm ---
+
+def reference_arm(args) -> dict:
+    """The oracle as it stands, on the host cores: each step is a bounded
+    sample of the same workload (64 tokens through the block's linears)."""
+    _oracle_weights()
+    for _ in range(args.warmup):
+        cpu_baseline(sample_tokens=16)
+    t0 = time.perf_counter()
+    res = None
+    for _ in range(args.steps):
+        res = cpu_baseline(sample_tokens=64)
+    dt = (time.perf_counter() - t0) / args.steps
+    value = 64 / dt
+    return {"impl": "reference", "metric": METRIC, "value": round(value, 3), "unit": "tokens/s",
+            "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(dt * 1e3, 1), "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": "llama3-8b-block-linears-fwd-bwd", "tokens": T},
+            "cpu_baseline": {"value": round(value, 3), "unit": "tokens/s", "cores": res["cores"],
+                             "kind": "oracle", "sample": "64 tokens per step through the block's 4 linears"},
+            "e2e": {"value": round(value, 3), "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="fa4", choices=["fa4", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--quick", action="store_true", help="skip the quantizer sweep")
+    ap.add_argument("--profile", default=None,
+                    help="KIND:LAYER -- run only that call (for a single-kernel profiler capture)")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        if rank == 0:
+            print(json.dumps(reference_arm(args)), flush=True)
+        return
+
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    if world > 1:
+        import datetime
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                             device_id=device)
+    if args.profile:
+        print(json.dumps(profile_arm(args, device)), flush=True)
+        return
+    try:
+        res = fa4_arm(args, rank, world, device)
+        if rank == 0 and res is not None:
+            print(json.dumps(res), flush=True)
+    finally:
+        if world > 1:
+            torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()
