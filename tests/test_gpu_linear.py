@@ -58,7 +58,7 @@ def test_linear_wgrad(rnd):
     # the Hadamard preconditioning leaves dW = dY^T X (up to FP4 error)
     exact = dy.double().T.numpy() @ x.double().numpy()
     rel = np.linalg.norm(dw.cpu().numpy() - exact) / np.linalg.norm(exact)
-    assert rel < 0.2, rel
+    assert rel < (0.2 if rnd == fa.RNE else 0.3), rel  # SR adds zero-mean noise
 
 
 @pytest.mark.parametrize("layer", list(workloads.LLAMA8B_LINEARS), ids=str)
@@ -104,3 +104,21 @@ def test_bounded_wait_times_out_and_context_survives():
     assert fa.check_device_status(ws) == 0
     want = O.gemm(O.quantize(x[:, :256].contiguous(), O.MXFP4), O.quantize(x[:128, 256:].contiguous(), O.MXFP4))
     assert np.allclose(d.cpu().numpy(), want, rtol=0, atol=1e-2)
+
+
+def test_bounded_wait_times_out_in_the_two_sm_kernel():
+    """Same check for the cluster (2-SM) GEMM path (M and N multiples of 256):
+    both CTAs of the pair give up, release their tensor memory and return."""
+    need_gpu()
+    x = workloads.tiny(1)
+    a = torch.cat([x[:, :256], x[:, 256:]], 0)[:256].contiguous()
+    b = x[:, 256:].contiguous()
+    A = to_gpu_qt(O.quantize(a, O.NVFP4_GLOBAL))
+    B = to_gpu_qt(O.quantize(b, O.NVFP4_GLOBAL))
+    ws = fa.workspace(4096)
+    fa.debug_gemm_timeout(A, B, skip_k_tile=0, timeout_ns=20_000_000, ws=ws)
+    assert fa.check_device_status(ws) == 7
+    d = fa.gemm(A, B, ws=ws)
+    assert fa.check_device_status(ws) == 0
+    Ao, Bo = O.quantize(a, O.NVFP4_GLOBAL), O.quantize(b, O.NVFP4_GLOBAL)
+    assert np.abs(d.cpu().numpy() - O.gemm(Ao, Bo)).max() <= O.gemm_tolerance(Ao, Bo)
