@@ -539,384 +539,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 }  // namespace gemm
 
 // ==========================================================================
-// Scale staging by tcgen05.st with a separate scale pipeline.
-//
-// Same output tiles as gemm_kernel (128 x BN per CTA, persistent), but the
-// scale factors take their own path to tensor memory:
-//   warp 10      scale producer: per k-tile, the A and B scale atoms
-//                (contiguous 512-byte runs) by cp.async.bulk into a deep
-//                ring of small shared-memory stages (SF_STAGES);
-//   warps 2..9   scale staging + epilogue: they read each k-tile's atoms
-//                from shared memory and write, with tcgen05.st, only the
-//                words their 32-lane quadrant's MMA slice reads (row 32q + l
-//                of A in column 4a + q; all B rows of atom a in columns
-//                (BN/32)a ..) into a ring of NBUF tensor-memory buffers, up
-//                to NBUF k-tiles ahead of the MMA; at the end of each tile
-//                they drain the accumulator and store it;
-//   warp 0       A/B producer: two TMA tile loads per k-tile (AB_STAGES);
-//   warp 1       MMA issue.
-// Neither tcgen05.cp (whose per-instruction cost in the tensor pipe rivals
-// an MMA) nor the scale staging sits between an A/B stage landing and its
-// MMAs, and the A/B producer issues only two copies per k-tile.
-// ==========================================================================
-namespace gemm_st {
-
-using namespace fa4::gemm;
-
-constexpr int NBUF = 5;       // scale buffers in tensor memory
-constexpr int SF_BASE = 256;  // first column after the accumulator
-constexpr int NUM_THREADS_ST = 352;  // 11 warps
-
-template <int KIND, int BN>
-struct CfgSt {
-  using C = Cfg<KIND>;
-  static constexpr int A_BYTES = BM * BKB;
-  static constexpr int B_BYTES = BN * BKB;
-  static constexpr int SFA_BYTES = C::SFA_BYTES;                  // 128 rows
-  static constexpr int SFB_BYTES = C::SFA_BYTES * (BN / 128);
-  static constexpr int AB_BYTES = A_BYTES + B_BYTES;
-  static constexpr int SF_BYTES = SFA_BYTES + SFB_BYTES;
-  static constexpr int SF_STAGES = (KIND == kMX && BN == 256) ? 8 : 12;
-  static constexpr int BUDGET = 220 * 1024;
-  static constexpr int AB_STAGES_RAW = (BUDGET - SF_STAGES * SF_BYTES) / AB_BYTES;
-  static constexpr int AB_STAGES = AB_STAGES_RAW > 6 ? 6 : AB_STAGES_RAW;
-  static constexpr int OFF_A = 0;
-  static constexpr int OFF_B = OFF_A + AB_STAGES * A_BYTES;
-  static constexpr int OFF_SF = OFF_B + AB_STAGES * B_BYTES;
-  static constexpr int OFF_CTRL = OFF_SF + SF_STAGES * SF_BYTES;
-  // tensor-memory columns of one scale buffer
-  static constexpr int COLS_A = C::ATOMS_K * 4;
-  static constexpr int COLS_B = C::ATOMS_K * (BN / 32);
-  static constexpr int COLS_BUF = COLS_A + COLS_B;
-  static_assert(AB_STAGES >= 2, "shared-memory budget");
-  static_assert(SF_BASE + NBUF * COLS_BUF <= TMEM_COLS, "tensor-memory budget");
-};
-
-struct SmemSt {
-  uint64_t ab_full[6], ab_empty[6];
-  uint64_t sfs_full[12], sfs_empty[12];    // scale stages in shared memory
-  uint64_t sft_full[NBUF], sft_empty[NBUF];  // scale buffers in tensor memory
-  uint64_t acc_full, acc_empty, mma_done;
-  uint32_t tmem_base;
-  int abort;
-};
-
-template <int KIND, int BN>
-constexpr int total_smem_st() {
-  return CfgSt<KIND, BN>::OFF_CTRL + (int)sizeof(SmemSt) + 1024;
-}
-
-__device__ __forceinline__ bool wait_st(uint32_t bar, uint32_t parity, SmemSt *sm, const Params &p,
-                                        uint32_t where) {
-  if (mbar_try_wait(bar, parity)) return true;
-  const uint64_t t0 = globaltimer();
-  while (true) {
-    if (mbar_try_wait(bar, parity)) return true;
-    if (*(volatile int *)&sm->abort) return false;
-    if (globaltimer() - t0 > p.timeout_ns) {
-      *(volatile int *)&sm->abort = 1;
-      if (atomicCAS(p.status, 0u, kStatusTimeout) == 0u) atomicExch(p.status + 1, where);
-      return false;
-    }
-  }
-}
-__device__ __forceinline__ bool warp_wait_st(uint32_t bar, uint32_t parity, SmemSt *sm,
-                                             const Params &p, uint32_t where) {
-  int ok = 0;
-  if ((threadIdx.x & 31) == 0) ok = wait_st(bar, parity, sm, p, where) ? 1 : 0;
-  return __shfl_sync(0xFFFFFFFFu, ok, 0) != 0;
-}
-// wait until the last copy issued into each stage of a ring has landed
-__device__ __forceinline__ void drain_ring(uint64_t *full, int n, uint32_t issued,
-                                           uint32_t last_parity, const Params &p, uint32_t where) {
-  for (int s = 0; s < n; ++s) {
-    if (!((issued >> s) & 1u)) continue;
-    const uint32_t par = (last_parity >> s) & 1u;
-    const uint64_t t0 = globaltimer();
-    while (!mbar_try_wait(smem_u32(&full[s]), par)) {
-      if (globaltimer() - t0 > p.timeout_ns) {
-        if (atomicCAS(p.status, 0u, kStatusTimeout) == 0u) atomicExch(p.status + 1, where | s);
-        break;
-      }
-    }
-  }
-}
-
-__device__ __forceinline__ void tmem_st1(uint32_t taddr, uint32_t v) {
-  asm volatile("tcgen05.st.sync.aligned.32x32b.x1.b32 [%0], {%1};" ::"r"(taddr), "r"(v) : "memory");
-}
-__device__ __forceinline__ void tmem_st4(uint32_t taddr, const uint4 &v) {
-  asm volatile("tcgen05.st.sync.aligned.32x32b.x4.b32 [%0], {%1,%2,%3,%4};" ::"r"(taddr), "r"(v.x),
-               "r"(v.y), "r"(v.z), "r"(v.w)
-               : "memory");
-}
-
-template <int KIND, int BN>
-__global__ void __launch_bounds__(NUM_THREADS_ST, 1)
-    gemm_st_kernel(const __grid_constant__ CUtensorMap map_a,
-                   const __grid_constant__ CUtensorMap map_b, const Params p) {
-  using CS = CfgSt<KIND, BN>;
-  using C = Cfg<KIND>;
-  constexpr int ABS = CS::AB_STAGES, SFS = CS::SF_STAGES;
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                              ~uintptr_t(1023));
-  SmemSt *sm = reinterpret_cast<SmemSt *>(smem + CS::OFF_CTRL);
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-
-  const int num_m = (int)(p.M / BM), num_n = (int)(p.N / BN);
-  const int num_tiles = num_m * num_n;
-  const int KT = (int)(p.K / BK);
-  const int64_t kbt4 = (p.K / C::BS) / 4;
-  const int my_tiles =
-      (int)blockIdx.x < num_tiles ? (num_tiles - (int)blockIdx.x + (int)gridDim.x - 1) / (int)gridDim.x : 0;
-  const int total = my_tiles * KT;  // k-tiles this CTA processes
-
-  if (threadIdx.x == 0) {
-    for (int s = 0; s < ABS; ++s) {
-      mbar_init(smem_u32(&sm->ab_full[s]), 1);
-      mbar_init(smem_u32(&sm->ab_empty[s]), 1);
-    }
-    for (int s = 0; s < SFS; ++s) {
-      mbar_init(smem_u32(&sm->sfs_full[s]), 1);
-      mbar_init(smem_u32(&sm->sfs_empty[s]), 8);
-    }
-    for (int b = 0; b < NBUF; ++b) {
-      mbar_init(smem_u32(&sm->sft_full[b]), 8);
-      mbar_init(smem_u32(&sm->sft_empty[b]), 1);
-    }
-    mbar_init(smem_u32(&sm->acc_full), 1);
-    mbar_init(smem_u32(&sm->acc_empty), 8);
-    mbar_init(smem_u32(&sm->mma_done), 1);
-    sm->abort = 0;
-    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-  }
-  if (warp == 1) {
-    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
-                     smem_u32(&sm->tmem_base)),
-                 "r"(TMEM_COLS)
-                 : "memory");
-    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
-  }
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  const uint32_t tmem = sm->tmem_base;
-
-  if (warp == 0) {
-    // ------------------------------------------------------ A/B producer
-    if (lane == 0) {
-      uint32_t issued = 0, last_parity = 0;
-      int g = 0;
-      bool ok = true;
-      for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
-        int mt, nt;
-        tile_coords(tile, num_m, num_n, p.n_fastest, mt, nt);
-        for (int kt = 0; kt < KT; ++kt, ++g) {
-          const int s = g % ABS;
-          const uint32_t ph = (uint32_t)((g / ABS) & 1);
-          if (!wait_st(smem_u32(&sm->ab_empty[s]), ph ^ 1u, sm, p, 0x100u | s)) {
-            ok = false;
-            break;
-          }
-          if (g == p.debug_skip_stage) continue;
-          const uint32_t fb = smem_u32(&sm->ab_full[s]);
-          mbar_arrive_expect_tx(fb, CS::AB_BYTES);
-          tma_load_2d(smem_u32(smem + CS::OFF_A + s * CS::A_BYTES), &map_a, kt * BKB, mt * BM, fb);
-          tma_load_2d(smem_u32(smem + CS::OFF_B + s * CS::B_BYTES), &map_b, kt * BKB, nt * BN, fb);
-          issued |= 1u << s;
-          last_parity = (last_parity & ~(1u << s)) | (ph << s);
-        }
-      }
-      drain_ring(sm->ab_full, ABS, issued, last_parity, p, 0x400u);
-    }
-  } else if (warp == 10) {
-    // --------------------------------------------------- scale producer
-    if (lane == 0) {
-      uint32_t issued = 0, last_parity = 0;
-      int g = 0;
-      bool ok = true;
-      for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
-        int mt, nt;
-        tile_coords(tile, num_m, num_n, p.n_fastest, mt, nt);
-        for (int kt = 0; kt < KT; ++kt, ++g) {
-          const int s = g % SFS;
-          const uint32_t ph = (uint32_t)((g / SFS) & 1);
-          if (!wait_st(smem_u32(&sm->sfs_empty[s]), ph ^ 1u, sm, p, 0x120u | s)) {
-            ok = false;
-            break;
-          }
-          const uint32_t fb = smem_u32(&sm->sfs_full[s]);
-          mbar_arrive_expect_tx(fb, CS::SF_BYTES);
-          const uint32_t dst = smem_u32(smem + CS::OFF_SF + s * CS::SF_BYTES);
-          bulk_load(dst, p.a_scales + ((int64_t)mt * kbt4 + (int64_t)kt * C::ATOMS_K) * 512,
-                    CS::SFA_BYTES, fb);
-#pragma unroll
-          for (int nb = 0; nb < BN / 128; ++nb)
-            bulk_load(dst + CS::SFA_BYTES + nb * C::SFA_BYTES,
-                      p.b_scales + ((int64_t)(nt * (BN / 128) + nb) * kbt4 + (int64_t)kt * C::ATOMS_K) * 512,
-                      C::SFA_BYTES, fb);
-          issued |= 1u << s;
-          last_parity = (last_parity & ~(1u << s)) | (ph << s);
-        }
-      }
-      drain_ring(sm->sfs_full, SFS, issued, last_parity, p, 0x420u);
-    }
-  } else if (warp == 1) {
-    // ----------------------------------------------------------- MMA issue
-    if (lane == 0) {
-      uint32_t acc_phase = 0;
-      bool ok = true;
-      int g = 0;
-      for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
-        if (!wait_st(smem_u32(&sm->acc_empty), acc_phase ^ 1u, sm, p, 0x200u)) break;
-        tc_fence_after();
-        for (int kt = 0; kt < KT; ++kt, ++g) {
-          const int s = g % ABS, b = g % NBUF;
-          if (!wait_st(smem_u32(&sm->sft_full[b]), (uint32_t)((g / NBUF) & 1), sm, p, 0x230u | b) ||
-              !wait_st(smem_u32(&sm->ab_full[s]), (uint32_t)((g / ABS) & 1), sm, p, 0x210u | s)) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-          const uint32_t a_base = smem_u32(smem + CS::OFF_A + s * CS::A_BYTES);
-          const uint32_t b_base = smem_u32(smem + CS::OFF_B + s * CS::B_BYTES);
-          const uint32_t sf_col = tmem + SF_BASE + b * CS::COLS_BUF;
-#pragma unroll
-          for (int j = 0; j < BK / 64; ++j) {
-            const int a = (KIND == kMX) ? (j >> 1) : j;
-            const uint32_t sf_id = (KIND == kMX) ? (uint32_t)(2 * (j & 1)) : 0u;
-            const uint32_t sfa = (sf_col + 4 * a) | (sf_id << 30);
-            const uint32_t sfb = (sf_col + CS::COLS_A + (BN / 32) * a) | (sf_id << 30);
-            tc_mma<KIND>(tmem, operand_desc(a_base + j * 32), operand_desc(b_base + j * 32),
-                         instr_desc<KIND, BN>(sf_id), sfa, sfb, (kt > 0 || j > 0) ? 1u : 0u);
-          }
-          tc_commit(smem_u32(&sm->ab_empty[s]));
-          tc_commit(smem_u32(&sm->sft_empty[b]));
-        }
-        if (ok) tc_commit(smem_u32(&sm->acc_full));
-        acc_phase ^= 1u;
-      }
-      tc_commit(smem_u32(&sm->mma_done));
-      const uint64_t t0 = globaltimer();
-      while (!mbar_try_wait(smem_u32(&sm->mma_done), 0)) {
-        if (globaltimer() - t0 > p.timeout_ns) {
-          if (atomicCAS(p.status, 0u, kStatusTimeout) == 0u) atomicExch(p.status + 1, 0x500u);
-          break;
-        }
-      }
-    }
-  } else {
-    // ----------------------------------------- scale staging + epilogue
-    const int q = warp & 3;         // tensor-memory lane quadrant of this warp
-    const int h = (warp - 2) >> 2;  // which of the quadrant's two warps
-    const uint32_t lane_base = tmem + ((uint32_t)(32 * q) << 16);
-    constexpr int COLS = BN / 2;
-    constexpr int NCH = COLS / 32;
-    float alpha_g = p.alpha;
-    if constexpr (KIND == kNVG) alpha_g = p.alpha * p.a_ts[0] * p.b_ts[0];
-
-    // stage the scales of k-tile g into tensor-memory buffer g % NBUF
-    auto stage_scales = [&](int g) -> bool {
-      const int s = g % SFS, b = g % NBUF;
-      if (!warp_wait_st(smem_u32(&sm->sfs_full[s]), (uint32_t)((g / SFS) & 1), sm, p, 0x320u | s))
-        return false;
-      if (g >= NBUF &&
-          !warp_wait_st(smem_u32(&sm->sft_empty[b]), (uint32_t)(((g / NBUF) & 1) ^ 1), sm, p, 0x330u | b))
-        return false;
-      tc_fence_after();
-      const uint8_t *sfa_s = smem + CS::OFF_SF + s * CS::SF_BYTES;
-      const uint8_t *sfb_s = sfa_s + CS::SFA_BYTES;
-      const uint32_t col = lane_base + SF_BASE + b * CS::COLS_BUF;
-      if (h == 0) {
-        // A: row 32q + lane is word q of atom row `lane`
-#pragma unroll
-        for (int a = 0; a < C::ATOMS_K; ++a)
-          tmem_st1(col + 4 * a + q, *reinterpret_cast<const uint32_t *>(sfa_s + a * 512 + lane * 16 + 4 * q));
-      }
-      // B: atom a of each 128-row block: row 32w + lane is word w of atom row `lane`
-#pragma unroll
-      for (int a = h; a < C::ATOMS_K; a += 2) {
-#pragma unroll
-        for (int nb = 0; nb < BN / 128; ++nb)
-          tmem_st4(col + CS::COLS_A + (BN / 32) * a + 4 * nb,
-                   *reinterpret_cast<const uint4 *>(sfb_s + nb * C::SFA_BYTES + a * 512 + lane * 16));
-      }
-      asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) {
-        mbar_arrive(smem_u32(&sm->sfs_empty[s]));
-        mbar_arrive(smem_u32(&sm->sft_full[b]));
-      }
-      return true;
-    };
-
-    uint32_t acc_phase = 0;
-    int g = 0;
-    bool ok = true;
-    int it = 0;
-    for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x, ++it) {
-      // scales for the rest of this tile and the first NBUF k-tiles of the
-      // next one, then this tile's epilogue
-      const int until = min(total, (it + 1) * KT + NBUF);
-      for (; g < until; ++g)
-        if (!stage_scales(g)) {
-          ok = false;
-          break;
-        }
-      if (!ok) break;
-      int mt, nt;
-        tile_coords(tile, num_m, num_n, p.n_fastest, mt, nt);
-      if (!warp_wait_st(smem_u32(&sm->acc_full), acc_phase, sm, p, 0x310u)) break;
-      tc_fence_after();
-      uint32_t r[COLS];
-#pragma unroll
-      for (int c = 0; c < NCH; ++c) tmem_ld32(lane_base + h * COLS + 32 * c, &r[32 * c]);
-      tmem_wait_ld();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(smem_u32(&sm->acc_empty));
-      acc_phase ^= 1u;
-      const int64_t row = (int64_t)mt * BM + 32 * q + lane;
-      const int64_t colg = (int64_t)nt * BN + h * COLS;
-      if (p.out_fp32) {
-        float *dst = reinterpret_cast<float *>(p.D) + row * p.ldd + colg;
-#pragma unroll
-        for (int i = 0; i < COLS; i += 4)
-          *reinterpret_cast<float4 *>(dst + i) =
-              make_float4(__uint_as_float(r[i]) * alpha_g, __uint_as_float(r[i + 1]) * alpha_g,
-                          __uint_as_float(r[i + 2]) * alpha_g, __uint_as_float(r[i + 3]) * alpha_g);
-      } else {
-        uint16_t *dst = reinterpret_cast<uint16_t *>(p.D) + row * p.ldd + colg;
-#pragma unroll
-        for (int i = 0; i < COLS; i += 8) {
-          uint32_t w[4];
-#pragma unroll
-          for (int u = 0; u < 4; ++u) {
-            __nv_bfloat162 b2 = __floats2bfloat162_rn(__uint_as_float(r[i + 2 * u]) * alpha_g,
-                                                      __uint_as_float(r[i + 2 * u + 1]) * alpha_g);
-            w[u] = *reinterpret_cast<uint32_t *>(&b2);
-          }
-          *reinterpret_cast<uint4 *>(dst + i) = make_uint4(w[0], w[1], w[2], w[3]);
-        }
-      }
-    }
-  }
-
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  if (warp == 1) {
-    __syncwarp();
-    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(TMEM_COLS)
-                 : "memory");
-  }
-}
-
-}  // namespace gemm_st
-
-// ==========================================================================
 // 2-SM variant.  A cluster of two CTAs (ranks 0 and 1) computes a 256 x 256
 // output tile with tcgen05.mma.cta_group::2 (M = 256, N = 256): CTA r holds
 // A rows 128r..128r+127 and B rows 128r..128r+127 of the pair tile in its
@@ -1264,6 +886,475 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 }
 
 }  // namespace gemm2
+
+// ==========================================================================
+// Scale staging by tcgen05.st with a separate scale pipeline.
+//
+// Output tiles of 128 x BN per CTA (PAIR = false) or 256 x 256 per cluster
+// pair with tcgen05.mma.cta_group::2 (PAIR = true, see gemm2), persistent.
+// The scale factors take their own path to tensor memory:
+//   warp 10      scale producer: per k-tile, the A and B scale atoms
+//                (contiguous 512-byte runs) by cp.async.bulk into a deep
+//                ring of small shared-memory stages (SF_STAGES);
+//   warps 2..9   scale staging + epilogue: they read each k-tile's atoms
+//                from shared memory and write, with tcgen05.st, only the
+//                words their 32-lane quadrant's MMA slice reads (row 32q + l
+//                of A in column 4a + q; all B rows of atom a in columns
+//                (BN/32)a ..) into a ring of NBUF tensor-memory buffers, up
+//                to NBUF k-tiles ahead of the MMA; at the end of each tile
+//                they drain the accumulator and store it;
+//   warp 0       A/B producer: two TMA tile loads per k-tile (AB_STAGES);
+//   warp 1       MMA issue (the pair's leader only).
+// Neither tcgen05.cp (whose per-instruction cost in the tensor pipe rivals
+// an MMA) nor the scale staging sits between an A/B stage landing and its
+// MMAs, and the A/B producer issues only two copies per k-tile.  In a pair
+// each CTA stages its own A rows' scales and all 256 B rows' scales into its
+// own tensor memory; the leader's MMA waits for both CTAs' stagers.
+// ==========================================================================
+namespace gemm_st {
+
+using namespace fa4::gemm;
+using namespace fa4::gemm2;
+
+constexpr int NBUF = 5;       // scale buffers in tensor memory
+constexpr int SF_BASE = 256;  // first column after the accumulator
+constexpr int NUM_THREADS_ST = 352;  // 11 warps
+
+template <int KIND, int BN, bool PAIR>
+struct CfgSt {
+  using C = Cfg<KIND>;
+  static constexpr int TILE_M = PAIR ? 256 : 128;
+  static constexpr int B_ROWS = PAIR ? 128 : BN;               // B rows in this CTA
+  static constexpr int A_BYTES = 128 * BKB;
+  static constexpr int B_BYTES = B_ROWS * BKB;
+  static constexpr int SFA_BYTES = C::SFA_BYTES;                // 128 rows
+  static constexpr int SFB_BYTES = C::SFA_BYTES * (BN / 128);   // all BN rows
+  static constexpr int AB_BYTES = A_BYTES + B_BYTES;
+  static constexpr int SF_BYTES = SFA_BYTES + SFB_BYTES;
+  static constexpr int SF_STAGES = (PAIR || (KIND == kMX && BN == 256)) ? 8 : 12;
+  static constexpr int BUDGET = 220 * 1024;
+  static constexpr int AB_STAGES_RAW = (BUDGET - SF_STAGES * SF_BYTES) / AB_BYTES;
+  static constexpr int AB_STAGES = AB_STAGES_RAW > 6 ? 6 : AB_STAGES_RAW;
+  static constexpr int OFF_A = 0;
+  static constexpr int OFF_B = OFF_A + AB_STAGES * A_BYTES;
+  static constexpr int OFF_SF = OFF_B + AB_STAGES * B_BYTES;
+  static constexpr int OFF_CTRL = OFF_SF + SF_STAGES * SF_BYTES;
+  // tensor-memory columns of one scale buffer
+  static constexpr int COLS_A = C::ATOMS_K * 4;
+  static constexpr int COLS_B = C::ATOMS_K * (BN / 32);
+  static constexpr int COLS_BUF = COLS_A + COLS_B;
+  static constexpr int ARRIVALS = PAIR ? 16 : 8;  // stager / epilogue warps feeding the MMA
+  static_assert(!PAIR || BN == 256, "a pair computes 256-wide tiles");
+  static_assert(AB_STAGES >= 2, "shared-memory budget");
+  static_assert(SF_BASE + NBUF * COLS_BUF <= TMEM_COLS, "tensor-memory budget");
+};
+
+struct SmemSt {
+  uint64_t ab_full[6], ab_empty[6];
+  uint64_t sfs_full[12], sfs_empty[12];      // scale stages in shared memory
+  uint64_t sft_full[NBUF], sft_empty[NBUF];  // scale buffers in tensor memory
+  uint64_t acc_full, acc_empty, mma_done;
+  uint32_t tmem_base;
+  int abort;
+};
+
+template <int KIND, int BN, bool PAIR>
+constexpr int total_smem_st() {
+  return CfgSt<KIND, BN, PAIR>::OFF_CTRL + (int)sizeof(SmemSt) + 1024;
+}
+
+__device__ __forceinline__ bool wait_st(uint32_t bar, uint32_t parity, SmemSt *sm, const Params &p,
+                                        uint32_t where) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = globaltimer();
+  while (true) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if (*(volatile int *)&sm->abort) return false;
+    if (globaltimer() - t0 > p.timeout_ns) {
+      *(volatile int *)&sm->abort = 1;
+      if (atomicCAS(p.status, 0u, kStatusTimeout) == 0u) atomicExch(p.status + 1, where);
+      return false;
+    }
+  }
+}
+__device__ __forceinline__ bool warp_wait_st(uint32_t bar, uint32_t parity, SmemSt *sm,
+                                             const Params &p, uint32_t where) {
+  int ok = 0;
+  if ((threadIdx.x & 31) == 0) ok = wait_st(bar, parity, sm, p, where) ? 1 : 0;
+  return __shfl_sync(0xFFFFFFFFu, ok, 0) != 0;
+}
+// wait until the last copy issued into each stage of a ring has landed
+__device__ __forceinline__ void drain_ring(uint64_t *full, int n, uint32_t issued,
+                                           uint32_t last_parity, const Params &p, uint32_t where) {
+  for (int s = 0; s < n; ++s) {
+    if (!((issued >> s) & 1u)) continue;
+    const uint32_t par = (last_parity >> s) & 1u;
+    const uint64_t t0 = globaltimer();
+    while (!mbar_try_wait(smem_u32(&full[s]), par)) {
+      if (globaltimer() - t0 > p.timeout_ns) {
+        if (atomicCAS(p.status, 0u, kStatusTimeout) == 0u) atomicExch(p.status + 1, where | s);
+        break;
+      }
+    }
+  }
+}
+
+// Arrive on a barrier of the pair's leader from the peer CTA.  Relaxed: what
+// the arrival publishes is tensor memory already completed by
+// tcgen05.wait::st / wait::ld and ordered by tcgen05.fence, and a release at
+// cluster scope would also wait for this thread's outstanding global stores
+// (measured ~1000 cycles per arrival).
+__device__ __forceinline__ void mbar_arrive_remote_relaxed(uint32_t bar_cluster) {
+  asm volatile("mbarrier.arrive.relaxed.cluster.shared::cluster.b64 _, [%0];" ::"r"(bar_cluster)
+               : "memory");
+}
+
+__device__ __forceinline__ void tmem_st1(uint32_t taddr, uint32_t v) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x1.b32 [%0], {%1};" ::"r"(taddr), "r"(v) : "memory");
+}
+__device__ __forceinline__ void tmem_st4(uint32_t taddr, const uint4 &v) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x4.b32 [%0], {%1,%2,%3,%4};" ::"r"(taddr), "r"(v.x),
+               "r"(v.y), "r"(v.z), "r"(v.w)
+               : "memory");
+}
+
+template <int KIND, int BN, bool PAIR>
+__global__ void __launch_bounds__(NUM_THREADS_ST, 1)
+    gemm_st_kernel(const __grid_constant__ CUtensorMap map_a,
+                   const __grid_constant__ CUtensorMap map_b, const Params p) {
+  using CS = CfgSt<KIND, BN, PAIR>;
+  using C = Cfg<KIND>;
+  constexpr int ABS = CS::AB_STAGES, SFS = CS::SF_STAGES;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                              ~uintptr_t(1023));
+  SmemSt *sm = reinterpret_cast<SmemSt *>(smem + CS::OFF_CTRL);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = PAIR ? cluster_rank() : 0u;
+  const int unit = PAIR ? (int)(blockIdx.x >> 1) : (int)blockIdx.x;      // tile-walking unit
+  const int nunits = PAIR ? (int)(gridDim.x >> 1) : (int)gridDim.x;
+
+  const int num_m = (int)(p.M / CS::TILE_M), num_n = (int)(p.N / BN);
+  const int num_tiles = num_m * num_n;
+  const int KT = (int)(p.K / BK);
+  const int64_t kbt4 = (p.K / C::BS) / 4;
+  const int my_tiles = unit < num_tiles ? (num_tiles - unit + nunits - 1) / nunits : 0;
+  const int total = my_tiles * KT;  // k-tiles this CTA processes
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < ABS; ++s) {
+      mbar_init(smem_u32(&sm->ab_full[s]), 1);
+      mbar_init(smem_u32(&sm->ab_empty[s]), 1);
+    }
+    for (int s = 0; s < SFS; ++s) {
+      mbar_init(smem_u32(&sm->sfs_full[s]), 1);
+      mbar_init(smem_u32(&sm->sfs_empty[s]), 8);
+    }
+    for (int b = 0; b < NBUF; ++b) {
+      mbar_init(smem_u32(&sm->sft_full[b]), CS::ARRIVALS);
+      mbar_init(smem_u32(&sm->sft_empty[b]), 1);
+    }
+    mbar_init(smem_u32(&sm->acc_full), 1);
+    mbar_init(smem_u32(&sm->acc_empty), CS::ARRIVALS);
+    mbar_init(smem_u32(&sm->mma_done), 1);
+    sm->abort = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (warp == 1) {
+    if constexpr (PAIR) {
+      asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                       smem_u32(&sm->tmem_base)),
+                   "r"(TMEM_COLS)
+                   : "memory");
+      asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+    } else {
+      asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                       smem_u32(&sm->tmem_base)),
+                   "r"(TMEM_COLS)
+                   : "memory");
+      asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if constexpr (PAIR) {
+    __syncwarp();
+    cluster_sync();  // the peer's barriers exist before any remote arrive
+  }
+  tc_fence_after();
+  const uint32_t tmem = sm->tmem_base;
+  // barriers the pair's MMA waits on live in the leader (rank 0)
+  auto leader_addr = [&](const void *local) -> uint32_t {
+    return PAIR ? map_to_rank(smem_u32(local), 0) : smem_u32(local);
+  };
+
+  if (warp == 0) {
+    // ------------------------------------------------------ A/B producer
+    if (lane == 0) {
+      uint32_t issued = 0, last_parity = 0;
+      int g = 0;
+      bool ok = true;
+      for (int tile = unit; tile < num_tiles && ok; tile += nunits) {
+        int mt, nt;
+        tile_coords(tile, num_m, num_n, p.n_fastest, mt, nt);
+        for (int kt = 0; kt < KT; ++kt, ++g) {
+          const int s = g % ABS;
+          const uint32_t ph = (uint32_t)((g / ABS) & 1);
+          if (!wait_st(smem_u32(&sm->ab_empty[s]), ph ^ 1u, sm, p, 0x100u | s)) {
+            ok = false;
+            break;
+          }
+          if (g == p.debug_skip_stage) continue;
+          const uint32_t a_dst = smem_u32(smem + CS::OFF_A + s * CS::A_BYTES);
+          const uint32_t b_dst = smem_u32(smem + CS::OFF_B + s * CS::B_BYTES);
+          if constexpr (PAIR) {
+            const uint32_t fb = leader_addr(&sm->ab_full[s]);
+            if (rank == 0) mbar_arrive_expect_tx(smem_u32(&sm->ab_full[s]), 2 * CS::AB_BYTES);
+            tma_load_2d_pair(a_dst, &map_a, kt * BKB, mt * 256 + (int)rank * 128, fb);
+            tma_load_2d_pair(b_dst, &map_b, kt * BKB, nt * 256 + (int)rank * 128, fb);
+          } else {
+            const uint32_t fb = smem_u32(&sm->ab_full[s]);
+            mbar_arrive_expect_tx(fb, CS::AB_BYTES);
+            tma_load_2d(a_dst, &map_a, kt * BKB, mt * BM, fb);
+            tma_load_2d(b_dst, &map_b, kt * BKB, nt * BN, fb);
+          }
+          issued |= 1u << s;
+          last_parity = (last_parity & ~(1u << s)) | (ph << s);
+        }
+      }
+      if (!PAIR || rank == 0) {
+        drain_ring(sm->ab_full, ABS, issued, last_parity, p, 0x400u);
+      } else if (!ok) {
+        // the peer's copies complete on the leader's barriers: give any
+        // copy still in flight time to land before this CTA can leave
+        const uint64_t t0 = globaltimer();
+        while (globaltimer() - t0 < 200000ull) {
+        }
+      }
+    }
+  } else if (warp == 10) {
+    // --------------------------------------------------- scale producer
+    if (lane == 0) {
+      uint32_t issued = 0, last_parity = 0;
+      int g = 0;
+      bool ok = true;
+      for (int tile = unit; tile < num_tiles && ok; tile += nunits) {
+        int mt, nt;
+        tile_coords(tile, num_m, num_n, p.n_fastest, mt, nt);
+        const int rb_a = PAIR ? mt * 2 + (int)rank : mt;
+        for (int kt = 0; kt < KT; ++kt, ++g) {
+          const int s = g % SFS;
+          const uint32_t ph = (uint32_t)((g / SFS) & 1);
+          if (!wait_st(smem_u32(&sm->sfs_empty[s]), ph ^ 1u, sm, p, 0x120u | s)) {
+            ok = false;
+            break;
+          }
+          const uint32_t fb = smem_u32(&sm->sfs_full[s]);
+          mbar_arrive_expect_tx(fb, CS::SF_BYTES);
+          const uint32_t dst = smem_u32(smem + CS::OFF_SF + s * CS::SF_BYTES);
+          bulk_load(dst, p.a_scales + ((int64_t)rb_a * kbt4 + (int64_t)kt * C::ATOMS_K) * 512,
+                    CS::SFA_BYTES, fb);
+#pragma unroll
+          for (int nb = 0; nb < BN / 128; ++nb)
+            bulk_load(dst + CS::SFA_BYTES + nb * C::SFA_BYTES,
+                      p.b_scales + ((int64_t)(nt * (BN / 128) + nb) * kbt4 + (int64_t)kt * C::ATOMS_K) * 512,
+                      C::SFA_BYTES, fb);
+          issued |= 1u << s;
+          last_parity = (last_parity & ~(1u << s)) | (ph << s);
+        }
+      }
+      drain_ring(sm->sfs_full, SFS, issued, last_parity, p, 0x420u);
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------ MMA issue (leader)
+    if (lane == 0 && rank == 0) {
+      uint32_t acc_phase = 0;
+      bool ok = true;
+      int g = 0;
+      for (int tile = unit; tile < num_tiles && ok; tile += nunits) {
+        if (!wait_st(smem_u32(&sm->acc_empty), acc_phase ^ 1u, sm, p, 0x200u)) break;
+        tc_fence_after();
+        for (int kt = 0; kt < KT; ++kt, ++g) {
+          const int s = g % ABS, b = g % NBUF;
+          if (!wait_st(smem_u32(&sm->sft_full[b]), (uint32_t)((g / NBUF) & 1), sm, p, 0x230u | b) ||
+              !wait_st(smem_u32(&sm->ab_full[s]), (uint32_t)((g / ABS) & 1), sm, p, 0x210u | s)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a_base = smem_u32(smem + CS::OFF_A + s * CS::A_BYTES);
+          const uint32_t b_base = smem_u32(smem + CS::OFF_B + s * CS::B_BYTES);
+          const uint32_t sf_col = tmem + SF_BASE + b * CS::COLS_BUF;
+#pragma unroll
+          for (int j = 0; j < BK / 64; ++j) {
+            const int a = (KIND == kMX) ? (j >> 1) : j;
+            const uint32_t sf_id = (KIND == kMX) ? (uint32_t)(2 * (j & 1)) : 0u;
+            const uint32_t sfa = (sf_col + 4 * a) | (sf_id << 30);
+            const uint32_t sfb = (sf_col + CS::COLS_A + (BN / 32) * a) | (sf_id << 30);
+            const uint32_t acc = (kt > 0 || j > 0) ? 1u : 0u;
+            if constexpr (PAIR)
+              tc_mma_pair<KIND>(tmem, operand_desc(a_base + j * 32), operand_desc(b_base + j * 32),
+                                instr_desc_pair<KIND>(sf_id), sfa, sfb, acc);
+            else
+              tc_mma<KIND>(tmem, operand_desc(a_base + j * 32), operand_desc(b_base + j * 32),
+                           instr_desc<KIND, BN>(sf_id), sfa, sfb, acc);
+          }
+          if constexpr (PAIR) {
+            tc_commit_pair(smem_u32(&sm->ab_empty[s]), (uint16_t)3);
+            tc_commit_pair(smem_u32(&sm->sft_empty[b]), (uint16_t)3);
+          } else {
+            tc_commit(smem_u32(&sm->ab_empty[s]));
+            tc_commit(smem_u32(&sm->sft_empty[b]));
+          }
+        }
+        if (ok) {
+          if constexpr (PAIR)
+            tc_commit_pair(smem_u32(&sm->acc_full), (uint16_t)3);
+          else
+            tc_commit(smem_u32(&sm->acc_full));
+        }
+        acc_phase ^= 1u;
+      }
+      if constexpr (PAIR)
+        tc_commit_pair(smem_u32(&sm->mma_done), (uint16_t)1);
+      else
+        tc_commit(smem_u32(&sm->mma_done));
+      const uint64_t t0 = globaltimer();
+      while (!mbar_try_wait(smem_u32(&sm->mma_done), 0)) {
+        if (globaltimer() - t0 > p.timeout_ns) {
+          if (atomicCAS(p.status, 0u, kStatusTimeout) == 0u) atomicExch(p.status + 1, 0x500u);
+          break;
+        }
+      }
+    }
+  } else {
+    // ----------------------------------------- scale staging + epilogue
+    const int q = warp & 3;         // tensor-memory lane quadrant of this warp
+    const int h = (warp - 2) >> 2;  // which of the quadrant's two warps
+    const uint32_t lane_base = tmem + ((uint32_t)(32 * q) << 16);
+    constexpr int COLS = BN / 2;
+    constexpr int NCH = COLS / 32;
+    float alpha_g = p.alpha;
+    if constexpr (KIND == kNVG) alpha_g = p.alpha * p.a_ts[0] * p.b_ts[0];
+    const uint32_t acc_empty_l = leader_addr(&sm->acc_empty);
+
+    // stage the scales of k-tile g into tensor-memory buffer g % NBUF
+    auto stage_scales = [&](int g) -> bool {
+      const int s = g % SFS, b = g % NBUF;
+      if (!warp_wait_st(smem_u32(&sm->sfs_full[s]), (uint32_t)((g / SFS) & 1), sm, p, 0x320u | s))
+        return false;
+      if (g >= NBUF &&
+          !warp_wait_st(smem_u32(&sm->sft_empty[b]), (uint32_t)(((g / NBUF) & 1) ^ 1), sm, p, 0x330u | b))
+        return false;
+      tc_fence_after();
+      const uint8_t *sfa_s = smem + CS::OFF_SF + s * CS::SF_BYTES;
+      const uint8_t *sfb_s = sfa_s + CS::SFA_BYTES;
+      const uint32_t col = lane_base + SF_BASE + b * CS::COLS_BUF;
+      if (h == 0) {
+        // A: row 32q + lane is word q of atom row `lane`
+#pragma unroll
+        for (int a = 0; a < C::ATOMS_K; ++a)
+          tmem_st1(col + 4 * a + q, *reinterpret_cast<const uint32_t *>(sfa_s + a * 512 + lane * 16 + 4 * q));
+      }
+      // B: atom a of each 128-row block: row 32w + lane is word w of atom row `lane`
+#pragma unroll
+      for (int a = h; a < C::ATOMS_K; a += 2) {
+#pragma unroll
+        for (int nb = 0; nb < BN / 128; ++nb)
+          tmem_st4(col + CS::COLS_A + (BN / 32) * a + 4 * nb,
+                   *reinterpret_cast<const uint4 *>(sfb_s + nb * C::SFA_BYTES + a * 512 + lane * 16));
+      }
+      asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) {
+        mbar_arrive(smem_u32(&sm->sfs_empty[s]));
+        if (PAIR && rank != 0)
+          mbar_arrive_remote_relaxed(leader_addr(&sm->sft_full[b]));
+        else
+          mbar_arrive(smem_u32(&sm->sft_full[b]));
+      }
+      return true;
+    };
+
+    uint32_t acc_phase = 0;
+    int g = 0;
+    bool ok = true;
+    int it = 0;
+    for (int tile = unit; tile < num_tiles && ok; tile += nunits, ++it) {
+      // scales for the rest of this tile and the first NBUF k-tiles of the
+      // next one, then this tile's epilogue
+      const int until = min(total, (it + 1) * KT + NBUF);
+      for (; g < until; ++g)
+        if (!stage_scales(g)) {
+          ok = false;
+          break;
+        }
+      if (!ok) break;
+      int mt, nt;
+      tile_coords(tile, num_m, num_n, p.n_fastest, mt, nt);
+      if (!warp_wait_st(smem_u32(&sm->acc_full), acc_phase, sm, p, 0x310u)) break;
+      tc_fence_after();
+      uint32_t r[COLS];
+#pragma unroll
+      for (int c = 0; c < NCH; ++c) tmem_ld32(lane_base + h * COLS + 32 * c, &r[32 * c]);
+      tmem_wait_ld();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) {
+        if (PAIR && rank != 0)
+          mbar_arrive_remote_relaxed(acc_empty_l);
+        else
+          mbar_arrive(smem_u32(&sm->acc_empty));
+      }
+      acc_phase ^= 1u;
+      const int64_t row = (int64_t)mt * CS::TILE_M + (int64_t)rank * 128 + 32 * q + lane;
+      const int64_t colg = (int64_t)nt * BN + h * COLS;
+      if (p.out_fp32) {
+        float *dst = reinterpret_cast<float *>(p.D) + row * p.ldd + colg;
+#pragma unroll
+        for (int i = 0; i < COLS; i += 4)
+          *reinterpret_cast<float4 *>(dst + i) =
+              make_float4(__uint_as_float(r[i]) * alpha_g, __uint_as_float(r[i + 1]) * alpha_g,
+                          __uint_as_float(r[i + 2]) * alpha_g, __uint_as_float(r[i + 3]) * alpha_g);
+      } else {
+        uint16_t *dst = reinterpret_cast<uint16_t *>(p.D) + row * p.ldd + colg;
+#pragma unroll
+        for (int i = 0; i < COLS; i += 8) {
+          uint32_t w[4];
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            __nv_bfloat162 b2 = __floats2bfloat162_rn(__uint_as_float(r[i + 2 * u]) * alpha_g,
+                                                      __uint_as_float(r[i + 2 * u + 1]) * alpha_g);
+            w[u] = *reinterpret_cast<uint32_t *>(&b2);
+          }
+          *reinterpret_cast<uint4 *>(dst + i) = make_uint4(w[0], w[1], w[2], w[3]);
+        }
+      }
+    }
+  }
+
+  // in a pair neither CTA leaves (or frees tensor memory) while the pair's
+  // MMAs may still read its shared memory or write its tensor memory
+  tc_fence_before();
+  __syncthreads();
+  if constexpr (PAIR) {
+    __syncwarp();
+    cluster_sync();
+  }
+  tc_fence_after();
+  if (warp == 1) {
+    __syncwarp();
+    if constexpr (PAIR)
+      asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(TMEM_COLS)
+                   : "memory");
+    else
+      asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(TMEM_COLS)
+                   : "memory");
+  }
+}
+
+}  // namespace gemm_st
 }  // namespace fa4
 
 namespace fa4 {
@@ -1391,32 +1482,57 @@ static cudaError_t launch_t(const GemmArgs &a, cudaStream_t st) {
   return cudaGetLastError();
 }
 
-template <int KIND, int BN>
+template <int KIND, int BN, bool PAIR>
 static cudaError_t launch_st(const GemmArgs &a, cudaStream_t st) {
-  constexpr int smem = gemm_st::total_smem_st<KIND, BN>();
+  constexpr int smem = gemm_st::total_smem_st<KIND, BN, PAIR>();
   CUtensorMap ma, mb;
   if (!make_payload_map(&ma, a.a_payload, a.M, a.K, gemm::BM)) return cudaErrorInvalidValue;
-  if (!make_payload_map(&mb, a.b_payload, a.N, a.K, BN)) return cudaErrorInvalidValue;
+  if (!make_payload_map(&mb, a.b_payload, a.N, a.K, PAIR ? 128 : BN)) return cudaErrorInvalidValue;
   gemm::Params p = make_params(a);
-  auto kern = gemm_st::gemm_st_kernel<KIND, BN>;
+  auto kern = gemm_st::gemm_st_kernel<KIND, BN, PAIR>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  const int64_t tiles = (a.M / gemm::BM) * (a.N / BN);
-  const int grid = (int)(tiles < sms ? tiles : sms);
-  kern<<<grid, gemm_st::NUM_THREADS_ST, smem, st>>>(ma, mb, p);
+  const int64_t tiles = (a.M / (PAIR ? 256 : gemm::BM)) * (a.N / BN);
+  cudaLaunchConfig_t cfg = {};
+  cfg.blockDim = dim3(gemm_st::NUM_THREADS_ST);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = PAIR ? 2 : 1;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = PAIR ? 1 : 0;
+  // persistent grid: no more units than can be resident at once (pairs must
+  // sit in one GPC, so fewer than SMs/2 pairs may fit)
+  int units = PAIR ? sms / 2 : sms;
+  if (PAIR) {
+    int clusters = 0;
+    cfg.gridDim = dim3((unsigned)(2 * units));
+    if (cudaOccupancyMaxActiveClusters(&clusters, kern, &cfg) == cudaSuccess && clusters > 0 &&
+        clusters < units)
+      units = clusters;
+  }
+  const int grid_units = (int)(tiles < units ? tiles : units);
+  cfg.gridDim = dim3((unsigned)(PAIR ? 2 * grid_units : grid_units));
+  e = cudaLaunchKernelEx(&cfg, kern, ma, mb, p);
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 
 cudaError_t launch_gemm_blockscaled(const GemmArgs &a, cudaStream_t st) {
   const bool wide = (a.N % 256) == 0;
-  if (a.fmt == kMX) return wide ? launch_st<kMX, 256>(a, st) : launch_st<kMX, 128>(a, st);
-  if (a.fmt == kNVG) return wide ? launch_st<kNVG, 256>(a, st) : launch_st<kNVG, 128>(a, st);
   const bool pair = wide && (a.M % 256) == 0;
-  if (pair && a.fmt == kMX) return launch_pair<kMX>(a, st);
-  if (pair && a.fmt == kNVG) return launch_pair<kNVG>(a, st);
+  if (a.fmt == kMX)
+    return pair ? launch_st<kMX, 256, true>(a, st)
+                : (wide ? launch_st<kMX, 256, false>(a, st) : launch_st<kMX, 128, false>(a, st));
+  if (a.fmt == kNVG)
+    return pair ? launch_st<kNVG, 256, true>(a, st)
+                : (wide ? launch_st<kNVG, 256, false>(a, st) : launch_st<kNVG, 128, false>(a, st));
   switch (a.fmt) {
     case kMX:
       return wide ? launch_t<kMX, 256>(a, st) : launch_t<kMX, 128>(a, st);
