@@ -60,19 +60,28 @@ __device__ __forceinline__ uint32_t e2m1x8_rne(const float *v) {
 
 // Stochastic rounding of y to a neighbouring E2M1 value with 16 random bits
 // u: with lo <= |y| < hi the neighbouring grid magnitudes and g = hi - lo,
-// round up iff u < (|y| - lo) * 65536 / g.  Both factors are exact (lo and
-// |y| share a binade, g is a power of two), so this equals the definition
-// with f = (|y| - lo) / g computed first.  |y| >= 6 gives 6; the sign of y is
-// kept.  Grid magnitudes 0, .5, 1, 1.5, 2, 3, 4, 6.
+// round up iff u < t, t = (|y| - lo) / g * 65536; |y| >= 6 gives 6; the sign
+// of y is kept.  Grid magnitudes 0, .5, 1, 1.5, 2, 3, 4, 6.
+// Evaluated on the binary32 bits A of |y| (integer compares order
+// non-negative floats):
+//  * 1 <= |y| < 6: lo is |y| with all but the top mantissa bit cleared and g
+//    is half its binade, so t = (A & 0x3FFFFF) / 64 exactly and the lower
+//    code is (A >> 22) - 252 (exponent and top mantissa bit);
+//    u < t  <=>  (u << 6) < (A & 0x3FFFFF).
+//  * 0.5 <= |y| < 1: lo = g = 0.5, t = (A & 0x7FFFFF) / 128, lower code 1.
+//  * |y| < 0.5: lo = 0, t = |y| * 131072 (exact), compared as floats.
 __device__ __forceinline__ uint32_t e2m1_sr(float y, uint32_t u) {
-  const uint32_t s = (__float_as_uint(y) >> 28) & 8u;
-  const float a = fabsf(y);
-  if (a >= 6.0f) return s | 7u;
-  uint32_t c = (a >= 0.5f) + (a >= 1.0f) + (a >= 1.5f) + (a >= 2.0f) + (a >= 3.0f) + (a >= 4.0f);
-  const float lo = (c < 4) ? 0.5f * (float)c : (float)(c - 2);  // exact
-  const float k = (c < 4) ? 131072.0f : ((c < 6) ? 65536.0f : 32768.0f);
-  const float t = __fmul_rn(__fsub_rn(a, lo), k);
-  c += ((float)u < t) ? 1u : 0u;
+  const uint32_t bits = __float_as_uint(y);
+  const uint32_t s = (bits >> 28) & 8u;
+  const uint32_t A = bits & 0x7FFFFFFFu;
+  const uint32_t c_hi = (A >> 22) - 252u + (((u << 6) < (A & 0x3FFFFFu)) ? 1u : 0u);
+  const uint32_t c_mid = 1u + (((u << 7) < (A & 0x7FFFFFu)) ? 1u : 0u);
+  const float uf = __fsub_rn(__uint_as_float(u | 0x4B000000u), 8388608.0f);  // (float)u, exact
+  const uint32_t c_lo = (uf < __fmul_rn(__uint_as_float(A), 131072.0f)) ? 1u : 0u;
+  const uint32_t c = (A >= 0x40C00000u) ? 7u
+                     : (A >= 0x3F800000u) ? c_hi
+                     : (A >= 0x3F000000u) ? c_mid
+                                          : c_lo;
   return s | c;
 }
 
@@ -141,13 +150,14 @@ __device__ __forceinline__ u32x4 philox10(uint32_t c0, uint32_t c1, uint32_t c2,
                                           uint32_t k0, uint32_t k1) {
 #pragma unroll
   for (int r = 0; r < 10; ++r) {
-    const uint32_t lo0 = 0xD2511F53u * c0, hi0 = __umulhi(0xD2511F53u, c0);
-    const uint32_t lo1 = 0xCD9E8D57u * c2, hi1 = __umulhi(0xCD9E8D57u, c2);
-    const uint32_t n0 = hi1 ^ c1 ^ k0, n2 = hi0 ^ c3 ^ k1;
+    // one 32x32 -> 64-bit product per multiplier gives both halves
+    const uint64_t p0 = (uint64_t)0xD2511F53u * c0;
+    const uint64_t p1 = (uint64_t)0xCD9E8D57u * c2;
+    const uint32_t n0 = (uint32_t)(p1 >> 32) ^ c1 ^ k0, n2 = (uint32_t)(p0 >> 32) ^ c3 ^ k1;
+    c1 = (uint32_t)p1;
+    c3 = (uint32_t)p0;
     c0 = n0;
-    c1 = lo1;
     c2 = n2;
-    c3 = lo0;
     k0 += 0x9E3779B9u;
     k1 += 0xBB67AE85u;
   }

@@ -539,49 +539,19 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 }  // namespace gemm
 
 // ==========================================================================
-// 2-SM variant.  A cluster of two CTAs (ranks 0 and 1) computes a 256 x 256
-// output tile with tcgen05.mma.cta_group::2 (M = 256, N = 256): CTA r holds
-// A rows 128r..128r+127 and B rows 128r..128r+127 of the pair tile in its
-// shared memory, and receives D rows 128r..128r+127 (all 256 columns) in its
-// tensor memory.  Each SM therefore moves half the B operand of the 1-SM
-// tile through its shared memory for the same number of MMA cycles.  Both
-// CTAs' TMA loads complete on the leader's stage barrier; the leader's single
-// MMA thread issues the scale copies and MMAs for the pair and its commits
-// arrive on the barriers of both CTAs (commit multicast).  The B scale
-// factors (all 256 rows) are loaded by each CTA itself, since every SM needs
-// them for its half of the output; no TMA load uses cluster multicast.
+// PTX helpers for 2-SM (cta_group::2) tiles.  A cluster of two CTAs (ranks 0
+// and 1) computes a 256 x 256 output tile with tcgen05.mma.cta_group::2
+// (M = 256, N = 256): CTA r holds A rows 128r..128r+127 and B rows
+// 128r..128r+127 of the pair tile in its shared memory and receives D rows
+// 128r..128r+127 (all 256 columns) in its tensor memory, so each SM moves
+// half the B operand of a 1-SM tile for the same MMA work.  Both CTAs' TMA
+// loads complete on the leader's barrier; the leader's commits arrive on
+// the barriers of both CTAs (commit multicast).  No TMA load uses cluster
+// multicast.
 // ==========================================================================
 namespace gemm2 {
 
 using namespace fa4::gemm;
-
-template <int KIND>
-struct Cfg2 {
-  static constexpr int STAGES = (KIND == kMX) ? 6 : 5;
-  static constexpr int A_BYTES = 128 * BKB;                     // own 128 rows
-  static constexpr int B_BYTES = 128 * BKB;                     // own half of N
-  static constexpr int SFA_BYTES = Cfg<KIND>::SFA_BYTES;        // own 128 rows
-  static constexpr int SFB_BYTES = 2 * Cfg<KIND>::SFA_BYTES;    // all 256 N rows
-  static constexpr int SF_ROWS = Cfg<KIND>::SFA_BYTES / 256;    // 256-byte rows per chunk
-  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES;
-  static constexpr int OFF_A = 0;
-  static constexpr int OFF_B = OFF_A + STAGES * A_BYTES;
-  static constexpr int OFF_SFA = OFF_B + STAGES * B_BYTES;
-  static constexpr int OFF_SFB = OFF_SFA + STAGES * SFA_BYTES;
-  static constexpr int OFF_CTRL = OFF_SFB + STAGES * SFB_BYTES;
-};
-
-struct Smem2 {
-  uint64_t full[6], empty[6];
-  uint64_t acc_full, acc_empty, mma_done;
-  uint32_t tmem_base;
-  int abort;
-};
-
-template <int KIND>
-constexpr int total_smem2() {
-  return Cfg2<KIND>::OFF_CTRL + (int)sizeof(Smem2) + 1024;
-}
 
 __device__ __forceinline__ uint32_t cluster_rank() {
   uint32_t r;
@@ -621,10 +591,6 @@ __device__ __forceinline__ void tc_commit_pair(uint32_t bar, uint16_t mask) {
       "h"(mask)
       : "memory");
 }
-__device__ __forceinline__ void tc_cp_pair(uint32_t taddr, uint64_t sdesc) {
-  asm volatile("tcgen05.cp.cta_group::2.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc)
-               : "memory");
-}
 template <int KIND>
 __device__ __forceinline__ void tc_mma_pair(uint32_t d, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
                                             uint32_t sfa, uint32_t sfb, uint32_t accumulate) {
@@ -649,240 +615,6 @@ template <int KIND>
 __device__ __forceinline__ uint32_t instr_desc_pair(uint32_t sf_id) {
   return (1u << 7) | (1u << 10) | ((uint32_t)(256 >> 3) << 17) | ((KIND == kMX ? 1u : 0u) << 23) |
          ((uint32_t)(256 >> 4) << 24) | (sf_id << 4) | (sf_id << 29);
-}
-
-__device__ __forceinline__ bool wait_bar2(uint32_t bar, uint32_t parity, Smem2 *sm, const Params &p,
-                                          uint32_t where) {
-  if (mbar_try_wait(bar, parity)) return true;
-  const uint64_t t0 = globaltimer();
-  while (true) {
-    if (mbar_try_wait(bar, parity)) return true;
-    if (*(volatile int *)&sm->abort) return false;
-    if (globaltimer() - t0 > p.timeout_ns) {
-      *(volatile int *)&sm->abort = 1;
-      if (atomicCAS(p.status, 0u, kStatusTimeout) == 0u) atomicExch(p.status + 1, where);
-      return false;
-    }
-  }
-}
-__device__ __forceinline__ bool warp_wait_bar2(uint32_t bar, uint32_t parity, Smem2 *sm,
-                                               const Params &p, uint32_t where) {
-  int ok = 0;
-  if ((threadIdx.x & 31) == 0) ok = wait_bar2(bar, parity, sm, p, where) ? 1 : 0;
-  return __shfl_sync(0xFFFFFFFFu, ok, 0) != 0;
-}
-
-template <int KIND>
-__global__ void __launch_bounds__(NUM_THREADS, 1)
-    gemm2_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_b,
-                 const __grid_constant__ CUtensorMap map_sfa, const __grid_constant__ CUtensorMap map_sfb,
-                 const Params p) {
-  using C2 = Cfg2<KIND>;
-  using C = Cfg<KIND>;
-  constexpr int STAGES2 = C2::STAGES;
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                              ~uintptr_t(1023));
-  Smem2 *sm = reinterpret_cast<Smem2 *>(smem + C2::OFF_CTRL);
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const uint32_t rank = cluster_rank();
-  const int pair = (int)(blockIdx.x >> 1), npairs = (int)(gridDim.x >> 1);
-
-  const int num_m = (int)(p.M / 256), num_n = (int)(p.N / 256);
-  const int num_tiles = num_m * num_n;
-  const int KT = (int)(p.K / BK);
-  const int64_t kbt4 = (p.K / C::BS) / 4;  // scale atoms per 128 rows
-
-  if (threadIdx.x == 0) {
-    for (int s = 0; s < STAGES2; ++s) {
-      mbar_init(smem_u32(&sm->full[s]), 1);
-      mbar_init(smem_u32(&sm->empty[s]), 1);
-    }
-    mbar_init(smem_u32(&sm->acc_full), 1);
-    mbar_init(smem_u32(&sm->acc_empty), 16);  // 8 epilogue warps in each CTA
-    mbar_init(smem_u32(&sm->mma_done), 1);
-    sm->abort = 0;
-    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-  }
-  if (warp == 1) {
-    asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
-                     smem_u32(&sm->tmem_base)),
-                 "r"(TMEM_COLS)
-                 : "memory");
-    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
-  }
-  tc_fence_before();
-  __syncthreads();
-  __syncwarp();
-  cluster_sync();  // peer barriers initialised before any remote arrive
-  tc_fence_after();
-  const uint32_t tmem = sm->tmem_base;
-
-  if (warp == 0) {
-    // ------------------------------------------------------------ producer
-    if (lane == 0) {
-      int stage = 0;
-      uint32_t phase = 0;
-      bool ok = true;
-      int k_global = 0;
-      for (int tile = pair; tile < num_tiles && ok; tile += npairs) {
-        int mt, nt;
-        tile_coords(tile, num_m, num_n, p.n_fastest, mt, nt);
-        for (int kt = 0; kt < KT; ++kt, ++k_global) {
-          if (!wait_bar2(smem_u32(&sm->empty[stage]), phase ^ 1u, sm, p, 0x100u | stage)) {
-            ok = false;
-            break;
-          }
-          if (k_global != p.debug_skip_stage) {
-            const uint32_t fb_local = smem_u32(&sm->full[stage]);
-            const uint32_t fb = map_to_rank(fb_local, 0);
-            if (rank == 0) mbar_arrive_expect_tx(fb_local, 2 * C2::STAGE_BYTES);
-            tma_load_2d_pair(smem_u32(smem + C2::OFF_A + stage * C2::A_BYTES), &map_a, kt * BKB,
-                             mt * 256 + (int)rank * 128, fb);
-            tma_load_2d_pair(smem_u32(smem + C2::OFF_B + stage * C2::B_BYTES), &map_b, kt * BKB,
-                             nt * 256 + (int)rank * 128, fb);
-            // scale chunks: 256-byte rows of the scale buffers
-            const int rb_a = mt * 2 + (int)rank;
-            tma_load_2d_pair(smem_u32(smem + C2::OFF_SFA + stage * C2::SFA_BYTES), &map_sfa, 0,
-                             (int)((rb_a * kbt4 + (int64_t)kt * C::ATOMS_K) * 2), fb);
-#pragma unroll
-            for (int nb = 0; nb < 2; ++nb) {
-              const int rb_b = nt * 2 + nb;
-              tma_load_2d_pair(smem_u32(smem + C2::OFF_SFB + stage * C2::SFB_BYTES + nb * C::SFA_BYTES),
-                               &map_sfb, 0, (int)((rb_b * kbt4 + (int64_t)kt * C::ATOMS_K) * 2), fb);
-            }
-          }
-          if (++stage == STAGES2) {
-            stage = 0;
-            phase ^= 1u;
-          }
-        }
-      }
-      if (!ok) {
-        // let copies already issued land before this CTA can leave
-        const uint64_t t0 = globaltimer();
-        while (globaltimer() - t0 < 200000ull) {
-        }
-      }
-    }
-  } else if (warp == 1) {
-    // ------------------------------------------------- MMA issue (leader)
-    if (lane == 0 && rank == 0) {
-      int stage = 0;
-      uint32_t phase = 0, acc_phase = 0;
-      bool ok = true;
-      for (int tile = pair; tile < num_tiles && ok; tile += npairs) {
-        if (!wait_bar2(smem_u32(&sm->acc_empty), acc_phase ^ 1u, sm, p, 0x200u)) break;
-        tc_fence_after();
-        for (int kt = 0; kt < KT; ++kt) {
-          if (!wait_bar2(smem_u32(&sm->full[stage]), phase, sm, p, 0x210u | stage)) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-          const uint32_t a_base = smem_u32(smem + C2::OFF_A + stage * C2::A_BYTES);
-          const uint32_t b_base = smem_u32(smem + C2::OFF_B + stage * C2::B_BYTES);
-          const uint32_t sfa_base = smem_u32(smem + C2::OFF_SFA + stage * C2::SFA_BYTES);
-          const uint32_t sfb_base = smem_u32(smem + C2::OFF_SFB + stage * C2::SFB_BYTES);
-          // scale atoms -> tensor memory of both CTAs (each from its own
-          // shared memory): A atom a at SFA_COL + 4a; B atom (row block nb,
-          // a) at SFB_COL + 8a + 4nb
-#pragma unroll
-          for (int a = 0; a < C::ATOMS_K; ++a) {
-            tc_cp_pair(tmem + SFA_COL + 4 * a, scale_desc(sfa_base + a * 512));
-#pragma unroll
-            for (int nb = 0; nb < 2; ++nb)
-              tc_cp_pair(tmem + SFB_COL + 8 * a + 4 * nb,
-                         scale_desc(sfb_base + nb * C::SFA_BYTES + a * 512));
-          }
-#pragma unroll
-          for (int j = 0; j < BK / 64; ++j) {
-            const int a = (KIND == kMX) ? (j >> 1) : j;
-            const uint32_t sf_id = (KIND == kMX) ? (uint32_t)(2 * (j & 1)) : 0u;
-            const uint32_t sfa = (tmem + SFA_COL + 4 * a) | (sf_id << 30);
-            const uint32_t sfb = (tmem + SFB_COL + 8 * a) | (sf_id << 30);
-            tc_mma_pair<KIND>(tmem, operand_desc(a_base + j * 32), operand_desc(b_base + j * 32),
-                              instr_desc_pair<KIND>(sf_id), sfa, sfb, (kt > 0 || j > 0) ? 1u : 0u);
-          }
-          tc_commit_pair(smem_u32(&sm->empty[stage]), (uint16_t)3);
-          if (++stage == STAGES2) {
-            stage = 0;
-            phase ^= 1u;
-          }
-        }
-        if (ok) tc_commit_pair(smem_u32(&sm->acc_full), (uint16_t)3);
-        acc_phase ^= 1u;
-      }
-      tc_commit_pair(smem_u32(&sm->mma_done), (uint16_t)1);
-      const uint64_t t0 = globaltimer();
-      while (!mbar_try_wait(smem_u32(&sm->mma_done), 0)) {
-        if (globaltimer() - t0 > p.timeout_ns) {
-          if (atomicCAS(p.status, 0u, kStatusTimeout) == 0u) atomicExch(p.status + 1, 0x500u);
-          break;
-        }
-      }
-    }
-  } else {
-    // ------------------------------------------------------------ epilogue
-    const int q = warp & 3;
-    const int h = (warp - 2) >> 2;
-    constexpr int COLS = 128;
-    const uint32_t acc_empty_leader = map_to_rank(smem_u32(&sm->acc_empty), 0);
-    uint32_t acc_phase = 0;
-    float alpha_g = p.alpha;
-    if constexpr (KIND == kNVG) alpha_g = p.alpha * p.a_ts[0] * p.b_ts[0];
-    for (int tile = pair; tile < num_tiles; tile += npairs) {
-      int mt, nt;
-        tile_coords(tile, num_m, num_n, p.n_fastest, mt, nt);
-      if (!warp_wait_bar2(smem_u32(&sm->acc_full), acc_phase, sm, p, 0x310u)) break;
-      tc_fence_after();
-      uint32_t r[COLS];
-#pragma unroll
-      for (int c = 0; c < COLS / 32; ++c)
-        tmem_ld32(tmem + ((uint32_t)(32 * q) << 16) + h * COLS + 32 * c, &r[32 * c]);
-      tmem_wait_ld();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive_cluster(acc_empty_leader);
-      acc_phase ^= 1u;
-      const int64_t row = (int64_t)mt * 256 + (int64_t)rank * 128 + 32 * q + lane;
-      const int64_t col = (int64_t)nt * 256 + h * COLS;
-      if (p.out_fp32) {
-        float *dst = reinterpret_cast<float *>(p.D) + row * p.ldd + col;
-#pragma unroll
-        for (int i = 0; i < COLS; i += 4)
-          *reinterpret_cast<float4 *>(dst + i) =
-              make_float4(__uint_as_float(r[i]) * alpha_g, __uint_as_float(r[i + 1]) * alpha_g,
-                          __uint_as_float(r[i + 2]) * alpha_g, __uint_as_float(r[i + 3]) * alpha_g);
-      } else {
-        uint16_t *dst = reinterpret_cast<uint16_t *>(p.D) + row * p.ldd + col;
-#pragma unroll
-        for (int i = 0; i < COLS; i += 8) {
-          uint32_t w[4];
-#pragma unroll
-          for (int u = 0; u < 4; ++u) {
-            __nv_bfloat162 b2 = __floats2bfloat162_rn(__uint_as_float(r[i + 2 * u]) * alpha_g,
-                                                      __uint_as_float(r[i + 2 * u + 1]) * alpha_g);
-            w[u] = *reinterpret_cast<uint32_t *>(&b2);
-          }
-          *reinterpret_cast<uint4 *>(dst + i) = make_uint4(w[0], w[1], w[2], w[3]);
-        }
-      }
-    }
-  }
-
-  // neither CTA leaves (or frees tensor memory) while the pair's MMAs may
-  // still read its shared memory or write its tensor memory
-  tc_fence_before();
-  __syncthreads();
-  __syncwarp();
-  cluster_sync();
-  tc_fence_after();
-  if (warp == 1) {
-    __syncwarp();
-    asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(TMEM_COLS)
-                 : "memory");
-  }
 }
 
 }  // namespace gemm2
@@ -1392,20 +1124,6 @@ static bool make_payload_map(CUtensorMap *m, const void *base, int64_t rows, int
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// Scale-buffer map: the R*Kb scale bytes viewed as rows of 256 bytes; one
-// 128-row x 256-K chunk of atoms is `rows_per_box` consecutive rows.
-static bool make_scale_map(CUtensorMap *m, const void *base, int64_t total_bytes, int rows_per_box) {
-  PFN_encodeTiled enc = get_encode();
-  if (!enc) return false;
-  cuuint64_t dims[2] = {256, (cuuint64_t)(total_bytes / 256)};
-  cuuint64_t strides[1] = {256};
-  cuuint32_t box[2] = {256, (cuuint32_t)rows_per_box};
-  cuuint32_t estr[2] = {1, 1};
-  return enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void *>(base), dims, strides, box, estr,
-             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
-             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
 static gemm::Params make_params(const GemmArgs &a) {
   gemm::Params p;
   p.a_scales = a.a_scales;
@@ -1425,42 +1143,6 @@ static gemm::Params make_params(const GemmArgs &a) {
   // keep the smaller operand resident in L2 and stream the larger one once
   p.n_fastest = (a.N <= a.M) ? 1 : 0;
   return p;
-}
-
-template <int KIND>
-static cudaError_t launch_pair(const GemmArgs &a, cudaStream_t st) {
-  using C2 = gemm2::Cfg2<KIND>;
-  const int bs = (KIND == kMX) ? 32 : 16;
-  CUtensorMap ma, mb, msa, msb;
-  if (!make_payload_map(&ma, a.a_payload, a.M, a.K, 128)) return cudaErrorInvalidValue;
-  if (!make_payload_map(&mb, a.b_payload, a.N, a.K, 128)) return cudaErrorInvalidValue;
-  if (!make_scale_map(&msa, a.a_scales, a.M * (a.K / bs), C2::SF_ROWS)) return cudaErrorInvalidValue;
-  if (!make_scale_map(&msb, a.b_scales, a.N * (a.K / bs), C2::SF_ROWS)) return cudaErrorInvalidValue;
-  gemm::Params p = make_params(a);
-  auto kern = gemm2::gemm2_kernel<KIND>;
-  constexpr int smem = gemm2::total_smem2<KIND>();
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-  if (e != cudaSuccess) return e;
-  int dev = 0, sms = 148;
-  cudaGetDevice(&dev);
-  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  const int64_t tiles = (a.M / 256) * (a.N / 256);
-  const int pairs = (int)(tiles < sms / 2 ? tiles : sms / 2);
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3((unsigned)(2 * pairs));
-  cfg.blockDim = dim3(gemm::NUM_THREADS);
-  cfg.dynamicSmemBytes = smem;
-  cfg.stream = st;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = 2;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  e = cudaLaunchKernelEx(&cfg, kern, ma, mb, msa, msb, p);
-  if (e != cudaSuccess) return e;
-  return cudaGetLastError();
 }
 
 template <int KIND, int BN>
