@@ -87,6 +87,7 @@ def _declare(L: ctypes.CDLL) -> ctypes.CDLL:
         "fa4_debug_convert": [P, P, i64, P, P, P, P],
         "fa4_debug_sr_bits": [u64, P, i64, P, P],
         "fa4_debug_gemm_timeout": [_QT, _QT, i64, i64, i64, ci, P, i64, ci, u64, P, sz, P],
+        "fa4_quantize_nvfp4_global_noalloc": [P, i64, i64, i64, ci, ci, u64, _QT, P],
     }
     for name, args in sig.items():
         fn = getattr(L, name)
@@ -175,6 +176,19 @@ def quantize(x: torch.Tensor, fmt: int, rnd: int = RNE, orient: int = ROWWISE, s
     ws = _ws(ws, need, x.device)
     _check(lib().fa4_quantize(_ptr(x), rows, cols, ld, fmt, rnd, orient, seed, out.c(), _ptr(ws),
                               ws.numel(), _stream(x.device)), "fa4_quantize")
+    return out
+
+
+def quantize_nvfp4_global_noalloc(x: torch.Tensor, rnd: int = RNE, orient: int = ROWWISE,
+                                  seed: int = 0, out: QTensor | None = None) -> QTensor:
+    """NVFP4-global quantization without a workspace: the amax scratch lives
+    in a fixed array inside the library (see include/fa4.h)."""
+    ld = _as_bf16_2d(x, "x")
+    rows, cols = x.shape
+    out = out or empty_qtensor(rows, cols, NVFP4_GLOBAL, orient, x.device)
+    _check(lib().fa4_quantize_nvfp4_global_noalloc(_ptr(x), rows, cols, ld, rnd, orient, seed,
+                                                   out.c(), _stream(x.device)),
+           "fa4_quantize_nvfp4_global_noalloc")
     return out
 
 

@@ -189,6 +189,27 @@ FA4_API fa4_status fa4_linear_wgrad(const void *dY, const void *X, int64_t T, in
                             fa4_out_dtype out_dtype, void *workspace, size_t workspace_bytes,
                             void *stream);
 
+/* NVFP4-global quantization that allocates nothing and takes no workspace.
+ * (No counterpart on the pages: it exists for callers, not for the method.)
+ * For callers that cannot provide device scratch: a runtime that reserves
+ * all device memory up front under a fixed plan, or code that must not call
+ * cudaMalloc at that point (it can synchronize the device, or the allocator
+ * belongs to someone else).  Same result, bytes and error checks as
+ * fa4_quantize(x, rows, cols, ld, FA4_NVFP4_GLOBAL, rnd, orient, seed, out,
+ * ...); the amax pass keeps its per-CTA partial maxima in a fixed array of
+ * 1184 floats (4736 bytes) inside the library, which every GPU that loads
+ * the library holds until the process exits.  A call needing more partials
+ * than that returns FA4_ERR_WORKSPACE (the launch configuration never does).
+ * The first call on a device looks up that array's device address (once per
+ * device); make that first call before any stream capture.  Every call
+ * shares the one array per device: calls that may run at the same time on
+ * the GPU (different streams, no ordering between them) race on it and must
+ * be serialized by the caller.  Errors: SHAPE, ALIGN, INVALID_ARG, WORKSPACE,
+ * CUDA, UNSUPPORTED (device ordinal >= 64). */
+FA4_API fa4_status fa4_quantize_nvfp4_global_noalloc(const void *x, int64_t rows, int64_t cols,
+                                                     int64_t ld, fa4_round rnd, fa4_orient orient,
+                                                     uint64_t seed, fa4_qtensor out, void *stream);
+
 /* Zero the workspace header (stream-ordered memset of FA4_WS_HEADER_BYTES). */
 FA4_API fa4_status fa4_workspace_init(void *workspace, size_t workspace_bytes, void *stream);
 

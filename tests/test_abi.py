@@ -155,3 +155,15 @@ def test_product_package_does_not_import_the_oracle():
             if f.endswith((".cu", ".cuh", ".h", ".cpp")):
                 assert "fa4_oracle" not in open(path).read(), path
                 assert "orc_" not in open(path).read(), path
+
+
+def test_noalloc_quantize_rejects_bad_arguments():
+    L = fa.lib()
+    q = _qt()
+    assert L.fa4_quantize_nvfp4_global_noalloc(None, 256, 256, 256, 0, 0, 0, q, None) == 1
+    assert L.fa4_quantize_nvfp4_global_noalloc(DEV, 250, 256, 256, 0, 0, 0, q, None) == 2
+    assert L.fa4_quantize_nvfp4_global_noalloc(DEV, 256, 256, 200, 0, 0, 0, q, None) == 2
+    assert L.fa4_quantize_nvfp4_global_noalloc(DEV + 4, 256, 256, 256, 0, 0, 0, q, None) == 3
+    assert L.fa4_quantize_nvfp4_global_noalloc(DEV, 256, 256, 256, 3, 0, 0, q, None) == 1
+    assert L.fa4_quantize_nvfp4_global_noalloc(DEV, 256, 256, 256, 0, 0, 0,
+                                               fa._QT(0x10000, 0x20000, 0), None) == 1
