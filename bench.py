@@ -120,16 +120,23 @@ def _f(s):
 
 # ------------------------------------------------------------ fa4 arm ---
 
+def input_seeds(rank: int, layer: int) -> tuple[int, int, int]:
+    """Seeds of (X, dY, W) of one layer on one rank (ranks < 1000 and
+    layers < 100 never share a seed)."""
+    s = rank * 1000 + 10 * layer
+    return s, s + 1, s + 2
+
+
 class Block:
     """Inputs, quantized weights and output buffers of one block's linears."""
 
     def __init__(self, fa, seed: int, device):
         self.layers = {}
         for i, (name, (cin, cout)) in enumerate(LAYERS.items()):
-            s = seed * 1000 + 10 * i
-            x = workloads.act(T, cin, seed=s, device=device)
-            dy = workloads.grad(T, cout, seed=s + 1, device=device)
-            w = workloads.weight(cout, cin, seed=s + 2, device=device)
+            sx, sdy, sw = input_seeds(seed, i)
+            x = workloads.act(T, cin, seed=sx, device=device)
+            dy = workloads.grad(T, cout, seed=sdy, device=device)
+            w = workloads.weight(cout, cin, seed=sw, device=device)
             L = dict(cin=cin, cout=cout, x=x, dy=dy, w=w)
             L["xq"] = fa.empty_qtensor(T, cin, fa.NVFP4_GLOBAL, fa.ROWWISE, device)
             L["gq"] = fa.empty_qtensor(T, cout, fa.MXFP4, fa.ROWWISE, device)
@@ -320,6 +327,41 @@ def cpu_baseline(sample_tokens: int = 128) -> dict:
                       f"(weights prepared by the oracle before timing)"}
 
 
+def max_over_ranks(x: float, device) -> float:
+    """Max of x over the ranks of the default process group (x itself when
+    there is no group or one rank).  Every rank must call it."""
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def bench_config(world: int) -> dict:
+    return {"workload": "llama3-8b-block-linears-fwd-bwd", "tokens": T,
+            "layers": {k: list(v) for k, v in LAYERS.items()},
+            "fwd": "NVFP4-global RNE", "dgrad": "MXFP4 row-wise SR",
+            "wgrad": "MXFP4 column-wise fixed-sign Hadamard-32 RNE, alpha 1/32",
+            "parallelism": f"replicas x{world}", "l2": "inputs > L2 (1.1 GB bf16 read per step)"}
+
+
+def whole_job_tokens_per_s(world: int, ms_step: float) -> float:
+    """Weak scaling: every rank runs its own replica of the step on T tokens,
+    so the job processes world * T tokens in the slowest rank's step time."""
+    return world * T / (ms_step * 1e-3)
+
+
+def init_ranks(world: int, device, backend: str = "nccl"):
+    """One process per GPU; a short timeout so ranks that wait on a dead peer
+    end with an error instead of hanging."""
+    if world <= 1:
+        return
+    import datetime
+    kw = {"device_id": device} if backend == "nccl" else {}
+    torch.distributed.init_process_group(backend, timeout=datetime.timedelta(seconds=120), **kw)
+
+
 def fa4_arm(args, rank, world, device) -> dict | None:
     import fp4_quantization_block_b200 as fa
     fa.lib()
@@ -353,11 +395,7 @@ def fa4_arm(args, rank, world, device) -> dict | None:
         torch.distributed.barrier()
     if fa.check_device_status(blk.ws) != 0:
         raise RuntimeError("device status set during the timed region")
-    ms_total = start.elapsed_time(end)
-    if world > 1:
-        t = torch.tensor([ms_total], dtype=torch.float64, device=device)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        ms_total = float(t.item())
+    ms_total = max_over_ranks(start.elapsed_time(end), device)
     ms_step = ms_total / args.steps
 
     # per-kind durations from consecutive events (previous event = start of call)
@@ -390,7 +428,7 @@ def fa4_arm(args, rank, world, device) -> dict | None:
         sweep = quantize_sweep(fa, device) if not args.quick else []
         e2e = e2e_run(fa, blk, max(2, min(args.steps, 5)), device)
         cpu = cpu_baseline() if (world == 1 and not args.no_cpu_baseline) else None
-        tok_s = world * T / (ms_step * 1e-3)
+        tok_s = whole_job_tokens_per_s(world, ms_step)
         result = {
             "metric": METRIC,
             "value": round(tok_s, 1),
@@ -405,11 +443,7 @@ def fa4_arm(args, rank, world, device) -> dict | None:
             "dtype": "e2m1",
             "data": "synthetic (seeded generators: act N(0,1)+0.5% channels x20, W N(0,0.02), "
                     "dY N(0,1e-3) x lognormal rows)",
-            "config": {"workload": "llama3-8b-block-linears-fwd-bwd", "tokens": T,
-                       "layers": {k: list(v) for k, v in LAYERS.items()},
-                       "fwd": "NVFP4-global RNE", "dgrad": "MXFP4 row-wise SR",
-                       "wgrad": "MXFP4 column-wise fixed-sign Hadamard-32 RNE, alpha 1/32",
-                       "parallelism": f"replicas x{world}", "l2": "inputs > L2 (1.1 GB bf16 read per step)"},
+            "config": bench_config(world),
             "metrics": {"linear_tokens_per_s": round(tok_s, 1),
                         "fp4_gemm_TFLOPS": round(gemm_tflops, 1),
                         "fused_quantize_GBps": round(q_gbs, 1),
@@ -506,10 +540,10 @@ def reference_arm(args) -> dict:
     dt = (time.perf_counter() - t0) / args.steps
     value = 64 / dt
     return {"impl": "reference", "metric": METRIC, "value": round(value, 3), "unit": "tokens/s",
-            "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
+            "n_gpus": int(os.environ.get("WORLD_SIZE", "1")), "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": round(dt * 1e3, 1), "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": "llama3-8b-block-linears-fwd-bwd", "tokens": T},
+            "config": bench_config(int(os.environ.get("WORLD_SIZE", "1"))),
             "cpu_baseline": {"value": round(value, 3), "unit": "tokens/s", "cores": res["cores"],
                              "kind": "oracle", "sample": "64 tokens per step through the block's 4 linears"},
             "e2e": {"value": round(value, 3), "unit": "tokens/s", "h2d_bytes_per_step": 0,
@@ -541,10 +575,7 @@ def main():
 
     device = torch.device("cuda", local)
     torch.cuda.set_device(device)
-    if world > 1:
-        import datetime
-        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                             device_id=device)
+    init_ranks(world, device)
     if args.profile:
         print(json.dumps(profile_arm(args, device)), flush=True)
         return
