@@ -675,7 +675,10 @@ struct CfgSt {
   static constexpr int COLS_A = C::ATOMS_K * 4;
   static constexpr int COLS_B = C::ATOMS_K * (BN / 32);
   static constexpr int COLS_BUF = COLS_A + COLS_B;
-  static constexpr int ARRIVALS = PAIR ? 16 : 8;  // stager / epilogue warps feeding the MMA
+  // warps arriving per k-tile on a scale buffer (one per lane quadrant, in
+  // each CTA of a pair) and per tile on the accumulator (two per quadrant)
+  static constexpr int SF_ARRIVALS = PAIR ? 8 : 4;
+  static constexpr int ACC_ARRIVALS = PAIR ? 16 : 8;
   static_assert(!PAIR || BN == 256, "a pair computes 256-wide tiles");
   static_assert(AB_STAGES >= 2, "shared-memory budget");
   static_assert(SF_BASE + NBUF * COLS_BUF <= TMEM_COLS, "tensor-memory budget");
@@ -780,14 +783,14 @@ __global__ void __launch_bounds__(NUM_THREADS_ST, 1)
     }
     for (int s = 0; s < SFS; ++s) {
       mbar_init(smem_u32(&sm->sfs_full[s]), 1);
-      mbar_init(smem_u32(&sm->sfs_empty[s]), 8);
+      mbar_init(smem_u32(&sm->sfs_empty[s]), 4);
     }
     for (int b = 0; b < NBUF; ++b) {
-      mbar_init(smem_u32(&sm->sft_full[b]), CS::ARRIVALS);
+      mbar_init(smem_u32(&sm->sft_full[b]), CS::SF_ARRIVALS);
       mbar_init(smem_u32(&sm->sft_empty[b]), 1);
     }
     mbar_init(smem_u32(&sm->acc_full), 1);
-    mbar_init(smem_u32(&sm->acc_empty), CS::ARRIVALS);
+    mbar_init(smem_u32(&sm->acc_empty), CS::ACC_ARRIVALS);
     mbar_init(smem_u32(&sm->mma_done), 1);
     sm->abort = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -982,15 +985,13 @@ __global__ void __launch_bounds__(NUM_THREADS_ST, 1)
       const uint8_t *sfa_s = smem + CS::OFF_SF + s * CS::SF_BYTES;
       const uint8_t *sfb_s = sfa_s + CS::SFA_BYTES;
       const uint32_t col = lane_base + SF_BASE + b * CS::COLS_BUF;
-      if (h == 0) {
-        // A: row 32q + lane is word q of atom row `lane`
+      // A: row 32q + lane is word q of atom row `lane`
 #pragma unroll
-        for (int a = 0; a < C::ATOMS_K; ++a)
-          tmem_st1(col + 4 * a + q, *reinterpret_cast<const uint32_t *>(sfa_s + a * 512 + lane * 16 + 4 * q));
-      }
+      for (int a = 0; a < C::ATOMS_K; ++a)
+        tmem_st1(col + 4 * a + q, *reinterpret_cast<const uint32_t *>(sfa_s + a * 512 + lane * 16 + 4 * q));
       // B: atom a of each 128-row block: row 32w + lane is word w of atom row `lane`
 #pragma unroll
-      for (int a = h; a < C::ATOMS_K; a += 2) {
+      for (int a = 0; a < C::ATOMS_K; ++a) {
 #pragma unroll
         for (int nb = 0; nb < BN / 128; ++nb)
           tmem_st4(col + CS::COLS_A + (BN / 32) * a + 4 * nb,
@@ -1009,15 +1010,16 @@ __global__ void __launch_bounds__(NUM_THREADS_ST, 1)
       return true;
     };
 
+    // the quadrant's two warps stage alternate k-tiles (h = 0 the even ones)
     uint32_t acc_phase = 0;
-    int g = 0;
+    int g = h;
     bool ok = true;
     int it = 0;
     for (int tile = unit; tile < num_tiles && ok; tile += nunits, ++it) {
       // scales for the rest of this tile and the first NBUF k-tiles of the
       // next one, then this tile's epilogue
       const int until = min(total, (it + 1) * KT + NBUF);
-      for (; g < until; ++g)
+      for (; g < until; g += 2)
         if (!stage_scales(g)) {
           ok = false;
           break;
