@@ -219,6 +219,7 @@ struct Params {
   int debug_skip_stage;
   uint64_t timeout_ns;
   int n_fastest;  // tile order: 1 = walk N first (B stays in L2), 0 = walk M first
+  int wide_store; // D and every row of it 32-byte aligned: 256-bit stores
 };
 
 // Output tile coordinates of linear tile index t.  Concurrently running CTAs
@@ -744,6 +745,13 @@ __device__ __forceinline__ void mbar_arrive_remote_relaxed(uint32_t bar_cluster)
                : "memory");
 }
 
+// 256-bit global store (sm_100): one full 32-byte sector per thread
+__device__ __forceinline__ void st_global_v8(void *ptr, const uint32_t (&v)[8]) {
+  asm volatile("st.global.v8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"l"(ptr), "r"(v[0]), "r"(v[1]),
+               "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7])
+               : "memory");
+}
+
 __device__ __forceinline__ void tmem_st1(uint32_t taddr, uint32_t v) {
   asm volatile("tcgen05.st.sync.aligned.32x32b.x1.b32 [%0], {%1};" ::"r"(taddr), "r"(v) : "memory");
 }
@@ -1044,25 +1052,50 @@ __global__ void __launch_bounds__(NUM_THREADS_ST, 1)
       acc_phase ^= 1u;
       const int64_t row = (int64_t)mt * CS::TILE_M + (int64_t)rank * 128 + 32 * q + lane;
       const int64_t colg = (int64_t)nt * BN + h * COLS;
+      // each thread writes one row: 32-byte pieces when D allows
       if (p.out_fp32) {
         float *dst = reinterpret_cast<float *>(p.D) + row * p.ldd + colg;
+        if (p.wide_store) {
 #pragma unroll
-        for (int i = 0; i < COLS; i += 4)
-          *reinterpret_cast<float4 *>(dst + i) =
-              make_float4(__uint_as_float(r[i]) * alpha_g, __uint_as_float(r[i + 1]) * alpha_g,
-                          __uint_as_float(r[i + 2]) * alpha_g, __uint_as_float(r[i + 3]) * alpha_g);
+          for (int i = 0; i < COLS; i += 8) {
+            uint32_t w[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) w[u] = __float_as_uint(__uint_as_float(r[i + u]) * alpha_g);
+            st_global_v8(dst + i, w);
+          }
+        } else {
+#pragma unroll
+          for (int i = 0; i < COLS; i += 4)
+            *reinterpret_cast<float4 *>(dst + i) =
+                make_float4(__uint_as_float(r[i]) * alpha_g, __uint_as_float(r[i + 1]) * alpha_g,
+                            __uint_as_float(r[i + 2]) * alpha_g, __uint_as_float(r[i + 3]) * alpha_g);
+        }
       } else {
         uint16_t *dst = reinterpret_cast<uint16_t *>(p.D) + row * p.ldd + colg;
+        if (p.wide_store) {
 #pragma unroll
-        for (int i = 0; i < COLS; i += 8) {
-          uint32_t w[4];
+          for (int i = 0; i < COLS; i += 16) {
+            uint32_t w[8];
 #pragma unroll
-          for (int u = 0; u < 4; ++u) {
-            __nv_bfloat162 b2 = __floats2bfloat162_rn(__uint_as_float(r[i + 2 * u]) * alpha_g,
-                                                      __uint_as_float(r[i + 2 * u + 1]) * alpha_g);
-            w[u] = *reinterpret_cast<uint32_t *>(&b2);
+            for (int u = 0; u < 8; ++u) {
+              __nv_bfloat162 b2 = __floats2bfloat162_rn(__uint_as_float(r[i + 2 * u]) * alpha_g,
+                                                        __uint_as_float(r[i + 2 * u + 1]) * alpha_g);
+              w[u] = *reinterpret_cast<uint32_t *>(&b2);
+            }
+            st_global_v8(dst + i, w);
           }
-          *reinterpret_cast<uint4 *>(dst + i) = make_uint4(w[0], w[1], w[2], w[3]);
+        } else {
+#pragma unroll
+          for (int i = 0; i < COLS; i += 8) {
+            uint32_t w[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+              __nv_bfloat162 b2 = __floats2bfloat162_rn(__uint_as_float(r[i + 2 * u]) * alpha_g,
+                                                        __uint_as_float(r[i + 2 * u + 1]) * alpha_g);
+              w[u] = *reinterpret_cast<uint32_t *>(&b2);
+            }
+            *reinterpret_cast<uint4 *>(dst + i) = make_uint4(w[0], w[1], w[2], w[3]);
+          }
         }
       }
     }
@@ -1144,6 +1177,8 @@ static gemm::Params make_params(const GemmArgs &a) {
   p.timeout_ns = a.timeout_ns;
   // keep the smaller operand resident in L2 and stream the larger one once
   p.n_fastest = (a.N <= a.M) ? 1 : 0;
+  const int64_t row_bytes = a.ldd * (a.out_fp32 ? 4 : 2);
+  p.wide_store = ((reinterpret_cast<uintptr_t>(a.D) & 31u) == 0 && row_bytes % 32 == 0) ? 1 : 0;
   return p;
 }
 
