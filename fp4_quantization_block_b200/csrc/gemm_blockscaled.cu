@@ -219,7 +219,6 @@ struct Params {
   int debug_skip_stage;
   uint64_t timeout_ns;
   int n_fastest;  // tile order: 1 = walk N first (B stays in L2), 0 = walk M first
-  int wide_store; // D and every row of it 32-byte aligned: 256-bit stores
 };
 
 // Output tile coordinates of linear tile index t.  Concurrently running CTAs
@@ -664,14 +663,21 @@ struct CfgSt {
   static constexpr int SFB_BYTES = C::SFA_BYTES * (BN / 128);   // all BN rows
   static constexpr int AB_BYTES = A_BYTES + B_BYTES;
   static constexpr int SF_BYTES = SFA_BYTES + SFB_BYTES;
-  static constexpr int SF_STAGES = (PAIR || (KIND == kMX && BN == 256)) ? 8 : 12;
-  static constexpr int BUDGET = 220 * 1024;
+  static constexpr int SF_STAGES = BN == 256 ? 5 : 8;
+  // epilogue staging: one 32-row x 64-byte output chunk per epilogue warp
+  static constexpr int EPI_WARP_BYTES = 2048;
+  static constexpr int EPI_BYTES = 8 * EPI_WARP_BYTES;
+  static constexpr int SMEM_LIMIT = 232448;  // 227 KB per block (opt-in)
+  static constexpr int RESERVE = 2048;       // control block + alignment slack
+  static constexpr int BUDGET = SMEM_LIMIT - RESERVE - EPI_BYTES;
   static constexpr int AB_STAGES_RAW = (BUDGET - SF_STAGES * SF_BYTES) / AB_BYTES;
   static constexpr int AB_STAGES = AB_STAGES_RAW > 6 ? 6 : AB_STAGES_RAW;
   static constexpr int OFF_A = 0;
   static constexpr int OFF_B = OFF_A + AB_STAGES * A_BYTES;
   static constexpr int OFF_SF = OFF_B + AB_STAGES * B_BYTES;
-  static constexpr int OFF_CTRL = OFF_SF + SF_STAGES * SF_BYTES;
+  static constexpr int OFF_EPI = OFF_SF + SF_STAGES * SF_BYTES;
+  static constexpr int OFF_CTRL = OFF_EPI + EPI_BYTES;
+  static_assert(OFF_EPI % 1024 == 0, "64-byte swizzle needs 512-byte aligned chunks");
   // tensor-memory columns of one scale buffer
   static constexpr int COLS_A = C::ATOMS_K * 4;
   static constexpr int COLS_B = C::ATOMS_K * (BN / 32);
@@ -696,6 +702,9 @@ struct SmemSt {
 
 template <int KIND, int BN, bool PAIR>
 constexpr int total_smem_st() {
+  static_assert(CfgSt<KIND, BN, PAIR>::OFF_CTRL + (int)sizeof(SmemSt) + 1024 <=
+                    CfgSt<KIND, BN, PAIR>::SMEM_LIMIT,
+                "shared-memory limit");
   return CfgSt<KIND, BN, PAIR>::OFF_CTRL + (int)sizeof(SmemSt) + 1024;
 }
 
@@ -745,11 +754,32 @@ __device__ __forceinline__ void mbar_arrive_remote_relaxed(uint32_t bar_cluster)
                : "memory");
 }
 
-// 256-bit global store (sm_100): one full 32-byte sector per thread
-__device__ __forceinline__ void st_global_v8(void *ptr, const uint32_t (&v)[8]) {
-  asm volatile("st.global.v8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"l"(ptr), "r"(v[0]), "r"(v[1]),
-               "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7])
+// Output tile store through shared memory: the bulk-tensor (TMA) engine
+// writes whole lines, so the epilogue issues no per-row global stores.
+__device__ __forceinline__ void sts128(uint32_t addr, uint32_t a, uint32_t b, uint32_t c,
+                                       uint32_t d) {
+  asm volatile("st.shared.v4.b32 [%0], {%1,%2,%3,%4};" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d)
                : "memory");
+}
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+__device__ __forceinline__ void tma_store_2d(const CUtensorMap *map, uint32_t src, int x, int y) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%1, %2}], [%3];" ::"l"(map),
+      "r"(x), "r"(y), "r"(src)
+      : "memory");
+}
+__device__ __forceinline__ void bulk_commit() {
+  asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+}
+// the shared-memory source of every committed store has been read
+__device__ __forceinline__ void bulk_wait_read_all() {
+  asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+}
+// every committed store has completed
+__device__ __forceinline__ void bulk_wait_all() {
+  asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
 }
 
 __device__ __forceinline__ void tmem_st1(uint32_t taddr, uint32_t v) {
@@ -764,7 +794,8 @@ __device__ __forceinline__ void tmem_st4(uint32_t taddr, const uint4 &v) {
 template <int KIND, int BN, bool PAIR>
 __global__ void __launch_bounds__(NUM_THREADS_ST, 1)
     gemm_st_kernel(const __grid_constant__ CUtensorMap map_a,
-                   const __grid_constant__ CUtensorMap map_b, const Params p) {
+                   const __grid_constant__ CUtensorMap map_b,
+                   const __grid_constant__ CUtensorMap map_d, const Params p) {
   using CS = CfgSt<KIND, BN, PAIR>;
   using C = Cfg<KIND>;
   constexpr int ABS = CS::AB_STAGES, SFS = CS::SF_STAGES;
@@ -975,6 +1006,7 @@ __global__ void __launch_bounds__(NUM_THREADS_ST, 1)
     const int q = warp & 3;         // tensor-memory lane quadrant of this warp
     const int h = (warp - 2) >> 2;  // which of the quadrant's two warps
     const uint32_t lane_base = tmem + ((uint32_t)(32 * q) << 16);
+    const uint32_t ebuf = smem_u32(smem + CS::OFF_EPI + (warp - 2) * CS::EPI_WARP_BYTES);
     constexpr int COLS = BN / 2;
     constexpr int NCH = COLS / 32;
     float alpha_g = p.alpha;
@@ -1050,55 +1082,65 @@ __global__ void __launch_bounds__(NUM_THREADS_ST, 1)
           mbar_arrive(smem_u32(&sm->acc_empty));
       }
       acc_phase ^= 1u;
-      const int64_t row = (int64_t)mt * CS::TILE_M + (int64_t)rank * 128 + 32 * q + lane;
-      const int64_t colg = (int64_t)nt * BN + h * COLS;
-      // each thread writes one row: 32-byte pieces when D allows
+      // stage 32 rows x 64 bytes at a time in this warp's buffer (16-byte
+      // pieces placed with the 64-byte swizzle: piece j of row r at
+      // j ^ ((r >> 1) & 3), which the tensor map undoes) and store it with
+      // the bulk-tensor engine; the buffer is reused once the previous store
+      // has read it
+      const int y0 = mt * CS::TILE_M + (int)rank * 128 + 32 * q;
+      const int x0 = nt * BN + h * COLS;
+      const uint32_t row_base = ebuf + lane * 64;
+      const int sw = (lane >> 1) & 3;
       if (p.out_fp32) {
-        float *dst = reinterpret_cast<float *>(p.D) + row * p.ldd + colg;
-        if (p.wide_store) {
 #pragma unroll
-          for (int i = 0; i < COLS; i += 8) {
-            uint32_t w[8];
+        for (int ch = 0; ch < COLS / 16; ++ch) {
+          if (lane == 0) bulk_wait_read_all();
+          __syncwarp();
 #pragma unroll
-            for (int u = 0; u < 8; ++u) w[u] = __float_as_uint(__uint_as_float(r[i + u]) * alpha_g);
-            st_global_v8(dst + i, w);
+          for (int j = 0; j < 4; ++j) {
+            const uint32_t *v = &r[16 * ch + 4 * j];
+            sts128(row_base + 16 * (j ^ sw), __float_as_uint(__uint_as_float(v[0]) * alpha_g),
+                   __float_as_uint(__uint_as_float(v[1]) * alpha_g),
+                   __float_as_uint(__uint_as_float(v[2]) * alpha_g),
+                   __float_as_uint(__uint_as_float(v[3]) * alpha_g));
           }
-        } else {
-#pragma unroll
-          for (int i = 0; i < COLS; i += 4)
-            *reinterpret_cast<float4 *>(dst + i) =
-                make_float4(__uint_as_float(r[i]) * alpha_g, __uint_as_float(r[i + 1]) * alpha_g,
-                            __uint_as_float(r[i + 2]) * alpha_g, __uint_as_float(r[i + 3]) * alpha_g);
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            tma_store_2d(&map_d, ebuf, x0 + 16 * ch, y0);
+            bulk_commit();
+          }
         }
       } else {
-        uint16_t *dst = reinterpret_cast<uint16_t *>(p.D) + row * p.ldd + colg;
-        if (p.wide_store) {
 #pragma unroll
-          for (int i = 0; i < COLS; i += 16) {
-            uint32_t w[8];
+        for (int ch = 0; ch < COLS / 32; ++ch) {
+          if (lane == 0) bulk_wait_read_all();
+          __syncwarp();
 #pragma unroll
-            for (int u = 0; u < 8; ++u) {
-              __nv_bfloat162 b2 = __floats2bfloat162_rn(__uint_as_float(r[i + 2 * u]) * alpha_g,
-                                                        __uint_as_float(r[i + 2 * u + 1]) * alpha_g);
-              w[u] = *reinterpret_cast<uint32_t *>(&b2);
-            }
-            st_global_v8(dst + i, w);
-          }
-        } else {
-#pragma unroll
-          for (int i = 0; i < COLS; i += 8) {
+          for (int j = 0; j < 4; ++j) {
             uint32_t w[4];
 #pragma unroll
             for (int u = 0; u < 4; ++u) {
-              __nv_bfloat162 b2 = __floats2bfloat162_rn(__uint_as_float(r[i + 2 * u]) * alpha_g,
-                                                        __uint_as_float(r[i + 2 * u + 1]) * alpha_g);
+              const int i = 32 * ch + 8 * j + 2 * u;
+              __nv_bfloat162 b2 = __floats2bfloat162_rn(__uint_as_float(r[i]) * alpha_g,
+                                                        __uint_as_float(r[i + 1]) * alpha_g);
               w[u] = *reinterpret_cast<uint32_t *>(&b2);
             }
-            *reinterpret_cast<uint4 *>(dst + i) = make_uint4(w[0], w[1], w[2], w[3]);
+            sts128(row_base + 16 * (j ^ sw), w[0], w[1], w[2], w[3]);
+          }
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            tma_store_2d(&map_d, ebuf, x0 + 32 * ch, y0);
+            bulk_commit();
           }
         }
       }
     }
+    // the stores read shared memory and write D after this: both done
+    // before the block can leave
+    if (lane == 0) bulk_wait_all();
+    __syncwarp();
   }
 
   // in a pair neither CTA leaves (or frees tensor memory) while the pair's
@@ -1159,6 +1201,22 @@ static bool make_payload_map(CUtensorMap *m, const void *base, int64_t rows, int
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// Output map for the bulk-tensor stores: D [M, N] bf16 or fp32 with row
+// stride ldd, box 64 bytes x 32 rows, 64-byte swizzle.
+static bool make_out_map(CUtensorMap *m, const GemmArgs &a) {
+  PFN_encodeTiled enc = get_encode();
+  if (!enc) return false;
+  const int esz = a.out_fp32 ? 4 : 2;
+  cuuint64_t dims[2] = {(cuuint64_t)a.N, (cuuint64_t)a.M};
+  cuuint64_t strides[1] = {(cuuint64_t)(a.ldd * esz)};
+  cuuint32_t box[2] = {(cuuint32_t)(64 / esz), 32};
+  cuuint32_t estr[2] = {1, 1};
+  return enc(m, a.out_fp32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
+             a.D, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+             CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 static gemm::Params make_params(const GemmArgs &a) {
   gemm::Params p;
   p.a_scales = a.a_scales;
@@ -1177,8 +1235,6 @@ static gemm::Params make_params(const GemmArgs &a) {
   p.timeout_ns = a.timeout_ns;
   // keep the smaller operand resident in L2 and stream the larger one once
   p.n_fastest = (a.N <= a.M) ? 1 : 0;
-  const int64_t row_bytes = a.ldd * (a.out_fp32 ? 4 : 2);
-  p.wide_store = ((reinterpret_cast<uintptr_t>(a.D) & 31u) == 0 && row_bytes % 32 == 0) ? 1 : 0;
   return p;
 }
 
@@ -1207,6 +1263,8 @@ static cudaError_t launch_st(const GemmArgs &a, cudaStream_t st) {
   CUtensorMap ma, mb;
   if (!make_payload_map(&ma, a.a_payload, a.M, a.K, gemm::BM)) return cudaErrorInvalidValue;
   if (!make_payload_map(&mb, a.b_payload, a.N, a.K, PAIR ? 128 : BN)) return cudaErrorInvalidValue;
+  CUtensorMap md;
+  if (!make_out_map(&md, a)) return cudaErrorInvalidValue;
   gemm::Params p = make_params(a);
   auto kern = gemm_st::gemm_st_kernel<KIND, BN, PAIR>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
@@ -1238,7 +1296,7 @@ static cudaError_t launch_st(const GemmArgs &a, cudaStream_t st) {
   }
   const int grid_units = (int)(tiles < units ? tiles : units);
   cfg.gridDim = dim3((unsigned)(PAIR ? 2 * grid_units : grid_units));
-  e = cudaLaunchKernelEx(&cfg, kern, ma, mb, p);
+  e = cudaLaunchKernelEx(&cfg, kern, ma, mb, md, p);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
