@@ -203,30 +203,46 @@ def launches_per_step() -> int:
 
 
 def quantize_sweep(fa, device, reps: int = 20) -> list[dict]:
-    """Quantizer sweep shapes (0.5*t_3 with outlier columns), row-wise RNE,
-    rotating over enough input copies that the working set exceeds L2."""
+    """Quantizer sweep shapes (0.5*t_3 with 1% outlier columns x50): every
+    format x rounding x orientation, plus the column-wise Hadamard MXFP4
+    quantizer, rotating over enough input copies that the working set
+    exceeds L2 (>= 256 MB)."""
+    hbm = _peaks()[0]
     out = []
+    cases = [(fmt, key, rnd, orient, False)
+             for orient in (fa.ROWWISE, fa.COLWISE)
+             for fmt, key in ((fa.MXFP4, "mx"), (fa.NVFP4_GLOBAL, "nvg"), (fa.NVFP4_CTA, "nvc"))
+             for rnd in (fa.RNE, fa.SR)]
+    cases += [(fa.MXFP4, "mx", rnd, fa.COLWISE, True) for rnd in (fa.RNE, fa.SR)]
     for rows, cols in workloads.SWEEP_SHAPES:
         nbuf = max(1, (512 << 20) // (rows * cols * 2))
         xs = [workloads.sweep(rows, cols, seed=i, device=device) for i in range(min(nbuf, 8))]
-        for fmt, key in ((fa.MXFP4, "mx"), (fa.NVFP4_GLOBAL, "nvg"), (fa.NVFP4_CTA, "nvc")):
-            for rnd in (fa.RNE, fa.SR):
-                qs = [fa.empty_qtensor(rows, cols, fmt, fa.ROWWISE, device) for _ in xs]
-                ws = fa.workspace(1 << 16, device)
-                for i in range(3):
-                    fa.quantize(xs[i % len(xs)], fmt, rnd, fa.ROWWISE, 1, out=qs[i % len(xs)], ws=ws)
-                torch.cuda.synchronize()
-                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-                e0.record()
-                for i in range(reps):
-                    fa.quantize(xs[i % len(xs)], fmt, rnd, fa.ROWWISE, 1, out=qs[i % len(xs)], ws=ws)
-                e1.record()
-                torch.cuda.synchronize()
-                us = e0.elapsed_time(e1) * 1000.0 / reps
-                gbs = BYTES_PER_ELEM[key] * rows * cols / (us * 1e-6) / 1e9
-                out.append({"shape": [rows, cols], "fmt": key, "rnd": "sr" if rnd else "rne",
-                            "us": round(us, 2), "GBps": round(gbs, 1)})
-                del qs
+        ws = fa.workspace(1 << 16, device)
+        for fmt, key, rnd, orient, had in cases:
+            qs = [fa.empty_qtensor(rows, cols, fmt, orient, device) for _ in xs]
+
+            def call(i):
+                if had:
+                    fa.hadamard32_quantize(xs[i % len(xs)], SIGN_MASK, rnd, 1, out=qs[i % len(xs)],
+                                           ws=ws)
+                else:
+                    fa.quantize(xs[i % len(xs)], fmt, rnd, orient, 1, out=qs[i % len(xs)], ws=ws)
+
+            for i in range(3):
+                call(i)
+            torch.cuda.synchronize()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            for i in range(reps):
+                call(i)
+            e1.record()
+            torch.cuda.synchronize()
+            us = e0.elapsed_time(e1) * 1000.0 / reps
+            gbs = BYTES_PER_ELEM[key] * rows * cols / (us * 1e-6) / 1e9
+            out.append({"shape": [rows, cols], "fmt": key, "rnd": "sr" if rnd else "rne",
+                        "orient": ("col" if orient else "row") + ("+had32" if had else ""),
+                        "us": round(us, 2), "GBps": round(gbs, 1), "frac_hbm": round(gbs / hbm, 3)})
+            del qs
         del xs
         torch.cuda.empty_cache()
     return out
