@@ -7,8 +7,10 @@ tokens, forward and backward:
   dgrad  dX = dY W      dY quantized row-wise MXFP4 with stochastic rounding
   wgrad  dW = dY^T X    dY and X quantized column-wise MXFP4 with the
                         fixed-sign 32-point Hadamard (RNE), GEMM with alpha 1/32
-Weights are quantized once before timing (row-wise NVFP4-global for fwd,
-column-wise MXFP4 for dgrad).  Inputs are synthetic (seeded generators in
+X and dY are each read once by the dual-orientation producer: X gives the
+forward operand and the saved wgrad operand, dY the dgrad and wgrad
+operands.  Weights are quantized once before timing (row-wise NVFP4-global
+for fwd, column-wise MXFP4 for dgrad).  Inputs are synthetic (seeded generators in
 workloads.py).  Each step reads ~1.1 GB of bf16 inputs, more than the 126 MB
 L2, so no timed iteration finds its inputs in L2.
 
@@ -41,7 +43,10 @@ SIGN_MASK = 0x2545F491
 T = workloads.LLAMA8B_TOKENS
 LAYERS = workloads.LLAMA8B_LINEARS
 BYTES_PER_ELEM = {"mx": 2.0 + 0.5 + 1.0 / 32, "nvg": 2.0 + 2.0 + 0.5 + 1.0 / 16,
-                  "nvc": 2.0 + 0.5 + 1.0 / 16 + 4.0 / (128 * 128)}
+                  "nvc": 2.0 + 0.5 + 1.0 / 16 + 4.0 / (128 * 128),
+                  # dual producers: one read, both operands written (+ the NVFP4-global amax read)
+                  "nvg_dual": 2.0 + 2.0 + (0.5 + 1.0 / 16) + (0.5 + 1.0 / 32),
+                  "mx_dual": 2.0 + (0.5 + 1.0 / 32) + (0.5 + 1.0 / 32)}
 
 
 # DRAM bytes (read + write) per launch of the dominant kernel, the MXFP4
@@ -174,8 +179,7 @@ class Block:
             L["wc"] = fa.quantize(L["w"], fa.MXFP4, fa.RNE, fa.COLWISE, ws=self.ws)
 
 
-KINDS = ["quant_fwd_nvg", "gemm_fwd", "quant_dgrad_mx_sr", "gemm_dgrad", "quant_wgrad_had",
-         "gemm_wgrad"]
+KINDS = ["quant_fwd_dual", "gemm_fwd", "quant_bwd_dual", "gemm_dgrad", "gemm_wgrad"]
 
 
 def run_step(fa, blk: Block, step: int, events=None):
@@ -191,17 +195,18 @@ def run_step(fa, blk: Block, step: int, events=None):
             events.append((kind, name, e))
 
     for name, L in blk.layers.items():
-        fa.quantize(L["x"], fa.NVFP4_GLOBAL, fa.RNE, fa.ROWWISE, out=L["xq"], ws=blk.ws)
-        mark("quant_fwd_nvg", name)
+        # forward: X -> NVFP4-global operand + saved MXFP4 Hadamard wgrad operand
+        fa.quantize_dual(L["x"], fa.NVFP4_GLOBAL, fa.RNE, 0, col_hadamard=True,
+                         sign_mask=SIGN_MASK, row_out=L["xq"], col_out=L["xc"], ws=blk.ws)
+        mark("quant_fwd_dual", name)
         fa.gemm(L["xq"], L["wq"], 1.0, out=L["y"], ws=blk.ws)
         mark("gemm_fwd", name)
-        fa.quantize(L["dy"], fa.MXFP4, fa.SR, fa.ROWWISE, seed=seed, out=L["gq"], ws=blk.ws)
-        mark("quant_dgrad_mx_sr", name)
+        # backward: dY -> MXFP4 SR dgrad operand + MXFP4 Hadamard wgrad operand
+        fa.quantize_dual(L["dy"], fa.MXFP4, fa.SR, seed, col_hadamard=True, sign_mask=SIGN_MASK,
+                         row_out=L["gq"], col_out=L["gc"], ws=blk.ws)
+        mark("quant_bwd_dual", name)
         fa.gemm(L["gq"], L["wc"], 1.0, out=L["dx"], ws=blk.ws)
         mark("gemm_dgrad", name)
-        fa.hadamard32_quantize(L["dy"], SIGN_MASK, fa.RNE, out=L["gc"], ws=blk.ws)
-        fa.hadamard32_quantize(L["x"], SIGN_MASK, fa.RNE, out=L["xc"], ws=blk.ws)
-        mark("quant_wgrad_had", name)
         fa.gemm(L["gc"], L["xc"], 1.0 / 32, out=L["dw"], ws=blk.ws)
         mark("gemm_wgrad", name)
 
@@ -210,16 +215,20 @@ def kernel_work(kind: str, cin: int, cout: int) -> tuple[float, str]:
     """Algorithmic work of one call: bytes (quantizers) or FLOPs (GEMMs)."""
     if kind.startswith("gemm"):
         return 2.0 * T * cin * cout, "flop"
+    if kind == "quant_fwd_dual":
+        return BYTES_PER_ELEM["nvg_dual"] * T * cin, "byte"
+    if kind == "quant_bwd_dual":
+        return BYTES_PER_ELEM["mx_dual"] * T * cout, "byte"
     if kind == "quant_fwd_nvg":
         return BYTES_PER_ELEM["nvg"] * T * cin, "byte"
     if kind == "quant_dgrad_mx_sr":
         return BYTES_PER_ELEM["mx"] * T * cout, "byte"
-    return BYTES_PER_ELEM["mx"] * T * (cin + cout), "byte"  # two Hadamard quantizations
+    return BYTES_PER_ELEM["mx"] * T * cout, "byte"  # one Hadamard quantization of dY
 
 
 def launches_per_step() -> int:
-    # per layer: amax + quant (NVG), gemm, quant (SR), gemm, 2 Hadamard quants, gemm
-    return len(LAYERS) * 8
+    # per layer: amax + dual (X), GEMM, dual (dY), GEMM, GEMM
+    return len(LAYERS) * 6
 
 
 def quantize_sweep(fa, device, reps: int = 20) -> list[dict]:
@@ -269,7 +278,8 @@ def quantize_sweep(fa, device, reps: int = 20) -> list[dict]:
 
 
 def e2e_run(fa, blk: Block, steps: int, device) -> dict:
-    """Same step through the public linear_* calls with host (pinned) inputs
+    """Same step through the public training-form linear calls
+    (linear_fwd_save, linear_bwd) with host (pinned) inputs
     and outputs: the H2D copy of X and dY and the D2H copy of Y, dX and dW of
     every layer are inside the timed region."""
     host = {}
@@ -281,8 +291,8 @@ def e2e_run(fa, blk: Block, steps: int, device) -> dict:
                           dw=torch.empty_like(L["dw"], device="cpu").pin_memory())
         h2d += L["x"].numel() * 2 + L["dy"].numel() * 2
         d2h += L["y"].numel() * 2 + L["dx"].numel() * 2 + L["dw"].numel() * 4
-    wsz = max(fa.linear_ws_bytes(k, T, cin, cout, fa.NVFP4_GLOBAL if k == 0 else fa.MXFP4)
-              for k in range(3) for cin, cout in LAYERS.values())
+    wsz = max(fa.linear_ws_bytes(k, T, cin, cout, fa.NVFP4_GLOBAL if k == 3 else fa.MXFP4)
+              for k in (3, 4) for cin, cout in LAYERS.values())
     ws = fa.workspace(wsz, device)
 
     def one(step):
@@ -290,9 +300,10 @@ def e2e_run(fa, blk: Block, steps: int, device) -> dict:
             H = host[name]
             L["x"].copy_(H["x"], non_blocking=True)
             L["dy"].copy_(H["dy"], non_blocking=True)
-            fa.linear_fwd(L["x"], L["wq"], fa.NVFP4_GLOBAL, out=L["y"], ws=ws)
-            fa.linear_dgrad(L["dy"], L["wc"], fa.MXFP4, fa.SR, seed=step, out=L["dx"], ws=ws)
-            fa.linear_wgrad(L["dy"], L["x"], SIGN_MASK, fa.RNE, seed=step, out=L["dw"], ws=ws)
+            fa.linear_fwd_save(L["x"], L["wq"], fa.NVFP4_GLOBAL, SIGN_MASK, out=L["y"],
+                               xcol=L["xc"], ws=ws)
+            fa.linear_bwd(L["dy"], L["wc"], L["xc"], fa.MXFP4, fa.SR, seed=step,
+                          sign_mask=SIGN_MASK, dx=L["dx"], dw=L["dw"], ws=ws)
             H["y"].copy_(L["y"], non_blocking=True)
             H["dx"].copy_(L["dx"], non_blocking=True)
             H["dw"].copy_(L["dw"], non_blocking=True)
@@ -379,6 +390,7 @@ def bench_config(world: int) -> dict:
             "layers": {k: list(v) for k, v in LAYERS.items()},
             "fwd": "NVFP4-global RNE", "dgrad": "MXFP4 row-wise SR",
             "wgrad": "MXFP4 column-wise fixed-sign Hadamard-32 RNE, alpha 1/32",
+            "producers": "dual-orientation: one read each of X and dY",
             "parallelism": f"replicas x{world}", "l2": "inputs > L2 (1.1 GB bf16 read per step)"}
 
 
@@ -518,7 +530,7 @@ def profile_arm(args, device) -> dict:
     """Run one call kind on one layer only (warm-up + steps launches), for a
     profiler capture of a single kernel: --profile KIND:LAYER, KIND one of
     gemm_fwd, gemm_dgrad, gemm_wgrad, quant_fwd_nvg, quant_dgrad_mx_sr,
-    quant_wgrad_had."""
+    quant_wgrad_had, quant_fwd_dual, quant_bwd_dual."""
     import fp4_quantization_block_b200 as fa
     kind, layer = args.profile.split(":")
     cin, cout = LAYERS[layer]
@@ -549,6 +561,16 @@ def profile_arm(args, device) -> dict:
     elif kind == "quant_wgrad_had":
         q = fa.empty_qtensor(T, cout, fa.MXFP4, fa.COLWISE, device)
         call = lambda: fa.hadamard32_quantize(dy, SIGN_MASK, out=q, ws=ws)
+    elif kind == "quant_fwd_dual":
+        qr = fa.empty_qtensor(T, cin, fa.NVFP4_GLOBAL, fa.ROWWISE, device)
+        qc = fa.empty_qtensor(T, cin, fa.MXFP4, fa.COLWISE, device)
+        call = lambda: fa.quantize_dual(x, fa.NVFP4_GLOBAL, fa.RNE, 0, True, SIGN_MASK,
+                                        row_out=qr, col_out=qc, ws=ws)
+    elif kind == "quant_bwd_dual":
+        qr = fa.empty_qtensor(T, cout, fa.MXFP4, fa.ROWWISE, device)
+        qc = fa.empty_qtensor(T, cout, fa.MXFP4, fa.COLWISE, device)
+        call = lambda: fa.quantize_dual(dy, fa.MXFP4, fa.SR, 1, True, SIGN_MASK,
+                                        row_out=qr, col_out=qc, ws=ws)
     else:
         raise SystemExit(f"unknown kind {kind}")
     for _ in range(args.warmup):

@@ -24,8 +24,8 @@ import torch
 __all__ = [
     "MXFP4", "NVFP4_GLOBAL", "NVFP4_CTA", "RNE", "SR", "ROWWISE", "COLWISE",
     "QTensor", "FA4Error", "lib", "library_path", "quant_sizes", "empty_qtensor", "quantize",
-    "hadamard32_quantize", "gemm", "linear_ws_bytes", "linear_fwd", "linear_dgrad",
-    "linear_wgrad", "workspace", "check_device_status",
+    "hadamard32_quantize", "quantize_dual", "gemm", "linear_ws_bytes", "linear_fwd", "linear_dgrad",
+    "linear_wgrad", "linear_fwd_save", "linear_bwd", "workspace", "check_device_status",
 ]
 
 MXFP4, NVFP4_GLOBAL, NVFP4_CTA = 0, 1, 2
@@ -77,11 +77,14 @@ def _declare(L: ctypes.CDLL) -> ctypes.CDLL:
         "fa4_quant_sizes": [i64, i64, ci, ci, PSZ, PSZ, PSZ, PSZ],
         "fa4_quantize": [P, i64, i64, i64, ci, ci, ci, u64, _QT, P, sz, P],
         "fa4_hadamard32_quantize": [P, i64, i64, i64, u32, ci, u64, _QT, P, sz, P],
+        "fa4_quantize_dual": [P, i64, i64, i64, ci, ci, u64, _QT, ci, u32, ci, u64, _QT, P, sz, P],
         "fa4_gemm_blockscaled": [_QT, _QT, i64, i64, i64, ci, f32, P, i64, ci, P, sz, P],
         "fa4_linear_ws_bytes": [ci, i64, i64, i64, ci, PSZ],
         "fa4_linear_fwd": [P, _QT, i64, i64, i64, ci, P, P, sz, P],
         "fa4_linear_dgrad": [P, _QT, i64, i64, i64, ci, ci, u64, P, P, sz, P],
         "fa4_linear_wgrad": [P, P, i64, i64, i64, u32, ci, u64, P, ci, P, sz, P],
+        "fa4_linear_fwd_save": [P, _QT, i64, i64, i64, ci, u32, P, _QT, P, sz, P],
+        "fa4_linear_bwd": [P, _QT, _QT, i64, i64, i64, ci, ci, u64, u32, P, P, ci, P, sz, P],
         "fa4_workspace_init": [P, sz, P],
         "fa4_check_device_status": [P, P],
         "fa4_debug_convert": [P, P, i64, P, P, P, P],
@@ -204,6 +207,26 @@ def hadamard32_quantize(x: torch.Tensor, sign_mask: int, rnd: int = RNE, seed: i
     return out
 
 
+def quantize_dual(x: torch.Tensor, row_fmt: int, row_rnd: int = RNE, row_seed: int = 0,
+                  col_hadamard: bool = True, sign_mask: int = 0, col_rnd: int = RNE,
+                  col_seed: int = 0, row_out: QTensor | None = None,
+                  col_out: QTensor | None = None,
+                  ws: torch.Tensor | None = None) -> tuple[QTensor, QTensor]:
+    """One read of x: the row-wise operand (any format) and the column-wise
+    MXFP4 operand (with the fixed-sign Hadamard when col_hadamard)."""
+    ld = _as_bf16_2d(x, "x")
+    rows, cols = x.shape
+    row_out = row_out or empty_qtensor(rows, cols, row_fmt, ROWWISE, x.device)
+    col_out = col_out or empty_qtensor(rows, cols, MXFP4, COLWISE, x.device)
+    need = quant_sizes(rows, cols, row_fmt, ROWWISE)[3]
+    ws = _ws(ws, need, x.device)
+    _check(lib().fa4_quantize_dual(_ptr(x), rows, cols, ld, row_fmt, row_rnd, row_seed,
+                                   row_out.c(), 1 if col_hadamard else 0, sign_mask & 0xFFFFFFFF,
+                                   col_rnd, col_seed, col_out.c(), _ptr(ws), ws.numel(),
+                                   _stream(x.device)), "fa4_quantize_dual")
+    return row_out, col_out
+
+
 def gemm(A: QTensor, B: QTensor, alpha: float = 1.0, out_dtype=torch.float32,
          out: torch.Tensor | None = None, ws: torch.Tensor | None = None) -> torch.Tensor:
     """D[M, N] = alpha * A B^T on the block-scaled FP4 tensor cores."""
@@ -305,3 +328,37 @@ def debug_gemm_timeout(A: QTensor, B: QTensor, skip_k_tile: int, timeout_ns: int
                                         skip_k_tile, timeout_ns, _ptr(ws), ws.numel(), _stream(dev)),
            "fa4_debug_gemm_timeout")
     return out
+
+
+def linear_fwd_save(X: torch.Tensor, Wq: QTensor, fmt: int, sign_mask: int,
+                    out: torch.Tensor | None = None, xcol: QTensor | None = None,
+                    ws: torch.Tensor | None = None) -> tuple[torch.Tensor, QTensor]:
+    """Y = X W^T, plus X's column-wise MXFP4 Hadamard operand for the
+    backward half (one read of X)."""
+    T, Cin = X.shape
+    Cout = Wq.R
+    Y = out if out is not None else torch.empty(T, Cout, dtype=torch.bfloat16, device=X.device)
+    xcol = xcol or empty_qtensor(T, Cin, MXFP4, COLWISE, X.device)
+    ws = _ws(ws, linear_ws_bytes(3, T, Cin, Cout, fmt), X.device)
+    _check(lib().fa4_linear_fwd_save(_ptr(X), Wq.c(), T, Cin, Cout, fmt, sign_mask & 0xFFFFFFFF,
+                                     _ptr(Y), xcol.c(), _ptr(ws), ws.numel(), _stream(X.device)),
+           "fa4_linear_fwd_save")
+    return Y, xcol
+
+
+def linear_bwd(dY: torch.Tensor, Wq_col: QTensor, xcol: QTensor, fmt: int, rnd: int = SR,
+               seed: int = 0, sign_mask: int = 0, dw_dtype=torch.float32,
+               dx: torch.Tensor | None = None, dw: torch.Tensor | None = None,
+               ws: torch.Tensor | None = None) -> tuple[torch.Tensor, torch.Tensor]:
+    """dX = dY W and dW = dY^T X from one read of dY (xcol from
+    linear_fwd_save with the same sign_mask)."""
+    T, Cout = dY.shape
+    Cin = Wq_col.R
+    dX = dx if dx is not None else torch.empty(T, Cin, dtype=torch.bfloat16, device=dY.device)
+    dW = dw if dw is not None else torch.empty(Cout, Cin, dtype=dw_dtype, device=dY.device)
+    od = OUT_FP32 if dW.dtype == torch.float32 else OUT_BF16
+    ws = _ws(ws, linear_ws_bytes(4, T, Cin, Cout, fmt), dY.device)
+    _check(lib().fa4_linear_bwd(_ptr(dY), Wq_col.c(), xcol.c(), T, Cin, Cout, fmt, rnd, seed,
+                                sign_mask & 0xFFFFFFFF, _ptr(dX), _ptr(dW), od, _ptr(ws),
+                                ws.numel(), _stream(dY.device)), "fa4_linear_bwd")
+    return dX, dW

@@ -89,6 +89,27 @@ fa4_status do_quantize(const void *x, int64_t rows, int64_t cols, int64_t ld, in
   return cuda_status(e);
 }
 
+// Both orientations from one read of x (the row-wise NVFP4-global amax pass
+// first, when needed).
+fa4_status do_quantize_dual(const void *x, int64_t rows, int64_t cols, int64_t ld, int row_fmt,
+                            int row_rnd, uint64_t row_seed, const fa4_qtensor &row_out,
+                            bool hadamard, uint32_t sign_mask, int col_rnd, uint64_t col_seed,
+                            const fa4_qtensor &col_out, uint8_t *ws, cudaStream_t st) {
+  const uint16_t *xb = static_cast<const uint16_t *>(x);
+  float *partials = reinterpret_cast<float *>(ws + kHdr);
+  int np = 0;
+  if (row_fmt == FA4_NVFP4_GLOBAL) {
+    np = fa4::amax_partials_count(rows, cols);
+    cudaError_t e = fa4::launch_tensor_amax(xb, rows, cols, ld, partials, np, st);
+    if (e != cudaSuccess) return FA4_ERR_CUDA;
+  }
+  return cuda_status(fa4::launch_quant_dual(
+      row_fmt, row_rnd, col_rnd, hadamard, sign_mask, xb, rows, cols, ld,
+      static_cast<uint8_t *>(row_out.payload), static_cast<uint8_t *>(row_out.scales),
+      row_out.tensor_scale, static_cast<uint8_t *>(col_out.payload),
+      static_cast<uint8_t *>(col_out.scales), partials, np, row_seed, col_seed, st));
+}
+
 fa4_status do_gemm(const fa4_qtensor &A, const fa4_qtensor &B, int64_t M, int64_t N, int64_t K,
                    int fmt, float alpha, void *D, int64_t ldd, int out_dtype, uint8_t *ws,
                    cudaStream_t st, int skip, uint64_t timeout_ns) {
@@ -192,6 +213,25 @@ fa4_status fa4_hadamard32_quantize(const void *x, int64_t rows, int64_t cols, in
                      static_cast<uint8_t *>(workspace), S(stream));
 }
 
+fa4_status fa4_quantize_dual(const void *x, int64_t rows, int64_t cols, int64_t ld,
+                             fa4_format row_fmt, fa4_round row_rnd, uint64_t row_seed,
+                             fa4_qtensor row_out, int col_hadamard, uint32_t sign_mask,
+                             fa4_round col_rnd, uint64_t col_seed, fa4_qtensor col_out,
+                             void *workspace, size_t workspace_bytes, void *stream) {
+  if (!fmt_ok(row_fmt) || (row_rnd != FA4_RNE && row_rnd != FA4_SR) ||
+      (col_rnd != FA4_RNE && col_rnd != FA4_SR))
+    return FA4_ERR_INVALID_ARG;
+  fa4_status s = check_input(x, rows, cols, ld);
+  if (s != FA4_OK) return s;
+  if ((s = check_qt(row_out, row_fmt)) != FA4_OK) return s;
+  if ((s = check_qt(col_out, FA4_MXFP4)) != FA4_OK) return s;
+  if (!workspace || workspace_bytes < quant_ws(row_fmt)) return FA4_ERR_WORKSPACE;
+  if (!aligned16(workspace)) return FA4_ERR_ALIGN;
+  return do_quantize_dual(x, rows, cols, ld, row_fmt, row_rnd, row_seed, row_out, col_hadamard != 0,
+                          sign_mask, col_rnd, col_seed, col_out, static_cast<uint8_t *>(workspace),
+                          S(stream));
+}
+
 fa4_status fa4_gemm_blockscaled(fa4_qtensor A, fa4_qtensor B, int64_t M, int64_t N, int64_t K,
                                 fa4_format fmt, float alpha, void *D, int64_t ldd,
                                 fa4_out_dtype out_dtype, void *workspace, size_t workspace_bytes,
@@ -211,6 +251,8 @@ fa4_status fa4_linear_ws_bytes(int kind, int64_t T, int64_t Cin, int64_t Cout, f
     case 0: b += qt_ws_bytes(T, Cin, fmt); break;
     case 1: b += qt_ws_bytes(T, Cout, fmt); break;
     case 2: b += qt_ws_bytes(Cout, T, FA4_MXFP4) + qt_ws_bytes(Cin, T, FA4_MXFP4); break;
+    case 3: b += qt_ws_bytes(T, Cin, fmt); break;
+    case 4: b += qt_ws_bytes(T, Cout, fmt) + qt_ws_bytes(Cout, T, FA4_MXFP4); break;
     default: return FA4_ERR_INVALID_ARG;
   }
   *workspace_bytes = b;
@@ -281,6 +323,56 @@ fa4_status fa4_linear_wgrad(const void *dY, const void *X, int64_t T, int64_t Ci
                        S(stream))) != FA4_OK)
     return s;
   return do_gemm(gq, xq, Cout, Cin, T, FA4_MXFP4, 1.0f / 32.0f, dW, Cin, out_dtype, ws, S(stream),
+                 -1, kDefaultTimeoutNs);
+}
+
+fa4_status fa4_linear_fwd_save(const void *X, fa4_qtensor Wq, int64_t T, int64_t Cin, int64_t Cout,
+                               fa4_format fmt, uint32_t sign_mask, void *Y, fa4_qtensor Xcol,
+                               void *workspace, size_t workspace_bytes, void *stream) {
+  size_t need;
+  fa4_status s = fa4_linear_ws_bytes(3, T, Cin, Cout, fmt, &need);
+  if (s != FA4_OK) return s;
+  if ((s = check_input(X, T, Cin, Cin)) != FA4_OK) return s;
+  if ((s = check_qt(Xcol, FA4_MXFP4)) != FA4_OK) return s;
+  if (!workspace || workspace_bytes < need) return FA4_ERR_WORKSPACE;
+  if (!aligned16(workspace)) return FA4_ERR_ALIGN;
+  uint8_t *ws = static_cast<uint8_t *>(workspace);
+  fa4_qtensor xq = carve_qt(ws + kHdr + partials_bytes(), T, Cin, fmt);
+  if ((s = check_gemm(xq, Wq, T, Cout, Cin, fmt, Y, Cout, FA4_OUT_BF16, ws, workspace_bytes)) != FA4_OK)
+    return s;
+  if ((s = do_quantize_dual(X, T, Cin, Cin, fmt, FA4_RNE, 0u, xq, true, sign_mask, FA4_RNE, 0u, Xcol,
+                            ws, S(stream))) != FA4_OK)
+    return s;
+  return do_gemm(xq, Wq, T, Cout, Cin, fmt, 1.0f, Y, Cout, FA4_OUT_BF16, ws, S(stream), -1,
+                 kDefaultTimeoutNs);
+}
+
+fa4_status fa4_linear_bwd(const void *dY, fa4_qtensor Wq_col, fa4_qtensor Xcol, int64_t T,
+                          int64_t Cin, int64_t Cout, fa4_format fmt, fa4_round rnd, uint64_t seed,
+                          uint32_t sign_mask, void *dX, void *dW, fa4_out_dtype dw_dtype,
+                          void *workspace, size_t workspace_bytes, void *stream) {
+  if (rnd != FA4_RNE && rnd != FA4_SR) return FA4_ERR_INVALID_ARG;
+  size_t need;
+  fa4_status s = fa4_linear_ws_bytes(4, T, Cin, Cout, fmt, &need);
+  if (s != FA4_OK) return s;
+  if ((s = check_input(dY, T, Cout, Cout)) != FA4_OK) return s;
+  if (!workspace || workspace_bytes < need) return FA4_ERR_WORKSPACE;
+  if (!aligned16(workspace)) return FA4_ERR_ALIGN;
+  uint8_t *ws = static_cast<uint8_t *>(workspace);
+  uint8_t *base = ws + kHdr + partials_bytes();
+  fa4_qtensor gq = carve_qt(base, T, Cout, fmt);
+  fa4_qtensor gc = carve_qt(base + qt_ws_bytes(T, Cout, fmt), Cout, T, FA4_MXFP4);
+  if ((s = check_gemm(gq, Wq_col, T, Cin, Cout, fmt, dX, Cin, FA4_OUT_BF16, ws, workspace_bytes)) != FA4_OK)
+    return s;
+  if ((s = check_gemm(gc, Xcol, Cout, Cin, T, FA4_MXFP4, dW, Cin, dw_dtype, ws, workspace_bytes)) != FA4_OK)
+    return s;
+  if ((s = do_quantize_dual(dY, T, Cout, Cout, fmt, rnd, seed, gq, true, sign_mask, FA4_RNE, 0u, gc,
+                            ws, S(stream))) != FA4_OK)
+    return s;
+  if ((s = do_gemm(gq, Wq_col, T, Cin, Cout, fmt, 1.0f, dX, Cin, FA4_OUT_BF16, ws, S(stream), -1,
+                   kDefaultTimeoutNs)) != FA4_OK)
+    return s;
+  return do_gemm(gc, Xcol, Cout, Cin, T, FA4_MXFP4, 1.0f / 32.0f, dW, Cin, dw_dtype, ws, S(stream),
                  -1, kDefaultTimeoutNs);
 }
 

@@ -22,6 +22,12 @@ cudaError_t launch_quant_colwise(int fmt, int rnd, bool hadamard, uint32_t sign_
                                  uint8_t *payload, uint8_t *scales, float *ts,
                                  const float *partials, int n_partials, uint64_t seed,
                                  cudaStream_t st);
+cudaError_t launch_quant_dual(int row_fmt, int row_rnd, int col_rnd, bool hadamard,
+                              uint32_t sign_mask, const uint16_t *x, int64_t T, int64_t C,
+                              int64_t ld, uint8_t *row_payload, uint8_t *row_scales, float *row_ts,
+                              uint8_t *col_payload, uint8_t *col_scales, const float *partials,
+                              int n_partials, uint64_t row_seed, uint64_t col_seed,
+                              cudaStream_t st);
 cudaError_t launch_debug_convert(const float *y, const uint32_t *u16, int64_t n, uint8_t *rne,
                                  uint8_t *sr, uint8_t *e4m3, cudaStream_t st);
 cudaError_t launch_debug_sr_bits(uint64_t seed, const uint64_t *idx, int64_t n, uint32_t *bits,

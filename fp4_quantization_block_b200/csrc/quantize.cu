@@ -104,36 +104,17 @@ __global__ void __launch_bounds__(256) tensor_amax_kernel(const uint16_t *__rest
 // for steps s = 0..7, columns 8*(l&15) .. +8.  A half-warp covers one row;
 // NV blocks (16) are lane pairs, MX blocks (32) lane quads.
 // --------------------------------------------------------------------------
+// Row-wise quantization of one 128x128 tile of Q held in registers: v[s] is
+// row r0 + 16 s + 2 w + (l >> 4), columns k0 + 8 (l & 15) .. + 8.  s_enc is the
+// NVFP4 encode scale (unused for MXFP4).
 template <int FMT, int RND>
-__global__ void __launch_bounds__(256) quant_rowwise_kernel(
-    const uint16_t *__restrict__ x, int64_t R, int64_t K, int64_t ld, uint8_t *__restrict__ payload,
-    uint8_t *__restrict__ scales, float *__restrict__ ts, const float *__restrict__ partials,
-    int n_partials, uint64_t seed) {
-  __shared__ float red[8];
+__device__ __forceinline__ void rowwise_tile(const uint4 (&v)[8], int64_t r0, int64_t k0, int64_t K,
+                                             uint8_t *__restrict__ payload,
+                                             uint8_t *__restrict__ scales, float s_enc,
+                                             uint64_t seed) {
   const int w = threadIdx.x >> 5, l = threadIdx.x & 31;
-  const int64_t k0 = (int64_t)blockIdx.x * 128, r0 = (int64_t)blockIdx.y * 128;
   const int c = l & 15;          // 8-element chunk within the 128-wide row
   const int64_t kc = k0 + 8 * c;  // first column of the chunk
-
-  uint4 v[8];
-#pragma unroll
-  for (int s = 0; s < 8; ++s) {
-    const int64_t r = r0 + 16 * s + 2 * w + (l >> 4);
-    v[s] = ld_stream(x + r * ld + kc);
-  }
-
-  float s_enc = 1.0f;
-  if constexpr (FMT == kNVC) {
-    float m = 0.0f;
-#pragma unroll
-    for (int s = 0; s < 8; ++s) m = fmaxf(m, absmax8(v[s]));
-    s_enc = nv_encode_scale(cta_max256(m, red));
-    if (threadIdx.x == 0) ts[blockIdx.y * gridDim.x + blockIdx.x] = nv_decode_scale(s_enc);
-  } else if constexpr (FMT == kNVG) {
-    s_enc = nv_encode_scale(reduce_partials(partials, n_partials, red));
-    if (threadIdx.x == 0 && blockIdx.x == 0 && blockIdx.y == 0) ts[0] = nv_decode_scale(s_enc);
-  }
-
   const int64_t kbt = (FMT == kMX) ? (K >> 5) : (K >> 4);
 #pragma unroll
   for (int s = 0; s < 8; ++s) {
@@ -180,6 +161,53 @@ __global__ void __launch_bounds__(256) quant_rowwise_kernel(
   }
 }
 
+// Loads of one 128x128 tile in the row-wise thread layout (16-byte lanes, all
+// issued before any arithmetic).
+__device__ __forceinline__ void load_tile_rowwise(const uint16_t *__restrict__ x, int64_t ld,
+                                                  int64_t r0, int64_t k0, uint4 (&v)[8]) {
+  const int w = threadIdx.x >> 5, l = threadIdx.x & 31;
+#pragma unroll
+  for (int s = 0; s < 8; ++s) {
+    const int64_t r = r0 + 16 * s + 2 * w + (l >> 4);
+    v[s] = ld_stream(x + r * ld + k0 + 8 * (l & 15));
+  }
+}
+
+// NVFP4 encode scale of the tile's domain: CTA-local (this tile's amax, ts
+// written at ts_index) or global (reduced from the amax partials, ts[0]
+// written by block (0, 0)); 1 for MXFP4.
+template <int FMT>
+__device__ __forceinline__ float tile_encode_scale(const uint4 (&v)[8], float *__restrict__ ts,
+                                                   int64_t ts_index, const float *__restrict__ partials,
+                                                   int n_partials, float *red) {
+  float s_enc = 1.0f;
+  if constexpr (FMT == kNVC) {
+    float m = 0.0f;
+#pragma unroll
+    for (int s = 0; s < 8; ++s) m = fmaxf(m, absmax8(v[s]));
+    s_enc = nv_encode_scale(cta_max256(m, red));
+    if (threadIdx.x == 0) ts[ts_index] = nv_decode_scale(s_enc);
+  } else if constexpr (FMT == kNVG) {
+    s_enc = nv_encode_scale(reduce_partials(partials, n_partials, red));
+    if (threadIdx.x == 0 && blockIdx.x == 0 && blockIdx.y == 0) ts[0] = nv_decode_scale(s_enc);
+  }
+  return s_enc;
+}
+
+template <int FMT, int RND>
+__global__ void __launch_bounds__(256) quant_rowwise_kernel(
+    const uint16_t *__restrict__ x, int64_t R, int64_t K, int64_t ld, uint8_t *__restrict__ payload,
+    uint8_t *__restrict__ scales, float *__restrict__ ts, const float *__restrict__ partials,
+    int n_partials, uint64_t seed) {
+  __shared__ float red[8];
+  const int64_t k0 = (int64_t)blockIdx.x * 128, r0 = (int64_t)blockIdx.y * 128;
+  uint4 v[8];
+  load_tile_rowwise(x, ld, r0, k0, v);
+  const float s_enc = tile_encode_scale<FMT>(v, ts, (int64_t)blockIdx.y * gridDim.x + blockIdx.x,
+                                             partials, n_partials, red);
+  rowwise_tile<FMT, RND>(v, r0, k0, K, payload, scales, s_enc, seed);
+}
+
 // --------------------------------------------------------------------------
 // Column-wise quantizer: Q = x^T, x[T, C] row-major; Q[R = C, K = T].
 // The 128(tokens) x 128(channels) tile is staged in shared memory; each
@@ -202,47 +230,16 @@ __device__ __forceinline__ void fwht32(float *v) {
   }
 }
 
+// Column-wise quantization of the 128 (tokens) x 128 (channels) tile staged
+// in shared memory (tile[token][channel]; complete before the call): Q = x^T,
+// rows c0 .. c0+127 of Q, K range t0 .. t0+127.  sbuf holds 128 x 8 scale
+// bytes.  Ends with the tile's scale words written.
 template <int FMT, int RND, bool HAD>
-__global__ void __launch_bounds__(256) quant_colwise_kernel(
-    const uint16_t *__restrict__ x, int64_t T, int64_t C, int64_t ld, uint8_t *__restrict__ payload,
-    uint8_t *__restrict__ scales, float *__restrict__ ts, const float *__restrict__ partials,
-    int n_partials, uint64_t seed, uint32_t sign_mask) {
-  __shared__ __align__(16) uint16_t tile[128 * 128];  // [token][channel]
-  __shared__ __align__(16) uint8_t sbuf[128 * 8];     // [channel][block in tile]
-  __shared__ float red[8];
+__device__ __forceinline__ void colwise_tile(const uint16_t *tile, uint8_t *sbuf, int64_t c0,
+                                             int64_t t0, int64_t T, uint8_t *__restrict__ payload,
+                                             uint8_t *__restrict__ scales, float s_enc,
+                                             uint64_t seed, uint32_t sign_mask) {
   const int w = threadIdx.x >> 5, l = threadIdx.x & 31;
-  const int64_t c0 = (int64_t)blockIdx.x * 128;  // channel = row of Q
-  const int64_t t0 = (int64_t)blockIdx.y * 128;  // token = K of Q
-
-  // stage the tile: half-warp per token row, 16 bytes per lane
-  float s_enc_tile = 1.0f;
-  {
-    uint4 v[8];
-#pragma unroll
-    for (int s = 0; s < 8; ++s) {
-      const int64_t t = t0 + 16 * s + 2 * w + (l >> 4);
-      v[s] = ld_stream(x + t * ld + c0 + 8 * (l & 15));
-    }
-    float m = 0.0f;
-#pragma unroll
-    for (int s = 0; s < 8; ++s) {
-      const int tt = 16 * s + 2 * w + (l >> 4);
-      *reinterpret_cast<uint4 *>(&tile[tt * 128 + 8 * (l & 15)]) = v[s];
-      if constexpr (FMT == kNVC) m = fmaxf(m, absmax8(v[s]));
-    }
-    if constexpr (FMT == kNVC) {
-      // every thread receives the same tile maximum
-      s_enc_tile = nv_encode_scale(cta_max256(m, red));
-      if (threadIdx.x == 0) ts[blockIdx.x * gridDim.y + blockIdx.y] = nv_decode_scale(s_enc_tile);
-    }
-  }
-  float s_enc = s_enc_tile;
-  if constexpr (FMT == kNVG) {
-    s_enc = nv_encode_scale(reduce_partials(partials, n_partials, red));
-    if (threadIdx.x == 0 && blockIdx.x == 0 && blockIdx.y == 0) ts[0] = nv_decode_scale(s_enc);
-  }
-  __syncthreads();
-
   const int p = (w & 1) * 32 + l;  // channel pair within the tile: 2p, 2p+1
   const int j = w >> 1;            // 32-token block within the tile
   float v0[32], v1[32];
@@ -313,6 +310,63 @@ __global__ void __launch_bounds__(256) quant_colwise_kernel(
     const uint32_t word = *reinterpret_cast<const uint32_t *>(&sbuf[cl * 8 + 4 * h]);
     *reinterpret_cast<uint32_t *>(scales + sf_offset(c0 + cl, (t0 >> 4) + 4 * h, kbt)) = word;
   }
+}
+
+template <int FMT, int RND, bool HAD>
+__global__ void __launch_bounds__(256) quant_colwise_kernel(
+    const uint16_t *__restrict__ x, int64_t T, int64_t C, int64_t ld, uint8_t *__restrict__ payload,
+    uint8_t *__restrict__ scales, float *__restrict__ ts, const float *__restrict__ partials,
+    int n_partials, uint64_t seed, uint32_t sign_mask) {
+  __shared__ __align__(16) uint16_t tile[128 * 128];  // [token][channel]
+  __shared__ __align__(16) uint8_t sbuf[128 * 8];     // [channel][block in tile]
+  __shared__ float red[8];
+  const int w = threadIdx.x >> 5, l = threadIdx.x & 31;
+  const int64_t c0 = (int64_t)blockIdx.x * 128;  // channel = row of Q
+  const int64_t t0 = (int64_t)blockIdx.y * 128;  // token = K of Q
+  // stage the tile: half-warp per token row, 16 bytes per lane
+  uint4 v[8];
+  load_tile_rowwise(x, ld, t0, c0, v);
+#pragma unroll
+  for (int s = 0; s < 8; ++s)
+    *reinterpret_cast<uint4 *>(&tile[(16 * s + 2 * w + (l >> 4)) * 128 + 8 * (l & 15)]) = v[s];
+  // the CTA-local tile of Q = x^T is this tile transposed: same maximum;
+  // its ts entry is [c0 / 128][t0 / 128]
+  const float s_enc = tile_encode_scale<FMT>(v, ts, (int64_t)blockIdx.x * gridDim.y + blockIdx.y,
+                                             partials, n_partials, red);
+  __syncthreads();
+  colwise_tile<FMT, RND, HAD>(tile, sbuf, c0, t0, T, payload, scales, s_enc, seed, sign_mask);
+}
+
+// --------------------------------------------------------------------------
+// Dual-orientation producer: one read of x[T, C] emits the row-wise operand
+// (Q = x, any format) and the column-wise MXFP4 operand (Q = x^T, optionally
+// with the fixed-sign Hadamard), e.g. the forward operand and the saved
+// weight-gradient operand of an activation, or the data-gradient and
+// weight-gradient operands of dY.  Bytes equal those of the two single-
+// orientation kernels.
+// --------------------------------------------------------------------------
+template <int RFMT, int RRND, int CRND, bool HAD>
+__global__ void __launch_bounds__(256) quant_dual_kernel(
+    const uint16_t *__restrict__ x, int64_t T, int64_t C, int64_t ld, uint8_t *__restrict__ row_payload,
+    uint8_t *__restrict__ row_scales, float *__restrict__ row_ts, uint8_t *__restrict__ col_payload,
+    uint8_t *__restrict__ col_scales, const float *__restrict__ partials, int n_partials,
+    uint64_t row_seed, uint64_t col_seed, uint32_t sign_mask) {
+  __shared__ __align__(16) uint16_t tile[128 * 128];  // [token][channel]
+  __shared__ __align__(16) uint8_t sbuf[128 * 8];
+  __shared__ float red[8];
+  const int w = threadIdx.x >> 5, l = threadIdx.x & 31;
+  const int64_t c0 = (int64_t)blockIdx.x * 128, t0 = (int64_t)blockIdx.y * 128;
+  uint4 v[8];
+  load_tile_rowwise(x, ld, t0, c0, v);
+#pragma unroll
+  for (int s = 0; s < 8; ++s)
+    *reinterpret_cast<uint4 *>(&tile[(16 * s + 2 * w + (l >> 4)) * 128 + 8 * (l & 15)]) = v[s];
+  const float s_enc = tile_encode_scale<RFMT>(v, row_ts, (int64_t)blockIdx.y * gridDim.x + blockIdx.x,
+                                              partials, n_partials, red);
+  rowwise_tile<RFMT, RRND>(v, t0, c0, C, row_payload, row_scales, s_enc, row_seed);
+  __syncthreads();
+  colwise_tile<kMX, CRND, HAD>(tile, sbuf, c0, t0, T, col_payload, col_scales, 1.0f, col_seed,
+                               sign_mask);
 }
 
 // --------------------------------------------------------------------------
@@ -396,6 +450,35 @@ cudaError_t launch_quant_colwise(int fmt, int rnd, bool hadamard, uint32_t sign_
   FA4_COL(kMX, kSR, true) FA4_COL(kNVG, kRNE, false) FA4_COL(kNVG, kSR, false)
   FA4_COL(kNVC, kRNE, false) FA4_COL(kNVC, kSR, false)
 #undef FA4_COL
+  return cudaGetLastError();
+}
+
+template <int RF, int RR, int CR, bool H>
+static void launch_dual_t(dim3 g, cudaStream_t st, const uint16_t *x, int64_t T, int64_t C,
+                          int64_t ld, uint8_t *rp, uint8_t *rs, float *rts, uint8_t *cp, uint8_t *cs,
+                          const float *part, int np, uint64_t rseed, uint64_t cseed, uint32_t mask) {
+  quant_dual_kernel<RF, RR, CR, H><<<g, 256, 0, st>>>(x, T, C, ld, rp, rs, rts, cp, cs, part, np,
+                                                      rseed, cseed, mask);
+}
+
+cudaError_t launch_quant_dual(int row_fmt, int row_rnd, int col_rnd, bool hadamard,
+                              uint32_t sign_mask, const uint16_t *x, int64_t T, int64_t C,
+                              int64_t ld, uint8_t *row_payload, uint8_t *row_scales, float *row_ts,
+                              uint8_t *col_payload, uint8_t *col_scales, const float *partials,
+                              int n_partials, uint64_t row_seed, uint64_t col_seed,
+                              cudaStream_t st) {
+  dim3 g((unsigned)(C / 128), (unsigned)(T / 128));
+#define FA4_DUAL(F, RR, CR, H)                                                                  \
+  if (row_fmt == F && row_rnd == RR && col_rnd == CR && hadamard == H)                          \
+    launch_dual_t<F, RR, CR, H>(g, st, x, T, C, ld, row_payload, row_scales, row_ts, col_payload, \
+                                col_scales, partials, n_partials, row_seed, col_seed, sign_mask);
+#define FA4_DUAL_F(F)                                                                 \
+  FA4_DUAL(F, kRNE, kRNE, false) FA4_DUAL(F, kRNE, kRNE, true) FA4_DUAL(F, kRNE, kSR, false) \
+  FA4_DUAL(F, kRNE, kSR, true) FA4_DUAL(F, kSR, kRNE, false) FA4_DUAL(F, kSR, kRNE, true)    \
+  FA4_DUAL(F, kSR, kSR, false) FA4_DUAL(F, kSR, kSR, true)
+  FA4_DUAL_F(kMX) FA4_DUAL_F(kNVG) FA4_DUAL_F(kNVC)
+#undef FA4_DUAL_F
+#undef FA4_DUAL
   return cudaGetLastError();
 }
 

@@ -147,6 +147,24 @@ FA4_API fa4_status fa4_hadamard32_quantize(const void *x, int64_t rows, int64_t 
                                    fa4_qtensor out, void *workspace, size_t workspace_bytes,
                                    void *stream);
 
+/* Dual-orientation producer: one read of bf16 x[rows, cols] writes two
+ * quantized operands ("Format-Aware Fusion...", section "The Design
+ * Philosophy of Format-Aware Fusion": the producer fused with its consumers'
+ * layouts; what the backward pass keeps of an activation is then its
+ * column-wise FP4 operand for the weight gradient):
+ *   row_out = fa4_quantize(x, row_fmt, row_rnd, FA4_ROWWISE, row_seed)
+ *   col_out = col_hadamard ? fa4_hadamard32_quantize(x, sign_mask, col_rnd, col_seed)
+ *                          : fa4_quantize(x, FA4_MXFP4, col_rnd, FA4_COLWISE, col_seed)
+ * byte for byte.  For an activation X this is the forward operand and the
+ * saved wgrad operand; for dY the dgrad and wgrad operands.  The column-wise
+ * operand is always MXFP4.  Workspace: as fa4_quantize for row_fmt (the
+ * NVFP4-global amax pass reads x once more).  Errors: as fa4_quantize. */
+FA4_API fa4_status fa4_quantize_dual(const void *x, int64_t rows, int64_t cols, int64_t ld,
+                             fa4_format row_fmt, fa4_round row_rnd, uint64_t row_seed,
+                             fa4_qtensor row_out, int col_hadamard, uint32_t sign_mask,
+                             fa4_round col_rnd, uint64_t col_seed, fa4_qtensor col_out,
+                             void *workspace, size_t workspace_bytes, void *stream);
+
 /* Block-scaled FP4 GEMM on the tcgen05 tensor cores:
  *   D[m][n] = alpha * sum_k A[m][k] * B[n][k]       (D = alpha A B^T)
  * with A[M, K] and B[N, K] quantized operands in the same format (both
@@ -175,7 +193,7 @@ FA4_API fa4_status fa4_gemm_blockscaled(fa4_qtensor A, fa4_qtensor B, int64_t M,
  *                   column-wise with the fixed-sign Hadamard (sign_mask) and
  *                   `rnd`, then multiplied with alpha = 1/32.
  * fa4_linear_ws_bytes gives the workspace each needs (kind 0 fwd, 1 dgrad,
- * 2 wgrad).  Errors: as the calls they are made of. */
+ * 2 wgrad, 3 fwd_save, 4 bwd; below).  Errors: as the calls they are made of. */
 FA4_API fa4_status fa4_linear_ws_bytes(int kind, int64_t T, int64_t Cin, int64_t Cout, fa4_format fmt,
                                size_t *workspace_bytes);
 FA4_API fa4_status fa4_linear_fwd(const void *X, fa4_qtensor Wq, int64_t T, int64_t Cin, int64_t Cout,
@@ -188,6 +206,33 @@ FA4_API fa4_status fa4_linear_wgrad(const void *dY, const void *X, int64_t T, in
                             uint32_t sign_mask, fa4_round rnd, uint64_t seed, void *dW,
                             fa4_out_dtype out_dtype, void *workspace, size_t workspace_bytes,
                             void *stream);
+
+/* Training form of the linear layer, forward half: Y = X W^T as
+ * fa4_linear_fwd (X row-wise in `fmt`, RNE), and from the same read of X its
+ * column-wise MXFP4 operand with the fixed-sign Hadamard (RNE) into the
+ * caller's Xcol ([Cin, T]: payload Cin*T/2 bytes, scales Cin*T/32 bytes), the
+ * state the backward half needs instead of the bf16 X ("Format-Aware
+ * Fusion...", section "The Design Philosophy of Format-Aware Fusion": the
+ * state kept for the backward pass is the FP4 operand, not the bf16 X).  Y and Xcol equal fa4_linear_fwd and
+ * fa4_hadamard32_quantize(X, sign_mask, FA4_RNE) byte for byte.
+ * Workspace: fa4_linear_ws_bytes(kind 3).  Errors: as fa4_linear_fwd. */
+FA4_API fa4_status fa4_linear_fwd_save(const void *X, fa4_qtensor Wq, int64_t T, int64_t Cin,
+                               int64_t Cout, fa4_format fmt, uint32_t sign_mask, void *Y,
+                               fa4_qtensor Xcol, void *workspace, size_t workspace_bytes,
+                               void *stream);
+
+/* Training form, backward half: one read of dY gives its row-wise operand
+ * (`fmt`, rounding rnd with seed) and its column-wise MXFP4 Hadamard operand
+ * (RNE); then dX = dY W (bf16, with Wq_col the column-wise W as in
+ * fa4_linear_dgrad) and dW = dY^T X = (1/32) * GEMM(dY col, Xcol) (fp32 or
+ * bf16 by dw_dtype) with Xcol from fa4_linear_fwd_save and the same
+ * sign_mask.  dX equals fa4_linear_dgrad(dY, Wq_col, fmt, rnd, seed) and dW
+ * equals fa4_linear_wgrad(dY, X, sign_mask, FA4_RNE, ...) byte for byte.
+ * Workspace: fa4_linear_ws_bytes(kind 4).  Errors: as fa4_linear_dgrad. */
+FA4_API fa4_status fa4_linear_bwd(const void *dY, fa4_qtensor Wq_col, fa4_qtensor Xcol, int64_t T,
+                          int64_t Cin, int64_t Cout, fa4_format fmt, fa4_round rnd, uint64_t seed,
+                          uint32_t sign_mask, void *dX, void *dW, fa4_out_dtype dw_dtype,
+                          void *workspace, size_t workspace_bytes, void *stream);
 
 /* NVFP4-global quantization that allocates nothing and takes no workspace.
  * (No counterpart on the pages: it exists for callers, not for the method.)

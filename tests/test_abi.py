@@ -167,3 +167,46 @@ def test_noalloc_quantize_rejects_bad_arguments():
     assert L.fa4_quantize_nvfp4_global_noalloc(DEV, 256, 256, 256, 3, 0, 0, q, None) == 1
     assert L.fa4_quantize_nvfp4_global_noalloc(DEV, 256, 256, 256, 0, 0, 0,
                                                fa._QT(0x10000, 0x20000, 0), None) == 1
+
+
+def test_dual_quantize_rejects_bad_arguments():
+    L = fa.lib()
+    q = _qt()
+    args = lambda **k: dict(dict(x=DEV, rows=256, cols=256, ld=256, rf=fa.MXFP4, rr=0, cr=0,
+                                 row=q, col=q, ws=DEV + 4096, wsb=1 << 20), **k)
+
+    def call(a):
+        return L.fa4_quantize_dual(a["x"], a["rows"], a["cols"], a["ld"], a["rf"], a["rr"], 0,
+                                   a["row"], 1, 0x1234, a["cr"], 0, a["col"], a["ws"], a["wsb"],
+                                   None)
+    assert call(args(x=None)) == 1
+    assert call(args(rows=200)) == 2
+    assert call(args(ld=136)) == 2
+    assert call(args(x=DEV + 2)) == 3
+    assert call(args(rf=5)) == 1
+    assert call(args(rr=2)) == 1
+    assert call(args(cr=7)) == 1
+    assert call(args(col=fa._QT(0, 0x20000, 0))) == 1
+    assert call(args(row=fa._QT(0x10000, 0x20008, 0))) == 3
+    assert call(args(rf=fa.NVFP4_GLOBAL, row=fa._QT(0x10000, 0x20000, 0))) == 1
+    assert call(args(rf=fa.NVFP4_GLOBAL, wsb=256)) == 5
+    assert call(args(ws=None)) == 5
+
+
+def test_training_linear_rejects_bad_arguments():
+    L = fa.lib()
+    q = _qt()
+    n = ctypes.c_size_t()
+    assert L.fa4_linear_ws_bytes(3, 256, 256, 384, fa.MXFP4, ctypes.byref(n)) == 0
+    assert n.value >= 256 * 256 // 2
+    assert L.fa4_linear_ws_bytes(4, 256, 256, 384, fa.MXFP4, ctypes.byref(n)) == 0
+    assert n.value >= 2 * 256 * 384 // 2
+    assert L.fa4_linear_fwd_save(None, q, 256, 256, 384, 0, 1, DEV, q, DEV, 1 << 24, None) == 1
+    assert L.fa4_linear_fwd_save(DEV, q, 256, 256, 384, 0, 1, DEV, fa._QT(0, 0, 0), DEV, 1 << 24,
+                                 None) == 1
+    assert L.fa4_linear_fwd_save(DEV, q, 256, 256, 384, 0, 1, DEV, q, DEV, 64, None) == 5
+    assert L.fa4_linear_bwd(DEV, q, q, 256, 256, 384, 0, 3, 0, 1, DEV, DEV, 1, DEV, 1 << 24,
+                            None) == 1
+    assert L.fa4_linear_bwd(DEV, q, q, 250, 256, 384, 0, 1, 0, 1, DEV, DEV, 1, DEV, 1 << 24,
+                            None) == 2
+    assert L.fa4_linear_bwd(DEV, q, q, 256, 256, 384, 0, 1, 0, 1, DEV, DEV, 1, DEV, 64, None) == 5
