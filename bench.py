@@ -277,6 +277,39 @@ def quantize_sweep(fa, device, reps: int = 20) -> list[dict]:
     return out
 
 
+def gemm_sweep(fa, device, reps: int = 10) -> list[dict]:
+    """Block-scaled GEMM of each scale domain (MXFP4, NVFP4-global,
+    NVFP4-CTA-local) on the 8B forward shapes (M = 8192 tokens), bf16 out."""
+    fp4_peak = 4.0 * _peaks()[1]
+    out = []
+    for name, (cin, cout) in LAYERS.items():
+        a = workloads.act(T, cin, seed=5, device=device)
+        b = workloads.weight(cout, cin, seed=6, device=device)
+        d = torch.empty(T, cout, dtype=torch.bfloat16, device=device)
+        ws = fa.workspace(1 << 16, device)
+        for fmt, key in ((fa.MXFP4, "mx"), (fa.NVFP4_GLOBAL, "nvg"), (fa.NVFP4_CTA, "nvc")):
+            A, B = fa.quantize(a, fmt, ws=ws), fa.quantize(b, fmt, ws=ws)
+            for _ in range(3):
+                fa.gemm(A, B, 1.0, out=d, ws=ws)
+            torch.cuda.synchronize()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            for _ in range(reps):
+                fa.gemm(A, B, 1.0, out=d, ws=ws)
+            e1.record()
+            torch.cuda.synchronize()
+            us = e0.elapsed_time(e1) * 1000.0 / reps
+            tf = 2.0 * T * cin * cout / (us * 1e-6) / 1e12
+            out.append({"layer": name, "M": T, "N": cout, "K": cin, "fmt": key, "us": round(us, 1),
+                        "TFLOPS": round(tf, 1), "frac": round(tf / fp4_peak, 3)})
+            del A, B
+        del a, b, d
+    if fa.check_device_status(ws) != 0:
+        raise RuntimeError("device status set during the GEMM sweep")
+    torch.cuda.empty_cache()
+    return out
+
+
 def e2e_run(fa, blk: Block, steps: int, device) -> dict:
     """Same step through the public training-form linear calls
     (linear_fwd_save, linear_bwd) with host (pinned) inputs
@@ -478,6 +511,7 @@ def fa4_arm(args, rank, world, device) -> dict | None:
     result = None
     if rank == 0:
         sweep = quantize_sweep(fa, device) if not args.quick else []
+        gsweep = gemm_sweep(fa, device) if not args.quick else []
         e2e = e2e_run(fa, blk, max(2, min(args.steps, 5)), device)
         cpu = cpu_baseline() if (world == 1 and not args.no_cpu_baseline) else None
         tok_s = whole_job_tokens_per_s(world, ms_step)
@@ -501,7 +535,8 @@ def fa4_arm(args, rank, world, device) -> dict | None:
                         "fused_quantize_GBps": round(q_gbs, 1),
                         "breakdown": breakdown,
                         "weight_quantize_s": round(t_wq, 4),
-                        "quantize_sweep": sweep},
+                        "quantize_sweep": sweep,
+                        "gemm_sweep": gsweep},
             "roofline": {"bound": "tensor", "achieved": round(dom_tflops, 1),
                          "peak": round(fp4_peak, 1), "unit": "TFLOP/s",
                          "frac": round(dom_tflops / fp4_peak, 4), "traffic": dominant_traffic(),

@@ -63,26 +63,24 @@ __device__ __forceinline__ uint32_t e2m1x8_rne(const float *v) {
 // round up iff u < t, t = (|y| - lo) / g * 65536; |y| >= 6 gives 6; the sign
 // of y is kept.  Grid magnitudes 0, .5, 1, 1.5, 2, 3, 4, 6.
 // Evaluated on the binary32 bits A of |y| (integer compares order
-// non-negative floats):
-//  * 1 <= |y| < 6: lo is |y| with all but the top mantissa bit cleared and g
-//    is half its binade, so t = (A & 0x3FFFFF) / 64 exactly and the lower
-//    code is (A >> 22) - 252 (exponent and top mantissa bit);
-//    u < t  <=>  (u << 6) < (A & 0x3FFFFF).
-//  * 0.5 <= |y| < 1: lo = g = 0.5, t = (A & 0x7FFFFF) / 128, lower code 1.
+// non-negative floats), with |y| >= 6 first replaced by 6:
+//  * 1 <= |y| <= 6: the lower code is bits 22..30 of A minus 252 (exponent
+//    and top mantissa bit) and t = (A & 0x3FFFFF) / 64, so u < t iff adding
+//    0x3FFFFF - (u << 6) to A carries into bit 22: the code is
+//    ((A + 0x3FFFFF - (u << 6)) >> 22) - 252 (6 itself has a zero fraction
+//    and stays code 7).
+//  * 0.5 <= |y| < 1: lo = g = 0.5, t = (A & 0x7FFFFF) / 128; likewise the
+//    code is ((A + 0x7FFFFF - (u << 7)) >> 23) - 125, i.e. 1 or 2.
 //  * |y| < 0.5: lo = 0, t = |y| * 131072 (exact), compared as floats.
 __device__ __forceinline__ uint32_t e2m1_sr(float y, uint32_t u) {
   const uint32_t bits = __float_as_uint(y);
-  const uint32_t s = (bits >> 28) & 8u;
-  const uint32_t A = bits & 0x7FFFFFFFu;
-  const uint32_t c_hi = (A >> 22) - 252u + (((u << 6) < (A & 0x3FFFFFu)) ? 1u : 0u);
-  const uint32_t c_mid = 1u + (((u << 7) < (A & 0x7FFFFFu)) ? 1u : 0u);
+  const uint32_t A = min(bits & 0x7FFFFFFFu, 0x40C00000u);
+  const uint32_t c_hi = ((A + 0x3FFFFFu - (u << 6)) >> 22) - 252u;
+  const uint32_t c_mid = ((A + 0x7FFFFFu - (u << 7)) >> 23) - 125u;
   const float uf = __fsub_rn(__uint_as_float(u | 0x4B000000u), 8388608.0f);  // (float)u, exact
   const uint32_t c_lo = (uf < __fmul_rn(__uint_as_float(A), 131072.0f)) ? 1u : 0u;
-  const uint32_t c = (A >= 0x40C00000u) ? 7u
-                     : (A >= 0x3F800000u) ? c_hi
-                     : (A >= 0x3F000000u) ? c_mid
-                                          : c_lo;
-  return s | c;
+  const uint32_t c = (A >= 0x3F800000u) ? c_hi : (A >= 0x3F000000u) ? c_mid : c_lo;
+  return ((bits >> 28) & 8u) | c;
 }
 
 // ---------------------------------------------------------------- E4M3 ---
