@@ -55,8 +55,8 @@ BYTES_PER_ELEM = {"mx": 2.0 + 0.5 + 1.0 / 32, "nvg": 2.0 + 2.0 + 0.5 + 1.0 / 16,
 # They hold only for the kernel source they were taken on, identified by its
 # SHA-256; after any change the traffic is reported as null until re-taken.
 GEMM_SOURCE = os.path.join(ROOT, "fp4_quantization_block_b200", "csrc", "gemm_blockscaled.cu")
-DOMINANT_TRAFFIC = {"source_sha256": "2ea8bd3043da5905be476b70682279d78166be75377ec891660058f258316295",
-                    "bytes_per_launch": 246957472}
+DOMINANT_TRAFFIC = {"source_sha256": "3c69a3bac97a3ae7cbac2625ed7de8cd19d56536bc26d2f20b7ce7cbb8523411",
+                    "bytes_per_launch": 243078592}
 
 
 def dominant_traffic():
@@ -310,11 +310,45 @@ def gemm_sweep(fa, device, reps: int = 10) -> list[dict]:
     return out
 
 
+def epilogue_quant_run(fa, device, reps: int = 10) -> dict:
+    """The gate+up forward GEMM followed by the MXFP4 quantization of its bf16
+    output: separate calls against the quantizer fused into the GEMM epilogue
+    (with and without storing the bf16 output)."""
+    cin, cout = LAYERS["gate_up"]
+    x = workloads.act(T, cin, seed=7, device=device)
+    w = workloads.weight(cout, cin, seed=8, device=device)
+    ws = fa.workspace(1 << 16, device)
+    A, B = fa.quantize(x, fa.NVFP4_GLOBAL, ws=ws), fa.quantize(w, fa.NVFP4_GLOBAL, ws=ws)
+    d = torch.empty(T, cout, dtype=torch.bfloat16, device=device)
+    q = fa.empty_qtensor(T, cout, fa.MXFP4, fa.ROWWISE, device)
+    runs = {"separate": lambda: (fa.gemm(A, B, 1.0, out=d, ws=ws),
+                                 fa.quantize(d, fa.MXFP4, out=q, ws=ws)),
+            "fused": lambda: fa.gemm_mxout(A, B, 1.0, out=d, qout=q, ws=ws),
+            "fused_no_bf16": lambda: fa.gemm_mxout(A, B, 1.0, store_d=False, qout=q, ws=ws)}
+    res = {"shape": [T, cout, cin]}
+    for name, fn in runs.items():
+        for _ in range(3):
+            fn()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(reps):
+            fn()
+        e1.record()
+        torch.cuda.synchronize()
+        res[name + "_us"] = round(e0.elapsed_time(e1) * 1000.0 / reps, 1)
+    if fa.check_device_status(ws) != 0:
+        raise RuntimeError("device status set during the epilogue-quantization run")
+    return res
+
+
 def e2e_run(fa, blk: Block, steps: int, device) -> dict:
     """Same step through the public training-form linear calls
-    (linear_fwd_save, linear_bwd) with host (pinned) inputs
-    and outputs: the H2D copy of X and dY and the D2H copy of Y, dX and dW of
-    every layer are inside the timed region."""
+    (linear_fwd_save, linear_bwd) with host (pinned) inputs and outputs: the
+    H2D copy of X and dY and the D2H copy of Y, dX and dW of every layer are
+    inside the timed region.  Copies run on their own streams, layer by
+    layer, so the H2D of one layer, the kernels of another and the D2H of a
+    third overlap (PCIe is full duplex); events order each buffer's reuse."""
     host = {}
     h2d = d2h = 0
     for name, L in blk.layers.items():
@@ -327,27 +361,44 @@ def e2e_run(fa, blk: Block, steps: int, device) -> dict:
     wsz = max(fa.linear_ws_bytes(k, T, cin, cout, fa.NVFP4_GLOBAL if k == 3 else fa.MXFP4)
               for k in (3, 4) for cin, cout in LAYERS.values())
     ws = fa.workspace(wsz, device)
+    comp = torch.cuda.current_stream(device)
+    s_in, s_out = torch.cuda.Stream(device), torch.cuda.Stream(device)
+    ev = {name: {"loaded": torch.cuda.Event(), "computed": torch.cuda.Event(),
+                 "stored": torch.cuda.Event(), "used": False} for name in blk.layers}
 
     def one(step):
         for name, L in blk.layers.items():
-            H = host[name]
-            L["x"].copy_(H["x"], non_blocking=True)
-            L["dy"].copy_(H["dy"], non_blocking=True)
+            H, E = host[name], ev[name]
+            with torch.cuda.stream(s_in):
+                if E["used"]:
+                    s_in.wait_event(E["computed"])  # the last step's kernels have read x, dy
+                L["x"].copy_(H["x"], non_blocking=True)
+                L["dy"].copy_(H["dy"], non_blocking=True)
+                E["loaded"].record(s_in)
+            comp.wait_event(E["loaded"])
+            if E["used"]:
+                comp.wait_event(E["stored"])  # the last step's outputs have left the device
             fa.linear_fwd_save(L["x"], L["wq"], fa.NVFP4_GLOBAL, SIGN_MASK, out=L["y"],
                                xcol=L["xc"], ws=ws)
             fa.linear_bwd(L["dy"], L["wc"], L["xc"], fa.MXFP4, fa.SR, seed=step,
                           sign_mask=SIGN_MASK, dx=L["dx"], dw=L["dw"], ws=ws)
-            H["y"].copy_(L["y"], non_blocking=True)
-            H["dx"].copy_(L["dx"], non_blocking=True)
-            H["dw"].copy_(L["dw"], non_blocking=True)
+            E["computed"].record(comp)
+            with torch.cuda.stream(s_out):
+                s_out.wait_event(E["computed"])
+                H["y"].copy_(L["y"], non_blocking=True)
+                H["dx"].copy_(L["dx"], non_blocking=True)
+                H["dw"].copy_(L["dw"], non_blocking=True)
+                E["stored"].record(s_out)
+            E["used"] = True
 
     one(0)
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record()
+    e0.record(comp)
     for s in range(steps):
         one(s + 1)
-    e1.record()
+    comp.wait_stream(s_out)
+    e1.record(comp)
     torch.cuda.synchronize()
     if fa.check_device_status(ws) != 0:
         raise RuntimeError("device status set during the e2e run")
@@ -512,6 +563,7 @@ def fa4_arm(args, rank, world, device) -> dict | None:
     if rank == 0:
         sweep = quantize_sweep(fa, device) if not args.quick else []
         gsweep = gemm_sweep(fa, device) if not args.quick else []
+        epiq = epilogue_quant_run(fa, device) if not args.quick else {}
         e2e = e2e_run(fa, blk, max(2, min(args.steps, 5)), device)
         cpu = cpu_baseline() if (world == 1 and not args.no_cpu_baseline) else None
         tok_s = whole_job_tokens_per_s(world, ms_step)
@@ -536,7 +588,8 @@ def fa4_arm(args, rank, world, device) -> dict | None:
                         "breakdown": breakdown,
                         "weight_quantize_s": round(t_wq, 4),
                         "quantize_sweep": sweep,
-                        "gemm_sweep": gsweep},
+                        "gemm_sweep": gsweep,
+                        "gemm_epilogue_mxfp4": epiq},
             "roofline": {"bound": "tensor", "achieved": round(dom_tflops, 1),
                          "peak": round(fp4_peak, 1), "unit": "TFLOP/s",
                          "frac": round(dom_tflops / fp4_peak, 4), "traffic": dominant_traffic(),

@@ -24,7 +24,7 @@ import torch
 __all__ = [
     "MXFP4", "NVFP4_GLOBAL", "NVFP4_CTA", "RNE", "SR", "ROWWISE", "COLWISE",
     "QTensor", "FA4Error", "lib", "library_path", "quant_sizes", "empty_qtensor", "quantize",
-    "hadamard32_quantize", "quantize_dual", "gemm", "linear_ws_bytes", "linear_fwd", "linear_dgrad",
+    "hadamard32_quantize", "quantize_dual", "gemm", "gemm_mxout", "linear_ws_bytes", "linear_fwd", "linear_dgrad",
     "linear_wgrad", "linear_fwd_save", "linear_bwd", "workspace", "check_device_status",
 ]
 
@@ -79,6 +79,7 @@ def _declare(L: ctypes.CDLL) -> ctypes.CDLL:
         "fa4_hadamard32_quantize": [P, i64, i64, i64, u32, ci, u64, _QT, P, sz, P],
         "fa4_quantize_dual": [P, i64, i64, i64, ci, ci, u64, _QT, ci, u32, ci, u64, _QT, P, sz, P],
         "fa4_gemm_blockscaled": [_QT, _QT, i64, i64, i64, ci, f32, P, i64, ci, P, sz, P],
+        "fa4_gemm_blockscaled_mxout": [_QT, _QT, i64, i64, i64, ci, f32, P, i64, _QT, P, sz, P],
         "fa4_linear_ws_bytes": [ci, i64, i64, i64, ci, PSZ],
         "fa4_linear_fwd": [P, _QT, i64, i64, i64, ci, P, P, sz, P],
         "fa4_linear_dgrad": [P, _QT, i64, i64, i64, ci, ci, u64, P, P, sz, P],
@@ -362,3 +363,23 @@ def linear_bwd(dY: torch.Tensor, Wq_col: QTensor, xcol: QTensor, fmt: int, rnd: 
                                 sign_mask & 0xFFFFFFFF, _ptr(dX), _ptr(dW), od, _ptr(ws),
                                 ws.numel(), _stream(dY.device)), "fa4_linear_bwd")
     return dX, dW
+
+
+def gemm_mxout(A: QTensor, B: QTensor, alpha: float = 1.0, store_d: bool = True,
+               out: torch.Tensor | None = None, qout: QTensor | None = None,
+               ws: torch.Tensor | None = None) -> tuple[torch.Tensor | None, QTensor]:
+    """D = alpha * A B^T (bf16, unless store_d is False) and D's row-wise
+    MXFP4 operand, quantized in the GEMM's epilogue."""
+    if A.K != B.K or A.fmt != B.fmt:
+        raise ValueError("A and B must share K and format")
+    dev = A.payload.device
+    if store_d and out is None:
+        out = torch.empty((A.R, B.R), dtype=torch.bfloat16, device=dev)
+    qout = qout or empty_qtensor(A.R, B.R, MXFP4, ROWWISE, dev)
+    ws = _ws(ws, WS_HEADER_BYTES, dev)
+    d_ptr = _ptr(out) if store_d else None
+    ldd = out.stride(0) if store_d else B.R
+    _check(lib().fa4_gemm_blockscaled_mxout(A.c(), B.c(), A.R, B.R, A.K, A.fmt, float(alpha), d_ptr,
+                                            ldd, qout.c(), _ptr(ws), ws.numel(), _stream(dev)),
+           "fa4_gemm_blockscaled_mxout")
+    return (out if store_d else None), qout

@@ -112,7 +112,8 @@ fa4_status do_quantize_dual(const void *x, int64_t rows, int64_t cols, int64_t l
 
 fa4_status do_gemm(const fa4_qtensor &A, const fa4_qtensor &B, int64_t M, int64_t N, int64_t K,
                    int fmt, float alpha, void *D, int64_t ldd, int out_dtype, uint8_t *ws,
-                   cudaStream_t st, int skip, uint64_t timeout_ns) {
+                   cudaStream_t st, int skip, uint64_t timeout_ns,
+                   const fa4_qtensor *dq = nullptr) {
   fa4::GemmArgs a;
   a.a_payload = static_cast<const uint8_t *>(A.payload);
   a.a_scales = static_cast<const uint8_t *>(A.scales);
@@ -131,6 +132,10 @@ fa4_status do_gemm(const fa4_qtensor &A, const fa4_qtensor &B, int64_t M, int64_
   a.status = reinterpret_cast<uint32_t *>(ws);
   a.debug_skip_stage = skip;
   a.timeout_ns = timeout_ns;
+  if (dq) {
+    a.q_payload = static_cast<uint8_t *>(dq->payload);
+    a.q_scales = static_cast<uint8_t *>(dq->scales);
+  }
   return cuda_status(fa4::launch_gemm_blockscaled(a, st));
 }
 
@@ -374,6 +379,24 @@ fa4_status fa4_linear_bwd(const void *dY, fa4_qtensor Wq_col, fa4_qtensor Xcol, 
     return s;
   return do_gemm(gc, Xcol, Cout, Cin, T, FA4_MXFP4, 1.0f / 32.0f, dW, Cin, dw_dtype, ws, S(stream),
                  -1, kDefaultTimeoutNs);
+}
+
+fa4_status fa4_gemm_blockscaled_mxout(fa4_qtensor A, fa4_qtensor B, int64_t M, int64_t N,
+                                      int64_t K, fa4_format fmt, float alpha, void *D, int64_t ldd,
+                                      fa4_qtensor Dq, void *workspace, size_t workspace_bytes,
+                                      void *stream) {
+  if (!fmt_ok(fmt)) return FA4_ERR_INVALID_ARG;
+  if (fmt == FA4_NVFP4_CTA) return FA4_ERR_UNSUPPORTED;
+  fa4_status s = check_qt(Dq, FA4_MXFP4);
+  if (s != FA4_OK) return s;
+  // D is optional: checked as a bf16 output when given
+  static const uint8_t dummy[16] __attribute__((aligned(16))) = {};
+  const void *dcheck = D ? D : static_cast<const void *>(dummy);
+  if ((s = check_gemm(A, B, M, N, K, fmt, dcheck, D ? ldd : N, FA4_OUT_BF16, workspace,
+                      workspace_bytes)) != FA4_OK)
+    return s;
+  return do_gemm(A, B, M, N, K, fmt, alpha, D, D ? ldd : N, FA4_OUT_BF16,
+                 static_cast<uint8_t *>(workspace), S(stream), -1, kDefaultTimeoutNs, &Dq);
 }
 
 fa4_status fa4_workspace_init(void *workspace, size_t workspace_bytes, void *stream) {

@@ -48,6 +48,10 @@ struct GemmArgs {
   uint32_t *status;
   int debug_skip_stage;     // < 0 normally; >= 0: the producer never loads that k-tile (test hook)
   uint64_t timeout_ns;      // bounded-wait limit
+  // optional: the bf16 output's row-wise MXFP4 operand written by the
+  // epilogue (payload [M, N/2], scales in the atom layout); null: none.
+  // D may then be null (the bf16 output is not stored).
+  uint8_t *q_payload = nullptr, *q_scales = nullptr;
 };
 cudaError_t launch_gemm_blockscaled(const GemmArgs &a, cudaStream_t st);
 

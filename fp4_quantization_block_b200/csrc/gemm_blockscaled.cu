@@ -35,6 +35,7 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
+#include <string.h>
 
 #include <cuda_bf16.h>
 
@@ -219,6 +220,10 @@ struct Params {
   int debug_skip_stage;
   uint64_t timeout_ns;
   int n_fastest;  // tile order: 1 = walk N first (B stays in L2), 0 = walk M first
+  // epilogue quantization of the bf16 output to its row-wise MXFP4 operand
+  // (payload [M, N/2], scales in the 128x4 atom layout); null: none
+  uint8_t *q_payload, *q_scales;
+  int store_d;  // 0: D is not written (only the quantized operand)
 };
 
 // Output tile coordinates of linear tile index t.  Concurrently running CTAs
@@ -791,7 +796,7 @@ __device__ __forceinline__ void tmem_st4(uint32_t taddr, const uint4 &v) {
                : "memory");
 }
 
-template <int KIND, int BN, bool PAIR>
+template <int KIND, int BN, bool PAIR, bool QOUT>
 __global__ void __launch_bounds__(NUM_THREADS_ST, 1)
     gemm_st_kernel(const __grid_constant__ CUtensorMap map_a,
                    const __grid_constant__ CUtensorMap map_b,
@@ -1112,28 +1117,61 @@ __global__ void __launch_bounds__(NUM_THREADS_ST, 1)
           }
         }
       } else {
+        const int64_t row = (int64_t)y0 + lane;
+        uint32_t sword = 0;  // this row's MXFP4 scale bytes, one per 32-column chunk
 #pragma unroll
         for (int ch = 0; ch < COLS / 32; ++ch) {
-          if (lane == 0) bulk_wait_read_all();
-          __syncwarp();
+          uint32_t w[16];  // the chunk's 32 bf16 values of D, packed in pairs
 #pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            uint32_t w[4];
+          for (int u = 0; u < 16; ++u) {
+            const int i = 32 * ch + 2 * u;
+            __nv_bfloat162 b2 = __floats2bfloat162_rn(__uint_as_float(r[i]) * alpha_g,
+                                                      __uint_as_float(r[i + 1]) * alpha_g);
+            w[u] = *reinterpret_cast<uint32_t *>(&b2);
+          }
+          if constexpr (QOUT) {
+            // the 32 bf16 values are one MXFP4 block of D's row-wise operand:
+            // the same steps as the row-wise quantizer (RNE)
+            float f[32];
+            float amax = 0.0f;
 #pragma unroll
-            for (int u = 0; u < 4; ++u) {
-              const int i = 32 * ch + 8 * j + 2 * u;
-              __nv_bfloat162 b2 = __floats2bfloat162_rn(__uint_as_float(r[i]) * alpha_g,
-                                                        __uint_as_float(r[i + 1]) * alpha_g);
-              w[u] = *reinterpret_cast<uint32_t *>(&b2);
+            for (int u = 0; u < 16; ++u) {
+              f[2 * u] = bf16lo(w[u]);
+              f[2 * u + 1] = bf16hi(w[u]);
+              amax = fmaxf(amax, fmaxf(fabsf(f[2 * u]), fabsf(f[2 * u + 1])));
             }
-            sts128(row_base + 16 * (j ^ sw), w[0], w[1], w[2], w[3]);
+            const uint32_t sbyte = mx_scale_byte(amax);
+            const float mult = mx_multiplier(sbyte);
+#pragma unroll
+            for (int e = 0; e < 32; ++e) f[e] = __fmul_rn(f[e], mult);
+            const uint4 codes = make_uint4(e2m1x8_rne(&f[0]), e2m1x8_rne(&f[8]),
+                                           e2m1x8_rne(&f[16]), e2m1x8_rne(&f[24]));
+            *reinterpret_cast<uint4 *>(p.q_payload + row * (p.N >> 1) + ((x0 + 32 * ch) >> 1)) =
+                codes;
+            sword |= sbyte << (8 * ch);
           }
-          fence_proxy_async_smem();
-          __syncwarp();
-          if (lane == 0) {
-            tma_store_2d(&map_d, ebuf, x0 + 32 * ch, y0);
-            bulk_commit();
+          if (p.store_d) {
+            if (lane == 0) bulk_wait_read_all();
+            __syncwarp();
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+              sts128(row_base + 16 * (j ^ sw), w[4 * j], w[4 * j + 1], w[4 * j + 2], w[4 * j + 3]);
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) {
+              tma_store_2d(&map_d, ebuf, x0 + 32 * ch, y0);
+              bulk_commit();
+            }
           }
+        }
+        if constexpr (QOUT) {
+          // blocks x0/32 .. of this row: a whole scale word (128 columns) or
+          // its half (64 columns, the other half is the quadrant's other warp)
+          uint8_t *sdst = p.q_scales + sf_offset(row, x0 >> 5, p.N >> 5);
+          if constexpr (COLS == 128)
+            *reinterpret_cast<uint32_t *>(sdst) = sword;
+          else
+            *reinterpret_cast<uint16_t *>(sdst) = (uint16_t)sword;
         }
       }
     }
@@ -1235,6 +1273,9 @@ static gemm::Params make_params(const GemmArgs &a) {
   p.timeout_ns = a.timeout_ns;
   // keep the smaller operand resident in L2 and stream the larger one once
   p.n_fastest = (a.N <= a.M) ? 1 : 0;
+  p.q_payload = a.q_payload;
+  p.q_scales = a.q_scales;
+  p.store_d = a.D != nullptr;
   return p;
 }
 
@@ -1257,16 +1298,17 @@ static cudaError_t launch_t(const GemmArgs &a, cudaStream_t st) {
   return cudaGetLastError();
 }
 
-template <int KIND, int BN, bool PAIR>
+template <int KIND, int BN, bool PAIR, bool QOUT>
 static cudaError_t launch_st(const GemmArgs &a, cudaStream_t st) {
   constexpr int smem = gemm_st::total_smem_st<KIND, BN, PAIR>();
   CUtensorMap ma, mb;
   if (!make_payload_map(&ma, a.a_payload, a.M, a.K, gemm::BM)) return cudaErrorInvalidValue;
   if (!make_payload_map(&mb, a.b_payload, a.N, a.K, PAIR ? 128 : BN)) return cudaErrorInvalidValue;
   CUtensorMap md;
-  if (!make_out_map(&md, a)) return cudaErrorInvalidValue;
+  memset(&md, 0, sizeof(md));
+  if (a.D && !make_out_map(&md, a)) return cudaErrorInvalidValue;
   gemm::Params p = make_params(a);
-  auto kern = gemm_st::gemm_st_kernel<KIND, BN, PAIR>;
+  auto kern = gemm_st::gemm_st_kernel<KIND, BN, PAIR, QOUT>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
   int dev = 0, sms = 148;
@@ -1301,25 +1343,28 @@ static cudaError_t launch_st(const GemmArgs &a, cudaStream_t st) {
   return cudaGetLastError();
 }
 
-cudaError_t launch_gemm_blockscaled(const GemmArgs &a, cudaStream_t st) {
+template <bool QOUT>
+static cudaError_t launch_st_any(const GemmArgs &a, cudaStream_t st) {
   const bool wide = (a.N % 256) == 0;
   const bool pair = wide && (a.M % 256) == 0;
   if (a.fmt == kMX)
-    return pair ? launch_st<kMX, 256, true>(a, st)
-                : (wide ? launch_st<kMX, 256, false>(a, st) : launch_st<kMX, 128, false>(a, st));
-  if (a.fmt == kNVG)
-    return pair ? launch_st<kNVG, 256, true>(a, st)
-                : (wide ? launch_st<kNVG, 256, false>(a, st) : launch_st<kNVG, 128, false>(a, st));
-  switch (a.fmt) {
-    case kMX:
-      return wide ? launch_t<kMX, 256>(a, st) : launch_t<kMX, 128>(a, st);
-    case kNVG:
-      return wide ? launch_t<kNVG, 256>(a, st) : launch_t<kNVG, 128>(a, st);
-    case kNVC:
-      return launch_t<kNVC, 128>(a, st);
-    default:
-      return cudaErrorInvalidValue;
+    return pair ? launch_st<kMX, 256, true, QOUT>(a, st)
+                : (wide ? launch_st<kMX, 256, false, QOUT>(a, st) : launch_st<kMX, 128, false, QOUT>(a, st));
+  return pair ? launch_st<kNVG, 256, true, QOUT>(a, st)
+              : (wide ? launch_st<kNVG, 256, false, QOUT>(a, st) : launch_st<kNVG, 128, false, QOUT>(a, st));
+}
+
+cudaError_t launch_gemm_blockscaled(const GemmArgs &a, cudaStream_t st) {
+  if (a.fmt == kMX || a.fmt == kNVG) {
+    if (a.q_payload) {
+      if (a.out_fp32) return cudaErrorInvalidValue;  // the quantized output comes from bf16 D
+      return launch_st_any<true>(a, st);
+    }
+    if (!a.D) return cudaErrorInvalidValue;
+    return launch_st_any<false>(a, st);
   }
+  if (a.fmt == kNVC && !a.q_payload && a.D) return launch_t<kNVC, 128>(a, st);
+  return cudaErrorInvalidValue;
 }
 
 }  // namespace fa4

@@ -178,6 +178,20 @@ FA4_API fa4_status fa4_gemm_blockscaled(fa4_qtensor A, fa4_qtensor B, int64_t M,
                                 fa4_out_dtype out_dtype, void *workspace, size_t workspace_bytes,
                                 void *stream);
 
+/* The same GEMM with the quantizer fused into its epilogue ("Format-Aware
+ * Fusion...", section "The Design Philosophy of Format-Aware Fusion": the
+ * producer of the next operand is the GEMM that computes it): the bf16
+ * output D = alpha * A B^T is written (when D is not NULL) and its row-wise
+ * MXFP4 operand (RNE) goes to Dq ([M, N/2] payload, M*N/32 scale bytes in
+ * the atom layout), byte-identical to fa4_quantize(D, FA4_MXFP4, FA4_RNE,
+ * FA4_ROWWISE) of that bf16 D, without reading D back.  fmt MXFP4 or
+ * NVFP4_GLOBAL (FA4_ERR_UNSUPPORTED for NVFP4_CTA).  Other requirements and
+ * errors as fa4_gemm_blockscaled. */
+FA4_API fa4_status fa4_gemm_blockscaled_mxout(fa4_qtensor A, fa4_qtensor B, int64_t M, int64_t N,
+                                      int64_t K, fa4_format fmt, float alpha, void *D, int64_t ldd,
+                                      fa4_qtensor Dq, void *workspace, size_t workspace_bytes,
+                                      void *stream);
+
 /* Linear layer compositions for T tokens, Cin inputs, Cout outputs (the
  * configurations the pages' Llama-3-8B results train: "Format-Aware
  * Fusion...", section "Empirical Results").  bf16 activations row-major.

@@ -210,3 +210,17 @@ def test_training_linear_rejects_bad_arguments():
     assert L.fa4_linear_bwd(DEV, q, q, 250, 256, 384, 0, 1, 0, 1, DEV, DEV, 1, DEV, 1 << 24,
                             None) == 2
     assert L.fa4_linear_bwd(DEV, q, q, 256, 256, 384, 0, 1, 0, 1, DEV, DEV, 1, DEV, 64, None) == 5
+
+
+def test_mxout_gemm_rejects_bad_arguments():
+    L = fa.lib()
+    q = _qt()
+    f = L.fa4_gemm_blockscaled_mxout
+    assert f(q, q, 256, 256, 512, fa.NVFP4_CTA, 1.0, DEV, 256, q, DEV, 4096, None) == 4
+    assert f(q, q, 256, 256, 512, 7, 1.0, DEV, 256, q, DEV, 4096, None) == 1
+    assert f(q, q, 256, 256, 384, fa.MXFP4, 1.0, DEV, 256, q, DEV, 4096, None) == 2
+    assert f(q, q, 256, 256, 512, fa.MXFP4, 1.0, DEV + 8, 256, q, DEV, 4096, None) == 3
+    assert f(q, q, 256, 256, 512, fa.MXFP4, 1.0, DEV, 256, fa._QT(0, 0, 0), DEV, 4096, None) == 1
+    assert f(q, q, 256, 256, 512, fa.MXFP4, 1.0, None, 0, fa._QT(0x10008, 0x20000, 0), DEV, 4096,
+             None) == 3
+    assert f(q, q, 256, 256, 512, fa.MXFP4, 1.0, None, 0, q, DEV, 8, None) == 5
