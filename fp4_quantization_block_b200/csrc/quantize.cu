@@ -379,7 +379,7 @@ __global__ void debug_convert_kernel(const float *y, const uint32_t *u16, int64_
   if (i >= n) return;
   const float v = y[i];
   rne[i] = (uint8_t)(e2m1x2_rne(v, 0.0f) & 0xF);
-  if (sr) sr[i] = (uint8_t)e2m1_sr(v, u16[i] & 0xFFFFu);
+  if (sr) sr[i] = (uint8_t)(e2m1x2_sr(v, 0.0f, u16[i] & 0xFFFFu) & 0xFu);
   if (e4m3) {
     const float sb = fminf(fmaxf(v, 0.001953125f), 448.0f);
     e4m3[i] = (uint8_t)e4m3_rne(sb);

@@ -65,8 +65,10 @@ extern "C" {
 typedef enum { FA4_MXFP4 = 0, FA4_NVFP4_GLOBAL = 1, FA4_NVFP4_CTA = 2 } fa4_format;
 
 /* E2M1 rounding: round-to-nearest-even, or stochastic rounding with 16
- * Philox4x32-10 bits per element keyed by `seed` ("Format-Aware Fusion...",
- * section "Two Key Numerical Techniques": row-gradient stochastic rounding). */
+ * Philox4x32-10 bits u per element keyed by `seed` ("Format-Aware Fusion...",
+ * section "Two Key Numerical Techniques": row-gradient stochastic rounding):
+ * between the neighbouring grid values lo <= |y| < hi, with
+ * t = (|y| - lo) / (hi - lo) * 65536, the value rounds up iff u < floor(t). */
 typedef enum { FA4_RNE = 0, FA4_SR = 1 } fa4_round;
 
 /* Orientation of the quantized operand Q[R, K] relative to the bf16 input

@@ -120,8 +120,9 @@ int orc_e2m1_rne(float y) {
  * [FAF "Two Key Numerical Techniques"]: round up or down with a probability
  * set by the distance, so that the expectation equals the input.
  * Reading: lo <= |y| < hi are the neighbouring grid values, g = hi - lo, the
- * fraction f = (|y| - lo)/g is exact in binary32 (g is a power of two); the
- * value rounds up iff (float)u16 < f * 65536.  |y| >= 6 gives 6.  Sign kept. */
+ * fraction f = (|y| - lo)/g is exact in binary32 (g is a power of two); with
+ * t = f * 65536 the value rounds up iff u16 < floor(t), i.e. for floor(t) of
+ * the 65536 draws (bias below g/65536).  |y| >= 6 gives 6.  Sign kept. */
 int orc_e2m1_sr(float y, uint32_t u16) {
   int s = signbit(y) ? 1 : 0;
   float a = fabsf(y);
@@ -133,10 +134,12 @@ int orc_e2m1_sr(float y, uint32_t u16) {
     double lo = floor((double)a / q) * q;
     float f = (a - (float)lo) / (float)q;  /* both exact */
     float t = f * 65536.0f;                /* exact */
+    /* round up iff u < floor(t): the integer part of t is the number of
+     * the 65536 draws that round up (P(up) = floor(t) / 65536) */
 #ifdef PLANT_SR_LE
-    int up = ((float)(u16 & 0xFFFFu) <= t) ? 1 : 0;
+    int up = ((float)(u16 & 0xFFFFu) <= floorf(t)) ? 1 : 0;
 #else
-    int up = ((float)(u16 & 0xFFFFu) < t) ? 1 : 0;
+    int up = ((float)(u16 & 0xFFFFu) < floorf(t)) ? 1 : 0;
 #endif
     double v = up ? lo + q : lo;
     mc = e2m1_mag_code(v);

@@ -127,7 +127,7 @@ def pin_e2m1_sr():
     # beyond 6 saturates
     assert np.all(O.e2m1_sr(np.full(65536, 7.5, np.float32), u) == 7)
     # exact expectation: averaging over all 2^16 draws gives
-    # lo + g * ceil(65536 f) / 65536, within g/65536 of y (unbiased)
+    # lo + g * floor(65536 f) / 65536, within g/65536 of y (unbiased to 2^-16 g)
     rng = np.random.default_rng(7)
     for y in list(rng.uniform(-6, 6, 24).astype(np.float32)) + [np.float32(0.3), np.float32(5.9)]:
         codes = O.e2m1_sr(np.full(65536, y, dtype=np.float32), u)
@@ -141,6 +141,20 @@ def pin_e2m1_sr():
         # only the two neighbours ever appear
         vals = {abs(O.e2m1_decode(c)) for c in range(16) if counts[c]}
         assert vals <= {lo, hi}
+    # the number of the 2^16 draws that round up is the integer part of
+    # 65536 f (f the fraction between the neighbours), computed here from the
+    # grid by exact rational arithmetic, including fractions with bits below
+    # 2^-16 (where the integer part and a plain comparison u < 65536 f differ)
+    from fractions import Fraction
+    for y in (1.0 + 0.5 * 12345.75 / 65536, 0.25 + 2.0 ** -20, 4.0 + 2.0 * 3.5 / 65536,
+              2.0 ** -17 * 1.5, 0.6 + 2.0 ** -19, 5.0 + 2.0 ** -21):
+        y32 = np.float32(y)
+        a = Fraction(float(y32))
+        lo = max(Fraction(v) for v in grid if Fraction(v) <= a)
+        hi = min(Fraction(v) for v in grid if Fraction(v) > a)
+        ups = int(np.sum(np.abs([O.e2m1_decode(c) for c in
+                                 O.e2m1_sr(np.full(65536, y32, np.float32), u)]) == float(hi)))
+        assert ups == int((a - lo) / (hi - lo) * 65536), (y, ups)
     # with the Philox stream: 10^5 draws, mean within 3 sigma
     for y in (np.float32(0.3), np.float32(-2.7), np.float32(4.9)):
         n = 100000
