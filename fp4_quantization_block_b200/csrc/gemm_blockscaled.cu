@@ -11,22 +11,19 @@
 // Fusion: The Engineering Practice That Doubles FP4 Pretraining Throughput",
 // section "The Design Philosophy of Format-Aware Fusion").
 //
-// Structure (one CTA per SM, persistent over output tiles, 10 warps):
-//   warp 0      TMA producer: per k-tile of 256 elements, the A tile
-//               (128 rows x 128 B) and B tile (BN rows x 128 B) by
-//               cp.async.bulk.tensor with 128-byte swizzle, and the scale
-//               atoms (contiguous 512-byte runs) by cp.async.bulk, into a
-//               4-stage shared-memory ring guarded by mbarriers.
-//   warp 1      MMA issuer: tcgen05.cp moves the scale atoms into tensor
-//               memory, tcgen05.mma kind::mxf4 (MX, 32-blocks, E8M0) or
-//               kind::mxf4nvf4 (NV, 16-blocks, E4M3) accumulates a 128 x BN
-//               FP32 tile in tensor memory; tcgen05.commit frees each stage.
-//   warps 2..9  epilogue: tcgen05.ld of the accumulator, alpha (and the
-//               NVFP4 second-level scales), conversion, global stores.
-// NVFP4-CTA-local: the second-level scale differs per 128-wide K chunk, so
-// each chunk accumulates into one of two tensor-memory partials and the
-// epilogue warps fold tsA[m/128][kc] * tsB[n/128][kc] * partial into FP32
-// registers.
+// Two kernels:
+//   gemm_st::gemm_st_kernel (MXFP4 and NVFP4-global; below): scale factors
+//     staged into tensor memory by tcgen05.st from their own pipeline, 1-SM
+//     or 2-SM (cta_group::2) tiles, output through shared memory and
+//     bulk-tensor stores, optionally the output's MXFP4 operand from the
+//     epilogue.
+//   gemm::gemm_kernel (NVFP4-CTA-local): one CTA per SM, persistent, 10
+//     warps: warp 0 loads A, B and the scale atoms into a 4-stage ring;
+//     warp 1 moves the atoms into tensor memory with tcgen05.cp and issues
+//     tcgen05.mma kind::mxf4nvf4; the second-level scale differs per
+//     128-wide K chunk, so each chunk accumulates into one of two
+//     tensor-memory partials and warps 2..9 fold
+//     tsA[m/128][kc] * tsB[n/128][kc] * partial into FP32 registers.
 //
 // Every mbarrier wait is bounded: past `timeout_ns` the waiting thread sets
 // the device status word, raises a CTA-wide abort flag and leaves its loop;
@@ -633,13 +630,18 @@ __device__ __forceinline__ uint32_t instr_desc_pair(uint32_t sf_id) {
 //   warp 10      scale producer: per k-tile, the A and B scale atoms
 //                (contiguous 512-byte runs) by cp.async.bulk into a deep
 //                ring of small shared-memory stages (SF_STAGES);
-//   warps 2..9   scale staging + epilogue: they read each k-tile's atoms
-//                from shared memory and write, with tcgen05.st, only the
-//                words their 32-lane quadrant's MMA slice reads (row 32q + l
-//                of A in column 4a + q; all B rows of atom a in columns
-//                (BN/32)a ..) into a ring of NBUF tensor-memory buffers, up
-//                to NBUF k-tiles ahead of the MMA; at the end of each tile
-//                they drain the accumulator and store it;
+//   warps 2..9   scale staging + epilogue, two warps per 32-lane quadrant
+//                taking alternate k-tiles: a warp reads its k-tile's atoms
+//                from shared memory and writes, with tcgen05.st, the words
+//                its quadrant's MMA slice reads (row 32q + l of A in column
+//                4a + q; all B rows of atom a in columns (BN/32)a ..) into a
+//                ring of NBUF tensor-memory buffers, up to NBUF k-tiles ahead
+//                of the MMA; at the end of each tile each warp reads half of
+//                its quadrant's accumulator columns, releases the
+//                accumulator, and writes 32 rows x 64 bytes at a time into a
+//                private shared-memory buffer that a bulk-tensor store copies
+//                to D (with QOUT it also quantizes each 32-column MXFP4 block
+//                of its rows);
 //   warp 0       A/B producer: two TMA tile loads per k-tile (AB_STAGES);
 //   warp 1       MMA issue (the pair's leader only).
 // Neither tcgen05.cp (whose per-instruction cost in the tensor pipe rivals

@@ -1,6 +1,6 @@
 // quantize.cu -- fused FP4 quantization producers for sm_100a.
 //
-// One kernel per orientation does the whole producer of "FP4 Is No Longer
+// One kernel per orientation (and one for both) does the whole producer of "FP4 Is No Longer
 // Just a Hardware Feature -- The NVFP4 Software Stack Is Taking Shape",
 // section "The first change" (block amax -> scale -> divide -> E2M1 -> pack
 // two values per byte) in registers, and writes the scale bytes straight into
