@@ -44,6 +44,7 @@ T = workloads.LLAMA8B_TOKENS
 LAYERS = workloads.LLAMA8B_LINEARS
 BYTES_PER_ELEM = {"mx": 2.0 + 0.5 + 1.0 / 32, "nvg": 2.0 + 2.0 + 0.5 + 1.0 / 16,
                   "nvc": 2.0 + 0.5 + 1.0 / 16 + 4.0 / (128 * 128),
+                  "mxnc": 2.0 + 0.5 + 1.0 / 32,
                   # dual producers: one read, both operands written (+ the NVFP4-global amax read)
                   "nvg_dual": 2.0 + 2.0 + (0.5 + 1.0 / 16) + (0.5 + 1.0 / 32),
                   "mx_dual": 2.0 + (0.5 + 1.0 / 32) + (0.5 + 1.0 / 32)}
@@ -240,7 +241,8 @@ def quantize_sweep(fa, device, reps: int = 20) -> list[dict]:
     out = []
     cases = [(fmt, key, rnd, orient, False)
              for orient in (fa.ROWWISE, fa.COLWISE)
-             for fmt, key in ((fa.MXFP4, "mx"), (fa.NVFP4_GLOBAL, "nvg"), (fa.NVFP4_CTA, "nvc"))
+             for fmt, key in ((fa.MXFP4, "mx"), (fa.NVFP4_GLOBAL, "nvg"), (fa.NVFP4_CTA, "nvc"),
+                              (fa.MXFP4_NOCLIP, "mxnc"))
              for rnd in (fa.RNE, fa.SR)]
     cases += [(fa.MXFP4, "mx", rnd, fa.COLWISE, True) for rnd in (fa.RNE, fa.SR)]
     for rows, cols in workloads.SWEEP_SHAPES:

@@ -22,18 +22,18 @@ from dataclasses import dataclass
 import torch
 
 __all__ = [
-    "MXFP4", "NVFP4_GLOBAL", "NVFP4_CTA", "RNE", "SR", "ROWWISE", "COLWISE",
+    "MXFP4", "NVFP4_GLOBAL", "NVFP4_CTA", "MXFP4_NOCLIP", "RNE", "SR", "ROWWISE", "COLWISE",
     "QTensor", "FA4Error", "lib", "library_path", "quant_sizes", "empty_qtensor", "quantize",
     "hadamard32_quantize", "quantize_dual", "gemm", "gemm_mxout", "linear_ws_bytes", "linear_fwd", "linear_dgrad",
     "linear_wgrad", "linear_fwd_save", "linear_bwd", "workspace", "check_device_status",
 ]
 
-MXFP4, NVFP4_GLOBAL, NVFP4_CTA = 0, 1, 2
+MXFP4, NVFP4_GLOBAL, NVFP4_CTA, MXFP4_NOCLIP = 0, 1, 2, 3
 RNE, SR = 0, 1
 ROWWISE, COLWISE = 0, 1
 OUT_BF16, OUT_FP32 = 0, 1
 WS_HEADER_BYTES = 256
-BLOCK = {MXFP4: 32, NVFP4_GLOBAL: 16, NVFP4_CTA: 16}
+BLOCK = {MXFP4: 32, NVFP4_GLOBAL: 16, NVFP4_CTA: 16, MXFP4_NOCLIP: 32}
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 library_path = os.path.join(_HERE, "libfa4.so")

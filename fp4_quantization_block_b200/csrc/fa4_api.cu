@@ -16,8 +16,11 @@ constexpr size_t kHdr = FA4_WS_HEADER_BYTES;
 inline size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
 inline bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 inline bool aligned4(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
-inline bool fmt_ok(int f) { return f == FA4_MXFP4 || f == FA4_NVFP4_GLOBAL || f == FA4_NVFP4_CTA; }
-inline int block_of(int f) { return f == FA4_MXFP4 ? 32 : 16; }
+inline bool fmt_ok(int f) {
+  return f == FA4_MXFP4 || f == FA4_NVFP4_GLOBAL || f == FA4_NVFP4_CTA || f == FA4_MXFP4_NOCLIP;
+}
+inline bool is_mx(int f) { return f == FA4_MXFP4 || f == FA4_MXFP4_NOCLIP; }
+inline int block_of(int f) { return is_mx(f) ? 32 : 16; }
 inline cudaStream_t S(void *s) { return reinterpret_cast<cudaStream_t>(s); }
 
 size_t partials_bytes() { return align256(sizeof(float) * fa4::kMaxAmaxPartials); }
@@ -55,7 +58,7 @@ fa4_status check_input(const void *x, int64_t rows, int64_t cols, int64_t ld) {
 
 fa4_status check_qt(const fa4_qtensor &q, int fmt) {
   if (!q.payload || !q.scales) return FA4_ERR_INVALID_ARG;
-  if (fmt != FA4_MXFP4 && !q.tensor_scale) return FA4_ERR_INVALID_ARG;
+  if (!is_mx(fmt) && !q.tensor_scale) return FA4_ERR_INVALID_ARG;
   if (!aligned16(q.payload) || !aligned16(q.scales)) return FA4_ERR_ALIGN;
   if (q.tensor_scale && !aligned4(q.tensor_scale)) return FA4_ERR_ALIGN;
   return FA4_OK;
@@ -124,7 +127,7 @@ fa4_status do_gemm(const fa4_qtensor &A, const fa4_qtensor &B, int64_t M, int64_
   a.M = M;
   a.N = N;
   a.K = K;
-  a.fmt = fmt;
+  a.fmt = fmt == FA4_MXFP4_NOCLIP ? FA4_MXFP4 : fmt;  // same layout and scale type
   a.alpha = alpha;
   a.D = D;
   a.ldd = ldd;

@@ -22,7 +22,10 @@
 
 namespace fa4 {
 
-enum : int { kMX = 0, kNVG = 1, kNVC = 2 };
+enum : int { kMX = 0, kNVG = 1, kNVC = 2, kMXN = 3 };  // kMXN: MXFP4 without clipping
+// both MXFP4 scale rules share the 32-value block and the E8M0 scale byte
+template <int FMT>
+__device__ __host__ constexpr bool is_mx() { return FMT == kMX || FMT == kMXN; }
 enum : int { kRNE = 0, kSR = 1 };
 
 // ---------------------------------------------------------------- bf16 ---
@@ -104,6 +107,20 @@ __device__ __forceinline__ float e4m3_to_float(uint32_t code) {
 __device__ __forceinline__ uint32_t mx_scale_byte(float amax) {
   const int E = (int)(__float_as_uint(amax) >> 23) & 0xFF;
   return (uint32_t)max(E - 2, 0);
+}
+// MXFP4 without clipping: the smallest e with amax <= 6 * 2^e, i.e. with
+// amax = m * 2^(E-127), 1 <= m < 2: e = E - 129 when m <= 1.5 (mantissa bits
+// <= 0x400000), else E - 128; clamped to [-127, 127] (E = 0 gives -127).
+// Stored byte e + 127.
+__device__ __forceinline__ uint32_t mx_scale_byte_noclip(float amax) {
+  const uint32_t b = __float_as_uint(amax);
+  const int E = (int)(b >> 23) & 0xFF;
+  if (E == 0) return 0u;
+  return (uint32_t)max(E - 2 + ((b & 0x7FFFFFu) > 0x400000u ? 1 : 0), 0);
+}
+template <int FMT>
+__device__ __forceinline__ uint32_t mx_byte(float amax) {
+  return FMT == kMXN ? mx_scale_byte_noclip(amax) : mx_scale_byte(amax);
 }
 __device__ __forceinline__ float mx_multiplier(uint32_t byte) {
   return __uint_as_float((254u - byte) << 23);

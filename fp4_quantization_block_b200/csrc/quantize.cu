@@ -115,7 +115,7 @@ __device__ __forceinline__ void rowwise_tile(const uint4 (&v)[8], int64_t r0, in
   const int w = threadIdx.x >> 5, l = threadIdx.x & 31;
   const int c = l & 15;          // 8-element chunk within the 128-wide row
   const int64_t kc = k0 + 8 * c;  // first column of the chunk
-  const int64_t kbt = (FMT == kMX) ? (K >> 5) : (K >> 4);
+  const int64_t kbt = is_mx<FMT>() ? (K >> 5) : (K >> 4);
 #pragma unroll
   for (int s = 0; s < 8; ++s) {
     const int64_t r = r0 + 16 * s + 2 * w + (l >> 4);
@@ -123,10 +123,10 @@ __device__ __forceinline__ void rowwise_tile(const uint4 (&v)[8], int64_t r0, in
     unpack8(v[s], f);
     float amax = absmax8(v[s]);
     amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, 1));
-    if constexpr (FMT == kMX) amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, 2));
+    if constexpr (is_mx<FMT>()) amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, 2));
     uint32_t sbyte;
-    if constexpr (FMT == kMX) {
-      sbyte = mx_scale_byte(amax);
+    if constexpr (is_mx<FMT>()) {
+      sbyte = mx_byte<FMT>(amax);
       const float mult = mx_multiplier(sbyte);
 #pragma unroll
       for (int e = 0; e < 8; ++e) f[e] = __fmul_rn(f[e], mult);
@@ -146,7 +146,7 @@ __device__ __forceinline__ void rowwise_tile(const uint4 (&v)[8], int64_t r0, in
 
     // gather four consecutive block scales of the row into one word
     uint32_t word;
-    if constexpr (FMT == kMX) {
+    if constexpr (is_mx<FMT>()) {
       word = sbyte << (8 * (c >> 2));
       word |= __shfl_xor_sync(0xFFFFFFFFu, word, 4);
       word |= __shfl_xor_sync(0xFFFFFFFFu, word, 8);
@@ -249,7 +249,7 @@ __device__ __forceinline__ void colwise_tile(const uint16_t *tile, uint8_t *sbuf
     v0[t] = bf16lo(pair);
     v1[t] = bf16hi(pair);
   }
-  const int64_t kbt = (FMT == kMX) ? (T >> 5) : (T >> 4);
+  const int64_t kbt = is_mx<FMT>() ? (T >> 5) : (T >> 4);
 
 #pragma unroll
   for (int half = 0; half < 2; ++half) {
@@ -264,11 +264,11 @@ __device__ __forceinline__ void colwise_tile(const uint16_t *tile, uint8_t *sbuf
     }
     uint32_t codes[4];
     const int64_t kfirst = t0 + 32 * j;  // first K index of this 32-block
-    if constexpr (FMT == kMX) {
+    if constexpr (is_mx<FMT>()) {
       float amax = 0.0f;
 #pragma unroll
       for (int t = 0; t < 32; ++t) amax = fmaxf(amax, fabsf(v[t]));
-      const uint32_t sbyte = mx_scale_byte(amax);
+      const uint32_t sbyte = mx_byte<FMT>(amax);
       const float mult = mx_multiplier(sbyte);
 #pragma unroll
       for (int t = 0; t < 32; ++t) v[t] = __fmul_rn(v[t], mult);
@@ -299,7 +299,7 @@ __device__ __forceinline__ void colwise_tile(const uint16_t *tile, uint8_t *sbuf
   }
   __syncthreads();
   // scale words: MX 4 blocks (one word) per channel, NV 8 blocks (two words)
-  if constexpr (FMT == kMX) {
+  if constexpr (is_mx<FMT>()) {
     if (threadIdx.x < 128) {
       const int cl = threadIdx.x;
       const uint32_t word = *reinterpret_cast<const uint32_t *>(&sbuf[cl * 8]);
@@ -424,6 +424,7 @@ cudaError_t launch_quant_rowwise(int fmt, int rnd, const uint16_t *x, int64_t R,
 #define FA4_ROW(F, Q) \
   if (fmt == F && rnd == Q) launch_row<F, Q>(g, st, x, R, K, ld, payload, scales, ts, partials, n_partials, seed);
   FA4_ROW(kMX, kRNE) FA4_ROW(kMX, kSR) FA4_ROW(kNVG, kRNE) FA4_ROW(kNVG, kSR) FA4_ROW(kNVC, kRNE)
+  FA4_ROW(kMXN, kRNE) FA4_ROW(kMXN, kSR)
   FA4_ROW(kNVC, kSR)
 #undef FA4_ROW
   return cudaGetLastError();
@@ -448,6 +449,7 @@ cudaError_t launch_quant_colwise(int fmt, int rnd, bool hadamard, uint32_t sign_
                         sign_mask);
   FA4_COL(kMX, kRNE, false) FA4_COL(kMX, kSR, false) FA4_COL(kMX, kRNE, true)
   FA4_COL(kMX, kSR, true) FA4_COL(kNVG, kRNE, false) FA4_COL(kNVG, kSR, false)
+  FA4_COL(kMXN, kRNE, false) FA4_COL(kMXN, kSR, false)
   FA4_COL(kNVC, kRNE, false) FA4_COL(kNVC, kSR, false)
 #undef FA4_COL
   return cudaGetLastError();
@@ -476,7 +478,7 @@ cudaError_t launch_quant_dual(int row_fmt, int row_rnd, int col_rnd, bool hadama
   FA4_DUAL(F, kRNE, kRNE, false) FA4_DUAL(F, kRNE, kRNE, true) FA4_DUAL(F, kRNE, kSR, false) \
   FA4_DUAL(F, kRNE, kSR, true) FA4_DUAL(F, kSR, kRNE, false) FA4_DUAL(F, kSR, kRNE, true)    \
   FA4_DUAL(F, kSR, kSR, false) FA4_DUAL(F, kSR, kSR, true)
-  FA4_DUAL_F(kMX) FA4_DUAL_F(kNVG) FA4_DUAL_F(kNVC)
+  FA4_DUAL_F(kMX) FA4_DUAL_F(kNVG) FA4_DUAL_F(kNVC) FA4_DUAL_F(kMXN)
 #undef FA4_DUAL_F
 #undef FA4_DUAL
   return cudaGetLastError();

@@ -61,8 +61,19 @@ extern "C" {
  *                   for the tensor ("FP4 Is No Longer Just a Hardware
  *                   Feature...", section "NVFP4 is more than a 4-bit value").
  *  FA4_NVFP4_CTA    as NVFP4_GLOBAL but one FP32 decode scale per 128x128
- *                   tile of the quantized operand, [R/128][K/128]. */
-typedef enum { FA4_MXFP4 = 0, FA4_NVFP4_GLOBAL = 1, FA4_NVFP4_CTA = 2 } fa4_format;
+ *                   tile of the quantized operand, [R/128][K/128].
+ *  FA4_MXFP4_NOCLIP MXFP4 with the other power-of-two scale rule: the
+ *                   smallest e with amax <= 6 * 2^e, so no value saturates
+ *                   (FA4_MXFP4 takes floor(log2 amax) - 2 and saturates
+ *                   the top of the range).  Same payload, scale layout and
+ *                   scale type as FA4_MXFP4: its operands multiply in a GEMM
+ *                   called with FA4_MXFP4 or FA4_MXFP4_NOCLIP alike. */
+typedef enum {
+  FA4_MXFP4 = 0,
+  FA4_NVFP4_GLOBAL = 1,
+  FA4_NVFP4_CTA = 2,
+  FA4_MXFP4_NOCLIP = 3
+} fa4_format;
 
 /* E2M1 rounding: round-to-nearest-even, or stochastic rounding with 16
  * Philox4x32-10 bits u per element keyed by `seed` ("Format-Aware Fusion...",

@@ -29,10 +29,10 @@ import numpy as np
 
 from . import build as _build
 
-MXFP4, NVFP4_GLOBAL, NVFP4_CTA = 0, 1, 2
+MXFP4, NVFP4_GLOBAL, NVFP4_CTA, MXFP4_NOCLIP = 0, 1, 2, 3
 RNE, SR = 0, 1
 ROWWISE, COLWISE = 0, 1
-BLOCK = {MXFP4: 32, NVFP4_GLOBAL: 16, NVFP4_CTA: 16}
+BLOCK = {MXFP4: 32, NVFP4_GLOBAL: 16, NVFP4_CTA: 16, MXFP4_NOCLIP: 32}
 
 _lib = None
 
@@ -76,6 +76,7 @@ def _setup(lib: ctypes.CDLL) -> ctypes.CDLL:
         "orc_e4m3_decode": (f64, [ci]),
         "orc_e4m3_rne": (ci, [f32]),
         "orc_mx_exponent": (ci, [f32]),
+        "orc_mx_exponent_noclip": (ci, [f32]),
         "orc_nv_encode_scale": (f32, [f32]),
         "orc_nv_decode_scale": (f32, [f32]),
         "orc_nv_block_scale": (ci, [f32, f32, P]),
@@ -140,6 +141,10 @@ def e4m3_rne(v) -> np.ndarray:
 
 def mx_exponent(amax: float) -> int:
     return load().orc_mx_exponent(float(amax))
+
+
+def mx_exponent_noclip(amax: float) -> int:
+    return load().orc_mx_exponent_noclip(float(amax))
 
 
 def nv_encode_scale(amax_t: float) -> float:
@@ -243,7 +248,7 @@ def quantize(x, fmt: int, rnd: int = RNE, orient: int = ROWWISE, seed: int = 0,
                              0 if row_range is None else int(row_range[1]))
     if rc != 0:
         raise ValueError(f"oracle quantize rejected the arguments (rc={rc})")
-    if fmt == MXFP4:
+    if fmt in (MXFP4, MXFP4_NOCLIP):
         ts = np.zeros(0, dtype=np.float32)
     return QTensor(payload, scales, ts, R, K, fmt)
 

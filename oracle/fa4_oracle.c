@@ -43,6 +43,8 @@
 #define ORC_MXFP4 0
 #define ORC_NVFP4_GLOBAL 1
 #define ORC_NVFP4_CTA 2
+#define ORC_MXFP4_NOCLIP 3
+#define ORC_IS_MX(f) ((f) == ORC_MXFP4 || (f) == ORC_MXFP4_NOCLIP)
 #define ORC_RNE 0
 #define ORC_SR 1
 
@@ -199,6 +201,20 @@ int orc_mx_exponent(float amax) {
 #else
   int e = (ex - 1) - 2;
 #endif
+  if (e < -127) e = -127;
+  if (e > 127) e = 127;
+  return e;
+}
+
+/* MXFP4 without clipping: the smallest e with amax <= 6 * 2^e (so no element
+ * of the block saturates), clamped to [-127, 127]; amax = 0 gives -127.
+ * With amax = m * 2^E, 1 <= m < 2: e = E - 2 when m <= 1.5, else E - 1. */
+int orc_mx_exponent_noclip(float amax) {
+  if (!(amax > 0.0f)) return -127;
+  int ex;
+  float fr = frexpf(amax, &ex); /* amax = fr * 2^ex, 0.5 <= fr < 1 */
+  int E = ex - 1;                /* m = 2 fr */
+  int e = (2.0f * fr <= 1.5f) ? E - 2 : E - 1;
   if (e < -127) e = -127;
   if (e > 127) e = 127;
   return e;
@@ -380,7 +396,7 @@ int orc_quantize(const uint16_t *x, int64_t rows, int64_t cols, int64_t ld, int 
                  uint8_t *scales, float *ts, int64_t r_begin, int64_t r_end) {
   int64_t R = orient == 0 ? rows : cols;
   int64_t K = orient == 0 ? cols : rows;
-  int bs = (fmt == ORC_MXFP4) ? 32 : 16;
+  int bs = ORC_IS_MX(fmt) ? 32 : 16;
   if (hadamard && fmt != ORC_MXFP4) return -1;
   if (K % bs != 0 || (K & 1)) return -1;
   if (fmt == ORC_NVFP4_CTA && (R % 128 != 0 || K % 128 != 0)) return -1;
@@ -439,8 +455,8 @@ int orc_quantize(const uint16_t *x, int64_t rows, int64_t cols, int64_t ld, int 
       uint8_t sbyte;
       int mx_e = 0;
       float mult = 1.0f; /* NVFP4: y = v * mult */
-      if (fmt == ORC_MXFP4) {
-        mx_e = orc_mx_exponent(amax_b);
+      if (ORC_IS_MX(fmt)) {
+        mx_e = (fmt == ORC_MXFP4) ? orc_mx_exponent(amax_b) : orc_mx_exponent_noclip(amax_b);
         sbyte = (uint8_t)(mx_e + 127);
       } else {
         float se = (fmt == ORC_NVFP4_CTA) ? s_enc[(r / 128) * n_tk + (kb * bs) / 128] : s_enc[0];
@@ -450,7 +466,7 @@ int orc_quantize(const uint16_t *x, int64_t rows, int64_t cols, int64_t ld, int 
       for (int j = 0; j < bs; ++j) {
         int64_t k = kb * bs + j;
         /* MXFP4: exact multiplication by 2^-e; NVFP4: one binary32 multiply */
-        float y = (fmt == ORC_MXFP4) ? ldexpf(v[j], -mx_e) : v[j] * mult;
+        float y = ORC_IS_MX(fmt) ? ldexpf(v[j], -mx_e) : v[j] * mult;
         int code;
         if (rnd == ORC_SR) code = orc_e2m1_sr(y, orc_sr_bits(seed, (uint64_t)(r * K + k)));
         else code = orc_e2m1_rne(y);
@@ -470,7 +486,7 @@ int orc_quantize(const uint16_t *x, int64_t rows, int64_t cols, int64_t ld, int 
 
 int orc_dequantize_blocks(const uint8_t *payload, const uint8_t *scales, int64_t R, int64_t K,
                           int fmt, const int64_t *row_idx, int64_t n_rows, double *out) {
-  int bs = (fmt == ORC_MXFP4) ? 32 : 16;
+  int bs = ORC_IS_MX(fmt) ? 32 : 16;
   int64_t kb_total = K / bs;
   for (int64_t i = 0; i < n_rows; ++i) {
     int64_t r = row_idx ? row_idx[i] : i;
@@ -479,7 +495,7 @@ int orc_dequantize_blocks(const uint8_t *payload, const uint8_t *scales, int64_t
       uint8_t byte = payload[r * (K / 2) + k / 2];
       int code = (k & 1) ? (byte >> 4) : (byte & 0xF);
       uint8_t sb = scales[orc_sf_offset(r, k / bs, kb_total)];
-      double scale = (fmt == ORC_MXFP4) ? ldexp(1.0, (int)sb - 127) : orc_e4m3_decode(sb);
+      double scale = ORC_IS_MX(fmt) ? ldexp(1.0, (int)sb - 127) : orc_e4m3_decode(sb);
       out[i * K + k] = orc_e2m1_decode(code) * scale;
     }
   }

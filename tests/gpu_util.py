@@ -8,8 +8,8 @@ import torch
 import fp4_quantization_block_b200 as fa
 import oracle as O
 
-FMTS = [fa.MXFP4, fa.NVFP4_GLOBAL, fa.NVFP4_CTA]
-FMT_IDS = {fa.MXFP4: "mx", fa.NVFP4_GLOBAL: "nvg", fa.NVFP4_CTA: "nvc"}
+FMTS = [fa.MXFP4, fa.NVFP4_GLOBAL, fa.NVFP4_CTA, fa.MXFP4_NOCLIP]
+FMT_IDS = {fa.MXFP4: "mx", fa.NVFP4_GLOBAL: "nvg", fa.NVFP4_CTA: "nvc", fa.MXFP4_NOCLIP: "mxnc"}
 
 
 def need_gpu():

@@ -228,6 +228,39 @@ def pin_mx_exponent():
     assert O.mx_exponent(3.99) == -1
 
 
+
+def pin_mx_exponent_noclip():
+    """The no-clip MXFP4 exponent is the smallest e with amax <= 6 * 2^e
+    (clamped to [-127, 127]): checked by its definition on every positive
+    finite bf16 value, and no element of a no-clip block saturates."""
+    bits = np.arange(1, 0x7F80, dtype=np.uint32) << 16          # positive finite bf16
+    vals = bits.view(np.float32)
+    for a in vals[:: 7]:
+        a = float(a)
+        e = O.mx_exponent_noclip(a)
+        if e > -127:
+            assert a <= 6.0 * 2.0 ** e and a > 6.0 * 2.0 ** (e - 1), (a, e)
+        else:
+            assert a <= 6.0 * 2.0 ** -127 or a <= 6.0 * 2.0 ** e, (a, e)
+    assert O.mx_exponent_noclip(0.0) == -127
+    assert O.mx_exponent_noclip(6.0) == 0 and O.mx_exponent_noclip(6.0000005) == 1
+    assert O.mx_exponent_noclip(1.5) == -2 and O.mx_exponent_noclip(1.5000001) == -1
+    # a block quantized with it never saturates: the block max lands on a
+    # grid value within half a grid step, never clipped to 6 from above
+    rng = np.random.default_rng(3)
+    x = torch.from_numpy((rng.standard_normal((128, 256)) * 3).astype(np.float32)).to(torch.bfloat16)
+    q = O.quantize(x, O.MXFP4_NOCLIP)
+    d = O.dequantize(q)
+    xf = x.float().numpy().astype(np.float64)
+    for r in range(0, 128, 17):
+        for kb in range(0, 256, 32):
+            blk = xf[r, kb:kb + 32]
+            e = O.mx_exponent_noclip(float(np.abs(blk).max()))
+            assert np.all(np.abs(blk) * 2.0 ** -e <= 6.0)
+            step = 2.0 ** (e + 1)                                  # largest grid step (4 -> 6)
+            assert np.all(np.abs(d[r, kb:kb + 32] - blk) <= step / 2 + 1e-30)
+
+
 def pin_nv_scales():
     g = _golden("nvfp4_contract.txt")
     emax = float(g["e4m3_max"][0])
@@ -527,7 +560,8 @@ def pin_philox_structure():
     assert int(hi[0]) == int(w2[0]) & 0xFFFF
 
 
-ALL_PINS = [pin_e2m1_decode, pin_e2m1_rne, pin_e2m1_sr, pin_e4m3, pin_mx_exponent, pin_nv_scales,
+ALL_PINS = [pin_e2m1_decode, pin_e2m1_rne, pin_e2m1_sr, pin_e4m3, pin_mx_exponent,
+            pin_mx_exponent_noclip, pin_nv_scales,
             pin_hadamard, pin_swizzle, pin_quantize_rne, pin_quantize_sr, pin_quantize_orientation,
             pin_quantize_hadamard, pin_packing, pin_gemm_bruteforce, pin_gemm_approximates_matmul,
             pin_philox_structure]

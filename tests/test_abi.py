@@ -39,7 +39,7 @@ def test_version_and_status_strings():
     assert L.fa4_status_string(99) == b"unknown status"
 
 
-@pytest.mark.parametrize("fmt", [fa.MXFP4, fa.NVFP4_GLOBAL, fa.NVFP4_CTA])
+@pytest.mark.parametrize("fmt", [fa.MXFP4, fa.NVFP4_GLOBAL, fa.NVFP4_CTA, fa.MXFP4_NOCLIP])
 @pytest.mark.parametrize("orient", [fa.ROWWISE, fa.COLWISE])
 def test_quant_sizes_match_the_layout(fmt, orient):
     rows, cols = 384, 640
@@ -66,6 +66,7 @@ DEV = 0x7F0000000000  # never dereferenced: every call below fails validation fi
     (dict(ld=132), 2),
     (dict(x=DEV + 8), 3),
     (dict(fmt=7), 1),
+    (dict(fmt=4), 1),
     (dict(rnd=5), 1),
     (dict(orient=3), 1),
     (dict(ws=None), 5),
