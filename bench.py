@@ -688,7 +688,7 @@ def reference_arm(args) -> dict:
     sample of the same workload (64 tokens through the block's linears)."""
     _oracle_weights()
     for _ in range(args.warmup):
-        cpu_baseline(sample_tokens=16)
+        cpu_baseline(sample_tokens=32)  # the smallest sample the 32-token MXFP4 blocks allow
     t0 = time.perf_counter()
     res = None
     for _ in range(args.steps):

@@ -81,3 +81,25 @@ def test_every_rank_draws_distinct_inputs():
     seeds = [s for rank in range(8) for i in range(len(bench.LAYERS))
              for s in bench.input_seeds(rank, i)]
     assert len(seeds) == len(set(seeds))
+
+
+@pytest.mark.timeout(900)
+def test_reference_arm_prints_the_contract_line():
+    """The oracle arm on rank 0: one JSON line with the kernel arm's metric,
+    unit and config, the oracle's cpu_baseline and an e2e with no copies."""
+    import json
+    import bench
+    env = dict(os.environ, RANK="0", WORLD_SIZE="1", LOCAL_RANK="0")
+    p = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference",
+                        "--steps", "1", "--warmup", "3"], env=env, capture_output=True,
+                       text=True, timeout=880)
+    assert p.returncode == 0, p.stderr[-2000:]
+    lines = [l for l in p.stdout.splitlines() if l.strip()]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    assert d["impl"] == "reference" and d["metric"] == bench.METRIC and d["unit"] == "tokens/s"
+    assert d["config"] == bench.bench_config(1) and d["higher_is_better"] is True
+    assert d["value"] > 0 and d["cpu_baseline"]["kind"] == "oracle"
+    assert d["cpu_baseline"]["value"] == d["value"] and d["cpu_baseline"]["cores"] >= 1
+    assert d["e2e"] == {"value": d["value"], "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                        "d2h_bytes_per_step": 0}
