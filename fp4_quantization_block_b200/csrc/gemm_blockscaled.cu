@@ -11,19 +11,14 @@
 // Fusion: The Engineering Practice That Doubles FP4 Pretraining Throughput",
 // section "The Design Philosophy of Format-Aware Fusion").
 //
-// Two kernels:
-//   gemm_st::gemm_st_kernel (MXFP4 and NVFP4-global; below): scale factors
-//     staged into tensor memory by tcgen05.st from their own pipeline, 1-SM
-//     or 2-SM (cta_group::2) tiles, output through shared memory and
-//     bulk-tensor stores, optionally the output's MXFP4 operand from the
-//     epilogue.
-//   gemm::gemm_kernel (NVFP4-CTA-local): one CTA per SM, persistent, 10
-//     warps: warp 0 loads A, B and the scale atoms into a 4-stage ring;
-//     warp 1 moves the atoms into tensor memory with tcgen05.cp and issues
-//     tcgen05.mma kind::mxf4nvf4; the second-level scale differs per
-//     128-wide K chunk, so each chunk accumulates into one of two
-//     tensor-memory partials and warps 2..9 fold
-//     tsA[m/128][kc] * tsB[n/128][kc] * partial into FP32 registers.
+// The kernel (gemm_st::gemm_st_kernel, below): scale factors staged into
+// tensor memory by tcgen05.st from their own pipeline, 1-SM or 2-SM
+// (cta_group::2) tiles, output through shared memory and bulk-tensor
+// stores, optionally the output's MXFP4 operand from the epilogue.
+// NVFP4-CTA-local: the second-level scale differs per 128-wide K chunk, so
+// each chunk accumulates into one of two tensor-memory partials that the
+// epilogue warps fold, tsA[m/128][kc] * tsB[n/128][kc] * partial, into FP32
+// registers as soon as the chunk's MMAs complete.
 //
 // Every mbarrier wait is bounded: past `timeout_ns` the waiting thread sets
 // the device status word, raises a CTA-wide abort flag and leaves its loop;
@@ -45,11 +40,7 @@ namespace gemm {
 constexpr int BM = 128;
 constexpr int BK = 256;            // elements per k-tile (128 bytes per row)
 constexpr int BKB = BK / 2;        // bytes per row per k-tile
-constexpr int STAGES = 4;
-constexpr int NUM_THREADS = 320;   // 10 warps
 constexpr int TMEM_COLS = 512;
-constexpr int SFA_COL = 256;       // tensor-memory column of the A scale atoms
-constexpr int SFB_COL = 288;       // ... of the B scale atoms
 constexpr uint32_t kStatusTimeout = 7;
 
 // ------------------------------------------------------------ PTX wrappers
@@ -109,10 +100,6 @@ __device__ __forceinline__ void tc_commit(uint32_t bar) {
                    bar)
                : "memory");
 }
-__device__ __forceinline__ void tc_cp_32x128b_warpx4(uint32_t taddr, uint64_t sdesc) {
-  asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc)
-               : "memory");
-}
 template <int KIND>
 __device__ __forceinline__ void tc_mma(uint32_t d, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
                                        uint32_t sfa, uint32_t sfb, uint32_t accumulate) {
@@ -161,10 +148,6 @@ __device__ __forceinline__ uint64_t smem_desc(uint32_t addr, uint32_t lbo, uint3
 __device__ __forceinline__ uint64_t operand_desc(uint32_t addr) {
   return smem_desc(addr, 16, 1024, 2);
 }
-// One 512-byte scale atom: 32 rows of 16 bytes, 8-row core matrices 128
-// bytes apart, no swizzle.
-__device__ __forceinline__ uint64_t scale_desc(uint32_t addr) { return smem_desc(addr, 0, 128, 0); }
-
 // Block-scaled instruction descriptor: E2M1 A and B (format 1), K-major,
 // N >> 3 in bits 17-22, scale type in bit 23 (1 = E8M0, 0 = E4M3), M >> 4
 // in bits 24-28, scale-factor byte ids in bits 4-5 (B) and 29-30 (A).
@@ -181,28 +164,6 @@ struct Cfg {  // KIND kMX: 32-blocks; kNVG / kNVC: 16-blocks
   static constexpr int SF_PER_ROW = BK / BS;           // scale bytes per row per k-tile
   static constexpr int ATOMS_K = SF_PER_ROW / 4;       // 128x4 atoms along K per k-tile
   static constexpr int SFA_BYTES = ATOMS_K * 512;      // per 128 rows
-};
-
-struct Smem {
-  uint64_t full[STAGES], empty[STAGES];
-  uint64_t acc_full, acc_empty, part_full[2], part_empty[2], mma_done;
-  uint32_t tmem_base;
-  int abort;
-};
-
-template <int KIND, int BN>
-struct Layout {
-  static constexpr int A_BYTES = BM * BKB;                       // 16 KB
-  static constexpr int B_BYTES = BN * BKB;                       // 16 or 32 KB
-  static constexpr int SFA_BYTES = Cfg<KIND>::SFA_BYTES;
-  static constexpr int SFB_BYTES = Cfg<KIND>::SFA_BYTES * (BN / 128);
-  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES;
-  static constexpr int OFF_A = 0;
-  static constexpr int OFF_B = OFF_A + STAGES * A_BYTES;
-  static constexpr int OFF_SFA = OFF_B + STAGES * B_BYTES;
-  static constexpr int OFF_SFB = OFF_SFA + STAGES * SFA_BYTES;
-  static constexpr int OFF_CTRL = OFF_SFB + STAGES * SFB_BYTES;
-  static constexpr int TOTAL = OFF_CTRL + (int)sizeof(Smem) + 1024;  // + alignment slack
 };
 
 struct Params {
@@ -234,307 +195,6 @@ __device__ __forceinline__ void tile_coords(int t, int num_m, int num_n, int n_f
   } else {
     mt = t % num_m;
     nt = t / num_m;
-  }
-}
-
-// Bounded wait.  Returns false on timeout (status set, abort raised) or when
-// another role already aborted.
-__device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, Smem *sm, const Params &p,
-                                         uint32_t where) {
-  if (mbar_try_wait(bar, parity)) return true;
-  const uint64_t t0 = globaltimer();
-  while (true) {
-    if (mbar_try_wait(bar, parity)) return true;
-    if (*(volatile int *)&sm->abort) return false;
-    if (globaltimer() - t0 > p.timeout_ns) {
-      *(volatile int *)&sm->abort = 1;
-      if (atomicCAS(p.status, 0u, kStatusTimeout) == 0u) atomicExch(p.status + 1, where);
-      return false;
-    }
-  }
-}
-
-// Warp-uniform bounded wait: lane 0 waits, every lane gets the result, and
-// the warp is converged afterwards (the .sync.aligned tcgen05 loads that
-// follow need all 32 lanes together).
-__device__ __forceinline__ bool warp_wait_bar(uint32_t bar, uint32_t parity, Smem *sm,
-                                              const Params &p, uint32_t where) {
-  int ok = 0;
-  if ((threadIdx.x & 31) == 0) ok = wait_bar(bar, parity, sm, p, where) ? 1 : 0;
-  ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
-  return ok != 0;
-}
-
-// KIND: kMX, kNVG or kNVC (CTA-local second-level scales).
-template <int KIND, int BN>
-__global__ void __launch_bounds__(NUM_THREADS, 1)
-    gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_b,
-                const Params p) {
-  constexpr bool CTA = (KIND == kNVC);
-  using L = Layout<KIND, BN>;
-  using C = Cfg<KIND>;
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                              ~uintptr_t(1023));
-  Smem *sm = reinterpret_cast<Smem *>(smem + L::OFF_CTRL);
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-
-  const int num_m = (int)(p.M / BM), num_n = (int)(p.N / BN);
-  const int num_tiles = num_m * num_n;
-  const int KT = (int)(p.K / BK);
-  const int64_t kbt4 = (p.K / C::BS) / 4;  // scale atoms per 128 rows
-
-  if (threadIdx.x == 0) {
-    for (int s = 0; s < STAGES; ++s) {
-      mbar_init(smem_u32(&sm->full[s]), 1);
-      mbar_init(smem_u32(&sm->empty[s]), 1);
-    }
-    mbar_init(smem_u32(&sm->acc_full), 1);
-    mbar_init(smem_u32(&sm->acc_empty), 8);
-    for (int i = 0; i < 2; ++i) {
-      mbar_init(smem_u32(&sm->part_full[i]), 1);
-      mbar_init(smem_u32(&sm->part_empty[i]), 8);
-    }
-    mbar_init(smem_u32(&sm->mma_done), 1);
-    sm->abort = 0;
-    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-  }
-  if (warp == 1) {
-    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
-                     smem_u32(&sm->tmem_base)),
-                 "r"(TMEM_COLS)
-                 : "memory");
-    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
-  }
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  const uint32_t tmem = sm->tmem_base;
-
-  if (warp == 0) {
-    // ------------------------------------------------------------ producer
-    if (lane == 0) {
-      int stage = 0;
-      uint32_t phase = 0;
-      uint32_t issued = 0;       // stages with a load in flight or landed
-      uint32_t last_parity = 0;  // parity bit of the last load issued per stage
-      bool ok = true;
-      int k_global = 0;
-      for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
-        int mt, nt;
-        tile_coords(tile, num_m, num_n, p.n_fastest, mt, nt);
-        for (int kt = 0; kt < KT; ++kt, ++k_global) {
-          if (!wait_bar(smem_u32(&sm->empty[stage]), phase ^ 1u, sm, p, 0x100u | stage)) {
-            ok = false;
-            break;
-          }
-          if (k_global != p.debug_skip_stage) {
-            const uint32_t fb = smem_u32(&sm->full[stage]);
-            mbar_arrive_expect_tx(fb, L::STAGE_BYTES);
-            tma_load_2d(smem_u32(smem + L::OFF_A + stage * L::A_BYTES), &map_a, kt * BKB, mt * BM, fb);
-            tma_load_2d(smem_u32(smem + L::OFF_B + stage * L::B_BYTES), &map_b, kt * BKB, nt * BN, fb);
-            const uint8_t *sa = p.a_scales + ((int64_t)mt * kbt4 + (int64_t)kt * C::ATOMS_K) * 512;
-            bulk_load(smem_u32(smem + L::OFF_SFA + stage * L::SFA_BYTES), sa, L::SFA_BYTES, fb);
-#pragma unroll
-            for (int nb = 0; nb < BN / 128; ++nb) {
-              const uint8_t *sb =
-                  p.b_scales + ((int64_t)(nt * (BN / 128) + nb) * kbt4 + (int64_t)kt * C::ATOMS_K) * 512;
-              bulk_load(smem_u32(smem + L::OFF_SFB + stage * L::SFB_BYTES + nb * C::SFA_BYTES), sb,
-                        C::SFA_BYTES, fb);
-            }
-            issued |= 1u << stage;
-            last_parity = (last_parity & ~(1u << stage)) | (phase << stage);
-          }
-          if (++stage == STAGES) {
-            stage = 0;
-            phase ^= 1u;
-          }
-        }
-      }
-      // never leave with a copy in flight into this CTA's shared memory
-      for (int s = 0; s < STAGES; ++s) {
-        if (!((issued >> s) & 1u)) continue;
-        const uint32_t par = (last_parity >> s) & 1u;
-        const uint64_t t0 = globaltimer();
-        while (!mbar_try_wait(smem_u32(&sm->full[s]), par)) {
-          if (globaltimer() - t0 > p.timeout_ns) {
-            if (atomicCAS(p.status, 0u, kStatusTimeout) == 0u) atomicExch(p.status + 1, 0x400u | s);
-            break;
-          }
-        }
-      }
-    }
-  } else if (warp == 1) {
-    // ----------------------------------------------------------- MMA issue
-    if (lane == 0) {
-      int stage = 0;
-      uint32_t phase = 0, acc_phase = 0;
-      uint32_t chunk = 0;  // CTA-local: global 128-K chunk counter
-      bool ok = true;
-      for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
-        if constexpr (!CTA) {
-          if (!wait_bar(smem_u32(&sm->acc_empty), acc_phase ^ 1u, sm, p, 0x200u)) break;
-          tc_fence_after();
-        }
-        for (int kt = 0; kt < KT; ++kt) {
-          if (!wait_bar(smem_u32(&sm->full[stage]), phase, sm, p, 0x210u | stage)) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-          const uint32_t a_base = smem_u32(smem + L::OFF_A + stage * L::A_BYTES);
-          const uint32_t b_base = smem_u32(smem + L::OFF_B + stage * L::B_BYTES);
-          const uint32_t sfa_base = smem_u32(smem + L::OFF_SFA + stage * L::SFA_BYTES);
-          const uint32_t sfb_base = smem_u32(smem + L::OFF_SFB + stage * L::SFB_BYTES);
-          // scale atoms -> tensor memory: A atom a at column SFA_COL + 4a; B
-          // atom (row block nb, a) at SFB_COL + (BN/32)*a + 4*nb
-#pragma unroll
-          for (int a = 0; a < C::ATOMS_K; ++a) {
-            tc_cp_32x128b_warpx4(tmem + SFA_COL + 4 * a, scale_desc(sfa_base + a * 512));
-#pragma unroll
-            for (int nb = 0; nb < BN / 128; ++nb)
-              tc_cp_32x128b_warpx4(tmem + SFB_COL + (BN / 32) * a + 4 * nb,
-                                   scale_desc(sfb_base + nb * C::SFA_BYTES + a * 512));
-          }
-#pragma unroll
-          for (int j = 0; j < BK / 64; ++j) {
-            // MX: two MMAs share one atom (scale bytes 0-1 and 2-3 of the
-            // word); NV: one atom per MMA
-            const int a = (KIND == kMX) ? (j >> 1) : j;
-            const uint32_t sf_id = (KIND == kMX) ? (uint32_t)(2 * (j & 1)) : 0u;
-            const uint32_t sfa = (tmem + SFA_COL + 4 * a) | (sf_id << 30);
-            const uint32_t sfb = (tmem + SFB_COL + (BN / 32) * a) | (sf_id << 30);
-            const uint64_t ad = operand_desc(a_base + j * 32);
-            const uint64_t bd = operand_desc(b_base + j * 32);
-            if constexpr (CTA) {
-              const int c = j >> 1;  // 128-K chunk within the k-tile
-              const uint32_t pb = (chunk + c) & 1u;
-              if ((j & 1) == 0) {
-                if (!wait_bar(smem_u32(&sm->part_empty[pb]), (((chunk + c) >> 1) & 1u) ^ 1u, sm, p,
-                              0x220u | pb)) {
-                  ok = false;
-                  break;
-                }
-                tc_fence_after();
-              }
-              tc_mma<KIND>(tmem + pb * 128, ad, bd, instr_desc<KIND, BN>(sf_id), sfa, sfb,
-                           (uint32_t)(j & 1));
-              if (j & 1) tc_commit(smem_u32(&sm->part_full[pb]));
-            } else {
-              tc_mma<KIND>(tmem, ad, bd, instr_desc<KIND, BN>(sf_id), sfa, sfb,
-                           (kt > 0 || j > 0) ? 1u : 0u);
-            }
-          }
-          if constexpr (CTA) chunk += BK / 128;
-          tc_commit(smem_u32(&sm->empty[stage]));
-          if (!ok) break;
-          if (++stage == STAGES) {
-            stage = 0;
-            phase ^= 1u;
-          }
-        }
-        if constexpr (!CTA) {
-          if (ok) tc_commit(smem_u32(&sm->acc_full));
-          acc_phase ^= 1u;
-        }
-      }
-      // all MMAs issued by this thread have completed before tensor memory
-      // is released
-      tc_commit(smem_u32(&sm->mma_done));
-      const uint64_t t0 = globaltimer();
-      while (!mbar_try_wait(smem_u32(&sm->mma_done), 0)) {
-        if (globaltimer() - t0 > p.timeout_ns) {
-          if (atomicCAS(p.status, 0u, kStatusTimeout) == 0u) atomicExch(p.status + 1, 0x500u);
-          break;
-        }
-      }
-    }
-  } else {
-    // ------------------------------------------------------------ epilogue
-    const int q = warp & 3;          // tensor-memory lane quadrant this warp may access
-    const int h = (warp - 2) >> 2;   // column half
-    constexpr int COLS = BN / 2;     // columns per warp
-    constexpr int NCH = COLS / 32;   // 32-column loads
-    const int nk = (int)(p.K / 128);
-    uint32_t acc_phase = 0, chunk = 0;
-    float alpha_g = p.alpha;
-    if constexpr (KIND == kNVG && !CTA) alpha_g = p.alpha * p.a_ts[0] * p.b_ts[0];
-    for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
-      int mt, nt;
-        tile_coords(tile, num_m, num_n, p.n_fastest, mt, nt);
-      float v[COLS];
-      bool ok = true;
-      if constexpr (CTA) {
-#pragma unroll
-        for (int i = 0; i < COLS; ++i) v[i] = 0.0f;
-        for (int kc = 0; kc < nk; ++kc, ++chunk) {
-          const uint32_t pb = chunk & 1u;
-          if (!warp_wait_bar(smem_u32(&sm->part_full[pb]), (chunk >> 1) & 1u, sm, p, 0x300u | pb)) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-          uint32_t r[COLS];
-#pragma unroll
-          for (int c = 0; c < NCH; ++c)
-            tmem_ld32(tmem + ((uint32_t)(32 * q) << 16) + pb * 128 + h * COLS + 32 * c, &r[32 * c]);
-          tmem_wait_ld();
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(smem_u32(&sm->part_empty[pb]));
-          const float s = p.a_ts[(int64_t)mt * nk + kc] * p.b_ts[(int64_t)nt * nk + kc];
-#pragma unroll
-          for (int i = 0; i < COLS; ++i) v[i] = fmaf(s, __uint_as_float(r[i]), v[i]);
-        }
-        if (!ok) break;
-#pragma unroll
-        for (int i = 0; i < COLS; ++i) v[i] *= p.alpha;
-      } else {
-        if (!warp_wait_bar(smem_u32(&sm->acc_full), acc_phase, sm, p, 0x310u)) break;
-        tc_fence_after();
-        uint32_t r[COLS];
-#pragma unroll
-        for (int c = 0; c < NCH; ++c)
-          tmem_ld32(tmem + ((uint32_t)(32 * q) << 16) + h * COLS + 32 * c, &r[32 * c]);
-        tmem_wait_ld();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(smem_u32(&sm->acc_empty));
-        acc_phase ^= 1u;
-#pragma unroll
-        for (int i = 0; i < COLS; ++i) v[i] = __uint_as_float(r[i]) * alpha_g;
-      }
-      // each thread owns one output row segment of COLS columns
-      const int64_t row = (int64_t)mt * BM + 32 * q + lane;
-      const int64_t col = (int64_t)nt * BN + h * COLS;
-      if (p.out_fp32) {
-        float *dst = reinterpret_cast<float *>(p.D) + row * p.ldd + col;
-#pragma unroll
-        for (int i = 0; i < COLS; i += 4)
-          *reinterpret_cast<float4 *>(dst + i) = make_float4(v[i], v[i + 1], v[i + 2], v[i + 3]);
-      } else {
-        uint16_t *dst = reinterpret_cast<uint16_t *>(p.D) + row * p.ldd + col;
-#pragma unroll
-        for (int i = 0; i < COLS; i += 8) {
-          uint32_t w[4];
-#pragma unroll
-          for (int u = 0; u < 4; ++u) {
-            __nv_bfloat162 b2 = __floats2bfloat162_rn(v[i + 2 * u], v[i + 2 * u + 1]);
-            w[u] = *reinterpret_cast<uint32_t *>(&b2);
-          }
-          *reinterpret_cast<uint4 *>(dst + i) = make_uint4(w[0], w[1], w[2], w[3]);
-        }
-      }
-    }
-  }
-
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  if (warp == 1) {
-    __syncwarp();
-    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(TMEM_COLS)
-                 : "memory");
   }
 }
 
@@ -703,6 +363,7 @@ struct SmemSt {
   uint64_t sfs_full[12], sfs_empty[12];      // scale stages in shared memory
   uint64_t sft_full[NBUF], sft_empty[NBUF];  // scale buffers in tensor memory
   uint64_t acc_full, acc_empty, mma_done;
+  uint64_t part_full[2], part_empty[2];  // CTA-local NVFP4: the two 128-K chunk partials
   uint32_t tmem_base;
   int abort;
 };
@@ -837,6 +498,10 @@ __global__ void __launch_bounds__(NUM_THREADS_ST, 1)
     }
     mbar_init(smem_u32(&sm->acc_full), 1);
     mbar_init(smem_u32(&sm->acc_empty), CS::ACC_ARRIVALS);
+    for (int c = 0; c < 2; ++c) {
+      mbar_init(smem_u32(&sm->part_full[c]), 1);
+      mbar_init(smem_u32(&sm->part_empty[c]), CS::ACC_ARRIVALS);
+    }
     mbar_init(smem_u32(&sm->mma_done), 1);
     sm->abort = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -953,8 +618,10 @@ __global__ void __launch_bounds__(NUM_THREADS_ST, 1)
       bool ok = true;
       int g = 0;
       for (int tile = unit; tile < num_tiles && ok; tile += nunits) {
-        if (!wait_st(smem_u32(&sm->acc_empty), acc_phase ^ 1u, sm, p, 0x200u)) break;
-        tc_fence_after();
+        if constexpr (KIND != kNVC) {
+          if (!wait_st(smem_u32(&sm->acc_empty), acc_phase ^ 1u, sm, p, 0x200u)) break;
+          tc_fence_after();
+        }
         for (int kt = 0; kt < KT; ++kt, ++g) {
           const int s = g % ABS, b = g % NBUF;
           if (!wait_st(smem_u32(&sm->sft_full[b]), (uint32_t)((g / NBUF) & 1), sm, p, 0x230u | b) ||
@@ -972,14 +639,33 @@ __global__ void __launch_bounds__(NUM_THREADS_ST, 1)
             const uint32_t sf_id = (KIND == kMX) ? (uint32_t)(2 * (j & 1)) : 0u;
             const uint32_t sfa = (sf_col + 4 * a) | (sf_id << 30);
             const uint32_t sfb = (sf_col + CS::COLS_A + (BN / 32) * a) | (sf_id << 30);
-            const uint32_t acc = (kt > 0 || j > 0) ? 1u : 0u;
-            if constexpr (PAIR)
-              tc_mma_pair<KIND>(tmem, operand_desc(a_base + j * 32), operand_desc(b_base + j * 32),
-                                instr_desc_pair<KIND>(sf_id), sfa, sfb, acc);
-            else
-              tc_mma<KIND>(tmem, operand_desc(a_base + j * 32), operand_desc(b_base + j * 32),
-                           instr_desc<KIND, BN>(sf_id), sfa, sfb, acc);
+            if constexpr (KIND == kNVC) {
+              // each 128-K chunk (MMAs 2c, 2c+1) starts a fresh partial in
+              // columns 128c.. once the fold has read its previous content
+              const int c = j >> 1;
+              if ((j & 1) == 0) {
+                if (!wait_st(smem_u32(&sm->part_empty[c]), (uint32_t)((g & 1) ^ 1), sm, p,
+                             0x240u | c)) {
+                  ok = false;
+                  break;
+                }
+                tc_fence_after();
+              }
+              tc_mma<KIND>(tmem + 128 * c, operand_desc(a_base + j * 32),
+                           operand_desc(b_base + j * 32), instr_desc<KIND, BN>(sf_id), sfa, sfb,
+                           (uint32_t)(j & 1));
+              if (j & 1) tc_commit(smem_u32(&sm->part_full[c]));
+            } else {
+              const uint32_t acc = (kt > 0 || j > 0) ? 1u : 0u;
+              if constexpr (PAIR)
+                tc_mma_pair<KIND>(tmem, operand_desc(a_base + j * 32), operand_desc(b_base + j * 32),
+                                  instr_desc_pair<KIND>(sf_id), sfa, sfb, acc);
+              else
+                tc_mma<KIND>(tmem, operand_desc(a_base + j * 32), operand_desc(b_base + j * 32),
+                             instr_desc<KIND, BN>(sf_id), sfa, sfb, acc);
+            }
           }
+          if (!ok) break;
           if constexpr (PAIR) {
             tc_commit_pair(smem_u32(&sm->ab_empty[s]), (uint16_t)3);
             tc_commit_pair(smem_u32(&sm->sft_empty[b]), (uint16_t)3);
@@ -988,7 +674,7 @@ __global__ void __launch_bounds__(NUM_THREADS_ST, 1)
             tc_commit(smem_u32(&sm->sft_empty[b]));
           }
         }
-        if (ok) {
+        if (ok && KIND != kNVC) {
           if constexpr (PAIR)
             tc_commit_pair(smem_u32(&sm->acc_full), (uint16_t)3);
           else
@@ -1057,38 +743,9 @@ __global__ void __launch_bounds__(NUM_THREADS_ST, 1)
       return true;
     };
 
-    // the quadrant's two warps stage alternate k-tiles (h = 0 the even ones)
-    uint32_t acc_phase = 0;
-    int g = h;
-    bool ok = true;
-    int it = 0;
-    for (int tile = unit; tile < num_tiles && ok; tile += nunits, ++it) {
-      // scales for the rest of this tile and the first NBUF k-tiles of the
-      // next one, then this tile's epilogue
-      const int until = min(total, (it + 1) * KT + NBUF);
-      for (; g < until; g += 2)
-        if (!stage_scales(g)) {
-          ok = false;
-          break;
-        }
-      if (!ok) break;
-      int mt, nt;
-      tile_coords(tile, num_m, num_n, p.n_fastest, mt, nt);
-      if (!warp_wait_st(smem_u32(&sm->acc_full), acc_phase, sm, p, 0x310u)) break;
-      tc_fence_after();
-      uint32_t r[COLS];
-#pragma unroll
-      for (int c = 0; c < NCH; ++c) tmem_ld32(lane_base + h * COLS + 32 * c, &r[32 * c]);
-      tmem_wait_ld();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) {
-        if (PAIR && rank != 0)
-          mbar_arrive_remote_relaxed(acc_empty_l);
-        else
-          mbar_arrive(smem_u32(&sm->acc_empty));
-      }
-      acc_phase ^= 1u;
+    // write one output tile (this warp's 32 rows x COLS columns, accumulator
+    // words in r) through the shared-memory buffer and bulk-tensor stores
+    auto store_tile = [&](const uint32_t (&r)[COLS], int mt, int nt) {
       // stage 32 rows x 64 bytes at a time in this warp's buffer (16-byte
       // pieces placed with the 64-byte swizzle: piece j of row r at
       // j ^ ((r >> 1) & 3), which the tensor map undoes) and store it with
@@ -1176,6 +833,91 @@ __global__ void __launch_bounds__(NUM_THREADS_ST, 1)
             *reinterpret_cast<uint16_t *>(sdst) = (uint16_t)sword;
         }
       }
+    };
+
+    if constexpr (KIND == kNVC) {
+      // CTA-local NVFP4: per k-tile, stage this warp's scales up to NBUF
+      // k-tiles ahead, then fold both 128-K chunk partials into FP32
+      // registers, acc += tsA[m/128][kc] * tsB[n/128][kc] * partial, and
+      // release each partial as soon as it is read; store at the tile's end
+      const int nk = (int)(p.K / 128);
+      int g_st = h, g = 0;
+      bool ok = true;
+      for (int tile = unit; tile < num_tiles && ok; tile += nunits) {
+        int mt, nt;
+        tile_coords(tile, num_m, num_n, p.n_fastest, mt, nt);
+        float acc[COLS];
+#pragma unroll
+        for (int i = 0; i < COLS; ++i) acc[i] = 0.0f;
+        for (int kt = 0; kt < KT && ok; ++kt, ++g) {
+          for (; g_st < total && g_st < g + NBUF; g_st += 2)
+            if (!stage_scales(g_st)) {
+              ok = false;
+              break;
+            }
+          if (!ok) break;
+#pragma unroll
+          for (int c = 0; c < 2; ++c) {
+            if (!warp_wait_st(smem_u32(&sm->part_full[c]), (uint32_t)(g & 1), sm, p, 0x340u | c)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            uint32_t r[COLS];
+#pragma unroll
+            for (int ch = 0; ch < NCH; ++ch)
+              tmem_ld32(lane_base + 128 * c + h * COLS + 32 * ch, &r[32 * ch]);
+            tmem_wait_ld();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(smem_u32(&sm->part_empty[c]));
+            const int kc = 2 * kt + c;
+            const float f = p.a_ts[(int64_t)mt * nk + kc] * p.b_ts[(int64_t)nt * nk + kc];
+#pragma unroll
+            for (int i = 0; i < COLS; ++i) acc[i] = fmaf(f, __uint_as_float(r[i]), acc[i]);
+          }
+        }
+        if (!ok) break;
+        uint32_t r[COLS];
+#pragma unroll
+        for (int i = 0; i < COLS; ++i) r[i] = __float_as_uint(acc[i]);
+        store_tile(r, mt, nt);
+      }
+    } else {
+    // the quadrant's two warps stage alternate k-tiles (h = 0 the even ones)
+    uint32_t acc_phase = 0;
+    int g = h;
+    bool ok = true;
+    int it = 0;
+    for (int tile = unit; tile < num_tiles && ok; tile += nunits, ++it) {
+      // scales for the rest of this tile and the first NBUF k-tiles of the
+      // next one, then this tile's epilogue
+      const int until = min(total, (it + 1) * KT + NBUF);
+      for (; g < until; g += 2)
+        if (!stage_scales(g)) {
+          ok = false;
+          break;
+        }
+      if (!ok) break;
+      int mt, nt;
+      tile_coords(tile, num_m, num_n, p.n_fastest, mt, nt);
+      if (!warp_wait_st(smem_u32(&sm->acc_full), acc_phase, sm, p, 0x310u)) break;
+      tc_fence_after();
+      uint32_t r[COLS];
+#pragma unroll
+      for (int c = 0; c < NCH; ++c) tmem_ld32(lane_base + h * COLS + 32 * c, &r[32 * c]);
+      tmem_wait_ld();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) {
+        if (PAIR && rank != 0)
+          mbar_arrive_remote_relaxed(acc_empty_l);
+        else
+          mbar_arrive(smem_u32(&sm->acc_empty));
+      }
+      acc_phase ^= 1u;
+      store_tile(r, mt, nt);
+    }
     }
     // the stores read shared memory and write D after this: both done
     // before the block can leave
@@ -1281,25 +1023,6 @@ static gemm::Params make_params(const GemmArgs &a) {
   return p;
 }
 
-template <int KIND, int BN>
-static cudaError_t launch_t(const GemmArgs &a, cudaStream_t st) {
-  using L = gemm::Layout<KIND, BN>;
-  CUtensorMap ma, mb;
-  if (!make_payload_map(&ma, a.a_payload, a.M, a.K, gemm::BM)) return cudaErrorInvalidValue;
-  if (!make_payload_map(&mb, a.b_payload, a.N, a.K, BN)) return cudaErrorInvalidValue;
-  gemm::Params p = make_params(a);
-  auto kern = gemm::gemm_kernel<KIND, BN>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::TOTAL);
-  if (e != cudaSuccess) return e;
-  int dev = 0, sms = 148;
-  cudaGetDevice(&dev);
-  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  const int64_t tiles = (a.M / gemm::BM) * (a.N / BN);
-  const int grid = (int)(tiles < sms ? tiles : sms);
-  kern<<<grid, gemm::NUM_THREADS, L::TOTAL, st>>>(ma, mb, p);
-  return cudaGetLastError();
-}
-
 template <int KIND, int BN, bool PAIR, bool QOUT>
 static cudaError_t launch_st(const GemmArgs &a, cudaStream_t st) {
   constexpr int smem = gemm_st::total_smem_st<KIND, BN, PAIR>();
@@ -1365,7 +1088,7 @@ cudaError_t launch_gemm_blockscaled(const GemmArgs &a, cudaStream_t st) {
     if (!a.D) return cudaErrorInvalidValue;
     return launch_st_any<false>(a, st);
   }
-  if (a.fmt == kNVC && !a.q_payload && a.D) return launch_t<kNVC, 128>(a, st);
+  if (a.fmt == kNVC && !a.q_payload && a.D) return launch_st<kNVC, 128, false, false>(a, st);
   return cudaErrorInvalidValue;
 }
 
