@@ -140,6 +140,8 @@ int orc_e2m1_sr(float y, uint32_t u16) {
      * the 65536 draws that round up (P(up) = floor(t) / 65536) */
 #ifdef PLANT_SR_LE
     int up = ((float)(u16 & 0xFFFFu) <= floorf(t)) ? 1 : 0;
+#elif defined(PLANT_SR_NOFLOOR)
+    int up = ((float)(u16 & 0xFFFFu) < t) ? 1 : 0;
 #else
     int up = ((float)(u16 & 0xFFFFu) < floorf(t)) ? 1 : 0;
 #endif
@@ -214,7 +216,12 @@ int orc_mx_exponent_noclip(float amax) {
   int ex;
   float fr = frexpf(amax, &ex); /* amax = fr * 2^ex, 0.5 <= fr < 1 */
   int E = ex - 1;                /* m = 2 fr */
+#ifdef PLANT_MX_NOCLIP_FLOOR
+  int e = E - 2; /* the clipping rule's exponent */
+  (void)fr;
+#else
   int e = (2.0f * fr <= 1.5f) ? E - 2 : E - 1;
+#endif
   if (e < -127) e = -127;
   if (e > 127) e = 127;
   return e;

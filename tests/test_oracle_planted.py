@@ -14,6 +14,8 @@ import oracle_pins as P
 PLANTS = {
     "PLANT_TIE_AWAY": [P.pin_e2m1_rne],
     "PLANT_SR_LE": [P.pin_e2m1_sr],
+    "PLANT_SR_NOFLOOR": [P.pin_e2m1_sr],
+    "PLANT_MX_NOCLIP_FLOOR": [P.pin_mx_exponent_noclip],
     "PLANT_MX_EMAX": [P.pin_mx_exponent, P.pin_quantize_rne],
     "PLANT_SWIZZLE": [P.pin_swizzle],
     "PLANT_HAD_SIGN_AFTER": [P.pin_hadamard, P.pin_quantize_hadamard],
