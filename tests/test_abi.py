@@ -225,3 +225,34 @@ def test_mxout_gemm_rejects_bad_arguments():
     assert f(q, q, 256, 256, 512, fa.MXFP4, 1.0, None, 0, fa._QT(0x10008, 0x20000, 0), DEV, 4096,
              None) == 3
     assert f(q, q, 256, 256, 512, fa.MXFP4, 1.0, None, 0, q, DEV, 8, None) == 5
+
+
+def test_header_is_plain_c_and_links_from_c(tmp_path):
+    """The boundary is a C ABI: include/fa4.h compiles as strict C99 and a C
+    program links against libfa4.so and calls host-only entry points."""
+    import shutil
+    import subprocess
+    if not shutil.which("gcc"):
+        pytest.skip("no C compiler")
+    src = tmp_path / "abi.c"
+    src.write_text(
+        '#include "fa4.h"\n#include <stdio.h>\n#include <string.h>\n'
+        "int main(void) {\n"
+        "  size_t pb = 0, sb = 0, tc = 0, ws = 0;\n"
+        "  if (fa4_version() < 100) return 1;\n"
+        "  if (strcmp(fa4_status_string(FA4_OK), \"ok\") != 0) return 2;\n"
+        "  if (fa4_quant_sizes(256, 512, FA4_NVFP4_GLOBAL, FA4_ROWWISE, &pb, &sb, &tc, &ws) != FA4_OK)\n"
+        "    return 3;\n"
+        "  if (pb != 256 * 256 || sb != 256 * 32 || tc != 1) return 4;\n"
+        "  if (fa4_quantize(NULL, 256, 512, 512, FA4_MXFP4, FA4_RNE, FA4_ROWWISE, 0,\n"
+        "                   (fa4_qtensor){0, 0, 0}, NULL, 0, NULL) != FA4_ERR_INVALID_ARG) return 5;\n"
+        "  puts(\"c-abi ok\");\n  return 0;\n}\n")
+    exe = tmp_path / "abi"
+    lib_dir = os.path.dirname(fa.library_path)
+    cc = subprocess.run(["gcc", "-std=c99", "-Wall", "-Wextra", "-pedantic", "-Werror",
+                         "-I", os.path.join(ROOT, "include"), str(src), "-o", str(exe),
+                         "-L", lib_dir, "-l:libfa4.so", f"-Wl,-rpath,{lib_dir}"],
+                        capture_output=True, text=True)
+    assert cc.returncode == 0, cc.stderr
+    run = subprocess.run([str(exe)], capture_output=True, text=True, timeout=60)
+    assert run.returncode == 0 and "c-abi ok" in run.stdout, (run.returncode, run.stderr)
