@@ -184,7 +184,9 @@ FA4_API fa4_status fa4_quantize_dual(const void *x, int64_t rows, int64_t cols, 
  * K-major).  NVFP4_GLOBAL multiplies by the two tensor decode scales;
  * NVFP4_CTA multiplies every 128-wide K chunk by tsA[m/128][kc] *
  * tsB[n/128][kc].  FP32 accumulation.  D is row-major [M, N] with leading
- * dimension ldd elements, bf16 or fp32.  M, N, K multiples of 128.
+ * dimension ldd elements (a multiple of 8, at least N), bf16 or fp32.  M and
+ * N multiples of 128, K a multiple of 256 (one k-tile).  Workspace: at least
+ * FA4_WS_HEADER_BYTES (the bounded-wait status word).
  * Errors: SHAPE, ALIGN, INVALID_ARG, UNSUPPORTED, WORKSPACE, CUDA. */
 FA4_API fa4_status fa4_gemm_blockscaled(fa4_qtensor A, fa4_qtensor B, int64_t M, int64_t N, int64_t K,
                                 fa4_format fmt, float alpha, void *D, int64_t ldd,
