@@ -561,12 +561,21 @@ def fa4_arm(args, rank, world, device) -> dict | None:
                  for k, v in per_kind.items()}
     clocks = clk.summary()
 
+    # end to end on every rank (each GPU has its own host link): whole-job
+    # tokens/s from the slowest rank, like the device-timed value
+    e2e = e2e_run(fa, blk, max(2, min(args.steps, 5)), device)
+    e2e_ms = max_over_ranks(e2e["ms_per_step"], device)
+    e2e["ms_per_step"] = e2e_ms
+    e2e["tokens_per_s"] = whole_job_tokens_per_s(world, e2e_ms)
+    e2e["h2d_bytes_per_step"] *= world  # all ranks' copies, like the whole-job tokens
+    e2e["d2h_bytes_per_step"] *= world
     result = None
     if rank == 0:
-        sweep = quantize_sweep(fa, device) if not args.quick else []
-        gsweep = gemm_sweep(fa, device) if not args.quick else []
-        epiq = epilogue_quant_run(fa, device) if not args.quick else {}
-        e2e = e2e_run(fa, blk, max(2, min(args.steps, 5)), device)
+        # single-GPU microbenchmarks and the oracle baseline: one GPU only
+        solo = world == 1 and not args.quick
+        sweep = quantize_sweep(fa, device) if solo else []
+        gsweep = gemm_sweep(fa, device) if solo else []
+        epiq = epilogue_quant_run(fa, device) if solo else {}
         cpu = cpu_baseline() if (world == 1 and not args.no_cpu_baseline) else None
         tok_s = whole_job_tokens_per_s(world, ms_step)
         result = {
