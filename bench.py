@@ -344,6 +344,125 @@ def epilogue_quant_run(fa, device, reps: int = 10) -> dict:
     return res
 
 
+STACK_LAYERS = 32
+STACK_BF16_LAYERS = 4          # the last four blocks keep bf16 linears
+STACK_TOKENS = 2 * T           # sequence 8192 x batch 2
+
+
+def stack_run(fa, device, steps: int = 3, warmup: int = 3) -> dict:
+    """The linears of a 32-layer Llama-3-8B-shaped stack, forward then
+    backward, at 16384 tokens: layers 0-27 on the FP4 path (the block step's
+    calls), layers 28-31 as bf16 cuBLAS matmuls through torch.  Every layer
+    has its own seeded weights (FP4 layers keep only their quantized copies);
+    activations and gradients are one buffer per linear shape, shared by the
+    layers (each is larger than L2 or read beside others that are, so no
+    layer finds its inputs in L2).  No attention, normalisation or optimizer:
+    the stack's linears only."""
+    Ts = STACK_TOKENS
+    n_fp4 = STACK_LAYERS - STACK_BF16_LAYERS
+    ws = fa.workspace(1 << 16, device)
+    act = {}
+    for i, (name, (cin, cout)) in enumerate(LAYERS.items()):
+        a = dict(cin=cin, cout=cout,
+                 x=workloads.act(Ts, cin, seed=70000 + i, device=device),
+                 dy=workloads.grad(Ts, cout, seed=70010 + i, device=device))
+        a["xq"] = fa.empty_qtensor(Ts, cin, fa.NVFP4_GLOBAL, fa.ROWWISE, device)
+        a["xc"] = fa.empty_qtensor(Ts, cin, fa.MXFP4, fa.COLWISE, device)
+        a["gq"] = fa.empty_qtensor(Ts, cout, fa.MXFP4, fa.ROWWISE, device)
+        a["gc"] = fa.empty_qtensor(Ts, cout, fa.MXFP4, fa.COLWISE, device)
+        a["y"] = torch.empty(Ts, cout, dtype=torch.bfloat16, device=device)
+        a["dx"] = torch.empty(Ts, cin, dtype=torch.bfloat16, device=device)
+        a["dw"] = torch.empty(cout, cin, dtype=torch.float32, device=device)
+        a["dw16"] = torch.empty(cout, cin, dtype=torch.bfloat16, device=device)
+        act[name] = a
+    weights = []
+    t_wq = time.perf_counter()
+    for layer in range(STACK_LAYERS):
+        lw = {}
+        for i, (name, (cin, cout)) in enumerate(LAYERS.items()):
+            w = workloads.weight(cout, cin, seed=80000 + 10 * layer + i, device=device)
+            if layer < n_fp4:
+                lw[name] = (fa.quantize(w, fa.NVFP4_GLOBAL, fa.RNE, fa.ROWWISE, ws=ws),
+                            fa.quantize(w, fa.MXFP4, fa.RNE, fa.COLWISE, ws=ws))
+                del w
+            else:
+                lw[name] = w
+        weights.append(lw)
+    torch.cuda.synchronize()
+    t_wq = time.perf_counter() - t_wq
+
+    def fwd(layer):
+        for name, a in act.items():
+            if layer < n_fp4:
+                wq, _ = weights[layer][name]
+                fa.quantize_dual(a["x"], fa.NVFP4_GLOBAL, fa.RNE, 0, col_hadamard=True,
+                                 sign_mask=SIGN_MASK, row_out=a["xq"], col_out=a["xc"], ws=ws)
+                fa.gemm(a["xq"], wq, 1.0, out=a["y"], ws=ws)
+            else:
+                torch.matmul(a["x"], weights[layer][name].t(), out=a["y"])
+
+    def bwd(layer, seed):
+        for name, a in act.items():
+            if layer < n_fp4:
+                _, wc = weights[layer][name]
+                fa.quantize_dual(a["dy"], fa.MXFP4, fa.SR, seed, col_hadamard=True,
+                                 sign_mask=SIGN_MASK, row_out=a["gq"], col_out=a["gc"], ws=ws)
+                fa.gemm(a["gq"], wc, 1.0, out=a["dx"], ws=ws)
+                fa.gemm(a["gc"], a["xc"], 1.0 / 32, out=a["dw"], ws=ws)
+            else:
+                w = weights[layer][name]
+                torch.matmul(a["dy"], w, out=a["dx"])
+                torch.matmul(a["dy"].t(), a["x"], out=a["dw16"])
+
+    stream = torch.cuda.current_stream(device)
+    marks = []
+
+    def step(s, timed):
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(5)] if timed else None
+        if timed:
+            ev[0].record(stream)
+        for layer in range(STACK_LAYERS):
+            fwd(layer)
+            if timed and layer == n_fp4 - 1:
+                ev[1].record(stream)
+        if timed:
+            ev[2].record(stream)
+        for layer in reversed(range(STACK_LAYERS)):
+            bwd(layer, 1000003 * (s + 1) + layer)
+            if timed and layer == n_fp4:
+                ev[3].record(stream)
+        if timed:
+            ev[4].record(stream)
+            marks.append(ev)
+
+    for s in range(warmup):
+        step(s, False)
+    torch.cuda.synchronize()
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(device.index if device.index is not None else 0) as clk:
+        start.record(stream)
+        for s in range(steps):
+            step(warmup + s, True)
+        end.record(stream)
+        torch.cuda.synchronize()
+    if fa.check_device_status(ws) != 0:
+        raise RuntimeError("device status set during the stack run")
+    ms = start.elapsed_time(end) / steps
+    fp4_ms = sum(e[0].elapsed_time(e[1]) + e[3].elapsed_time(e[4]) for e in marks) / steps
+    bf16_ms = sum(e[1].elapsed_time(e[2]) + e[2].elapsed_time(e[3]) for e in marks) / steps
+    flop_layer = 3 * 2.0 * Ts * sum(cin * cout for cin, cout in LAYERS.values())
+    return {"workload": "llama3-8b-32-layer-linear-stack-fwd-bwd", "tokens": Ts,
+            "layers": STACK_LAYERS, "bf16_layers": f"{n_fp4}-{STACK_LAYERS - 1}",
+            "steps": steps, "warmup": warmup, "ms_per_step": round(ms, 3),
+            "tokens_per_s": round(Ts / (ms * 1e-3), 1),
+            "fp4_layers_ms": round(fp4_ms, 3),
+            "fp4_layers_TFLOPS": round(n_fp4 * flop_layer / (fp4_ms * 1e-3) / 1e12, 1),
+            "bf16_layers_ms": round(bf16_ms, 3),
+            "bf16_layers_TFLOPS": round(STACK_BF16_LAYERS * flop_layer / (bf16_ms * 1e-3) / 1e12, 1),
+            "weight_quantize_s": round(t_wq, 3), "clocks": clk.summary(),
+            "scope": "linears only (no attention, norms or optimizer); activations shared by layers"}
+
+
 def e2e_run(fa, blk: Block, steps: int, device) -> dict:
     """Same step through the public training-form linear calls
     (linear_fwd_save, linear_bwd) with host (pinned) inputs and outputs: the
@@ -576,6 +695,12 @@ def fa4_arm(args, rank, world, device) -> dict | None:
         sweep = quantize_sweep(fa, device) if solo else []
         gsweep = gemm_sweep(fa, device) if solo else []
         epiq = epilogue_quant_run(fa, device) if solo else {}
+        stack = {}
+        if solo or args.stack:
+            try:
+                stack = stack_run(fa, device)
+            except (RuntimeError, torch.cuda.OutOfMemoryError) as e:
+                stack = {"error": f"{type(e).__name__}: {e}"}
         cpu = cpu_baseline() if (world == 1 and not args.no_cpu_baseline) else None
         tok_s = whole_job_tokens_per_s(world, ms_step)
         result = {
@@ -600,7 +725,8 @@ def fa4_arm(args, rank, world, device) -> dict | None:
                         "weight_quantize_s": round(t_wq, 4),
                         "quantize_sweep": sweep,
                         "gemm_sweep": gsweep,
-                        "gemm_epilogue_mxfp4": epiq},
+                        "gemm_epilogue_mxfp4": epiq,
+                        "linear_stack": stack},
             "roofline": {"bound": "tensor", "achieved": round(dom_tflops, 1),
                          "peak": round(fp4_peak, 1), "unit": "TFLOP/s",
                          "frac": round(dom_tflops / fp4_peak, 4), "traffic": dominant_traffic(),
@@ -722,7 +848,10 @@ def main():
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", default="fa4", choices=["fa4", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--quick", action="store_true", help="skip the quantizer sweep")
+    ap.add_argument("--quick", action="store_true",
+                    help="skip the single-GPU sweeps and the 32-layer stack")
+    ap.add_argument("--stack", action="store_true",
+                    help="run the 32-layer linear stack even with --quick")
     ap.add_argument("--profile", default=None,
                     help="KIND:LAYER -- run only that call (for a single-kernel profiler capture)")
     args = ap.parse_args()
