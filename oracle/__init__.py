@@ -224,7 +224,7 @@ def ts_count(R: int, K: int, fmt: int) -> int:
     if fmt == NVFP4_GLOBAL:
         return 1
     if fmt == NVFP4_CTA:
-        return (R // 128) * (K // 128)
+        return -(-R // 128) * -(-K // 128)
     return 0
 
 
@@ -272,9 +272,9 @@ def dequantize(q: QTensor, rows=None) -> np.ndarray:
     if q.fmt == NVFP4_GLOBAL:
         d *= float(q.ts[0])
     elif q.fmt == NVFP4_CTA:
-        nk = q.K // 128
-        t = q.ts.reshape(q.R // 128, nk).astype(np.float64)
-        d *= np.repeat(t[r // 128], 128, axis=1)
+        nk = -(-q.K // 128)
+        t = q.ts.reshape(-(-q.R // 128), nk).astype(np.float64)
+        d *= np.repeat(t[r // 128], 128, axis=1)[:, :q.K]
     return d
 
 
@@ -307,9 +307,9 @@ def gemm_sampled(A: QTensor, B: QTensor, alpha: float = 1.0, m_idx=None, n_idx=N
     mi = np.arange(A.R) if m_idx is None else np.asarray(m_idx, dtype=np.int64)
     ni = np.arange(B.R) if n_idx is None else np.asarray(n_idx, dtype=np.int64)
     if A.fmt == NVFP4_CTA:
-        nk = A.K // 128
-        ta = A.ts.reshape(A.R // 128, nk).astype(np.float64)[mi // 128]  # [nm, nk]
-        tb = B.ts.reshape(B.R // 128, nk).astype(np.float64)[ni // 128]  # [nn, nk]
+        nk = -(-A.K // 128)  # the last chunk ends at K
+        ta = A.ts.reshape(-(-A.R // 128), nk).astype(np.float64)[mi // 128]  # [nm, nk]
+        tb = B.ts.reshape(-(-B.R // 128), nk).astype(np.float64)[ni // 128]  # [nn, nk]
         d = np.zeros((a.shape[0], b.shape[0]), dtype=np.float64)
         for kc in range(nk):
             s = a[:, kc * 128:(kc + 1) * 128] @ b[:, kc * 128:(kc + 1) * 128].T

@@ -378,7 +378,10 @@ void orc_hadamard32(const float *x, uint32_t sign_mask, float *y) {
 /* (1 for NVFP4-global, [R/128][K/128] for NVFP4-CTA-local, none for MX).    */
 /* NVFP4-CTA-local [FAF "The Design Philosophy..."] takes the second-level   */
 /* amax over the 128x128 tile of Q that holds the block (reading; the pages  */
-/* name only "CTA-local nvfp").                                             */
+/* name only "CTA-local nvfp"); tiles at a ragged edge (R or K not a        */
+/* multiple of 128) hold fewer values and take the amax of those, so ts is  */
+/* [ceil(R/128)][ceil(K/128)].  R may be any positive count; K must be a    */
+/* multiple of the block size (32 MX, 16 NV).                               */
 /* hadamard: apply orc_hadamard32 to each 32-value block before the scale    */
 /* (MXFP4 only).  SR bits use i = r*K + k.  Only rows [r_begin, r_end) of Q  */
 /* are produced (all when r_end <= 0), for sampled checks of large tensors.  */
@@ -406,15 +409,14 @@ int orc_quantize(const uint16_t *x, int64_t rows, int64_t cols, int64_t ld, int 
   int bs = ORC_IS_MX(fmt) ? 32 : 16;
   if (hadamard && fmt != ORC_MXFP4) return -1;
   if (K % bs != 0 || (K & 1)) return -1;
-  if (fmt == ORC_NVFP4_CTA && (R % 128 != 0 || K % 128 != 0)) return -1;
   int64_t kb_total = K / bs;
   memset(scales, 0, (size_t)orc_sf_bytes(R, kb_total));
   memset(payload, 0, (size_t)(R * (K / 2)));
 
   /* second-level amax for NVFP4: one encode scale for the tensor (global) or
      one per 128x128 tile of Q (CTA-local) */
-  int64_t n_tk = K / 128;
-  int64_t n_tiles = (fmt == ORC_NVFP4_CTA) ? (R / 128) * n_tk : 1;
+  int64_t n_tk = (K + 127) / 128;
+  int64_t n_tiles = (fmt == ORC_NVFP4_CTA) ? (R + 127) / 128 * n_tk : 1;
   float *s_enc = (float *)malloc(sizeof(float) * (size_t)n_tiles);
   if (!s_enc) return -2;
   s_enc[0] = 1.0f;
@@ -429,11 +431,11 @@ int orc_quantize(const uint16_t *x, int64_t rows, int64_t cols, int64_t ld, int 
     ts[0] = orc_nv_decode_scale(s_enc[0]);
   }
   if (fmt == ORC_NVFP4_CTA) {
-    for (int64_t tr = 0; tr < R / 128; ++tr)
+    for (int64_t tr = 0; tr < (R + 127) / 128; ++tr)
       for (int64_t tk = 0; tk < n_tk; ++tk) {
         float amax_t = 0.0f;
-        for (int64_t r = tr * 128; r < tr * 128 + 128; ++r)
-          for (int64_t k = tk * 128; k < tk * 128 + 128; ++k) {
+        for (int64_t r = tr * 128; r < tr * 128 + 128 && r < R; ++r)
+          for (int64_t k = tk * 128; k < tk * 128 + 128 && k < K; ++k) {
             float a = fabsf(q_elem(x, ld, orient, r, k));
             if (a > amax_t) amax_t = a;
           }
@@ -515,7 +517,8 @@ int orc_dequantize_blocks(const uint8_t *payload, const uint8_t *scales, int64_t
 /* with E2M1 codes and E8M0/E4M3 block scales every product has at most 12   */
 /* significant bits, so the block sums are exact.  NVFP4-global multiplies    */
 /* by ts_A*ts_B; NVFP4-CTA-local multiplies each 128-wide K chunk by         */
-/* ts_A[m/128][kc] * ts_B[n/128][kc].  Computes the rows/columns listed in   */
+/* ts_A[m/128][kc] * ts_B[n/128][kc] (the last chunk ends at K when K is    */
+/* not a multiple of 128).  Computes the rows/columns listed in              */
 /* m_idx/n_idx (all when NULL); out is [n_m][n_n] row-major.                 */
 /* ------------------------------------------------------------------------ */
 
@@ -530,7 +533,7 @@ int orc_gemm(const uint8_t *pa, const uint8_t *sa, const float *tsa, const uint8
     free(brow);
     return -2;
   }
-  int64_t nk = K / 128;
+  int64_t nk = (K + 127) / 128;
   for (int64_t i = 0; i < n_m; ++i) {
     int64_t m = m_idx ? m_idx[i] : i;
     if (m < 0 || m >= M || orc_dequantize_blocks(pa, sa, M, K, fmt, &m, 1, arow) != 0) {
@@ -550,7 +553,7 @@ int orc_gemm(const uint8_t *pa, const uint8_t *sa, const float *tsa, const uint8
         d = 0.0;
         for (int64_t kc = 0; kc < nk; ++kc) {
           double s = 0.0;
-          for (int64_t k = kc * 128; k < kc * 128 + 128; ++k) s += arow[k] * brow[k];
+          for (int64_t k = kc * 128; k < kc * 128 + 128 && k < K; ++k) s += arow[k] * brow[k];
 #ifdef PLANT_CTA_TILE_INDEX
           d += (double)tsa[(m / 128) * nk + kc] * (double)tsb[(m / 128) * nk + kc] * s;
 #else

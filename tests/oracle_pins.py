@@ -376,11 +376,16 @@ def _check_quant_bounds(x: torch.Tensor, q: O.QTensor, fmt: int, orient: int,
             ts = np.full((R, K // bs), float(q.ts[0]))
             assert abs(float(q.ts[0]) * 2688.0 - amax_t) <= 3 * np.spacing(np.float32(amax_t)) or amax_t == 0
         else:
-            t = q.ts.reshape(R // 128, K // 128).astype(np.float64)
-            tile_amax = np.abs(Q).reshape(R // 128, 128, K // 128, 128).max(axis=(1, 3))
+            # 128x128 tiles; those at a ragged edge hold fewer values (zero
+            # padding leaves a tile's amax unchanged)
+            nr, nk = -(-R // 128), -(-K // 128)
+            t = q.ts.reshape(nr, nk).astype(np.float64)
+            Qa = np.zeros((nr * 128, nk * 128))
+            Qa[:R, :K] = np.abs(Q)
+            tile_amax = Qa.reshape(nr, 128, nk, 128).max(axis=(1, 3))
             nz = tile_amax > 0
             assert np.all(np.abs(t[nz] * 2688.0 - tile_amax[nz]) <= 3 * np.spacing(tile_amax[nz].astype(np.float32)))
-            ts = np.repeat(np.repeat(t, 128, axis=0), 128 // bs, axis=1)
+            ts = np.repeat(np.repeat(t, 128, axis=0), 128 // bs, axis=1)[:R, :K // bs]
         eff_b = sv * ts
         live = amax_b > 2 ** -9 * 448 * 6 * ts * 1.01 / 448  # not clamped at the bottom
         rel = np.abs(eff_b[live] - amax_b[live] / 6.0) / (amax_b[live] / 6.0)
@@ -481,6 +486,51 @@ def pin_packing():
     assert q.scales[O.sf_offset(0, 0, 4)] == 127  # 6 -> exponent 0
 
 
+def _valid_scale_offsets(R: int, kb_total: int) -> np.ndarray:
+    return np.array([O.sf_offset(r, k, kb_total) for r in range(R) for k in range(kb_total)])
+
+
+def pin_quantize_ragged():
+    """Row counts that are not a multiple of 128 and K that is not a multiple
+    of 128 (MX/NV blocks still whole): the closed-form bounds hold, and the
+    result equals the valid part of the same tensor zero-padded to whole
+    128x128 tiles -- zero rows and columns change no block, tensor or tile
+    amax.  Scale bytes outside the valid rows and blocks are zero."""
+    for (R, K) in ((200, 352), (1, 96), (129, 160)):
+        x = workloads.sweep(max(R, 2), K, seed=R + K)[:R].contiguous()
+        Rp, Kp = -(-R // 128) * 128, -(-K // 128) * 128
+        xp = torch.zeros(Rp, Kp, dtype=torch.bfloat16)
+        xp[:R, :K] = x
+        xr = torch.zeros(Rp, K, dtype=torch.bfloat16)  # rows padded only: same SR indices
+        xr[:R] = x
+        for fmt in (O.MXFP4, O.MXFP4_NOCLIP, O.NVFP4_GLOBAL, O.NVFP4_CTA):
+            bs = O.BLOCK[fmt]
+            q = O.quantize(x, fmt, O.RNE, O.ROWWISE)
+            if fmt != O.MXFP4_NOCLIP:
+                _check_quant_bounds(x, q, fmt, O.ROWWISE)
+            assert q.payload.shape == (R, K // 2)
+            assert q.scales.size == Rp * (-(-(K // bs) // 4) * 4)
+            assert q.ts.size == (0 if O.BLOCK[fmt] == 32 else O.ts_count(R, K, fmt))
+            valid = _valid_scale_offsets(R, K // bs)
+            pad = np.setdiff1d(np.arange(q.scales.size), valid)
+            assert np.all(q.scales[pad] == 0)
+            for xpad, rnd in ((xp, O.RNE), (xr, O.SR)):
+                p = O.quantize(xpad, fmt, rnd, O.ROWWISE, seed=5)
+                g = q if rnd == O.RNE else O.quantize(x, fmt, O.SR, O.ROWWISE, seed=5)
+                assert np.array_equal(g.payload, p.payload[:R, :K // 2]), (R, K, fmt, rnd)
+                Kbp = xpad.shape[1] // bs
+                vp = np.array([O.sf_offset(r, k, Kbp) for r in range(R) for k in range(K // bs)])
+                assert np.array_equal(g.scales[valid], p.scales[vp]), (R, K, fmt, rnd)
+                assert np.array_equal(g.ts, p.ts), (R, K, fmt, rnd)
+        # column-wise: the token dimension K of the quantized operand is ragged
+        xc = workloads.sweep(K, max(R, 2), seed=7)[:, :R].contiguous()
+        for fmt in (O.MXFP4, O.NVFP4_CTA):
+            a = O.quantize(xc, fmt, O.RNE, O.COLWISE)
+            b = O.quantize(xc.t().contiguous(), fmt, O.RNE, O.ROWWISE)
+            assert np.array_equal(a.payload, b.payload) and np.array_equal(a.scales, b.scales)
+            assert np.array_equal(a.ts, b.ts)
+
+
 # ------------------------------------------------------------------ GEMM ---
 
 def pin_gemm_bruteforce():
@@ -507,6 +557,31 @@ def pin_gemm_bruteforce():
                     assert abs(got[i, j] - want) <= 1e-12 * max(1.0, abs(want)), (fmt, K, i, j)
             # and the large-shape helper agrees
             assert np.allclose(O.gemm_sampled(A, B, alpha, mi, ni), got, rtol=1e-13, atol=0)
+
+
+def pin_gemm_ragged():
+    """M, N and K that are not multiples of 128: the GEMM equals the valid
+    block of the GEMM of the zero-padded operands (binary64 sums are exact,
+    so equality is exact), and exact rational brute force on sampled entries."""
+    rng = np.random.default_rng(23)
+    for fmt in (O.MXFP4, O.NVFP4_GLOBAL, O.NVFP4_CTA):
+        M, N, K = 200, 72, 352
+        xa = torch.from_numpy(rng.standard_normal((M, K)).astype(np.float32)).to(torch.bfloat16)
+        xb = torch.from_numpy((rng.standard_normal((N, K)) * 3).astype(np.float32)).to(torch.bfloat16)
+        xb[:, 300:] *= 50.0  # the ragged last K chunk gets its own tile scale
+        pa = torch.zeros(256, 384, dtype=torch.bfloat16)
+        pb = torch.zeros(128, 384, dtype=torch.bfloat16)
+        pa[:M, :K], pb[:N, :K] = xa, xb
+        A, B = O.quantize(xa, fmt), O.quantize(xb, fmt)
+        d = O.gemm(A, B, 0.5)
+        dp = O.gemm(O.quantize(pa, fmt), O.quantize(pb, fmt), 0.5)
+        assert np.array_equal(d, dp[:M, :N]), fmt
+        assert np.array_equal(O.gemm_sampled(A, B, 0.5), d), fmt
+        da, db = O.dequantize(A, [0, 199]), O.dequantize(B, [3, 71])
+        for i, m in enumerate((0, 199)):
+            for j, n in enumerate((3, 71)):
+                s = sum(Fraction(float(da[i, k])) * Fraction(float(db[j, k])) for k in range(K))
+                assert abs(d[m, n] - float(Fraction(1, 2) * s)) <= 1e-12 * max(1.0, abs(d[m, n]))
 
 
 def pin_gemm_approximates_matmul():
@@ -563,5 +638,6 @@ def pin_philox_structure():
 ALL_PINS = [pin_e2m1_decode, pin_e2m1_rne, pin_e2m1_sr, pin_e4m3, pin_mx_exponent,
             pin_mx_exponent_noclip, pin_nv_scales,
             pin_hadamard, pin_swizzle, pin_quantize_rne, pin_quantize_sr, pin_quantize_orientation,
-            pin_quantize_hadamard, pin_packing, pin_gemm_bruteforce, pin_gemm_approximates_matmul,
+            pin_quantize_hadamard, pin_packing, pin_quantize_ragged, pin_gemm_bruteforce,
+            pin_gemm_ragged, pin_gemm_approximates_matmul,
             pin_philox_structure]
