@@ -20,6 +20,13 @@
 // epilogue warps fold, tsA[m/128][kc] * tsB[n/128][kc] * partial, into FP32
 // registers as soon as the chunk's MMAs complete.
 //
+// Ragged shapes (M, N any; K a multiple of 32): the grid covers whole tiles;
+// TMA reads zeros for payload outside A and B, scale atoms that the operands
+// do not have (past the last 128-row block, or past the last atom along K)
+// are staged as zero bytes, and the stores skip what lies outside D.  Zero
+// payload times a finite scale adds nothing, so the padded tile computes
+// the exact result of the smaller one.
+//
 // Every mbarrier wait is bounded: past `timeout_ns` the waiting thread sets
 // the device status word, raises a CTA-wide abort flag and leaves its loop;
 // the CTA then waits (bounded) for its own copies in flight, frees its
@@ -182,6 +189,9 @@ struct Params {
   // (payload [M, N/2], scales in the 128x4 atom layout); null: none
   uint8_t *q_payload, *q_scales;
   int store_d;  // 0: D is not written (only the quantized operand)
+  // ragged shapes: some tile reaches past M, N or K (see the file comment)
+  int ragged;
+  int64_t rb_a, rb_b;  // 128-row blocks of A and B (atom rows of their scales)
 };
 
 // Output tile coordinates of linear tile index t.  Concurrently running CTAs
@@ -476,10 +486,11 @@ __global__ void __launch_bounds__(NUM_THREADS_ST, 1)
   const int unit = PAIR ? (int)(blockIdx.x >> 1) : (int)blockIdx.x;      // tile-walking unit
   const int nunits = PAIR ? (int)(gridDim.x >> 1) : (int)gridDim.x;
 
-  const int num_m = (int)(p.M / CS::TILE_M), num_n = (int)(p.N / BN);
+  const int num_m = (int)((p.M + CS::TILE_M - 1) / CS::TILE_M);
+  const int num_n = (int)((p.N + BN - 1) / BN);
   const int num_tiles = num_m * num_n;
-  const int KT = (int)(p.K / BK);
-  const int64_t kbt4 = (p.K / C::BS) / 4;
+  const int KT = (int)((p.K + BK - 1) / BK);
+  const int64_t kbt4 = (p.K / C::BS + 3) / 4;  // atoms along K per 128-row block
   const int my_tiles = unit < num_tiles ? (num_tiles - unit + nunits - 1) / nunits : 0;
   const int total = my_tiles * KT;  // k-tiles this CTA processes
 
@@ -596,15 +607,37 @@ __global__ void __launch_bounds__(NUM_THREADS_ST, 1)
             break;
           }
           const uint32_t fb = smem_u32(&sm->sfs_full[s]);
-          mbar_arrive_expect_tx(fb, CS::SF_BYTES);
           const uint32_t dst = smem_u32(smem + CS::OFF_SF + s * CS::SF_BYTES);
-          bulk_load(dst, p.a_scales + ((int64_t)rb_a * kbt4 + (int64_t)kt * C::ATOMS_K) * 512,
-                    CS::SFA_BYTES, fb);
+          if (!p.ragged) {
+            mbar_arrive_expect_tx(fb, CS::SF_BYTES);
+            bulk_load(dst, p.a_scales + ((int64_t)rb_a * kbt4 + (int64_t)kt * C::ATOMS_K) * 512,
+                      CS::SFA_BYTES, fb);
 #pragma unroll
-          for (int nb = 0; nb < BN / 128; ++nb)
-            bulk_load(dst + CS::SFA_BYTES + nb * C::SFA_BYTES,
-                      p.b_scales + ((int64_t)(nt * (BN / 128) + nb) * kbt4 + (int64_t)kt * C::ATOMS_K) * 512,
-                      C::SFA_BYTES, fb);
+            for (int nb = 0; nb < BN / 128; ++nb)
+              bulk_load(dst + CS::SFA_BYTES + nb * C::SFA_BYTES,
+                        p.b_scales + ((int64_t)(nt * (BN / 128) + nb) * kbt4 + (int64_t)kt * C::ATOMS_K) * 512,
+                        C::SFA_BYTES, fb);
+          } else {
+            // only the atoms the operands have: na along K, and no 128-row
+            // block past the last one (at least B's first block exists)
+            const int64_t left = kbt4 - (int64_t)kt * C::ATOMS_K;
+            const uint32_t bytes = (uint32_t)(left < C::ATOMS_K ? left : C::ATOMS_K) * 512u;
+            const bool a_in = rb_a < p.rb_a;
+            uint32_t total_bytes = a_in ? bytes : 0u;
+#pragma unroll
+            for (int nb = 0; nb < BN / 128; ++nb)
+              if (nt * (BN / 128) + nb < p.rb_b) total_bytes += bytes;
+            mbar_arrive_expect_tx(fb, total_bytes);
+            if (a_in)
+              bulk_load(dst, p.a_scales + ((int64_t)rb_a * kbt4 + (int64_t)kt * C::ATOMS_K) * 512,
+                        bytes, fb);
+#pragma unroll
+            for (int nb = 0; nb < BN / 128; ++nb)
+              if (nt * (BN / 128) + nb < p.rb_b)
+                bulk_load(dst + CS::SFA_BYTES + nb * C::SFA_BYTES,
+                          p.b_scales + ((int64_t)(nt * (BN / 128) + nb) * kbt4 + (int64_t)kt * C::ATOMS_K) * 512,
+                          bytes, fb);
+          }
           issued |= 1u << s;
           last_parity = (last_parity & ~(1u << s)) | (ph << s);
         }
@@ -718,17 +751,37 @@ __global__ void __launch_bounds__(NUM_THREADS_ST, 1)
       const uint8_t *sfa_s = smem + CS::OFF_SF + s * CS::SF_BYTES;
       const uint8_t *sfb_s = sfa_s + CS::SFA_BYTES;
       const uint32_t col = lane_base + SF_BASE + b * CS::COLS_BUF;
+      // ragged shapes: atoms the scale producer did not load are zero
+      int na = C::ATOMS_K;
+      bool a_in = true, b_in[BN / 128];
+#pragma unroll
+      for (int nb = 0; nb < BN / 128; ++nb) b_in[nb] = true;
+      if (p.ragged) {
+        const int kt = g % KT;
+        int mt, nt;
+        tile_coords(unit + (g / KT) * nunits, num_m, num_n, p.n_fastest, mt, nt);
+        const int64_t left = kbt4 - (int64_t)kt * C::ATOMS_K;
+        na = left < C::ATOMS_K ? (int)left : C::ATOMS_K;
+        a_in = (PAIR ? mt * 2 + (int)rank : mt) < p.rb_a;
+#pragma unroll
+        for (int nb = 0; nb < BN / 128; ++nb) b_in[nb] = nt * (BN / 128) + nb < p.rb_b;
+      }
       // A: row 32q + lane is word q of atom row `lane`
 #pragma unroll
       for (int a = 0; a < C::ATOMS_K; ++a)
-        tmem_st1(col + 4 * a + q, *reinterpret_cast<const uint32_t *>(sfa_s + a * 512 + lane * 16 + 4 * q));
+        tmem_st1(col + 4 * a + q,
+                 (a_in && a < na)
+                     ? *reinterpret_cast<const uint32_t *>(sfa_s + a * 512 + lane * 16 + 4 * q)
+                     : 0u);
       // B: atom a of each 128-row block: row 32w + lane is word w of atom row `lane`
 #pragma unroll
       for (int a = 0; a < C::ATOMS_K; ++a) {
 #pragma unroll
         for (int nb = 0; nb < BN / 128; ++nb)
           tmem_st4(col + CS::COLS_A + (BN / 32) * a + 4 * nb,
-                   *reinterpret_cast<const uint4 *>(sfb_s + nb * C::SFA_BYTES + a * 512 + lane * 16));
+                   (b_in[nb] && a < na)
+                       ? *reinterpret_cast<const uint4 *>(sfb_s + nb * C::SFA_BYTES + a * 512 + lane * 16)
+                       : make_uint4(0u, 0u, 0u, 0u));
       }
       asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
       tc_fence_before();
@@ -755,9 +808,13 @@ __global__ void __launch_bounds__(NUM_THREADS_ST, 1)
       const int x0 = nt * BN + h * COLS;
       const uint32_t row_base = ebuf + lane * 64;
       const int sw = (lane >> 1) & 3;
+      // ragged shapes: these 32 rows may lie wholly below D (the bulk-tensor
+      // store clips a box that only reaches past M or N)
+      const bool rows_in = !p.ragged || (int64_t)y0 < p.M;
       if (p.out_fp32) {
 #pragma unroll
         for (int ch = 0; ch < COLS / 16; ++ch) {
+          if (p.ragged && (!rows_in || (int64_t)(x0 + 16 * ch) >= p.N)) continue;
           if (lane == 0) bulk_wait_read_all();
           __syncwarp();
 #pragma unroll
@@ -780,6 +837,7 @@ __global__ void __launch_bounds__(NUM_THREADS_ST, 1)
         uint32_t sword = 0;  // this row's MXFP4 scale bytes, one per 32-column chunk
 #pragma unroll
         for (int ch = 0; ch < COLS / 32; ++ch) {
+          const bool chunk_in = !p.ragged || (rows_in && (int64_t)(x0 + 32 * ch) < p.N);
           uint32_t w[16];  // the chunk's 32 bf16 values of D, packed in pairs
 #pragma unroll
           for (int u = 0; u < 16; ++u) {
@@ -805,11 +863,13 @@ __global__ void __launch_bounds__(NUM_THREADS_ST, 1)
             for (int e = 0; e < 32; ++e) f[e] = __fmul_rn(f[e], mult);
             const uint4 codes = make_uint4(e2m1x8_rne(&f[0]), e2m1x8_rne(&f[8]),
                                            e2m1x8_rne(&f[16]), e2m1x8_rne(&f[24]));
-            *reinterpret_cast<uint4 *>(p.q_payload + row * (p.N >> 1) + ((x0 + 32 * ch) >> 1)) =
-                codes;
+            // rows and blocks outside D hold zero accumulators: scale byte 0
+            if (!p.ragged || (row < p.M && (int64_t)(x0 + 32 * ch) < p.N))
+              *reinterpret_cast<uint4 *>(p.q_payload + row * (p.N >> 1) + ((x0 + 32 * ch) >> 1)) =
+                  codes;
             sword |= sbyte << (8 * ch);
           }
-          if (p.store_d) {
+          if (p.store_d && chunk_in) {
             if (lane == 0) bulk_wait_read_all();
             __syncwarp();
 #pragma unroll
@@ -825,12 +885,17 @@ __global__ void __launch_bounds__(NUM_THREADS_ST, 1)
         }
         if constexpr (QOUT) {
           // blocks x0/32 .. of this row: a whole scale word (128 columns) or
-          // its half (64 columns, the other half is the quadrant's other warp)
-          uint8_t *sdst = p.q_scales + sf_offset(row, x0 >> 5, p.N >> 5);
-          if constexpr (COLS == 128)
-            *reinterpret_cast<uint32_t *>(sdst) = sword;
-          else
-            *reinterpret_cast<uint16_t *>(sdst) = (uint16_t)sword;
+          // its half (64 columns, the other half is the quadrant's other warp);
+          // ragged: rows up to the next multiple of 128 and blocks up to the
+          // next multiple of 4 are the operand's padding (written, zero)
+          const int64_t nbk = p.N >> 5;
+          if (!p.ragged || (row < p.rb_a * 128 && (int64_t)(x0 >> 5) < nbk)) {
+            uint8_t *sdst = p.q_scales + sf_offset(row, x0 >> 5, (nbk + 3) & ~int64_t(3));
+            if constexpr (COLS == 128)
+              *reinterpret_cast<uint32_t *>(sdst) = sword;
+            else
+              *reinterpret_cast<uint16_t *>(sdst) = (uint16_t)sword;
+          }
         }
       }
     };
@@ -840,7 +905,7 @@ __global__ void __launch_bounds__(NUM_THREADS_ST, 1)
       // k-tiles ahead, then fold both 128-K chunk partials into FP32
       // registers, acc += tsA[m/128][kc] * tsB[n/128][kc] * partial, and
       // release each partial as soon as it is read; store at the tile's end
-      const int nk = (int)(p.K / 128);
+      const int nk = (int)((p.K + 127) / 128);  // 128-wide K chunks (the last may be short)
       int g_st = h, g = 0;
       bool ok = true;
       for (int tile = unit; tile < num_tiles && ok; tile += nunits) {
@@ -872,7 +937,9 @@ __global__ void __launch_bounds__(NUM_THREADS_ST, 1)
             __syncwarp();
             if (lane == 0) mbar_arrive(smem_u32(&sm->part_empty[c]));
             const int kc = 2 * kt + c;
-            const float f = p.a_ts[(int64_t)mt * nk + kc] * p.b_ts[(int64_t)nt * nk + kc];
+            // a chunk wholly past K (ragged) holds a zero partial and no scale
+            const float f = kc < nk ? p.a_ts[(int64_t)mt * nk + kc] * p.b_ts[(int64_t)nt * nk + kc]
+                                    : 0.0f;
 #pragma unroll
             for (int i = 0; i < COLS; ++i) acc[i] = fmaf(f, __uint_as_float(r[i]), acc[i]);
           }
@@ -1020,6 +1087,9 @@ static gemm::Params make_params(const GemmArgs &a) {
   p.q_payload = a.q_payload;
   p.q_scales = a.q_scales;
   p.store_d = a.D != nullptr;
+  p.rb_a = (a.M + 127) / 128;
+  p.rb_b = (a.N + 127) / 128;
+  p.ragged = 0;  // set by the launcher for its tile shape
   return p;
 }
 
@@ -1033,13 +1103,15 @@ static cudaError_t launch_st(const GemmArgs &a, cudaStream_t st) {
   memset(&md, 0, sizeof(md));
   if (a.D && !make_out_map(&md, a)) return cudaErrorInvalidValue;
   gemm::Params p = make_params(a);
+  constexpr int TILE_M = PAIR ? 256 : gemm::BM;
+  p.ragged = (a.M % TILE_M) || (a.N % BN) || (a.K % gemm::BK);
   auto kern = gemm_st::gemm_st_kernel<KIND, BN, PAIR, QOUT>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  const int64_t tiles = (a.M / (PAIR ? 256 : gemm::BM)) * (a.N / BN);
+  const int64_t tiles = ((a.M + TILE_M - 1) / TILE_M) * ((a.N + BN - 1) / BN);
   cudaLaunchConfig_t cfg = {};
   cfg.blockDim = dim3(gemm_st::NUM_THREADS_ST);
   cfg.dynamicSmemBytes = smem;
@@ -1070,8 +1142,11 @@ static cudaError_t launch_st(const GemmArgs &a, cudaStream_t st) {
 
 template <bool QOUT>
 static cudaError_t launch_st_any(const GemmArgs &a, cudaStream_t st) {
-  const bool wide = (a.N % 256) == 0;
-  const bool pair = wide && (a.M % 256) == 0;
+  // 256-wide tiles (and 256-row pairs) where they cover no more than
+  // 128-wide (128-row) tiles would
+  auto up = [](int64_t v, int64_t m) { return (v + m - 1) / m * m; };
+  const bool wide = up(a.N, 256) == up(a.N, 128);
+  const bool pair = wide && up(a.M, 256) == up(a.M, 128);
   if (a.fmt == kMX)
     return pair ? launch_st<kMX, 256, true, QOUT>(a, st)
                 : (wide ? launch_st<kMX, 256, false, QOUT>(a, st) : launch_st<kMX, 128, false, QOUT>(a, st));
