@@ -1022,16 +1022,18 @@ using PFN_encodeTiled = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint3
                                      const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
                                      CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
 
+// The driver's tensor-map encoder, looked up once (a function-local static
+// is initialised exactly once even when several host threads call first).
 static PFN_encodeTiled get_encode() {
-  static PFN_encodeTiled fn = nullptr;
-  if (!fn) {
+  static const PFN_encodeTiled fn = []() -> PFN_encodeTiled {
     void *ptr = nullptr;
     cudaDriverEntryPointQueryResult q;
     if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
             cudaSuccess &&
         q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<PFN_encodeTiled>(ptr);
-  }
+      return reinterpret_cast<PFN_encodeTiled>(ptr);
+    return nullptr;
+  }();
   return fn;
 }
 

@@ -35,8 +35,11 @@
  *    status word that bounded waits inside the kernels set on timeout.  The
  *    caller zero-fills the workspace (or calls fa4_workspace_init) once
  *    before first use; fa4_check_device_status reads and clears the word.
- *  - Thread-safe: no global mutable state except a mutex-guarded cache of
- *    TMA descriptors keyed by pointer and shape.
+ *  - Thread-safe: tensor-memory-access descriptors are encoded on the host
+ *    for every call and passed by value to the kernel; the only global state
+ *    is the driver entry point looked up once and, for
+ *    fa4_quantize_nvfp4_global_noalloc, a mutex-guarded per-device pointer
+ *    to its static scratch array.
  */
 #ifndef FA4_H
 #define FA4_H
