@@ -249,15 +249,18 @@ __global__ void __launch_bounds__(256) quant_rowwise_kernel(
 // conflicts) and keeping all 64 values in registers, so the optional
 // Hadamard-32 is an in-register butterfly.
 // --------------------------------------------------------------------------
-__device__ __forceinline__ void fwht32(float *v) {
+// In-place butterfly with strides 1, 2, 4, 8, 16, (a, b) -> (a + b, a - b),
+// on packed pairs: lane lo and lane hi are two independent 32-value blocks
+// (two channels) taking the same steps.
+__device__ __forceinline__ void fwht32x2(uint64_t *v) {
 #pragma unroll
   for (int h = 1; h < 32; h <<= 1) {
 #pragma unroll
     for (int i = 0; i < 32; ++i) {
       if ((i & h) == 0) {
-        const float a = v[i], b = v[i + h];
-        v[i] = __fadd_rn(a, b);
-        v[i + h] = __fsub_rn(a, b);
+        const uint64_t a = v[i], b = v[i + h];
+        v[i] = f2_add(a, b);
+        v[i + h] = f2_sub(a, b);
       }
     }
   }
@@ -277,40 +280,48 @@ __device__ __forceinline__ void colwise_tile(const uint16_t *tile, uint8_t *sbuf
   const int w = threadIdx.x >> 5, l = threadIdx.x & 31;
   const int p = (w & 1) * 32 + l;  // channel pair within the tile: 2p, 2p+1
   const int j = w >> 1;            // 32-token block within the tile
-  float v0[32], v1[32];
+  float v0[32], v1[32];  // channels 2p and 2p+1
+  if constexpr (HAD) {
+    // the two channels' blocks take the same signs and butterfly: run them
+    // as packed pairs; a sign is the bf16 sign bit, flipped before widening
+    uint64_t w2[32];
 #pragma unroll
-  for (int t = 0; t < 32; ++t) {
-    const uint32_t pair = *reinterpret_cast<const uint32_t *>(&tile[(32 * j + t) * 128 + 2 * p]);
-    v0[t] = bf16lo(pair);
-    v1[t] = bf16hi(pair);
+    for (int t = 0; t < 32; ++t) {
+      uint32_t pair = *reinterpret_cast<const uint32_t *>(&tile[(32 * j + t) * 128 + 2 * p]);
+      if ((sign_mask >> t) & 1u) pair ^= 0x80008000u;
+      w2[t] = f2_pack(bf16lo(pair), bf16hi(pair));
+    }
+    fwht32x2(w2);
+#pragma unroll
+    for (int t = 0; t < 32; ++t) f2_unpack(w2[t], v0[t], v1[t]);
+  } else {
+#pragma unroll
+    for (int t = 0; t < 32; ++t) {
+      const uint32_t pair = *reinterpret_cast<const uint32_t *>(&tile[(32 * j + t) * 128 + 2 * p]);
+      v0[t] = bf16lo(pair);
+      v1[t] = bf16hi(pair);
+    }
   }
   const int64_t kb = is_mx<FMT>() ? (T >> 5) : (T >> 4);  // blocks per row of Q
   // blocks per atom row: padded to a multiple of 4 (already one unless EDGE)
   const int64_t kbt = EDGE ? ((kb + 3) & ~int64_t(3)) : kb;
 
+  // block scales of both channels (MX: one 32-block each; NV: two 16-blocks
+  // each, multiplier mult[half][hb])
+  const int64_t kfirst = t0 + 32 * j;  // first K index of this 32-block
+  float mult[2][2];
 #pragma unroll
   for (int half = 0; half < 2; ++half) {
-    float *v = half ? v1 : v0;
+    const float *v = half ? v1 : v0;
     const int cl = 2 * p + half;  // channel within the tile
-    const int64_t r = c0 + cl;
     // the thread's 32-token block is wholly inside or outside (T % 32 == 0)
-    const bool inside = !EDGE || (r < C && t0 + 32 * j < T);
-    if constexpr (HAD) {
-#pragma unroll
-      for (int t = 0; t < 32; ++t)
-        if ((sign_mask >> t) & 1u) v[t] = -v[t];
-      fwht32(v);
-    }
-    uint32_t codes[4];
-    const int64_t kfirst = t0 + 32 * j;  // first K index of this 32-block
+    const bool inside = !EDGE || (c0 + cl < C && kfirst < T);
     if constexpr (is_mx<FMT>()) {
       float amax = 0.0f;
 #pragma unroll
       for (int t = 0; t < 32; ++t) amax = fmaxf(amax, fabsf(v[t]));
       const uint32_t sbyte = mx_byte<FMT>(amax);
-      const float mult = mx_multiplier(sbyte);
-#pragma unroll
-      for (int t = 0; t < 32; ++t) v[t] = __fmul_rn(v[t], mult);
+      mult[half][0] = mult[half][1] = mx_multiplier(sbyte);
       sbuf[cl * 8 + j] = (EDGE && !inside) ? (uint8_t)0 : (uint8_t)sbyte;
     } else {
 #pragma unroll
@@ -318,13 +329,24 @@ __device__ __forceinline__ void colwise_tile(const uint16_t *tile, uint8_t *sbuf
         float amax = 0.0f;
 #pragma unroll
         for (int t = 0; t < 16; ++t) amax = fmaxf(amax, fabsf(v[16 * hb + t]));
-        float mult;
-        const uint32_t sbyte = nv_block_scale(amax, s_enc, &mult);
-#pragma unroll
-        for (int t = 0; t < 16; ++t) v[16 * hb + t] = __fmul_rn(v[16 * hb + t], mult);
+        const uint32_t sbyte = nv_block_scale(amax, s_enc, &mult[half][hb]);
         sbuf[cl * 8 + 2 * j + hb] = (EDGE && !inside) ? (uint8_t)0 : (uint8_t)sbyte;
       }
     }
+  }
+  // y = x * multiplier, both channels at once
+#pragma unroll
+  for (int t = 0; t < 32; ++t)
+    f2_unpack(f2_mul(f2_pack(v0[t], v1[t]), f2_pack(mult[0][t >> 4], mult[1][t >> 4])), v0[t],
+              v1[t]);
+
+#pragma unroll
+  for (int half = 0; half < 2; ++half) {
+    float *v = half ? v1 : v0;
+    const int cl = 2 * p + half;  // channel within the tile
+    const int64_t r = c0 + cl;
+    const bool inside = !EDGE || (r < C && kfirst < T);
+    uint32_t codes[4];
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
       if constexpr (RND == kSR) {
