@@ -915,6 +915,15 @@ __global__ void __launch_bounds__(NUM_THREADS_ST, 1)
 #pragma unroll
         for (int i = 0; i < COLS; ++i) acc[i] = 0.0f;
         for (int kt = 0; kt < KT && ok; ++kt, ++g) {
+          // the two chunks' factors, loaded before the waits below so that
+          // their global-memory latency overlaps them (a chunk wholly past K,
+          // ragged, holds a zero partial and gets no scale)
+          float fk[2];
+#pragma unroll
+          for (int c = 0; c < 2; ++c) {
+            const int kc = 2 * kt + c;
+            fk[c] = kc < nk ? p.a_ts[(int64_t)mt * nk + kc] * p.b_ts[(int64_t)nt * nk + kc] : 0.0f;
+          }
           for (; g_st < total && g_st < g + NBUF; g_st += 2)
             if (!stage_scales(g_st)) {
               ok = false;
@@ -936,10 +945,7 @@ __global__ void __launch_bounds__(NUM_THREADS_ST, 1)
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(smem_u32(&sm->part_empty[c]));
-            const int kc = 2 * kt + c;
-            // a chunk wholly past K (ragged) holds a zero partial and no scale
-            const float f = kc < nk ? p.a_ts[(int64_t)mt * nk + kc] * p.b_ts[(int64_t)nt * nk + kc]
-                                    : 0.0f;
+            const float f = fk[c];
 #pragma unroll
             for (int i = 0; i < COLS; ++i) acc[i] = fmaf(f, __uint_as_float(r[i]), acc[i]);
           }
