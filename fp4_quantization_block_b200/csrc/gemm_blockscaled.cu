@@ -911,9 +911,11 @@ __global__ void __launch_bounds__(NUM_THREADS_ST, 1)
       for (int tile = unit; tile < num_tiles && ok; tile += nunits) {
         int mt, nt;
         tile_coords(tile, num_m, num_n, p.n_fastest, mt, nt);
-        float acc[COLS];
+        // packed pairs of accumulator columns (2i, 2i+1): one fma.rn.f32x2
+        // folds both, the same rounding as fmaf on each
+        uint64_t acc2[COLS / 2];
 #pragma unroll
-        for (int i = 0; i < COLS; ++i) acc[i] = 0.0f;
+        for (int i = 0; i < COLS / 2; ++i) acc2[i] = 0ull;
         for (int kt = 0; kt < KT && ok; ++kt, ++g) {
           // the two chunks' factors, loaded before the waits below so that
           // their global-memory latency overlaps them (a chunk wholly past K,
@@ -945,15 +947,16 @@ __global__ void __launch_bounds__(NUM_THREADS_ST, 1)
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(smem_u32(&sm->part_empty[c]));
-            const float f = fk[c];
+            const uint64_t f2 = f2_pack(fk[c], fk[c]);
 #pragma unroll
-            for (int i = 0; i < COLS; ++i) acc[i] = fmaf(f, __uint_as_float(r[i]), acc[i]);
+            for (int i = 0; i < COLS / 2; ++i)
+              acc2[i] = f2_fma(f2, f2_pack_bits(r[2 * i], r[2 * i + 1]), acc2[i]);
           }
         }
         if (!ok) break;
         uint32_t r[COLS];
 #pragma unroll
-        for (int i = 0; i < COLS; ++i) r[i] = __float_as_uint(acc[i]);
+        for (int i = 0; i < COLS / 2; ++i) f2_unpack_bits(acc2[i], r[2 * i], r[2 * i + 1]);
         store_tile(r, mt, nt);
       }
     } else {
