@@ -16,9 +16,10 @@
 // (cta_group::2) tiles, output through shared memory and bulk-tensor
 // stores, optionally the output's MXFP4 operand from the epilogue.
 // NVFP4-CTA-local: the second-level scale differs per 128-wide K chunk, so
-// each chunk accumulates into one of two tensor-memory partials that the
-// epilogue warps fold, tsA[m/128][kc] * tsB[n/128][kc] * partial, into FP32
-// registers as soon as the chunk's MMAs complete.
+// each chunk accumulates into one of three tensor-memory partials (the MMAs
+// may run two chunks ahead) that the epilogue warps fold,
+// tsA[m/128][kc] * tsB[n/128][kc] * partial, into FP32 registers as soon as
+// the chunk's MMAs complete.
 //
 // Ragged shapes (M, N any; K a multiple of 32): the grid covers whole tiles;
 // TMA reads zeros for payload outside A and B, scale atoms that the operands
@@ -325,8 +326,8 @@ namespace gemm_st {
 using namespace fa4::gemm;
 using namespace fa4::gemm2;
 
-constexpr int NBUF = 5;       // scale buffers in tensor memory
-constexpr int SF_BASE = 256;  // first column after the accumulator
+constexpr int NBUF = 5;       // scale buffers in tensor memory (at most)
+constexpr int SF_BASE = 256;  // first column after a 256-column accumulator
 constexpr int NUM_THREADS_ST = 352;  // 11 warps
 
 template <int KIND, int BN, bool PAIR>
@@ -359,13 +360,20 @@ struct CfgSt {
   static constexpr int COLS_A = C::ATOMS_K * 4;
   static constexpr int COLS_B = C::ATOMS_K * (BN / 32);
   static constexpr int COLS_BUF = COLS_A + COLS_B;
+  // CTA-local NVFP4 keeps three 128-column chunk partials (the MMA may run
+  // two chunks ahead of the fold) and four scale buffers after them; the
+  // other formats one accumulator and five scale buffers
+  static constexpr int NPART = 3;
+  static constexpr int SF_COL0 = KIND == kNVC ? NPART * 128 : SF_BASE;
+  static constexpr int NBUF_ST = KIND == kNVC ? 4 : NBUF;
   // warps arriving per k-tile on a scale buffer (one per lane quadrant, in
   // each CTA of a pair) and per tile on the accumulator (two per quadrant)
   static constexpr int SF_ARRIVALS = PAIR ? 8 : 4;
   static constexpr int ACC_ARRIVALS = PAIR ? 16 : 8;
   static_assert(!PAIR || BN == 256, "a pair computes 256-wide tiles");
   static_assert(AB_STAGES >= 2, "shared-memory budget");
-  static_assert(SF_BASE + NBUF * COLS_BUF <= TMEM_COLS, "tensor-memory budget");
+  static_assert(SF_COL0 + NBUF_ST * COLS_BUF <= TMEM_COLS, "tensor-memory budget");
+  static_assert(NBUF_ST <= NBUF, "barrier arrays");
 };
 
 struct SmemSt {
@@ -373,7 +381,7 @@ struct SmemSt {
   uint64_t sfs_full[12], sfs_empty[12];      // scale stages in shared memory
   uint64_t sft_full[NBUF], sft_empty[NBUF];  // scale buffers in tensor memory
   uint64_t acc_full, acc_empty, mma_done;
-  uint64_t part_full[2], part_empty[2];  // CTA-local NVFP4: the two 128-K chunk partials
+  uint64_t part_full[3], part_empty[3];  // CTA-local NVFP4: the 128-K chunk partials
   uint32_t tmem_base;
   int abort;
 };
@@ -503,13 +511,13 @@ __global__ void __launch_bounds__(NUM_THREADS_ST, 1)
       mbar_init(smem_u32(&sm->sfs_full[s]), 1);
       mbar_init(smem_u32(&sm->sfs_empty[s]), 4);
     }
-    for (int b = 0; b < NBUF; ++b) {
+    for (int b = 0; b < CS::NBUF_ST; ++b) {
       mbar_init(smem_u32(&sm->sft_full[b]), CS::SF_ARRIVALS);
       mbar_init(smem_u32(&sm->sft_empty[b]), 1);
     }
     mbar_init(smem_u32(&sm->acc_full), 1);
     mbar_init(smem_u32(&sm->acc_empty), CS::ACC_ARRIVALS);
-    for (int c = 0; c < 2; ++c) {
+    for (int c = 0; c < CS::NPART; ++c) {
       mbar_init(smem_u32(&sm->part_full[c]), 1);
       mbar_init(smem_u32(&sm->part_empty[c]), CS::ACC_ARRIVALS);
     }
@@ -656,8 +664,8 @@ __global__ void __launch_bounds__(NUM_THREADS_ST, 1)
           tc_fence_after();
         }
         for (int kt = 0; kt < KT; ++kt, ++g) {
-          const int s = g % ABS, b = g % NBUF;
-          if (!wait_st(smem_u32(&sm->sft_full[b]), (uint32_t)((g / NBUF) & 1), sm, p, 0x230u | b) ||
+          const int s = g % ABS, b = g % CS::NBUF_ST;
+          if (!wait_st(smem_u32(&sm->sft_full[b]), (uint32_t)((g / CS::NBUF_ST) & 1), sm, p, 0x230u | b) ||
               !wait_st(smem_u32(&sm->ab_full[s]), (uint32_t)((g / ABS) & 1), sm, p, 0x210u | s)) {
             ok = false;
             break;
@@ -665,7 +673,7 @@ __global__ void __launch_bounds__(NUM_THREADS_ST, 1)
           tc_fence_after();
           const uint32_t a_base = smem_u32(smem + CS::OFF_A + s * CS::A_BYTES);
           const uint32_t b_base = smem_u32(smem + CS::OFF_B + s * CS::B_BYTES);
-          const uint32_t sf_col = tmem + SF_BASE + b * CS::COLS_BUF;
+          const uint32_t sf_col = tmem + CS::SF_COL0 + b * CS::COLS_BUF;
 #pragma unroll
           for (int j = 0; j < BK / 64; ++j) {
             const int a = (KIND == kMX) ? (j >> 1) : j;
@@ -673,21 +681,22 @@ __global__ void __launch_bounds__(NUM_THREADS_ST, 1)
             const uint32_t sfa = (sf_col + 4 * a) | (sf_id << 30);
             const uint32_t sfb = (sf_col + CS::COLS_A + (BN / 32) * a) | (sf_id << 30);
             if constexpr (KIND == kNVC) {
-              // each 128-K chunk (MMAs 2c, 2c+1) starts a fresh partial in
-              // columns 128c.. once the fold has read its previous content
-              const int c = j >> 1;
+              // chunk q = 2g + c (MMAs 2c, 2c+1 of this k-tile) starts a
+              // fresh partial in buffer q % 3 once the fold has read that
+              // buffer's previous chunk
+              const int q = 2 * g + (j >> 1), pb = q % CS::NPART;
               if ((j & 1) == 0) {
-                if (!wait_st(smem_u32(&sm->part_empty[c]), (uint32_t)((g & 1) ^ 1), sm, p,
-                             0x240u | c)) {
+                if (!wait_st(smem_u32(&sm->part_empty[pb]), (uint32_t)(((q / CS::NPART) & 1) ^ 1), sm,
+                             p, 0x240u | pb)) {
                   ok = false;
                   break;
                 }
                 tc_fence_after();
               }
-              tc_mma<KIND>(tmem + 128 * c, operand_desc(a_base + j * 32),
+              tc_mma<KIND>(tmem + 128 * pb, operand_desc(a_base + j * 32),
                            operand_desc(b_base + j * 32), instr_desc<KIND, BN>(sf_id), sfa, sfb,
                            (uint32_t)(j & 1));
-              if (j & 1) tc_commit(smem_u32(&sm->part_full[c]));
+              if (j & 1) tc_commit(smem_u32(&sm->part_full[pb]));
             } else {
               const uint32_t acc = (kt > 0 || j > 0) ? 1u : 0u;
               if constexpr (PAIR)
@@ -739,18 +748,19 @@ __global__ void __launch_bounds__(NUM_THREADS_ST, 1)
     if constexpr (KIND == kNVG) alpha_g = p.alpha * p.a_ts[0] * p.b_ts[0];
     const uint32_t acc_empty_l = leader_addr(&sm->acc_empty);
 
-    // stage the scales of k-tile g into tensor-memory buffer g % NBUF
+    // stage the scales of k-tile g into tensor-memory buffer g % NBUF_ST
     auto stage_scales = [&](int g) -> bool {
-      const int s = g % SFS, b = g % NBUF;
+      const int s = g % SFS, b = g % CS::NBUF_ST;
       if (!warp_wait_st(smem_u32(&sm->sfs_full[s]), (uint32_t)((g / SFS) & 1), sm, p, 0x320u | s))
         return false;
-      if (g >= NBUF &&
-          !warp_wait_st(smem_u32(&sm->sft_empty[b]), (uint32_t)(((g / NBUF) & 1) ^ 1), sm, p, 0x330u | b))
+      if (g >= CS::NBUF_ST &&
+          !warp_wait_st(smem_u32(&sm->sft_empty[b]), (uint32_t)(((g / CS::NBUF_ST) & 1) ^ 1), sm, p,
+                        0x330u | b))
         return false;
       tc_fence_after();
       const uint8_t *sfa_s = smem + CS::OFF_SF + s * CS::SF_BYTES;
       const uint8_t *sfb_s = sfa_s + CS::SFA_BYTES;
-      const uint32_t col = lane_base + SF_BASE + b * CS::COLS_BUF;
+      const uint32_t col = lane_base + CS::SF_COL0 + b * CS::COLS_BUF;
       // ragged shapes: atoms the scale producer did not load are zero
       int na = C::ATOMS_K;
       bool a_in = true, b_in[BN / 128];
@@ -901,8 +911,8 @@ __global__ void __launch_bounds__(NUM_THREADS_ST, 1)
     };
 
     if constexpr (KIND == kNVC) {
-      // CTA-local NVFP4: per k-tile, stage this warp's scales up to NBUF
-      // k-tiles ahead, then fold both 128-K chunk partials into FP32
+      // CTA-local NVFP4: per k-tile, stage this warp's scales up to NBUF_ST
+      // k-tiles ahead, then fold the k-tile's two 128-K chunk partials into FP32
       // registers, acc += tsA[m/128][kc] * tsB[n/128][kc] * partial, and
       // release each partial as soon as it is read; store at the tile's end
       const int nk = (int)((p.K + 127) / 128);  // 128-wide K chunks (the last may be short)
@@ -926,7 +936,7 @@ __global__ void __launch_bounds__(NUM_THREADS_ST, 1)
             const int kc = 2 * kt + c;
             fk[c] = kc < nk ? p.a_ts[(int64_t)mt * nk + kc] * p.b_ts[(int64_t)nt * nk + kc] : 0.0f;
           }
-          for (; g_st < total && g_st < g + NBUF; g_st += 2)
+          for (; g_st < total && g_st < g + CS::NBUF_ST; g_st += 2)
             if (!stage_scales(g_st)) {
               ok = false;
               break;
@@ -934,7 +944,9 @@ __global__ void __launch_bounds__(NUM_THREADS_ST, 1)
           if (!ok) break;
 #pragma unroll
           for (int c = 0; c < 2; ++c) {
-            if (!warp_wait_st(smem_u32(&sm->part_full[c]), (uint32_t)(g & 1), sm, p, 0x340u | c)) {
+            const int q = 2 * g + c, pb = q % CS::NPART;  // chunk q's partial buffer
+            if (!warp_wait_st(smem_u32(&sm->part_full[pb]), (uint32_t)((q / CS::NPART) & 1), sm, p,
+                              0x340u | pb)) {
               ok = false;
               break;
             }
@@ -942,11 +954,11 @@ __global__ void __launch_bounds__(NUM_THREADS_ST, 1)
             uint32_t r[COLS];
 #pragma unroll
             for (int ch = 0; ch < NCH; ++ch)
-              tmem_ld32(lane_base + 128 * c + h * COLS + 32 * ch, &r[32 * ch]);
+              tmem_ld32(lane_base + 128 * pb + h * COLS + 32 * ch, &r[32 * ch]);
             tmem_wait_ld();
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(smem_u32(&sm->part_empty[c]));
+            if (lane == 0) mbar_arrive(smem_u32(&sm->part_empty[pb]));
             const uint64_t f2 = f2_pack(fk[c], fk[c]);
 #pragma unroll
             for (int i = 0; i < COLS / 2; ++i)
@@ -968,7 +980,7 @@ __global__ void __launch_bounds__(NUM_THREADS_ST, 1)
     for (int tile = unit; tile < num_tiles && ok; tile += nunits, ++it) {
       // scales for the rest of this tile and the first NBUF k-tiles of the
       // next one, then this tile's epilogue
-      const int until = min(total, (it + 1) * KT + NBUF);
+      const int until = min(total, (it + 1) * KT + CS::NBUF_ST);
       for (; g < until; g += 2)
         if (!stage_scales(g)) {
           ok = false;
