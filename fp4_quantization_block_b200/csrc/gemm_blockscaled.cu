@@ -19,7 +19,8 @@
 // each chunk accumulates into one of three tensor-memory partials (the MMAs
 // may run two chunks ahead) that the epilogue warps fold,
 // tsA[m/128][kc] * tsB[n/128][kc] * partial, into FP32 registers as soon as
-// the chunk's MMAs complete.
+// the chunk's MMAs complete; 128-wide tiles, as 2-SM pairs (256 x 128) when
+// M allows.
 //
 // Ragged shapes (M, N any; K a multiple of 32): the grid covers whole tiles;
 // TMA reads zeros for payload outside A and B, scale atoms that the operands
@@ -283,10 +284,11 @@ __device__ __forceinline__ void tc_mma_pair(uint32_t d, uint64_t adesc, uint64_t
         : "memory");
   }
 }
-// instruction descriptor for the pair: M = 256
-template <int KIND>
+// instruction descriptor for the pair: M = 256, N = 256 (or 128: the
+// CTA-local form, whose chunk partials must leave room in tensor memory)
+template <int KIND, int N = 256>
 __device__ __forceinline__ uint32_t instr_desc_pair(uint32_t sf_id) {
-  return (1u << 7) | (1u << 10) | ((uint32_t)(256 >> 3) << 17) | ((KIND == kMX ? 1u : 0u) << 23) |
+  return (1u << 7) | (1u << 10) | ((uint32_t)(N >> 3) << 17) | ((KIND == kMX ? 1u : 0u) << 23) |
          ((uint32_t)(256 >> 4) << 24) | (sf_id << 4) | (sf_id << 29);
 }
 
@@ -334,7 +336,7 @@ template <int KIND, int BN, bool PAIR>
 struct CfgSt {
   using C = Cfg<KIND>;
   static constexpr int TILE_M = PAIR ? 256 : 128;
-  static constexpr int B_ROWS = PAIR ? 128 : BN;               // B rows in this CTA
+  static constexpr int B_ROWS = PAIR ? BN / 2 : BN;            // B rows in this CTA
   static constexpr int A_BYTES = 128 * BKB;
   static constexpr int B_BYTES = B_ROWS * BKB;
   static constexpr int SFA_BYTES = C::SFA_BYTES;                // 128 rows
@@ -370,7 +372,8 @@ struct CfgSt {
   // each CTA of a pair) and per tile on the accumulator (two per quadrant)
   static constexpr int SF_ARRIVALS = PAIR ? 8 : 4;
   static constexpr int ACC_ARRIVALS = PAIR ? 16 : 8;
-  static_assert(!PAIR || BN == 256, "a pair computes 256-wide tiles");
+  static_assert(!PAIR || BN == 256 || (KIND == kNVC && BN == 128),
+                "a pair computes 256-wide tiles (CTA-local NVFP4: 128-wide)");
   static_assert(AB_STAGES >= 2, "shared-memory budget");
   static_assert(SF_COL0 + NBUF_ST * COLS_BUF <= TMEM_COLS, "tensor-memory budget");
   static_assert(NBUF_ST <= NBUF, "barrier arrays");
@@ -576,7 +579,7 @@ __global__ void __launch_bounds__(NUM_THREADS_ST, 1)
             const uint32_t fb = leader_addr(&sm->ab_full[s]);
             if (rank == 0) mbar_arrive_expect_tx(smem_u32(&sm->ab_full[s]), 2 * CS::AB_BYTES);
             tma_load_2d_pair(a_dst, &map_a, kt * BKB, mt * 256 + (int)rank * 128, fb);
-            tma_load_2d_pair(b_dst, &map_b, kt * BKB, nt * 256 + (int)rank * 128, fb);
+            tma_load_2d_pair(b_dst, &map_b, kt * BKB, nt * BN + (int)rank * (BN / 2), fb);
           } else {
             const uint32_t fb = smem_u32(&sm->ab_full[s]);
             mbar_arrive_expect_tx(fb, CS::AB_BYTES);
@@ -693,10 +696,20 @@ __global__ void __launch_bounds__(NUM_THREADS_ST, 1)
                 }
                 tc_fence_after();
               }
-              tc_mma<KIND>(tmem + 128 * pb, operand_desc(a_base + j * 32),
-                           operand_desc(b_base + j * 32), instr_desc<KIND, BN>(sf_id), sfa, sfb,
-                           (uint32_t)(j & 1));
-              if (j & 1) tc_commit(smem_u32(&sm->part_full[pb]));
+              if constexpr (PAIR)
+                tc_mma_pair<KIND>(tmem + 128 * pb, operand_desc(a_base + j * 32),
+                                  operand_desc(b_base + j * 32), instr_desc_pair<KIND, BN>(sf_id),
+                                  sfa, sfb, (uint32_t)(j & 1));
+              else
+                tc_mma<KIND>(tmem + 128 * pb, operand_desc(a_base + j * 32),
+                             operand_desc(b_base + j * 32), instr_desc<KIND, BN>(sf_id), sfa, sfb,
+                             (uint32_t)(j & 1));
+              if (j & 1) {
+                if constexpr (PAIR)
+                  tc_commit_pair(smem_u32(&sm->part_full[pb]), (uint16_t)3);
+                else
+                  tc_commit(smem_u32(&sm->part_full[pb]));
+              }
             } else {
               const uint32_t acc = (kt > 0 || j > 0) ? 1u : 0u;
               if constexpr (PAIR)
@@ -934,7 +947,8 @@ __global__ void __launch_bounds__(NUM_THREADS_ST, 1)
 #pragma unroll
           for (int c = 0; c < 2; ++c) {
             const int kc = 2 * kt + c;
-            fk[c] = kc < nk ? p.a_ts[(int64_t)mt * nk + kc] * p.b_ts[(int64_t)nt * nk + kc] : 0.0f;
+            const int mb = PAIR ? mt * 2 + (int)rank : mt;  // this CTA's 128-row block of A
+            fk[c] = kc < nk ? p.a_ts[(int64_t)mb * nk + kc] * p.b_ts[(int64_t)nt * nk + kc] : 0.0f;
           }
           for (; g_st < total && g_st < g + CS::NBUF_ST; g_st += 2)
             if (!stage_scales(g_st)) {
@@ -958,7 +972,12 @@ __global__ void __launch_bounds__(NUM_THREADS_ST, 1)
             tmem_wait_ld();
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(smem_u32(&sm->part_empty[pb]));
+            if (lane == 0) {
+              if (PAIR && rank != 0)
+                mbar_arrive_remote_relaxed(leader_addr(&sm->part_empty[pb]));
+              else
+                mbar_arrive(smem_u32(&sm->part_empty[pb]));
+            }
             const uint64_t f2 = f2_pack(fk[c], fk[c]);
 #pragma unroll
             for (int i = 0; i < COLS / 2; ++i)
@@ -1121,7 +1140,7 @@ static cudaError_t launch_st(const GemmArgs &a, cudaStream_t st) {
   constexpr int smem = gemm_st::total_smem_st<KIND, BN, PAIR>();
   CUtensorMap ma, mb;
   if (!make_payload_map(&ma, a.a_payload, a.M, a.K, gemm::BM)) return cudaErrorInvalidValue;
-  if (!make_payload_map(&mb, a.b_payload, a.N, a.K, PAIR ? 128 : BN)) return cudaErrorInvalidValue;
+  if (!make_payload_map(&mb, a.b_payload, a.N, a.K, PAIR ? BN / 2 : BN)) return cudaErrorInvalidValue;
   CUtensorMap md;
   memset(&md, 0, sizeof(md));
   if (a.D && !make_out_map(&md, a)) return cudaErrorInvalidValue;
@@ -1186,7 +1205,12 @@ cudaError_t launch_gemm_blockscaled(const GemmArgs &a, cudaStream_t st) {
     if (!a.D) return cudaErrorInvalidValue;
     return launch_st_any<false>(a, st);
   }
-  if (a.fmt == kNVC && !a.q_payload && a.D) return launch_st<kNVC, 128, false, false>(a, st);
+  if (a.fmt == kNVC && !a.q_payload && a.D) {
+    // 2-SM pairs (M = 256 per pair) where they cover no more rows than
+    // 128-row tiles would
+    const bool pair = (a.M + 255) / 256 * 256 == (a.M + 127) / 128 * 128;
+    return pair ? launch_st<kNVC, 128, true, false>(a, st) : launch_st<kNVC, 128, false, false>(a, st);
+  }
   return cudaErrorInvalidValue;
 }
 
