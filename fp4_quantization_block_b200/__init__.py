@@ -172,6 +172,15 @@ def _as_bf16_2d(x: torch.Tensor, name: str):
     return x.stride(0)
 
 
+def _rowmajor_bf16(x: torch.Tensor, name: str) -> torch.Tensor:
+    """x as a contiguous row-major bf16 CUDA tensor (the linear calls take no
+    leading dimension).  A strided input is copied; the caller keeps the
+    returned tensor alive until the call has been enqueued."""
+    if x.dtype != torch.bfloat16 or x.dim() != 2 or not x.is_cuda:
+        raise ValueError(f"{name} must be a 2-D bf16 CUDA tensor")
+    return x if x.is_contiguous() else x.contiguous()
+
+
 def quantize(x: torch.Tensor, fmt: int, rnd: int = RNE, orient: int = ROWWISE, seed: int = 0,
              out: QTensor | None = None, ws: torch.Tensor | None = None) -> QTensor:
     ld = _as_bf16_2d(x, "x")
@@ -256,12 +265,12 @@ def linear_ws_bytes(kind: int, T: int, Cin: int, Cout: int, fmt: int) -> int:
 def linear_fwd(X: torch.Tensor, Wq: QTensor, fmt: int, out: torch.Tensor | None = None,
                ws: torch.Tensor | None = None) -> torch.Tensor:
     """Y = X W^T; Wq is W[Cout, Cin] quantized row-wise."""
+    X = _rowmajor_bf16(X, "X")
     T, Cin = X.shape
     Cout = Wq.R
-    _as_bf16_2d(X, "X")
     out = out if out is not None else torch.empty((T, Cout), dtype=torch.bfloat16, device=X.device)
     ws = _ws(ws, linear_ws_bytes(0, T, Cin, Cout, fmt), X.device)
-    _check(lib().fa4_linear_fwd(_ptr(X.contiguous()), Wq.c(), T, Cin, Cout, fmt, _ptr(out), _ptr(ws),
+    _check(lib().fa4_linear_fwd(_ptr(X), Wq.c(), T, Cin, Cout, fmt, _ptr(out), _ptr(ws),
                                 ws.numel(), _stream(X.device)), "fa4_linear_fwd")
     return out
 
@@ -269,12 +278,12 @@ def linear_fwd(X: torch.Tensor, Wq: QTensor, fmt: int, out: torch.Tensor | None 
 def linear_dgrad(dY: torch.Tensor, Wq_col: QTensor, fmt: int, rnd: int = SR, seed: int = 0,
                  out: torch.Tensor | None = None, ws: torch.Tensor | None = None) -> torch.Tensor:
     """dX = dY W; Wq_col is W[Cout, Cin] quantized column-wise ([Cin, Cout])."""
+    dY = _rowmajor_bf16(dY, "dY")
     T, Cout = dY.shape
     Cin = Wq_col.R
-    _as_bf16_2d(dY, "dY")
     out = out if out is not None else torch.empty((T, Cin), dtype=torch.bfloat16, device=dY.device)
     ws = _ws(ws, linear_ws_bytes(1, T, Cin, Cout, fmt), dY.device)
-    _check(lib().fa4_linear_dgrad(_ptr(dY.contiguous()), Wq_col.c(), T, Cin, Cout, fmt, rnd, seed,
+    _check(lib().fa4_linear_dgrad(_ptr(dY), Wq_col.c(), T, Cin, Cout, fmt, rnd, seed,
                                   _ptr(out), _ptr(ws), ws.numel(), _stream(dY.device)),
            "fa4_linear_dgrad")
     return out
@@ -284,15 +293,15 @@ def linear_wgrad(dY: torch.Tensor, X: torch.Tensor, sign_mask: int, rnd: int = R
                  out_dtype=torch.float32, out: torch.Tensor | None = None,
                  ws: torch.Tensor | None = None) -> torch.Tensor:
     """dW = dY^T X through column-wise fixed-sign Hadamard MXFP4 operands."""
+    dY = _rowmajor_bf16(dY, "dY")
+    X = _rowmajor_bf16(X, "X")
     T, Cout = dY.shape
     _, Cin = X.shape
-    _as_bf16_2d(dY, "dY")
-    _as_bf16_2d(X, "X")
     if out is None:
         out = torch.empty((Cout, Cin), dtype=out_dtype, device=dY.device)
     od = OUT_FP32 if out.dtype == torch.float32 else OUT_BF16
     ws = _ws(ws, linear_ws_bytes(2, T, Cin, Cout, MXFP4), dY.device)
-    _check(lib().fa4_linear_wgrad(_ptr(dY.contiguous()), _ptr(X.contiguous()), T, Cin, Cout,
+    _check(lib().fa4_linear_wgrad(_ptr(dY), _ptr(X), T, Cin, Cout,
                                   sign_mask & 0xFFFFFFFF, rnd, seed, _ptr(out), od, _ptr(ws),
                                   ws.numel(), _stream(dY.device)), "fa4_linear_wgrad")
     return out
@@ -339,6 +348,7 @@ def linear_fwd_save(X: torch.Tensor, Wq: QTensor, fmt: int, sign_mask: int,
                     ws: torch.Tensor | None = None) -> tuple[torch.Tensor, QTensor]:
     """Y = X W^T, plus X's column-wise MXFP4 Hadamard operand for the
     backward half (one read of X)."""
+    X = _rowmajor_bf16(X, "X")
     T, Cin = X.shape
     Cout = Wq.R
     Y = out if out is not None else torch.empty(T, Cout, dtype=torch.bfloat16, device=X.device)
@@ -356,6 +366,7 @@ def linear_bwd(dY: torch.Tensor, Wq_col: QTensor, xcol: QTensor, fmt: int, rnd: 
                ws: torch.Tensor | None = None) -> tuple[torch.Tensor, torch.Tensor]:
     """dX = dY W and dW = dY^T X from one read of dY (xcol from
     linear_fwd_save with the same sign_mask)."""
+    dY = _rowmajor_bf16(dY, "dY")
     T, Cout = dY.shape
     Cin = Wq_col.R
     dX = dx if dx is not None else torch.empty(T, Cin, dtype=torch.bfloat16, device=dY.device)

@@ -273,3 +273,21 @@ def test_header_is_plain_c_and_links_from_c(tmp_path):
     assert cc.returncode == 0, cc.stderr
     run = subprocess.run([str(exe)], capture_output=True, text=True, timeout=60)
     assert run.returncode == 0 and "c-abi ok" in run.stdout, (run.returncode, run.stderr)
+
+
+def test_linear_bindings_validate_inputs_before_any_call():
+    """The training-form and plain linear bindings reject a non-bf16 or
+    host tensor before reaching the library (the C calls take no leading
+    dimension, so a strided device input is copied, never passed as is)."""
+    import torch
+    x = torch.zeros(32, 32, dtype=torch.float32)
+    q = fa.QTensor(torch.zeros(1, dtype=torch.uint8), torch.zeros(1, dtype=torch.uint8), None, 32, 32,
+                   fa.MXFP4)
+    for call in (lambda: fa.linear_fwd(x, q, fa.MXFP4),
+                 lambda: fa.linear_dgrad(x, q, fa.MXFP4),
+                 lambda: fa.linear_wgrad(x, x, 1),
+                 lambda: fa.linear_fwd_save(x, q, fa.MXFP4, 1),
+                 lambda: fa.linear_bwd(x, q, q, fa.MXFP4),
+                 lambda: fa.linear_fwd(x.to(torch.bfloat16), q, fa.MXFP4)):
+        with pytest.raises(ValueError):
+            call()
