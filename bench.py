@@ -312,6 +312,72 @@ def gemm_sweep(fa, device, reps: int = 10) -> list[dict]:
     return out
 
 
+def ragged_sweep(fa, device, reps: int = 10) -> list[dict]:
+    """Ragged shapes beside the aligned shapes they approximate: the same
+    quantizers and GEMM with a row count, a block dimension (K) or GEMM M, N
+    and K that are not multiples of 128.  Rates use each shape's own
+    elements (FLOPs), so a ragged line's ratio to its aligned one is the cost
+    of the masked tiles."""
+    hbm = _peaks()[0]
+    fp4_peak = 4.0 * _peaks()[1]
+    ws = fa.workspace(1 << 16, device)
+    out = []
+
+    def timed(call):
+        for _ in range(3):
+            call()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(reps):
+            call()
+        e1.record()
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1) * 1000.0 / reps
+
+    # quantizers: (label, rows, cols, kind)
+    qcases = [("mx row rne", 8192, 14336, "row"), ("mx row rne", 8191, 14336, "row"),
+              ("mx row rne", 8192, 14304, "row"),
+              ("mx col+had32 rne", 8192, 14336, "had"), ("mx col+had32 rne", 8160, 14336, "had"),
+              ("dual mx sr + col had32", 8192, 4096, "dual"),
+              ("dual mx sr + col had32", 8160, 4096, "dual")]
+    for label, rows, cols, kind in qcases:
+        x = workloads.sweep(rows, cols, seed=3, device=device)
+        if kind == "row":
+            q = fa.empty_qtensor(rows, cols, fa.MXFP4, fa.ROWWISE, device)
+            us = timed(lambda: fa.quantize(x, fa.MXFP4, fa.RNE, fa.ROWWISE, 0, out=q, ws=ws))
+            bpe = BYTES_PER_ELEM["mx"]
+        elif kind == "had":
+            q = fa.empty_qtensor(rows, cols, fa.MXFP4, fa.COLWISE, device)
+            us = timed(lambda: fa.hadamard32_quantize(x, SIGN_MASK, fa.RNE, 0, out=q, ws=ws))
+            bpe = BYTES_PER_ELEM["mx"]
+        else:
+            r = fa.empty_qtensor(rows, cols, fa.MXFP4, fa.ROWWISE, device)
+            c = fa.empty_qtensor(rows, cols, fa.MXFP4, fa.COLWISE, device)
+            us = timed(lambda: fa.quantize_dual(x, fa.MXFP4, fa.SR, 1, col_hadamard=True,
+                                                sign_mask=SIGN_MASK, row_out=r, col_out=c, ws=ws))
+            bpe = BYTES_PER_ELEM["mx_dual"]
+        gbs = bpe * rows * cols / (us * 1e-6) / 1e9
+        out.append({"op": label, "shape": [rows, cols], "us": round(us, 2), "GBps": round(gbs, 1),
+                    "frac_hbm": round(gbs / hbm, 3)})
+        del x
+    # GEMM (MXFP4, bf16 out): the gate+up forward shape and a ragged neighbour
+    for M, N, K in ((8192, 28672, 4096), (8000, 28600, 4064)):
+        a = workloads.act(M, K, seed=5, device=device)
+        b = workloads.weight(N, K, seed=6, device=device)
+        A, B = fa.quantize(a, fa.MXFP4, ws=ws), fa.quantize(b, fa.MXFP4, ws=ws)
+        d = fa.gemm(A, B, 1.0, out_dtype=torch.bfloat16, ws=ws)
+        us = timed(lambda: fa.gemm(A, B, 1.0, out=d, ws=ws))
+        tf = 2.0 * M * N * K / (us * 1e-6) / 1e12
+        out.append({"op": "gemm mx", "shape": [M, N, K], "us": round(us, 1), "TFLOPS": round(tf, 1),
+                    "frac": round(tf / fp4_peak, 3)})
+        del a, b, A, B, d
+    if fa.check_device_status(ws) != 0:
+        raise RuntimeError("device status set during the ragged sweep")
+    torch.cuda.empty_cache()
+    return out
+
+
 def epilogue_quant_run(fa, device, reps: int = 10) -> dict:
     """The gate+up forward GEMM followed by the MXFP4 quantization of its bf16
     output: separate calls against the quantizer fused into the GEMM epilogue
@@ -695,6 +761,12 @@ def fa4_arm(args, rank, world, device) -> dict | None:
         sweep = quantize_sweep(fa, device) if solo else []
         gsweep = gemm_sweep(fa, device) if solo else []
         epiq = epilogue_quant_run(fa, device) if solo else {}
+        ragged = []
+        if solo:
+            try:
+                ragged = ragged_sweep(fa, device)
+            except (RuntimeError, torch.cuda.OutOfMemoryError) as e:
+                ragged = [{"error": f"{type(e).__name__}: {e}"}]
         stack = {}
         if solo or args.stack:
             try:
@@ -726,6 +798,7 @@ def fa4_arm(args, rank, world, device) -> dict | None:
                         "quantize_sweep": sweep,
                         "gemm_sweep": gsweep,
                         "gemm_epilogue_mxfp4": epiq,
+                        "ragged_sweep": ragged,
                         "linear_stack": stack},
             "roofline": {"bound": "tensor", "achieved": round(dom_tflops, 1),
                          "peak": round(fp4_peak, 1), "unit": "TFLOP/s",

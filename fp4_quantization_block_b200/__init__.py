@@ -120,9 +120,10 @@ def _stream(device: torch.device):
 @dataclass
 class QTensor:
     """Quantized operand Q[R, K]: ``payload`` uint8 [R, K/2] (K-major, element
-    2j in the low nibble of byte j), ``scales`` uint8 [R*K/block] in the 128x4
-    atom layout the block-scaled MMA reads, ``ts`` float32 second-level decode
-    scales (NVFP4) or None (MXFP4)."""
+    2j in the low nibble of byte j), ``scales`` uint8 in the 128x4 atom layout
+    the block-scaled MMA reads (rows padded to a multiple of 128, blocks to a
+    multiple of 4), ``ts`` float32 second-level decode scales (NVFP4) or None
+    (MXFP4)."""
     payload: torch.Tensor
     scales: torch.Tensor
     ts: torch.Tensor | None
@@ -244,7 +245,9 @@ def gemm(A: QTensor, B: QTensor, alpha: float = 1.0, out_dtype=torch.float32,
         raise ValueError("A and B must share K and format")
     dev = A.payload.device
     if out is None:
-        out = torch.empty((A.R, B.R), dtype=out_dtype, device=dev)
+        # leading dimension a multiple of 8 elements (the ABI's row alignment)
+        ldd = -(-B.R // 8) * 8
+        out = torch.empty((A.R, ldd), dtype=out_dtype, device=dev)[:, :B.R]
     od = OUT_FP32 if out.dtype == torch.float32 else OUT_BF16
     ws = _ws(ws, WS_HEADER_BYTES, dev)
     _check(lib().fa4_gemm_blockscaled(A.c(), B.c(), A.R, B.R, A.K, A.fmt, float(alpha), _ptr(out),

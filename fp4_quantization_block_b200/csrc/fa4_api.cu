@@ -25,12 +25,26 @@ inline cudaStream_t S(void *s) { return reinterpret_cast<cudaStream_t>(s); }
 
 size_t partials_bytes() { return align256(sizeof(float) * fa4::kMaxAmaxPartials); }
 
+inline int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
+
 size_t qt_payload(int64_t R, int64_t K) { return (size_t)(R * (K / 2)); }
-size_t qt_scales(int64_t R, int64_t K, int fmt) { return (size_t)(R * (K / block_of(fmt))); }
+// scale atoms: rows padded to a multiple of 128, blocks to a multiple of 4
+size_t qt_scales(int64_t R, int64_t K, int fmt) {
+  return (size_t)(ceil_div(R, 128) * 128 * (ceil_div(K / block_of(fmt), 4) * 4));
+}
 size_t qt_ts(int64_t R, int64_t K, int fmt) {
   if (fmt == FA4_NVFP4_GLOBAL) return 1;
-  if (fmt == FA4_NVFP4_CTA) return (size_t)((R / 128) * (K / 128));
+  if (fmt == FA4_NVFP4_CTA) return (size_t)(ceil_div(R, 128) * ceil_div(K, 128));
   return 0;
+}
+// Shape rule of a quantized operand Q[R, K] read from x[rows, cols]: any
+// positive R; K a multiple of 32 (whole MX blocks, and payload rows of a
+// multiple of 16 bytes for the GEMM's tensor-memory-access loads); x rows
+// read in 16-byte pieces, so cols is a multiple of 8.
+bool quant_shape_ok(int64_t rows, int64_t cols, int orient) {
+  if (rows <= 0 || cols <= 0 || cols % 8) return false;
+  const int64_t K = orient == FA4_ROWWISE ? cols : rows;
+  return K % 32 == 0;
 }
 size_t quant_ws(int fmt) { return kHdr + (fmt == FA4_NVFP4_GLOBAL ? partials_bytes() : 0); }
 // bytes of a quantized operand carved from a workspace (256-aligned parts)
@@ -48,9 +62,14 @@ fa4_qtensor carve_qt(uint8_t *base, int64_t R, int64_t K, int fmt) {
   return q;
 }
 
-fa4_status check_input(const void *x, int64_t rows, int64_t cols, int64_t ld) {
+// x[rows, cols] read for the given orientations (row-wise, column-wise or
+// both)
+fa4_status check_input(const void *x, int64_t rows, int64_t cols, int64_t ld, bool row = true,
+                       bool col = false) {
   if (!x) return FA4_ERR_INVALID_ARG;
-  if (rows <= 0 || cols <= 0 || rows % 128 || cols % 128) return FA4_ERR_SHAPE;
+  if ((row && !quant_shape_ok(rows, cols, FA4_ROWWISE)) ||
+      (col && !quant_shape_ok(rows, cols, FA4_COLWISE)))
+    return FA4_ERR_SHAPE;
   if (ld < cols || ld % 8) return FA4_ERR_SHAPE;
   if (!aligned16(x)) return FA4_ERR_ALIGN;
   return FA4_OK;
@@ -151,7 +170,7 @@ fa4_status check_gemm(const fa4_qtensor &A, const fa4_qtensor &B, int64_t M, int
   fa4_status s = check_qt(A, fmt);
   if (s != FA4_OK) return s;
   if ((s = check_qt(B, fmt)) != FA4_OK) return s;
-  if (M <= 0 || N <= 0 || K <= 0 || M % 128 || N % 128 || K % 256) return FA4_ERR_SHAPE;
+  if (M <= 0 || N <= 0 || K <= 0 || K % 32) return FA4_ERR_SHAPE;
   if (ldd < N || ldd % 8) return FA4_ERR_SHAPE;
   if (!aligned16(D)) return FA4_ERR_ALIGN;
   if (!ws || ws_bytes < kHdr) return FA4_ERR_WORKSPACE;
@@ -183,7 +202,7 @@ fa4_status fa4_quant_sizes(int64_t rows, int64_t cols, fa4_format fmt, fa4_orien
                            size_t *payload_bytes, size_t *scale_bytes, size_t *tscale_count,
                            size_t *workspace_bytes) {
   if (!fmt_ok(fmt) || (orient != FA4_ROWWISE && orient != FA4_COLWISE)) return FA4_ERR_INVALID_ARG;
-  if (rows <= 0 || cols <= 0 || rows % 128 || cols % 128) return FA4_ERR_SHAPE;
+  if (!quant_shape_ok(rows, cols, orient)) return FA4_ERR_SHAPE;
   const int64_t R = orient == FA4_ROWWISE ? rows : cols, K = orient == FA4_ROWWISE ? cols : rows;
   if (payload_bytes) *payload_bytes = qt_payload(R, K);
   if (scale_bytes) *scale_bytes = qt_scales(R, K, fmt);
@@ -198,7 +217,7 @@ fa4_status fa4_quantize(const void *x, int64_t rows, int64_t cols, int64_t ld, f
   if (!fmt_ok(fmt) || (rnd != FA4_RNE && rnd != FA4_SR) ||
       (orient != FA4_ROWWISE && orient != FA4_COLWISE))
     return FA4_ERR_INVALID_ARG;
-  fa4_status s = check_input(x, rows, cols, ld);
+  fa4_status s = check_input(x, rows, cols, ld, orient == FA4_ROWWISE, orient == FA4_COLWISE);
   if (s != FA4_OK) return s;
   if ((s = check_qt(out, fmt)) != FA4_OK) return s;
   if (!workspace || workspace_bytes < quant_ws(fmt)) return FA4_ERR_WORKSPACE;
@@ -212,7 +231,7 @@ fa4_status fa4_hadamard32_quantize(const void *x, int64_t rows, int64_t cols, in
                                    fa4_qtensor out, void *workspace, size_t workspace_bytes,
                                    void *stream) {
   if (rnd != FA4_RNE && rnd != FA4_SR) return FA4_ERR_INVALID_ARG;
-  fa4_status s = check_input(x, rows, cols, ld);
+  fa4_status s = check_input(x, rows, cols, ld, false, true);
   if (s != FA4_OK) return s;
   if ((s = check_qt(out, FA4_MXFP4)) != FA4_OK) return s;
   if (!workspace || workspace_bytes < quant_ws(FA4_MXFP4)) return FA4_ERR_WORKSPACE;
@@ -229,7 +248,7 @@ fa4_status fa4_quantize_dual(const void *x, int64_t rows, int64_t cols, int64_t 
   if (!fmt_ok(row_fmt) || (row_rnd != FA4_RNE && row_rnd != FA4_SR) ||
       (col_rnd != FA4_RNE && col_rnd != FA4_SR))
     return FA4_ERR_INVALID_ARG;
-  fa4_status s = check_input(x, rows, cols, ld);
+  fa4_status s = check_input(x, rows, cols, ld, true, true);
   if (s != FA4_OK) return s;
   if ((s = check_qt(row_out, row_fmt)) != FA4_OK) return s;
   if ((s = check_qt(col_out, FA4_MXFP4)) != FA4_OK) return s;
@@ -253,7 +272,7 @@ fa4_status fa4_gemm_blockscaled(fa4_qtensor A, fa4_qtensor B, int64_t M, int64_t
 fa4_status fa4_linear_ws_bytes(int kind, int64_t T, int64_t Cin, int64_t Cout, fa4_format fmt,
                                size_t *workspace_bytes) {
   if (!workspace_bytes || !fmt_ok(fmt)) return FA4_ERR_INVALID_ARG;
-  if (T <= 0 || Cin <= 0 || Cout <= 0 || T % 128 || Cin % 128 || Cout % 128) return FA4_ERR_SHAPE;
+  if (T <= 0 || Cin <= 0 || Cout <= 0 || T % 32 || Cin % 32 || Cout % 32) return FA4_ERR_SHAPE;
   size_t b = kHdr + partials_bytes();
   switch (kind) {
     case 0: b += qt_ws_bytes(T, Cin, fmt); break;
@@ -314,8 +333,8 @@ fa4_status fa4_linear_wgrad(const void *dY, const void *X, int64_t T, int64_t Ci
   size_t need;
   fa4_status s = fa4_linear_ws_bytes(2, T, Cin, Cout, FA4_MXFP4, &need);
   if (s != FA4_OK) return s;
-  if ((s = check_input(dY, T, Cout, Cout)) != FA4_OK) return s;
-  if ((s = check_input(X, T, Cin, Cin)) != FA4_OK) return s;
+  if ((s = check_input(dY, T, Cout, Cout, false, true)) != FA4_OK) return s;
+  if ((s = check_input(X, T, Cin, Cin, false, true)) != FA4_OK) return s;
   if (!workspace || workspace_bytes < need) return FA4_ERR_WORKSPACE;
   if (!aligned16(workspace)) return FA4_ERR_ALIGN;
   uint8_t *ws = static_cast<uint8_t *>(workspace);
@@ -340,7 +359,7 @@ fa4_status fa4_linear_fwd_save(const void *X, fa4_qtensor Wq, int64_t T, int64_t
   size_t need;
   fa4_status s = fa4_linear_ws_bytes(3, T, Cin, Cout, fmt, &need);
   if (s != FA4_OK) return s;
-  if ((s = check_input(X, T, Cin, Cin)) != FA4_OK) return s;
+  if ((s = check_input(X, T, Cin, Cin, true, true)) != FA4_OK) return s;
   if ((s = check_qt(Xcol, FA4_MXFP4)) != FA4_OK) return s;
   if (!workspace || workspace_bytes < need) return FA4_ERR_WORKSPACE;
   if (!aligned16(workspace)) return FA4_ERR_ALIGN;
@@ -363,7 +382,7 @@ fa4_status fa4_linear_bwd(const void *dY, fa4_qtensor Wq_col, fa4_qtensor Xcol, 
   size_t need;
   fa4_status s = fa4_linear_ws_bytes(4, T, Cin, Cout, fmt, &need);
   if (s != FA4_OK) return s;
-  if ((s = check_input(dY, T, Cout, Cout)) != FA4_OK) return s;
+  if ((s = check_input(dY, T, Cout, Cout, true, true)) != FA4_OK) return s;
   if (!workspace || workspace_bytes < need) return FA4_ERR_WORKSPACE;
   if (!aligned16(workspace)) return FA4_ERR_ALIGN;
   uint8_t *ws = static_cast<uint8_t *>(workspace);
@@ -390,6 +409,7 @@ fa4_status fa4_gemm_blockscaled_mxout(fa4_qtensor A, fa4_qtensor B, int64_t M, i
                                       void *stream) {
   if (!fmt_ok(fmt)) return FA4_ERR_INVALID_ARG;
   if (fmt == FA4_NVFP4_CTA) return FA4_ERR_UNSUPPORTED;
+  if (N % 32) return FA4_ERR_SHAPE;  // D's MXFP4 blocks run along N
   fa4_status s = check_qt(Dq, FA4_MXFP4);
   if (s != FA4_OK) return s;
   // D is optional: checked as a bf16 output when given

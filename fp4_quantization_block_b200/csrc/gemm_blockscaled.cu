@@ -16,9 +16,18 @@
 // (cta_group::2) tiles, output through shared memory and bulk-tensor
 // stores, optionally the output's MXFP4 operand from the epilogue.
 // NVFP4-CTA-local: the second-level scale differs per 128-wide K chunk, so
-// each chunk accumulates into one of two tensor-memory partials that the
-// epilogue warps fold, tsA[m/128][kc] * tsB[n/128][kc] * partial, into FP32
-// registers as soon as the chunk's MMAs complete.
+// each chunk accumulates into one of three tensor-memory partials (the MMAs
+// may run two chunks ahead) that the epilogue warps fold,
+// tsA[m/128][kc] * tsB[n/128][kc] * partial, into FP32 registers as soon as
+// the chunk's MMAs complete; 128-wide tiles, as 2-SM pairs (256 x 128) when
+// M allows.
+//
+// Ragged shapes (M, N any; K a multiple of 32): the grid covers whole tiles;
+// TMA reads zeros for payload outside A and B, scale atoms that the operands
+// do not have (past the last 128-row block, or past the last atom along K)
+// are staged as zero bytes, and the stores skip what lies outside D.  Zero
+// payload times a finite scale adds nothing, so the padded tile computes
+// the exact result of the smaller one.
 //
 // Every mbarrier wait is bounded: past `timeout_ns` the waiting thread sets
 // the device status word, raises a CTA-wide abort flag and leaves its loop;
@@ -182,6 +191,9 @@ struct Params {
   // (payload [M, N/2], scales in the 128x4 atom layout); null: none
   uint8_t *q_payload, *q_scales;
   int store_d;  // 0: D is not written (only the quantized operand)
+  // ragged shapes: some tile reaches past M, N or K (see the file comment)
+  int ragged;
+  int64_t rb_a, rb_b;  // 128-row blocks of A and B (atom rows of their scales)
 };
 
 // Output tile coordinates of linear tile index t.  Concurrently running CTAs
@@ -272,10 +284,11 @@ __device__ __forceinline__ void tc_mma_pair(uint32_t d, uint64_t adesc, uint64_t
         : "memory");
   }
 }
-// instruction descriptor for the pair: M = 256
-template <int KIND>
+// instruction descriptor for the pair: M = 256, N = 256 (or 128: the
+// CTA-local form, whose chunk partials must leave room in tensor memory)
+template <int KIND, int N = 256>
 __device__ __forceinline__ uint32_t instr_desc_pair(uint32_t sf_id) {
-  return (1u << 7) | (1u << 10) | ((uint32_t)(256 >> 3) << 17) | ((KIND == kMX ? 1u : 0u) << 23) |
+  return (1u << 7) | (1u << 10) | ((uint32_t)(N >> 3) << 17) | ((KIND == kMX ? 1u : 0u) << 23) |
          ((uint32_t)(256 >> 4) << 24) | (sf_id << 4) | (sf_id << 29);
 }
 
@@ -315,15 +328,15 @@ namespace gemm_st {
 using namespace fa4::gemm;
 using namespace fa4::gemm2;
 
-constexpr int NBUF = 5;       // scale buffers in tensor memory
-constexpr int SF_BASE = 256;  // first column after the accumulator
+constexpr int NBUF = 5;       // scale buffers in tensor memory (at most)
+constexpr int SF_BASE = 256;  // first column after a 256-column accumulator
 constexpr int NUM_THREADS_ST = 352;  // 11 warps
 
 template <int KIND, int BN, bool PAIR>
 struct CfgSt {
   using C = Cfg<KIND>;
   static constexpr int TILE_M = PAIR ? 256 : 128;
-  static constexpr int B_ROWS = PAIR ? 128 : BN;               // B rows in this CTA
+  static constexpr int B_ROWS = PAIR ? BN / 2 : BN;            // B rows in this CTA
   static constexpr int A_BYTES = 128 * BKB;
   static constexpr int B_BYTES = B_ROWS * BKB;
   static constexpr int SFA_BYTES = C::SFA_BYTES;                // 128 rows
@@ -349,13 +362,21 @@ struct CfgSt {
   static constexpr int COLS_A = C::ATOMS_K * 4;
   static constexpr int COLS_B = C::ATOMS_K * (BN / 32);
   static constexpr int COLS_BUF = COLS_A + COLS_B;
+  // CTA-local NVFP4 keeps three 128-column chunk partials (the MMA may run
+  // two chunks ahead of the fold) and four scale buffers after them; the
+  // other formats one accumulator and five scale buffers
+  static constexpr int NPART = 3;
+  static constexpr int SF_COL0 = KIND == kNVC ? NPART * 128 : SF_BASE;
+  static constexpr int NBUF_ST = KIND == kNVC ? 4 : NBUF;
   // warps arriving per k-tile on a scale buffer (one per lane quadrant, in
   // each CTA of a pair) and per tile on the accumulator (two per quadrant)
   static constexpr int SF_ARRIVALS = PAIR ? 8 : 4;
   static constexpr int ACC_ARRIVALS = PAIR ? 16 : 8;
-  static_assert(!PAIR || BN == 256, "a pair computes 256-wide tiles");
+  static_assert(!PAIR || BN == 256 || (KIND == kNVC && BN == 128),
+                "a pair computes 256-wide tiles (CTA-local NVFP4: 128-wide)");
   static_assert(AB_STAGES >= 2, "shared-memory budget");
-  static_assert(SF_BASE + NBUF * COLS_BUF <= TMEM_COLS, "tensor-memory budget");
+  static_assert(SF_COL0 + NBUF_ST * COLS_BUF <= TMEM_COLS, "tensor-memory budget");
+  static_assert(NBUF_ST <= NBUF, "barrier arrays");
 };
 
 struct SmemSt {
@@ -363,7 +384,7 @@ struct SmemSt {
   uint64_t sfs_full[12], sfs_empty[12];      // scale stages in shared memory
   uint64_t sft_full[NBUF], sft_empty[NBUF];  // scale buffers in tensor memory
   uint64_t acc_full, acc_empty, mma_done;
-  uint64_t part_full[2], part_empty[2];  // CTA-local NVFP4: the two 128-K chunk partials
+  uint64_t part_full[3], part_empty[3];  // CTA-local NVFP4: the 128-K chunk partials
   uint32_t tmem_base;
   int abort;
 };
@@ -476,10 +497,11 @@ __global__ void __launch_bounds__(NUM_THREADS_ST, 1)
   const int unit = PAIR ? (int)(blockIdx.x >> 1) : (int)blockIdx.x;      // tile-walking unit
   const int nunits = PAIR ? (int)(gridDim.x >> 1) : (int)gridDim.x;
 
-  const int num_m = (int)(p.M / CS::TILE_M), num_n = (int)(p.N / BN);
+  const int num_m = (int)((p.M + CS::TILE_M - 1) / CS::TILE_M);
+  const int num_n = (int)((p.N + BN - 1) / BN);
   const int num_tiles = num_m * num_n;
-  const int KT = (int)(p.K / BK);
-  const int64_t kbt4 = (p.K / C::BS) / 4;
+  const int KT = (int)((p.K + BK - 1) / BK);
+  const int64_t kbt4 = (p.K / C::BS + 3) / 4;  // atoms along K per 128-row block
   const int my_tiles = unit < num_tiles ? (num_tiles - unit + nunits - 1) / nunits : 0;
   const int total = my_tiles * KT;  // k-tiles this CTA processes
 
@@ -492,13 +514,13 @@ __global__ void __launch_bounds__(NUM_THREADS_ST, 1)
       mbar_init(smem_u32(&sm->sfs_full[s]), 1);
       mbar_init(smem_u32(&sm->sfs_empty[s]), 4);
     }
-    for (int b = 0; b < NBUF; ++b) {
+    for (int b = 0; b < CS::NBUF_ST; ++b) {
       mbar_init(smem_u32(&sm->sft_full[b]), CS::SF_ARRIVALS);
       mbar_init(smem_u32(&sm->sft_empty[b]), 1);
     }
     mbar_init(smem_u32(&sm->acc_full), 1);
     mbar_init(smem_u32(&sm->acc_empty), CS::ACC_ARRIVALS);
-    for (int c = 0; c < 2; ++c) {
+    for (int c = 0; c < CS::NPART; ++c) {
       mbar_init(smem_u32(&sm->part_full[c]), 1);
       mbar_init(smem_u32(&sm->part_empty[c]), CS::ACC_ARRIVALS);
     }
@@ -557,7 +579,7 @@ __global__ void __launch_bounds__(NUM_THREADS_ST, 1)
             const uint32_t fb = leader_addr(&sm->ab_full[s]);
             if (rank == 0) mbar_arrive_expect_tx(smem_u32(&sm->ab_full[s]), 2 * CS::AB_BYTES);
             tma_load_2d_pair(a_dst, &map_a, kt * BKB, mt * 256 + (int)rank * 128, fb);
-            tma_load_2d_pair(b_dst, &map_b, kt * BKB, nt * 256 + (int)rank * 128, fb);
+            tma_load_2d_pair(b_dst, &map_b, kt * BKB, nt * BN + (int)rank * (BN / 2), fb);
           } else {
             const uint32_t fb = smem_u32(&sm->ab_full[s]);
             mbar_arrive_expect_tx(fb, CS::AB_BYTES);
@@ -596,15 +618,37 @@ __global__ void __launch_bounds__(NUM_THREADS_ST, 1)
             break;
           }
           const uint32_t fb = smem_u32(&sm->sfs_full[s]);
-          mbar_arrive_expect_tx(fb, CS::SF_BYTES);
           const uint32_t dst = smem_u32(smem + CS::OFF_SF + s * CS::SF_BYTES);
-          bulk_load(dst, p.a_scales + ((int64_t)rb_a * kbt4 + (int64_t)kt * C::ATOMS_K) * 512,
-                    CS::SFA_BYTES, fb);
+          if (!p.ragged) {
+            mbar_arrive_expect_tx(fb, CS::SF_BYTES);
+            bulk_load(dst, p.a_scales + ((int64_t)rb_a * kbt4 + (int64_t)kt * C::ATOMS_K) * 512,
+                      CS::SFA_BYTES, fb);
 #pragma unroll
-          for (int nb = 0; nb < BN / 128; ++nb)
-            bulk_load(dst + CS::SFA_BYTES + nb * C::SFA_BYTES,
-                      p.b_scales + ((int64_t)(nt * (BN / 128) + nb) * kbt4 + (int64_t)kt * C::ATOMS_K) * 512,
-                      C::SFA_BYTES, fb);
+            for (int nb = 0; nb < BN / 128; ++nb)
+              bulk_load(dst + CS::SFA_BYTES + nb * C::SFA_BYTES,
+                        p.b_scales + ((int64_t)(nt * (BN / 128) + nb) * kbt4 + (int64_t)kt * C::ATOMS_K) * 512,
+                        C::SFA_BYTES, fb);
+          } else {
+            // only the atoms the operands have: na along K, and no 128-row
+            // block past the last one (at least B's first block exists)
+            const int64_t left = kbt4 - (int64_t)kt * C::ATOMS_K;
+            const uint32_t bytes = (uint32_t)(left < C::ATOMS_K ? left : C::ATOMS_K) * 512u;
+            const bool a_in = rb_a < p.rb_a;
+            uint32_t total_bytes = a_in ? bytes : 0u;
+#pragma unroll
+            for (int nb = 0; nb < BN / 128; ++nb)
+              if (nt * (BN / 128) + nb < p.rb_b) total_bytes += bytes;
+            mbar_arrive_expect_tx(fb, total_bytes);
+            if (a_in)
+              bulk_load(dst, p.a_scales + ((int64_t)rb_a * kbt4 + (int64_t)kt * C::ATOMS_K) * 512,
+                        bytes, fb);
+#pragma unroll
+            for (int nb = 0; nb < BN / 128; ++nb)
+              if (nt * (BN / 128) + nb < p.rb_b)
+                bulk_load(dst + CS::SFA_BYTES + nb * C::SFA_BYTES,
+                          p.b_scales + ((int64_t)(nt * (BN / 128) + nb) * kbt4 + (int64_t)kt * C::ATOMS_K) * 512,
+                          bytes, fb);
+          }
           issued |= 1u << s;
           last_parity = (last_parity & ~(1u << s)) | (ph << s);
         }
@@ -623,8 +667,8 @@ __global__ void __launch_bounds__(NUM_THREADS_ST, 1)
           tc_fence_after();
         }
         for (int kt = 0; kt < KT; ++kt, ++g) {
-          const int s = g % ABS, b = g % NBUF;
-          if (!wait_st(smem_u32(&sm->sft_full[b]), (uint32_t)((g / NBUF) & 1), sm, p, 0x230u | b) ||
+          const int s = g % ABS, b = g % CS::NBUF_ST;
+          if (!wait_st(smem_u32(&sm->sft_full[b]), (uint32_t)((g / CS::NBUF_ST) & 1), sm, p, 0x230u | b) ||
               !wait_st(smem_u32(&sm->ab_full[s]), (uint32_t)((g / ABS) & 1), sm, p, 0x210u | s)) {
             ok = false;
             break;
@@ -632,7 +676,7 @@ __global__ void __launch_bounds__(NUM_THREADS_ST, 1)
           tc_fence_after();
           const uint32_t a_base = smem_u32(smem + CS::OFF_A + s * CS::A_BYTES);
           const uint32_t b_base = smem_u32(smem + CS::OFF_B + s * CS::B_BYTES);
-          const uint32_t sf_col = tmem + SF_BASE + b * CS::COLS_BUF;
+          const uint32_t sf_col = tmem + CS::SF_COL0 + b * CS::COLS_BUF;
 #pragma unroll
           for (int j = 0; j < BK / 64; ++j) {
             const int a = (KIND == kMX) ? (j >> 1) : j;
@@ -640,21 +684,32 @@ __global__ void __launch_bounds__(NUM_THREADS_ST, 1)
             const uint32_t sfa = (sf_col + 4 * a) | (sf_id << 30);
             const uint32_t sfb = (sf_col + CS::COLS_A + (BN / 32) * a) | (sf_id << 30);
             if constexpr (KIND == kNVC) {
-              // each 128-K chunk (MMAs 2c, 2c+1) starts a fresh partial in
-              // columns 128c.. once the fold has read its previous content
-              const int c = j >> 1;
+              // chunk q = 2g + c (MMAs 2c, 2c+1 of this k-tile) starts a
+              // fresh partial in buffer q % 3 once the fold has read that
+              // buffer's previous chunk
+              const int q = 2 * g + (j >> 1), pb = q % CS::NPART;
               if ((j & 1) == 0) {
-                if (!wait_st(smem_u32(&sm->part_empty[c]), (uint32_t)((g & 1) ^ 1), sm, p,
-                             0x240u | c)) {
+                if (!wait_st(smem_u32(&sm->part_empty[pb]), (uint32_t)(((q / CS::NPART) & 1) ^ 1), sm,
+                             p, 0x240u | pb)) {
                   ok = false;
                   break;
                 }
                 tc_fence_after();
               }
-              tc_mma<KIND>(tmem + 128 * c, operand_desc(a_base + j * 32),
-                           operand_desc(b_base + j * 32), instr_desc<KIND, BN>(sf_id), sfa, sfb,
-                           (uint32_t)(j & 1));
-              if (j & 1) tc_commit(smem_u32(&sm->part_full[c]));
+              if constexpr (PAIR)
+                tc_mma_pair<KIND>(tmem + 128 * pb, operand_desc(a_base + j * 32),
+                                  operand_desc(b_base + j * 32), instr_desc_pair<KIND, BN>(sf_id),
+                                  sfa, sfb, (uint32_t)(j & 1));
+              else
+                tc_mma<KIND>(tmem + 128 * pb, operand_desc(a_base + j * 32),
+                             operand_desc(b_base + j * 32), instr_desc<KIND, BN>(sf_id), sfa, sfb,
+                             (uint32_t)(j & 1));
+              if (j & 1) {
+                if constexpr (PAIR)
+                  tc_commit_pair(smem_u32(&sm->part_full[pb]), (uint16_t)3);
+                else
+                  tc_commit(smem_u32(&sm->part_full[pb]));
+              }
             } else {
               const uint32_t acc = (kt > 0 || j > 0) ? 1u : 0u;
               if constexpr (PAIR)
@@ -706,29 +761,50 @@ __global__ void __launch_bounds__(NUM_THREADS_ST, 1)
     if constexpr (KIND == kNVG) alpha_g = p.alpha * p.a_ts[0] * p.b_ts[0];
     const uint32_t acc_empty_l = leader_addr(&sm->acc_empty);
 
-    // stage the scales of k-tile g into tensor-memory buffer g % NBUF
+    // stage the scales of k-tile g into tensor-memory buffer g % NBUF_ST
     auto stage_scales = [&](int g) -> bool {
-      const int s = g % SFS, b = g % NBUF;
+      const int s = g % SFS, b = g % CS::NBUF_ST;
       if (!warp_wait_st(smem_u32(&sm->sfs_full[s]), (uint32_t)((g / SFS) & 1), sm, p, 0x320u | s))
         return false;
-      if (g >= NBUF &&
-          !warp_wait_st(smem_u32(&sm->sft_empty[b]), (uint32_t)(((g / NBUF) & 1) ^ 1), sm, p, 0x330u | b))
+      if (g >= CS::NBUF_ST &&
+          !warp_wait_st(smem_u32(&sm->sft_empty[b]), (uint32_t)(((g / CS::NBUF_ST) & 1) ^ 1), sm, p,
+                        0x330u | b))
         return false;
       tc_fence_after();
       const uint8_t *sfa_s = smem + CS::OFF_SF + s * CS::SF_BYTES;
       const uint8_t *sfb_s = sfa_s + CS::SFA_BYTES;
-      const uint32_t col = lane_base + SF_BASE + b * CS::COLS_BUF;
+      const uint32_t col = lane_base + CS::SF_COL0 + b * CS::COLS_BUF;
+      // ragged shapes: atoms the scale producer did not load are zero
+      int na = C::ATOMS_K;
+      bool a_in = true, b_in[BN / 128];
+#pragma unroll
+      for (int nb = 0; nb < BN / 128; ++nb) b_in[nb] = true;
+      if (p.ragged) {
+        const int kt = g % KT;
+        int mt, nt;
+        tile_coords(unit + (g / KT) * nunits, num_m, num_n, p.n_fastest, mt, nt);
+        const int64_t left = kbt4 - (int64_t)kt * C::ATOMS_K;
+        na = left < C::ATOMS_K ? (int)left : C::ATOMS_K;
+        a_in = (PAIR ? mt * 2 + (int)rank : mt) < p.rb_a;
+#pragma unroll
+        for (int nb = 0; nb < BN / 128; ++nb) b_in[nb] = nt * (BN / 128) + nb < p.rb_b;
+      }
       // A: row 32q + lane is word q of atom row `lane`
 #pragma unroll
       for (int a = 0; a < C::ATOMS_K; ++a)
-        tmem_st1(col + 4 * a + q, *reinterpret_cast<const uint32_t *>(sfa_s + a * 512 + lane * 16 + 4 * q));
+        tmem_st1(col + 4 * a + q,
+                 (a_in && a < na)
+                     ? *reinterpret_cast<const uint32_t *>(sfa_s + a * 512 + lane * 16 + 4 * q)
+                     : 0u);
       // B: atom a of each 128-row block: row 32w + lane is word w of atom row `lane`
 #pragma unroll
       for (int a = 0; a < C::ATOMS_K; ++a) {
 #pragma unroll
         for (int nb = 0; nb < BN / 128; ++nb)
           tmem_st4(col + CS::COLS_A + (BN / 32) * a + 4 * nb,
-                   *reinterpret_cast<const uint4 *>(sfb_s + nb * C::SFA_BYTES + a * 512 + lane * 16));
+                   (b_in[nb] && a < na)
+                       ? *reinterpret_cast<const uint4 *>(sfb_s + nb * C::SFA_BYTES + a * 512 + lane * 16)
+                       : make_uint4(0u, 0u, 0u, 0u));
       }
       asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
       tc_fence_before();
@@ -755,9 +831,13 @@ __global__ void __launch_bounds__(NUM_THREADS_ST, 1)
       const int x0 = nt * BN + h * COLS;
       const uint32_t row_base = ebuf + lane * 64;
       const int sw = (lane >> 1) & 3;
+      // ragged shapes: these 32 rows may lie wholly below D (the bulk-tensor
+      // store clips a box that only reaches past M or N)
+      const bool rows_in = !p.ragged || (int64_t)y0 < p.M;
       if (p.out_fp32) {
 #pragma unroll
         for (int ch = 0; ch < COLS / 16; ++ch) {
+          if (p.ragged && (!rows_in || (int64_t)(x0 + 16 * ch) >= p.N)) continue;
           if (lane == 0) bulk_wait_read_all();
           __syncwarp();
 #pragma unroll
@@ -780,6 +860,7 @@ __global__ void __launch_bounds__(NUM_THREADS_ST, 1)
         uint32_t sword = 0;  // this row's MXFP4 scale bytes, one per 32-column chunk
 #pragma unroll
         for (int ch = 0; ch < COLS / 32; ++ch) {
+          const bool chunk_in = !p.ragged || (rows_in && (int64_t)(x0 + 32 * ch) < p.N);
           uint32_t w[16];  // the chunk's 32 bf16 values of D, packed in pairs
 #pragma unroll
           for (int u = 0; u < 16; ++u) {
@@ -805,11 +886,13 @@ __global__ void __launch_bounds__(NUM_THREADS_ST, 1)
             for (int e = 0; e < 32; ++e) f[e] = __fmul_rn(f[e], mult);
             const uint4 codes = make_uint4(e2m1x8_rne(&f[0]), e2m1x8_rne(&f[8]),
                                            e2m1x8_rne(&f[16]), e2m1x8_rne(&f[24]));
-            *reinterpret_cast<uint4 *>(p.q_payload + row * (p.N >> 1) + ((x0 + 32 * ch) >> 1)) =
-                codes;
+            // rows and blocks outside D hold zero accumulators: scale byte 0
+            if (!p.ragged || (row < p.M && (int64_t)(x0 + 32 * ch) < p.N))
+              *reinterpret_cast<uint4 *>(p.q_payload + row * (p.N >> 1) + ((x0 + 32 * ch) >> 1)) =
+                  codes;
             sword |= sbyte << (8 * ch);
           }
-          if (p.store_d) {
+          if (p.store_d && chunk_in) {
             if (lane == 0) bulk_wait_read_all();
             __syncwarp();
 #pragma unroll
@@ -825,32 +908,49 @@ __global__ void __launch_bounds__(NUM_THREADS_ST, 1)
         }
         if constexpr (QOUT) {
           // blocks x0/32 .. of this row: a whole scale word (128 columns) or
-          // its half (64 columns, the other half is the quadrant's other warp)
-          uint8_t *sdst = p.q_scales + sf_offset(row, x0 >> 5, p.N >> 5);
-          if constexpr (COLS == 128)
-            *reinterpret_cast<uint32_t *>(sdst) = sword;
-          else
-            *reinterpret_cast<uint16_t *>(sdst) = (uint16_t)sword;
+          // its half (64 columns, the other half is the quadrant's other warp);
+          // ragged: rows up to the next multiple of 128 and blocks up to the
+          // next multiple of 4 are the operand's padding (written, zero)
+          const int64_t nbk = p.N >> 5;
+          if (!p.ragged || (row < p.rb_a * 128 && (int64_t)(x0 >> 5) < nbk)) {
+            uint8_t *sdst = p.q_scales + sf_offset(row, x0 >> 5, (nbk + 3) & ~int64_t(3));
+            if constexpr (COLS == 128)
+              *reinterpret_cast<uint32_t *>(sdst) = sword;
+            else
+              *reinterpret_cast<uint16_t *>(sdst) = (uint16_t)sword;
+          }
         }
       }
     };
 
     if constexpr (KIND == kNVC) {
-      // CTA-local NVFP4: per k-tile, stage this warp's scales up to NBUF
-      // k-tiles ahead, then fold both 128-K chunk partials into FP32
+      // CTA-local NVFP4: per k-tile, stage this warp's scales up to NBUF_ST
+      // k-tiles ahead, then fold the k-tile's two 128-K chunk partials into FP32
       // registers, acc += tsA[m/128][kc] * tsB[n/128][kc] * partial, and
       // release each partial as soon as it is read; store at the tile's end
-      const int nk = (int)(p.K / 128);
+      const int nk = (int)((p.K + 127) / 128);  // 128-wide K chunks (the last may be short)
       int g_st = h, g = 0;
       bool ok = true;
       for (int tile = unit; tile < num_tiles && ok; tile += nunits) {
         int mt, nt;
         tile_coords(tile, num_m, num_n, p.n_fastest, mt, nt);
-        float acc[COLS];
+        // packed pairs of accumulator columns (2i, 2i+1): one fma.rn.f32x2
+        // folds both, the same rounding as fmaf on each
+        uint64_t acc2[COLS / 2];
 #pragma unroll
-        for (int i = 0; i < COLS; ++i) acc[i] = 0.0f;
+        for (int i = 0; i < COLS / 2; ++i) acc2[i] = 0ull;
         for (int kt = 0; kt < KT && ok; ++kt, ++g) {
-          for (; g_st < total && g_st < g + NBUF; g_st += 2)
+          // the two chunks' factors, loaded before the waits below so that
+          // their global-memory latency overlaps them (a chunk wholly past K,
+          // ragged, holds a zero partial and gets no scale)
+          float fk[2];
+#pragma unroll
+          for (int c = 0; c < 2; ++c) {
+            const int kc = 2 * kt + c;
+            const int mb = PAIR ? mt * 2 + (int)rank : mt;  // this CTA's 128-row block of A
+            fk[c] = kc < nk ? p.a_ts[(int64_t)mb * nk + kc] * p.b_ts[(int64_t)nt * nk + kc] : 0.0f;
+          }
+          for (; g_st < total && g_st < g + CS::NBUF_ST; g_st += 2)
             if (!stage_scales(g_st)) {
               ok = false;
               break;
@@ -858,7 +958,9 @@ __global__ void __launch_bounds__(NUM_THREADS_ST, 1)
           if (!ok) break;
 #pragma unroll
           for (int c = 0; c < 2; ++c) {
-            if (!warp_wait_st(smem_u32(&sm->part_full[c]), (uint32_t)(g & 1), sm, p, 0x340u | c)) {
+            const int q = 2 * g + c, pb = q % CS::NPART;  // chunk q's partial buffer
+            if (!warp_wait_st(smem_u32(&sm->part_full[pb]), (uint32_t)((q / CS::NPART) & 1), sm, p,
+                              0x340u | pb)) {
               ok = false;
               break;
             }
@@ -866,21 +968,26 @@ __global__ void __launch_bounds__(NUM_THREADS_ST, 1)
             uint32_t r[COLS];
 #pragma unroll
             for (int ch = 0; ch < NCH; ++ch)
-              tmem_ld32(lane_base + 128 * c + h * COLS + 32 * ch, &r[32 * ch]);
+              tmem_ld32(lane_base + 128 * pb + h * COLS + 32 * ch, &r[32 * ch]);
             tmem_wait_ld();
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(smem_u32(&sm->part_empty[c]));
-            const int kc = 2 * kt + c;
-            const float f = p.a_ts[(int64_t)mt * nk + kc] * p.b_ts[(int64_t)nt * nk + kc];
+            if (lane == 0) {
+              if (PAIR && rank != 0)
+                mbar_arrive_remote_relaxed(leader_addr(&sm->part_empty[pb]));
+              else
+                mbar_arrive(smem_u32(&sm->part_empty[pb]));
+            }
+            const uint64_t f2 = f2_pack(fk[c], fk[c]);
 #pragma unroll
-            for (int i = 0; i < COLS; ++i) acc[i] = fmaf(f, __uint_as_float(r[i]), acc[i]);
+            for (int i = 0; i < COLS / 2; ++i)
+              acc2[i] = f2_fma(f2, f2_pack_bits(r[2 * i], r[2 * i + 1]), acc2[i]);
           }
         }
         if (!ok) break;
         uint32_t r[COLS];
 #pragma unroll
-        for (int i = 0; i < COLS; ++i) r[i] = __float_as_uint(acc[i]);
+        for (int i = 0; i < COLS / 2; ++i) f2_unpack_bits(acc2[i], r[2 * i], r[2 * i + 1]);
         store_tile(r, mt, nt);
       }
     } else {
@@ -892,7 +999,7 @@ __global__ void __launch_bounds__(NUM_THREADS_ST, 1)
     for (int tile = unit; tile < num_tiles && ok; tile += nunits, ++it) {
       // scales for the rest of this tile and the first NBUF k-tiles of the
       // next one, then this tile's epilogue
-      const int until = min(total, (it + 1) * KT + NBUF);
+      const int until = min(total, (it + 1) * KT + CS::NBUF_ST);
       for (; g < until; g += 2)
         if (!stage_scales(g)) {
           ok = false;
@@ -1022,6 +1129,9 @@ static gemm::Params make_params(const GemmArgs &a) {
   p.q_payload = a.q_payload;
   p.q_scales = a.q_scales;
   p.store_d = a.D != nullptr;
+  p.rb_a = (a.M + 127) / 128;
+  p.rb_b = (a.N + 127) / 128;
+  p.ragged = 0;  // set by the launcher for its tile shape
   return p;
 }
 
@@ -1030,18 +1140,20 @@ static cudaError_t launch_st(const GemmArgs &a, cudaStream_t st) {
   constexpr int smem = gemm_st::total_smem_st<KIND, BN, PAIR>();
   CUtensorMap ma, mb;
   if (!make_payload_map(&ma, a.a_payload, a.M, a.K, gemm::BM)) return cudaErrorInvalidValue;
-  if (!make_payload_map(&mb, a.b_payload, a.N, a.K, PAIR ? 128 : BN)) return cudaErrorInvalidValue;
+  if (!make_payload_map(&mb, a.b_payload, a.N, a.K, PAIR ? BN / 2 : BN)) return cudaErrorInvalidValue;
   CUtensorMap md;
   memset(&md, 0, sizeof(md));
   if (a.D && !make_out_map(&md, a)) return cudaErrorInvalidValue;
   gemm::Params p = make_params(a);
+  constexpr int TILE_M = PAIR ? 256 : gemm::BM;
+  p.ragged = (a.M % TILE_M) || (a.N % BN) || (a.K % gemm::BK);
   auto kern = gemm_st::gemm_st_kernel<KIND, BN, PAIR, QOUT>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  const int64_t tiles = (a.M / (PAIR ? 256 : gemm::BM)) * (a.N / BN);
+  const int64_t tiles = ((a.M + TILE_M - 1) / TILE_M) * ((a.N + BN - 1) / BN);
   cudaLaunchConfig_t cfg = {};
   cfg.blockDim = dim3(gemm_st::NUM_THREADS_ST);
   cfg.dynamicSmemBytes = smem;
@@ -1072,8 +1184,11 @@ static cudaError_t launch_st(const GemmArgs &a, cudaStream_t st) {
 
 template <bool QOUT>
 static cudaError_t launch_st_any(const GemmArgs &a, cudaStream_t st) {
-  const bool wide = (a.N % 256) == 0;
-  const bool pair = wide && (a.M % 256) == 0;
+  // 256-wide tiles (and 256-row pairs) where they cover no more than
+  // 128-wide (128-row) tiles would
+  auto up = [](int64_t v, int64_t m) { return (v + m - 1) / m * m; };
+  const bool wide = up(a.N, 256) == up(a.N, 128);
+  const bool pair = wide && up(a.M, 256) == up(a.M, 128);
   if (a.fmt == kMX)
     return pair ? launch_st<kMX, 256, true, QOUT>(a, st)
                 : (wide ? launch_st<kMX, 256, false, QOUT>(a, st) : launch_st<kMX, 128, false, QOUT>(a, st));
@@ -1090,7 +1205,12 @@ cudaError_t launch_gemm_blockscaled(const GemmArgs &a, cudaStream_t st) {
     if (!a.D) return cudaErrorInvalidValue;
     return launch_st_any<false>(a, st);
   }
-  if (a.fmt == kNVC && !a.q_payload && a.D) return launch_st<kNVC, 128, false, false>(a, st);
+  if (a.fmt == kNVC && !a.q_payload && a.D) {
+    // 2-SM pairs (M = 256 per pair) where they cover no more rows than
+    // 128-row tiles would
+    const bool pair = (a.M + 255) / 256 * 256 == (a.M + 127) / 128 * 128;
+    return pair ? launch_st<kNVC, 128, true, false>(a, st) : launch_st<kNVC, 128, false, false>(a, st);
+  }
   return cudaErrorInvalidValue;
 }
 

@@ -60,7 +60,9 @@ fa4_status fa4_quantize_nvfp4_global_noalloc(const void *x, int64_t rows, int64_
   if ((rnd != FA4_RNE && rnd != FA4_SR) || (orient != FA4_ROWWISE && orient != FA4_COLWISE))
     return FA4_ERR_INVALID_ARG;
   if (!x || !out.payload || !out.scales || !out.tensor_scale) return FA4_ERR_INVALID_ARG;
-  if (rows <= 0 || cols <= 0 || rows % 128 || cols % 128 || ld < cols || ld % 8) return FA4_ERR_SHAPE;
+  // Q[R, K]: any R, K a multiple of 32; x rows read in 16-byte pieces
+  const int64_t K = orient == FA4_ROWWISE ? cols : rows;
+  if (rows <= 0 || cols <= 0 || cols % 8 || K % 32 || ld < cols || ld % 8) return FA4_ERR_SHAPE;
   if (!aligned16(x) || !aligned16(out.payload) || !aligned16(out.scales) ||
       (reinterpret_cast<uintptr_t>(out.tensor_scale) & 3u))
     return FA4_ERR_ALIGN;

@@ -22,8 +22,11 @@
  *  - Every function returns an fa4_status; nothing throws across the ABI.
  *    Argument errors are detected on the host before anything is launched.
  *    A launch failure returns FA4_ERR_CUDA (cudaGetLastError).
- *  - Shapes: rows and cols multiples of 128 (GEMM K a multiple of 256);
- *    leading dimensions in elements,
+ *  - Shapes: a quantized operand Q[R, K] may have any number of rows R and
+ *    K (the block dimension) a multiple of 32; an input x[rows, cols] has
+ *    cols a multiple of 8.  GEMM: any M and N, K a multiple of 32.  Scale
+ *    atoms are padded (rows to a multiple of 128, blocks to a multiple of 4,
+ *    the padding written as zero bytes).  Leading dimensions in elements,
  *    multiples of 8 and >= the row length; every pointer 16-byte aligned.
  *    Anything else returns FA4_ERR_SHAPE / FA4_ERR_ALIGN.
  *  - Inputs must be finite; with a non-finite input the output bytes are
@@ -64,7 +67,9 @@ extern "C" {
  *                   for the tensor ("FP4 Is No Longer Just a Hardware
  *                   Feature...", section "NVFP4 is more than a 4-bit value").
  *  FA4_NVFP4_CTA    as NVFP4_GLOBAL but one FP32 decode scale per 128x128
- *                   tile of the quantized operand, [R/128][K/128].
+ *                   tile of the quantized operand, [ceil(R/128)][ceil(K/128)]
+ *                   (a tile cut by the operand's edge takes the amax of the
+ *                   values it holds).
  *  FA4_MXFP4_NOCLIP MXFP4 with the other power-of-two scale rule: the
  *                   smallest e with amax <= 6 * 2^e, so no value saturates
  *                   (FA4_MXFP4 takes floor(log2 amax) - 2 and saturates
@@ -97,7 +102,7 @@ typedef enum { FA4_OUT_BF16 = 0, FA4_OUT_FP32 = 1 } fa4_out_dtype;
 typedef enum {
   FA4_OK = 0,
   FA4_ERR_INVALID_ARG = 1, /* null pointer, bad enum value */
-  FA4_ERR_SHAPE = 2,       /* size not a multiple of 128, bad ld, K mismatch */
+  FA4_ERR_SHAPE = 2,       /* K not a multiple of 32, bad ld, empty tensor */
   FA4_ERR_ALIGN = 3,       /* pointer not 16-byte aligned */
   FA4_ERR_UNSUPPORTED = 4, /* e.g. Hadamard with NVFP4, mixed GEMM formats */
   FA4_ERR_WORKSPACE = 5,   /* workspace missing or smaller than required */
@@ -111,12 +116,14 @@ typedef enum {
  *               sign<<3 | exponent<<1 | mantissa).
  *  scales       one byte per block (E8M0 for MXFP4, E4M3 for NVFP4) in the
  *               128-row x 4-block atom layout the block-scaled tensor-core
- *               MMA reads: byte offset of (row r, block kb), Kb = K/block,
- *               ((r/128)*(Kb/4) + kb/4)*512 + (r%32)*16 + ((r%128)/32)*4
- *               + kb%4.  R*Kb bytes.
+ *               MMA reads: byte offset of (row r, block kb), with Kb4 =
+ *               K/block rounded up to a multiple of 4,
+ *               ((r/128)*(Kb4/4) + kb/4)*512 + (r%32)*16 + ((r%128)/32)*4
+ *               + kb%4.  ceil(R/128)*128*Kb4 bytes; the bytes of rows >= R
+ *               and blocks >= K/block are zero.
  *  tensor_scale FP32 decode scales: NVFP4_GLOBAL 1 value, NVFP4_CTA
- *               (R/128)*(K/128) values, row-major; unused (may be NULL) for
- *               MXFP4.  value = e2m1 * block scale * tensor_scale. */
+ *               ceil(R/128)*ceil(K/128) values, row-major; unused (may be
+ *               NULL) for MXFP4.  value = e2m1 * block scale * tensor_scale. */
 typedef struct {
   void *payload;
   void *scales;
@@ -187,8 +194,9 @@ FA4_API fa4_status fa4_quantize_dual(const void *x, int64_t rows, int64_t cols, 
  * K-major).  NVFP4_GLOBAL multiplies by the two tensor decode scales;
  * NVFP4_CTA multiplies every 128-wide K chunk by tsA[m/128][kc] *
  * tsB[n/128][kc].  FP32 accumulation.  D is row-major [M, N] with leading
- * dimension ldd elements (a multiple of 8, at least N), bf16 or fp32.  M and
- * N multiples of 128, K a multiple of 256 (one k-tile).  Workspace: at least
+ * dimension ldd elements (a multiple of 8, at least N), bf16 or fp32.  Any
+ * M and N; K a multiple of 32 (the tiles past M, N or K compute on zero
+ * payload and zero scales).  Workspace: at least
  * FA4_WS_HEADER_BYTES (the bounded-wait status word).
  * Errors: SHAPE, ALIGN, INVALID_ARG, UNSUPPORTED, WORKSPACE, CUDA. */
 FA4_API fa4_status fa4_gemm_blockscaled(fa4_qtensor A, fa4_qtensor B, int64_t M, int64_t N, int64_t K,
@@ -200,11 +208,12 @@ FA4_API fa4_status fa4_gemm_blockscaled(fa4_qtensor A, fa4_qtensor B, int64_t M,
  * Fusion...", section "The Design Philosophy of Format-Aware Fusion": the
  * producer of the next operand is the GEMM that computes it): the bf16
  * output D = alpha * A B^T is written (when D is not NULL) and its row-wise
- * MXFP4 operand (RNE) goes to Dq ([M, N/2] payload, M*N/32 scale bytes in
- * the atom layout), byte-identical to fa4_quantize(D, FA4_MXFP4, FA4_RNE,
- * FA4_ROWWISE) of that bf16 D, without reading D back.  fmt MXFP4 or
- * NVFP4_GLOBAL (FA4_ERR_UNSUPPORTED for NVFP4_CTA).  Other requirements and
- * errors as fa4_gemm_blockscaled. */
+ * MXFP4 operand (RNE) goes to Dq ([M, N/2] payload, scale bytes in the
+ * padded atom layout of an [M, N] operand), byte-identical to
+ * fa4_quantize(D, FA4_MXFP4, FA4_RNE, FA4_ROWWISE) of that bf16 D, without
+ * reading D back.  N a multiple of 32.  fmt MXFP4 or NVFP4_GLOBAL
+ * (FA4_ERR_UNSUPPORTED for NVFP4_CTA).  Other requirements and errors as
+ * fa4_gemm_blockscaled. */
 FA4_API fa4_status fa4_gemm_blockscaled_mxout(fa4_qtensor A, fa4_qtensor B, int64_t M, int64_t N,
                                       int64_t K, fa4_format fmt, float alpha, void *D, int64_t ldd,
                                       fa4_qtensor Dq, void *workspace, size_t workspace_bytes,
@@ -212,7 +221,9 @@ FA4_API fa4_status fa4_gemm_blockscaled_mxout(fa4_qtensor A, fa4_qtensor B, int6
 
 /* Linear layer compositions for T tokens, Cin inputs, Cout outputs (the
  * configurations the pages' Llama-3-8B results train: "Format-Aware
- * Fusion...", section "Empirical Results").  bf16 activations row-major.
+ * Fusion...", section "Empirical Results").  bf16 activations row-major;
+ * T, Cin and Cout multiples of 32 (each is the block dimension of some
+ * operand).
  *
  * fa4_linear_fwd:   Y[T, Cout] (bf16) = X[T, Cin] W^T.  X is quantized
  *                   row-wise (RNE) in `fmt` into the workspace; Wq is W[Cout,
@@ -242,7 +253,7 @@ FA4_API fa4_status fa4_linear_wgrad(const void *dY, const void *X, int64_t T, in
 /* Training form of the linear layer, forward half: Y = X W^T as
  * fa4_linear_fwd (X row-wise in `fmt`, RNE), and from the same read of X its
  * column-wise MXFP4 operand with the fixed-sign Hadamard (RNE) into the
- * caller's Xcol ([Cin, T]: payload Cin*T/2 bytes, scales Cin*T/32 bytes), the
+ * caller's Xcol ([Cin, T]: payload Cin*T/2 bytes, scales as fa4_quant_sizes), the
  * state the backward half needs instead of the bf16 X ("Format-Aware
  * Fusion...", section "The Design Philosophy of Format-Aware Fusion": the
  * state kept for the backward pass is the FP4 operand, not the bf16 X).  Y and Xcol equal fa4_linear_fwd and

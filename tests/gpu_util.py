@@ -29,8 +29,10 @@ def to_gpu_qt(q: O.QTensor, device="cuda") -> fa.QTensor:
 
 
 def scale_byte_range(q: O.QTensor, r0: int, r1: int) -> slice:
-    kb4 = q.K // O.BLOCK[q.fmt] // 4
-    return slice((r0 // 128) * kb4 * 512, (r1 // 128) * kb4 * 512)
+    """Scale bytes of the 128-row atom rows that hold rows r0 .. r1-1 (with
+    the padding of a ragged last atom row)."""
+    kb4 = -(-(q.K // O.BLOCK[q.fmt]) // 4)
+    return slice((r0 // 128) * kb4 * 512, -(-r1 // 128) * kb4 * 512)
 
 
 def assert_qt_equal(g: O.QTensor, o: O.QTensor, row_range=None):
@@ -52,9 +54,9 @@ def assert_qt_equal(g: O.QTensor, o: O.QTensor, row_range=None):
     if g.fmt == O.NVFP4_GLOBAL:
         assert g.ts.view(np.uint32)[0] == o.ts.view(np.uint32)[0], (g.ts, o.ts)
     elif g.fmt == O.NVFP4_CTA:
-        nk = g.K // 128
-        gt = g.ts.reshape(-1, nk)[r0 // 128:r1 // 128]
-        ot = o.ts.reshape(-1, nk)[r0 // 128:r1 // 128]
+        nk = -(-g.K // 128)
+        gt = g.ts.reshape(-1, nk)[r0 // 128:-(-r1 // 128)]
+        ot = o.ts.reshape(-1, nk)[r0 // 128:-(-r1 // 128)]
         assert np.array_equal(gt.view(np.uint32), ot.view(np.uint32))
 
 

@@ -51,6 +51,19 @@ def test_quant_sizes_match_the_layout(fmt, orient):
     assert ws >= fa.WS_HEADER_BYTES
 
 
+@pytest.mark.parametrize("fmt", [fa.MXFP4, fa.NVFP4_GLOBAL, fa.NVFP4_CTA, fa.MXFP4_NOCLIP])
+@pytest.mark.parametrize("rows,cols,orient", [(200, 352, fa.ROWWISE), (352, 200, fa.COLWISE),
+                                              (1, 32, fa.ROWWISE), (32, 8, fa.COLWISE)])
+def test_quant_sizes_of_ragged_operands(fmt, rows, cols, orient):
+    """Rows of Q not a multiple of 128 and K not a multiple of 128: scale
+    atoms padded as the oracle pads them."""
+    pb, sb, tc, _ = fa.quant_sizes(rows, cols, fmt, orient)
+    R, K = (rows, cols) if orient == fa.ROWWISE else (cols, rows)
+    assert pb == R * K // 2
+    assert sb == O.sf_bytes(R, K // fa.BLOCK[fmt])
+    assert tc == O.ts_count(R, K, fmt)
+
+
 def _qt(p=0x10000, s=0x20000, t=0x30000):
     return fa._QT(p, s, t)
 
@@ -60,8 +73,10 @@ DEV = 0x7F0000000000  # never dereferenced: every call below fails validation fi
 
 @pytest.mark.parametrize("case,expect", [
     (dict(x=None), 1),
-    (dict(rows=100), 2),
-    (dict(cols=200), 2),
+    (dict(rows=0), 2),
+    (dict(cols=100), 2),        # x rows are read in 16-byte pieces
+    (dict(cols=200), 2),        # K (= cols, row-wise) a multiple of 32
+    (dict(rows=200, orient=1), 2),  # K (= rows, column-wise) a multiple of 32
     (dict(ld=120), 2),
     (dict(ld=132), 2),
     (dict(x=DEV + 8), 3),
@@ -94,8 +109,8 @@ def test_hadamard_quantize_rejects_bad_arguments():
 
 
 @pytest.mark.parametrize("case,expect", [
-    (dict(M=100), 2),
-    (dict(K=384), 2),          # K must be a multiple of 256
+    (dict(M=0), 2),
+    (dict(K=48), 2),           # K must be a multiple of 32
     (dict(ldd=100), 2),
     (dict(D=None), 1),
     (dict(D=DEV + 4), 3),
@@ -162,7 +177,8 @@ def test_noalloc_quantize_rejects_bad_arguments():
     L = fa.lib()
     q = _qt()
     assert L.fa4_quantize_nvfp4_global_noalloc(None, 256, 256, 256, 0, 0, 0, q, None) == 1
-    assert L.fa4_quantize_nvfp4_global_noalloc(DEV, 250, 256, 256, 0, 0, 0, q, None) == 2
+    assert L.fa4_quantize_nvfp4_global_noalloc(DEV, 256, 250, 256, 0, 0, 0, q, None) == 2
+    assert L.fa4_quantize_nvfp4_global_noalloc(DEV, 240, 256, 256, 0, 1, 0, q, None) == 2
     assert L.fa4_quantize_nvfp4_global_noalloc(DEV, 256, 256, 200, 0, 0, 0, q, None) == 2
     assert L.fa4_quantize_nvfp4_global_noalloc(DEV + 4, 256, 256, 256, 0, 0, 0, q, None) == 3
     assert L.fa4_quantize_nvfp4_global_noalloc(DEV, 256, 256, 256, 3, 0, 0, q, None) == 1
@@ -219,7 +235,8 @@ def test_mxout_gemm_rejects_bad_arguments():
     f = L.fa4_gemm_blockscaled_mxout
     assert f(q, q, 256, 256, 512, fa.NVFP4_CTA, 1.0, DEV, 256, q, DEV, 4096, None) == 4
     assert f(q, q, 256, 256, 512, 7, 1.0, DEV, 256, q, DEV, 4096, None) == 1
-    assert f(q, q, 256, 256, 384, fa.MXFP4, 1.0, DEV, 256, q, DEV, 4096, None) == 2
+    assert f(q, q, 256, 256, 48, fa.MXFP4, 1.0, DEV, 256, q, DEV, 4096, None) == 2
+    assert f(q, q, 256, 240, 512, fa.MXFP4, 1.0, DEV, 256, q, DEV, 4096, None) == 2  # N % 32
     assert f(q, q, 256, 256, 512, fa.MXFP4, 1.0, DEV + 8, 256, q, DEV, 4096, None) == 3
     assert f(q, q, 256, 256, 512, fa.MXFP4, 1.0, DEV, 256, fa._QT(0, 0, 0), DEV, 4096, None) == 1
     assert f(q, q, 256, 256, 512, fa.MXFP4, 1.0, None, 0, fa._QT(0x10008, 0x20000, 0), DEV, 4096,
