@@ -89,26 +89,38 @@ fa4_status cuda_status(cudaError_t e) { return e == cudaSuccess ? FA4_OK : FA4_E
 fa4_status do_quantize(const void *x, int64_t rows, int64_t cols, int64_t ld, int fmt, int rnd,
                        int orient, bool hadamard, uint32_t sign_mask, uint64_t seed,
                        const fa4_qtensor &out, uint8_t *ws, cudaStream_t st) {
-  const uint16_t *xb = static_cast<const uint16_t *>(x);
-  float *partials = reinterpret_cast<float *>(ws + kHdr);
-  int np = 0;
+  fa4::QuantArgs q;
+  q.x = static_cast<const uint16_t *>(x);
+  q.T = rows;
+  q.C = cols;
+  q.ld = ld;
+  q.status = reinterpret_cast<uint32_t *>(ws);
+  q.timeout_ns = kDefaultTimeoutNs;
   if (fmt == FA4_NVFP4_GLOBAL) {
-    np = fa4::amax_partials_count(rows, cols);
-    cudaError_t e = fa4::launch_tensor_amax(xb, rows, cols, ld, partials, np, st);
+    q.partials = reinterpret_cast<float *>(ws + kHdr);
+    q.n_partials = fa4::amax_partials_count(rows, cols);
+    cudaError_t e = fa4::launch_tensor_amax(q.x, rows, cols, ld, reinterpret_cast<float *>(ws + kHdr),
+                                            q.n_partials, st);
     if (e != cudaSuccess) return FA4_ERR_CUDA;
   }
-  cudaError_t e;
   if (orient == FA4_ROWWISE) {
-    e = fa4::launch_quant_rowwise(fmt, rnd, xb, rows, cols, ld, static_cast<uint8_t *>(out.payload),
-                                  static_cast<uint8_t *>(out.scales), out.tensor_scale, partials, np,
-                                  seed, st);
+    q.row_fmt = fmt;
+    q.row_rnd = rnd;
+    q.row_payload = static_cast<uint8_t *>(out.payload);
+    q.row_scales = static_cast<uint8_t *>(out.scales);
+    q.row_ts = out.tensor_scale;
+    q.row_seed = seed;
   } else {
-    e = fa4::launch_quant_colwise(fmt, rnd, hadamard, sign_mask, xb, rows, cols, ld,
-                                  static_cast<uint8_t *>(out.payload),
-                                  static_cast<uint8_t *>(out.scales), out.tensor_scale, partials, np,
-                                  seed, st);
+    q.col_fmt = fmt;
+    q.col_rnd = rnd;
+    q.hadamard = hadamard;
+    q.sign_mask = sign_mask;
+    q.col_payload = static_cast<uint8_t *>(out.payload);
+    q.col_scales = static_cast<uint8_t *>(out.scales);
+    q.col_ts = out.tensor_scale;
+    q.col_seed = seed;
   }
-  return cuda_status(e);
+  return cuda_status(fa4::launch_quantize(q, st));
 }
 
 // Both orientations from one read of x (the row-wise NVFP4-global amax pass
@@ -117,19 +129,35 @@ fa4_status do_quantize_dual(const void *x, int64_t rows, int64_t cols, int64_t l
                             int row_rnd, uint64_t row_seed, const fa4_qtensor &row_out,
                             bool hadamard, uint32_t sign_mask, int col_rnd, uint64_t col_seed,
                             const fa4_qtensor &col_out, uint8_t *ws, cudaStream_t st) {
-  const uint16_t *xb = static_cast<const uint16_t *>(x);
-  float *partials = reinterpret_cast<float *>(ws + kHdr);
-  int np = 0;
+  fa4::QuantArgs q;
+  q.x = static_cast<const uint16_t *>(x);
+  q.T = rows;
+  q.C = cols;
+  q.ld = ld;
+  q.status = reinterpret_cast<uint32_t *>(ws);
+  q.timeout_ns = kDefaultTimeoutNs;
   if (row_fmt == FA4_NVFP4_GLOBAL) {
-    np = fa4::amax_partials_count(rows, cols);
-    cudaError_t e = fa4::launch_tensor_amax(xb, rows, cols, ld, partials, np, st);
+    q.partials = reinterpret_cast<float *>(ws + kHdr);
+    q.n_partials = fa4::amax_partials_count(rows, cols);
+    cudaError_t e = fa4::launch_tensor_amax(q.x, rows, cols, ld, reinterpret_cast<float *>(ws + kHdr),
+                                            q.n_partials, st);
     if (e != cudaSuccess) return FA4_ERR_CUDA;
   }
-  return cuda_status(fa4::launch_quant_dual(
-      row_fmt, row_rnd, col_rnd, hadamard, sign_mask, xb, rows, cols, ld,
-      static_cast<uint8_t *>(row_out.payload), static_cast<uint8_t *>(row_out.scales),
-      row_out.tensor_scale, static_cast<uint8_t *>(col_out.payload),
-      static_cast<uint8_t *>(col_out.scales), partials, np, row_seed, col_seed, st));
+  q.row_fmt = row_fmt;
+  q.row_rnd = row_rnd;
+  q.row_payload = static_cast<uint8_t *>(row_out.payload);
+  q.row_scales = static_cast<uint8_t *>(row_out.scales);
+  q.row_ts = row_out.tensor_scale;
+  q.row_seed = row_seed;
+  q.col_fmt = FA4_MXFP4;
+  q.col_rnd = col_rnd;
+  q.hadamard = hadamard;
+  q.sign_mask = sign_mask;
+  q.col_payload = static_cast<uint8_t *>(col_out.payload);
+  q.col_scales = static_cast<uint8_t *>(col_out.scales);
+  q.col_ts = nullptr;
+  q.col_seed = col_seed;
+  return cuda_status(fa4::launch_quantize(q, st));
 }
 
 fa4_status do_gemm(const fa4_qtensor &A, const fa4_qtensor &B, int64_t M, int64_t N, int64_t K,

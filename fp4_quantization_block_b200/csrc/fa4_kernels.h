@@ -2,6 +2,7 @@
 // and the kernels.  Not installed; not part of the public ABI.
 #pragma once
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -13,21 +14,32 @@ constexpr int kMaxAmaxPartials = 1184;  // 8 CTAs x 148 SMs
 int amax_partials_count(int64_t rows, int64_t cols);
 cudaError_t launch_tensor_amax(const uint16_t *x, int64_t rows, int64_t cols, int64_t ld,
                                float *partials, int n_partials, cudaStream_t st);
-cudaError_t launch_quant_rowwise(int fmt, int rnd, const uint16_t *x, int64_t R, int64_t K,
-                                 int64_t ld, uint8_t *payload, uint8_t *scales, float *ts,
-                                 const float *partials, int n_partials, uint64_t seed,
-                                 cudaStream_t st);
-cudaError_t launch_quant_colwise(int fmt, int rnd, bool hadamard, uint32_t sign_mask,
-                                 const uint16_t *x, int64_t T, int64_t C, int64_t ld,
-                                 uint8_t *payload, uint8_t *scales, float *ts,
-                                 const float *partials, int n_partials, uint64_t seed,
-                                 cudaStream_t st);
-cudaError_t launch_quant_dual(int row_fmt, int row_rnd, int col_rnd, bool hadamard,
-                              uint32_t sign_mask, const uint16_t *x, int64_t T, int64_t C,
-                              int64_t ld, uint8_t *row_payload, uint8_t *row_scales, float *row_ts,
-                              uint8_t *col_payload, uint8_t *col_scales, const float *partials,
-                              int n_partials, uint64_t row_seed, uint64_t col_seed,
-                              cudaStream_t st);
+// One quantize launch: x[T, C] (bf16, leading dimension ld) to the row-wise
+// operand (Q = x), the column-wise operand (Q = x^T), or both.  A format of
+// -1 skips that orientation.  When both are produced the column-wise operand
+// is MXFP4 (optionally through the fixed-sign Hadamard).
+struct QuantArgs {
+  const uint16_t *x;
+  int64_t T, C, ld;
+  int row_fmt = -1, row_rnd = 0;
+  uint8_t *row_payload = nullptr, *row_scales = nullptr;
+  float *row_ts = nullptr;
+  uint64_t row_seed = 0;
+  int col_fmt = -1, col_rnd = 0;
+  bool hadamard = false;
+  uint32_t sign_mask = 0;
+  uint8_t *col_payload = nullptr, *col_scales = nullptr;
+  float *col_ts = nullptr;
+  uint64_t col_seed = 0;
+  const float *partials = nullptr;  // NVFP4-global amax partials (either orientation)
+  int n_partials = 0;
+  uint32_t *status = nullptr;  // bounded-wait status word (may be null)
+  uint64_t timeout_ns = 2000000000ull;
+};
+cudaError_t launch_quantize(const QuantArgs &a, cudaStream_t st);
+// Tensor map of a bf16 matrix [rows, cols] (row stride ld elements) in
+// 128 x 128 boxes, no swizzle, zero fill past the edges.
+bool make_bf16_tile_map(CUtensorMap *m, const void *base, int64_t rows, int64_t cols, int64_t ld);
 cudaError_t launch_debug_convert(const float *y, const uint32_t *u16, int64_t n, uint8_t *rne,
                                  uint8_t *sr, uint8_t *e4m3, cudaStream_t st);
 cudaError_t launch_debug_sr_bits(uint64_t seed, const uint64_t *idx, int64_t n, uint32_t *bits,

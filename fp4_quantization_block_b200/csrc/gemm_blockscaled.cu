@@ -929,6 +929,22 @@ __global__ void __launch_bounds__(NUM_THREADS_ST, 1)
       // registers, acc += tsA[m/128][kc] * tsB[n/128][kc] * partial, and
       // release each partial as soon as it is read; store at the tile's end
       const int nk = (int)((p.K + 127) / 128);  // 128-wide K chunks (the last may be short)
+      // The chunk factors tsA[mb][kc] * tsB[nt][kc] of this CTA's chunk
+      // sequence Q = (tile iteration) * 2 KT + kc, 32 at a time: lane i
+      // holds chunk 32 b + i of block b in fcur, the next block in fnext,
+      // loaded a whole block (32 chunks of MMAs) before it is needed (a
+      // chunk wholly past K, ragged, holds a zero partial and gets factor 0)
+      const int cpt = 2 * KT;  // chunks per tile
+      auto chunk_factor = [&](int Q) -> float {
+        if (Q >= total * 2) return 0.0f;
+        const int kc = Q % cpt;
+        if (kc >= nk) return 0.0f;
+        int mt, nt;
+        tile_coords(unit + (Q / cpt) * nunits, num_m, num_n, p.n_fastest, mt, nt);
+        const int mb = PAIR ? mt * 2 + (int)rank : mt;  // this CTA's 128-row block of A
+        return p.a_ts[(int64_t)mb * nk + kc] * p.b_ts[(int64_t)nt * nk + kc];
+      };
+      float fcur = chunk_factor(lane), fnext = chunk_factor(32 + lane);
       int g_st = h, g = 0;
       bool ok = true;
       for (int tile = unit; tile < num_tiles && ok; tile += nunits) {
@@ -940,15 +956,15 @@ __global__ void __launch_bounds__(NUM_THREADS_ST, 1)
 #pragma unroll
         for (int i = 0; i < COLS / 2; ++i) acc2[i] = 0ull;
         for (int kt = 0; kt < KT && ok; ++kt, ++g) {
-          // the two chunks' factors, loaded before the waits below so that
-          // their global-memory latency overlaps them (a chunk wholly past K,
-          // ragged, holds a zero partial and gets no scale)
           float fk[2];
 #pragma unroll
           for (int c = 0; c < 2; ++c) {
-            const int kc = 2 * kt + c;
-            const int mb = PAIR ? mt * 2 + (int)rank : mt;  // this CTA's 128-row block of A
-            fk[c] = kc < nk ? p.a_ts[(int64_t)mb * nk + kc] * p.b_ts[(int64_t)nt * nk + kc] : 0.0f;
+            const int Q = 2 * g + c;
+            fk[c] = __shfl_sync(0xFFFFFFFFu, fcur, Q & 31);
+            if ((Q & 31) == 31) {
+              fcur = fnext;
+              fnext = chunk_factor(Q + 33 + lane);
+            }
           }
           for (; g_st < total && g_st < g + CS::NBUF_ST; g_st += 2)
             if (!stage_scales(g_st)) {
@@ -1089,6 +1105,18 @@ static bool make_payload_map(CUtensorMap *m, const void *base, int64_t rows, int
   cuuint32_t estr[2] = {1, 1};
   return enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void *>(base), dims, strides, box, estr,
              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+bool make_bf16_tile_map(CUtensorMap *m, const void *base, int64_t rows, int64_t cols, int64_t ld) {
+  PFN_encodeTiled enc = get_encode();
+  if (!enc) return false;
+  cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)(ld * 2)};
+  cuuint32_t box[2] = {128, 128};
+  cuuint32_t estr[2] = {1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides, box,
+             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 

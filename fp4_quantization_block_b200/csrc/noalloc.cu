@@ -73,20 +73,30 @@ fa4_status fa4_quantize_nvfp4_global_noalloc(const void *x, int64_t rows, int64_
   fa4_status s = scratch_for_current_device(&partials);
   if (s != FA4_OK) return s;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  const uint16_t *xb = static_cast<const uint16_t *>(x);
-  if (fa4::launch_tensor_amax(xb, rows, cols, ld, partials, np, st) != cudaSuccess) return FA4_ERR_CUDA;
-  cudaError_t e;
-  if (orient == FA4_ROWWISE)
-    e = fa4::launch_quant_rowwise(FA4_NVFP4_GLOBAL, rnd, xb, rows, cols, ld,
-                                  static_cast<uint8_t *>(out.payload),
-                                  static_cast<uint8_t *>(out.scales), out.tensor_scale, partials,
-                                  np, seed, st);
-  else
-    e = fa4::launch_quant_colwise(FA4_NVFP4_GLOBAL, rnd, false, 0u, xb, rows, cols, ld,
-                                  static_cast<uint8_t *>(out.payload),
-                                  static_cast<uint8_t *>(out.scales), out.tensor_scale, partials,
-                                  np, seed, st);
-  return e == cudaSuccess ? FA4_OK : FA4_ERR_CUDA;
+  fa4::QuantArgs q;
+  q.x = static_cast<const uint16_t *>(x);
+  q.T = rows;
+  q.C = cols;
+  q.ld = ld;
+  q.partials = partials;
+  q.n_partials = np;
+  if (fa4::launch_tensor_amax(q.x, rows, cols, ld, partials, np, st) != cudaSuccess) return FA4_ERR_CUDA;
+  if (orient == FA4_ROWWISE) {
+    q.row_fmt = FA4_NVFP4_GLOBAL;
+    q.row_rnd = rnd;
+    q.row_payload = static_cast<uint8_t *>(out.payload);
+    q.row_scales = static_cast<uint8_t *>(out.scales);
+    q.row_ts = out.tensor_scale;
+    q.row_seed = seed;
+  } else {
+    q.col_fmt = FA4_NVFP4_GLOBAL;
+    q.col_rnd = rnd;
+    q.col_payload = static_cast<uint8_t *>(out.payload);
+    q.col_scales = static_cast<uint8_t *>(out.scales);
+    q.col_ts = out.tensor_scale;
+    q.col_seed = seed;
+  }
+  return fa4::launch_quantize(q, st) == cudaSuccess ? FA4_OK : FA4_ERR_CUDA;
 }
 
 }  // extern "C"

@@ -1,30 +1,51 @@
 // quantize.cu -- fused FP4 quantization producers for sm_100a.
 //
-// One kernel per orientation (and one for both) does the whole producer of "FP4 Is No Longer
-// Just a Hardware Feature -- The NVFP4 Software Stack Is Taking Shape",
-// section "The first change" (block amax -> scale -> divide -> E2M1 -> pack
-// two values per byte) in registers, and writes the scale bytes straight into
-// the 128x4 atoms the block-scaled MMA reads, so nothing intermediate goes to
+// One kernel template does the whole producer of "FP4 Is No Longer Just a
+// Hardware Feature -- The NVFP4 Software Stack Is Taking Shape", section
+// "The first change" (block amax -> scale -> divide -> E2M1 -> pack two
+// values per byte) in registers, and writes the scale bytes straight into the
+// 128x4 atoms the block-scaled MMA reads, so nothing intermediate goes to
 // memory (the unfused pipeline that section warns about writes amax and
 // scales and re-reads the tensor).  The scale domain is a template parameter
 // ("Format-Aware Fusion: The Engineering Practice That Doubles FP4
 // Pretraining Throughput", section "The Design Philosophy of Format-Aware
 // Fusion"): native MX, global NV (second pass after tensor_amax_kernel) or
 // CTA-local NV (the 128x128 tile amax is reduced inside the CTA that
-// quantizes the tile, so the tensor is read once).
+// quantizes the tile, so the tensor is read once).  One read of x emits the
+// row-wise operand (Q = x), the column-wise operand (Q = x^T, optionally
+// through the fixed-sign 32-point Hadamard of "Two Key Numerical
+// Techniques"), or both.
 //
-// Work unit: one CTA of 256 threads per 128x128 tile of the quantized
-// operand Q.  The tile (32 KB of bf16) is loaded with 16-byte coalesced
-// loads, all issued before any arithmetic.
+// Structure: persistent CTAs of 256 threads, two per SM.  Each CTA walks
+// 128 x 128 tiles of x; one thread brings tiles into a three-stage
+// shared-memory ring with bulk-tensor (TMA) loads issued two tiles ahead, so
+// the loads in flight do not depend on registers.  A TMA load past the edge
+// of x fills zeros, which change no block, tile or tensor amax.
+//   row-wise pass  warp w, lane l: rows 16 s + 2 w + (l >> 4) (s = 0..7),
+//                  columns 8 (l & 15) .. + 8 (16-byte shared-memory reads;
+//                  an MX block is a lane quad, an NV block a lane pair);
+//   column-wise    thread -> two adjacent channels and one 32-token block,
+//   pass           reading down the columns (a warp reads 128 contiguous
+//                  bytes per token), all 64 values in registers as packed
+//                  binary32 pairs, so the Hadamard is an in-register
+//                  butterfly on f32x2 adds.
+// Scale bytes are stored one byte per block straight into their atom slot.
+// Tiles cut by the tensor's edge take the EDGE path, which stores only the
+// payload inside the tensor and writes every scale byte of the padded atoms
+// (rows up to the next multiple of 128, blocks up to the next multiple of 4),
+// zero outside the tensor.
 //
-// Ragged shapes: Q[R, K] with any R and K a multiple of 32.  Tiles cut by
-// the tensor's edge run the EDGE variant of the kernel, which reads zeros
-// outside the tensor -- zeros change no block, tile or tensor amax -- and
-// stores only the payload inside it; every scale byte of the padded atoms
-// (rows up to the next multiple of 128, blocks up to the next multiple of
-// 4) is written, zero outside the tensor.  When only R is ragged the uncut
-// tiles run the unmasked kernel; when K is, every tile runs the EDGE
-// variant (the atom stride along K is then the padded one).
+// Instruction economy (the SR and Hadamard producers are bound by issue
+// slots): block amax on packed bf16 pairs (max.xorsign.abs), the MX scale
+// byte read off the bf16 exponent field, NV block scales with an exactly
+// rounded division by 6 and a per-tile table of the element multipliers
+// s_enc / decode(code), unpack-and-scale on packed pairs, the Philox round
+// keys as kernel parameters, and four values per stochastic conversion.
+//
+// Every wait on a tile load is bounded: past `timeout_ns` the CTA sets the
+// status word (when given), waits (bounded) for its own loads in flight and
+// returns.
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -41,22 +62,8 @@ __device__ __forceinline__ uint4 ld_stream(const void *p) {
   return v;
 }
 
-__device__ __forceinline__ void unpack8(const uint4 &w, float *f) {
-  f[0] = bf16lo(w.x); f[1] = bf16hi(w.x);
-  f[2] = bf16lo(w.y); f[3] = bf16hi(w.y);
-  f[4] = bf16lo(w.z); f[5] = bf16hi(w.z);
-  f[6] = bf16lo(w.w); f[7] = bf16hi(w.w);
-}
-
 __device__ __forceinline__ float absmax8(const uint4 &w) {
-  // |bf16| max on the packed pairs: clear sign bits, max of the magnitudes
-  // as unsigned integers orders non-negative floats correctly
-  const uint32_t m = 0x7FFF7FFFu;
-  uint32_t a = __vmaxu2(w.x & m, w.y & m);
-  uint32_t b = __vmaxu2(w.z & m, w.w & m);
-  a = __vmaxu2(a, b);
-  const uint32_t hi = a >> 16, lo = a & 0xFFFFu;
-  return __uint_as_float((hi > lo ? hi : lo) << 16);
+  return __uint_as_float((absmax8_bf16(w) & 0x7FFFu) << 16);
 }
 
 // CTA-wide max of one value per thread (256 threads).
@@ -70,13 +77,6 @@ __device__ __forceinline__ float cta_max256(float v, float *red) {
 #pragma unroll
   for (int i = 1; i < 8; ++i) r = fmaxf(r, red[i]);
   return r;
-}
-
-// Largest of the NV-global amax partials, read by every CTA.
-__device__ __forceinline__ float reduce_partials(const float *partials, int n, float *red) {
-  float m = 0.0f;
-  for (int i = threadIdx.x; i < n; i += blockDim.x) m = fmaxf(m, partials[i]);
-  return cta_max256(m, red);
 }
 
 // --------------------------------------------------------------------------
@@ -107,151 +107,203 @@ __global__ void __launch_bounds__(256) tensor_amax_kernel(const uint16_t *__rest
   if (threadIdx.x == 0) partials[blockIdx.x] = m;
 }
 
-// --------------------------------------------------------------------------
-// Row-wise quantizer: Q = x[R, K], blocks along a row.
-// Thread layout in a 128x128 tile: warp w, lane l -> rows 16*s + 2*w + (l>>4)
-// for steps s = 0..7, columns 8*(l&15) .. +8.  A half-warp covers one row;
-// NV blocks (16) are lane pairs, MX blocks (32) lane quads.
-// --------------------------------------------------------------------------
-// Row-wise quantization of one 128x128 tile of Q held in registers: v[s] is
-// row r0 + 16 s + 2 w + (l >> 4), columns k0 + 8 (l & 15) .. + 8.  s_enc is the
-// NVFP4 encode scale (unused for MXFP4).
-// EDGE: Q has R rows; chunks outside Q hold zeros and are not stored.
-template <int FMT, int RND, bool EDGE>
-__device__ __forceinline__ void rowwise_tile(const uint4 (&v)[8], int64_t r0, int64_t k0, int64_t R,
-                                             int64_t K, uint8_t *__restrict__ payload,
-                                             uint8_t *__restrict__ scales, float s_enc,
-                                             uint64_t seed) {
-  const int w = threadIdx.x >> 5, l = threadIdx.x & 31;
-  const int c = l & 15;          // 8-element chunk within the 128-wide row
-  const int64_t kc = k0 + 8 * c;  // first column of the chunk
-  const int64_t kb = is_mx<FMT>() ? (K >> 5) : (K >> 4);  // blocks per row
-  // blocks per atom row: padded to a multiple of 4 (already one unless EDGE)
-  const int64_t kbt = EDGE ? ((kb + 3) & ~int64_t(3)) : kb;
-#pragma unroll
-  for (int s = 0; s < 8; ++s) {
-    const int64_t r = r0 + 16 * s + 2 * w + (l >> 4);
-    const bool inside = !EDGE || (r < R && kc < K);
-    float f[8];
-    unpack8(v[s], f);
-    float amax = absmax8(v[s]);
-    amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, 1));
-    if constexpr (is_mx<FMT>()) amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, 2));
-    uint32_t sbyte;
-    if constexpr (is_mx<FMT>()) {
-      sbyte = mx_byte<FMT>(amax);
-      const float mult = mx_multiplier(sbyte);
-#pragma unroll
-      for (int e = 0; e < 8; ++e) f[e] = __fmul_rn(f[e], mult);
-    } else {
-      float mult;
-      sbyte = nv_block_scale(amax, s_enc, &mult);
-#pragma unroll
-      for (int e = 0; e < 8; ++e) f[e] = __fmul_rn(f[e], mult);
-    }
-    if (EDGE && !inside) sbyte = 0u;  // padding scale bytes are zero
-    uint32_t codes;
-    if constexpr (RND == kSR) {
-      codes = e2m1x8_sr(f, sr_block_bits(seed, (uint64_t)(r * K + kc) >> 3));
-    } else {
-      codes = e2m1x8_rne(f);
-    }
-    if (inside) *reinterpret_cast<uint32_t *>(payload + r * (K >> 1) + (kc >> 1)) = codes;
+namespace qk {
 
-    // gather four consecutive block scales of the row into one word
-    uint32_t word;
-    if constexpr (is_mx<FMT>()) {
-      word = sbyte << (8 * (c >> 2));
-      word |= __shfl_xor_sync(0xFFFFFFFFu, word, 4);
-      word |= __shfl_xor_sync(0xFFFFFFFFu, word, 8);
-      if (c == 0) *reinterpret_cast<uint32_t *>(scales + sf_offset(r, k0 >> 5, kbt)) = word;
-    } else {
-      word = sbyte << (8 * ((c >> 1) & 3));
-      word |= __shfl_xor_sync(0xFFFFFFFFu, word, 2);
-      word |= __shfl_xor_sync(0xFFFFFFFFu, word, 4);
-      // a word whose first block is past the row's last one lies outside
-      // the padded atoms (only in an EDGE tile)
-      if ((c & 7) == 0 && (!EDGE || (k0 >> 4) + 4 * (c >> 3) < kb))
-        *reinterpret_cast<uint32_t *>(scales + sf_offset(r, (k0 >> 4) + 4 * (c >> 3), kbt)) = word;
-    }
-  }
-}
+constexpr int kThreads = 256;
+constexpr int kStages = 3;
+constexpr int kTileBytes = 128 * 128 * 2;  // one 128 x 128 bf16 tile
+constexpr int kNone = -1;                  // orientation not produced
+constexpr uint32_t kStatusTimeout = 7;
 
-// Loads of one 128x128 tile in the row-wise thread layout (16-byte lanes, all
-// issued before any arithmetic).  EDGE: chunks outside x[rows, cols] read as
-// zeros (cols is a multiple of 8, so a chunk is wholly inside or outside).
-template <bool EDGE>
-__device__ __forceinline__ void load_tile_rowwise(const uint16_t *__restrict__ x, int64_t ld,
-                                                  int64_t r0, int64_t k0, int64_t rows,
-                                                  int64_t cols, uint4 (&v)[8]) {
-  const int w = threadIdx.x >> 5, l = threadIdx.x & 31;
-#pragma unroll
-  for (int s = 0; s < 8; ++s) {
-    const int64_t r = r0 + 16 * s + 2 * w + (l >> 4);
-    if (!EDGE || (r < rows && k0 + 8 * (l & 15) < cols))
-      v[s] = ld_stream(x + r * ld + k0 + 8 * (l & 15));
-    else
-      v[s] = make_uint4(0u, 0u, 0u, 0u);
-  }
-}
-
-// Tiles of an EDGE launch: blockIdx + (a0, b0) in a grid of n_a tiles along
-// the blockIdx.x dimension.  The unmasked launch covers the tiles from
-// (0, 0) with the grid's own extent.
-struct EdgeTiles {
-  int a0, b0, n_a;
+struct Params {
+  int64_t T, C;  // x[T, C]
+  int tiles_c, tiles_t, ntiles;
+  // row-wise operand Q = x [T, C]
+  uint8_t *rp, *rs;
+  float *rts;
+  // column-wise operand Q = x^T [C, T]
+  uint8_t *cp, *cs;
+  float *cts;
+  // Philox4x32-10 round keys of the two seeds (round 9's complemented, see
+  // sr_bits_not)
+  uint32_t rkey0[10], rkey1[10], ckey0[10], ckey1[10];
+  // fixed-sign Hadamard: 0x80000000 where token t of a 32-block is negated
+  uint32_t sgn[32];
+  const float *partials;  // NVFP4-global amax partials
+  int np;
+  uint32_t *status;  // may be null
+  uint64_t timeout_ns;
 };
 
-// NVFP4 encode scale of the tile's domain: CTA-local (this tile's amax, ts
-// written at ts_index) or global (reduced from the amax partials, ts[0]
-// written by the first tile); 1 for MXFP4.
-template <int FMT>
-__device__ __forceinline__ float tile_encode_scale(const uint4 (&v)[8], float *__restrict__ ts,
-                                                   int64_t ts_index, bool first_tile,
-                                                   const float *__restrict__ partials,
-                                                   int n_partials, float *red) {
-  float s_enc = 1.0f;
-  if constexpr (FMT == kNVC) {
-    float m = 0.0f;
+struct Ctrl {
+  uint64_t full[kStages];
+  float red[8];
+  float tab_r[128];  // NVFP4 row-wise element multipliers s_enc / decode(code)
+  float tab_c[128];  // column-wise
+};
+constexpr int kSmemBytes = kStages * kTileBytes + (int)sizeof(Ctrl) + 128;
+
+__device__ __forceinline__ uint32_t smem_u32(const void *p) {
+  return (uint32_t)__cvta_generic_to_shared(p);
+}
+__device__ __forceinline__ uint64_t globaltimer() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+__device__ __forceinline__ bool wait_bounded(uint32_t bar, uint32_t parity, uint64_t timeout_ns) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = globaltimer();
+  while (!mbar_try_wait(bar, parity))
+    if (globaltimer() - t0 > timeout_ns) return false;
+  return true;
+}
+__device__ __forceinline__ void issue_tile(uint8_t *smem, Ctrl *cb, const CUtensorMap *map,
+                                           const Params &p, int t, int s) {
+  const uint32_t bar = smem_u32(&cb->full[s]);
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar),
+               "r"(kTileBytes)
+               : "memory");
+  const int x = (t % p.tiles_c) * 128, y = (t / p.tiles_c) * 128;
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3}], [%4];" ::"r"(smem_u32(smem + s * kTileBytes)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar)
+      : "memory");
+}
+
+__device__ __forceinline__ uint4 lds128(const void *p) {
+  uint4 v;
+  asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "r"(smem_u32(p)));
+  return v;
+}
+__device__ __forceinline__ uint32_t lds32(const void *p) {
+  uint32_t v;
+  asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(smem_u32(p)));
+  return v;
+}
+
+// The complement of sr_block_bits(seed, i8) (65535 - u in every 16-bit
+// half, the form e2m1x8_sr_not takes), with the round keys in
+// kernel parameters.
+__device__ __forceinline__ u32x4 sr_bits_not(const uint32_t (&k0)[10], const uint32_t (&k1)[10],
+                                             uint64_t i8) {
+  uint32_t c0 = (uint32_t)i8, c1 = (uint32_t)(i8 >> 32), c2 = 0u, c3 = 0u;
 #pragma unroll
-    for (int s = 0; s < 8; ++s) m = fmaxf(m, absmax8(v[s]));
-    s_enc = nv_encode_scale(cta_max256(m, red));
-    if (threadIdx.x == 0) ts[ts_index] = nv_decode_scale(s_enc);
-  } else if constexpr (FMT == kNVG) {
-    s_enc = nv_encode_scale(reduce_partials(partials, n_partials, red));
-    if (threadIdx.x == 0 && first_tile) ts[0] = nv_decode_scale(s_enc);
+  for (int r = 0; r < 10; ++r) {
+    const uint64_t p0 = (uint64_t)0xD2511F53u * c0;
+    const uint64_t p1 = (uint64_t)0xCD9E8D57u * c2;
+    const uint32_t n0 = (uint32_t)(p1 >> 32) ^ c1 ^ k0[r], n2 = (uint32_t)(p0 >> 32) ^ c3 ^ k1[r];
+    c1 = (uint32_t)p1;
+    c3 = (uint32_t)p0;
+    c0 = n0;
+    c2 = n2;
   }
-  return s_enc;
+  return {c0, ~c1, c2, ~c3};
 }
 
-// tiles: x along K, y along R; the CTA-local ts index is [R tile][K tile]
+// MX scale byte from the bf16 bits of a block amax (either half of m): the
+// binary32 exponent field of a bf16 value is its own exponent field, so
+// e = floor(log2 amax) - 2 clamped at -127 gives byte max(E - 2, 0); without
+// clipping, one more when the mantissa exceeds 1.5 (bf16 mantissa > 0x40).
+template <int FMT>
+__device__ __forceinline__ uint32_t mx_byte_bf16(uint32_t m) {
+  const int E = (int)((m >> 7) & 0xFFu);
+  if constexpr (FMT == kMXN) {
+    if (E == 0) return 0u;
+    return (uint32_t)max(E - 2 + ((m & 0x7Fu) > 0x40u ? 1 : 0), 0);
+  } else {
+    return (uint32_t)max(E - 2, 0);
+  }
+}
+
+// NVFP4 block scale of a block amax (binary32) under encode scale s_enc:
+// s_b = (amax / 6) * s_enc clamped to [2^-9, 448], its E4M3 code, and the
+// element multiplier s_enc / decode(code) from the table.
+__device__ __forceinline__ uint32_t nv_code(float amax, float s_enc) {
+  float sb = __fmul_rn(div6_rn(amax), s_enc);
+  sb = fminf(fmaxf(sb, 0.001953125f), 448.0f);
+  return e4m3_rne(sb);
+}
+// tab[code] = s_enc / decode(code) for every E4M3 code (threads 0..127; the
+// caller synchronizes before use).  Codes 0 and 127 never occur.
+__device__ __forceinline__ void build_tab(float *tab, float s_enc) {
+  if (threadIdx.x < 128) tab[threadIdx.x] = __fdiv_rn(s_enc, e4m3_to_float(threadIdx.x));
+}
+
+// y = bf16 x * mult for the eight values of w, on packed pairs
+__device__ __forceinline__ void unpack_scale8(const uint4 &w, float mult, float *f) {
+  const uint64_t mm = f2_pack(mult, mult);
+  const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+    f2_unpack(f2_mul(f2_pack_bits(ws[i] << 16, ws[i] & 0xFFFF0000u), mm), f[2 * i], f[2 * i + 1]);
+}
+
+// ---------------------------------------------------------- row-wise pass
+// Q = x: rows t0.., K range c0..; R = T, K = C.
 template <int FMT, int RND, bool EDGE>
-__global__ void __launch_bounds__(256) quant_rowwise_kernel(
-    const uint16_t *__restrict__ x, int64_t R, int64_t K, int64_t ld, uint8_t *__restrict__ payload,
-    uint8_t *__restrict__ scales, float *__restrict__ ts, const float *__restrict__ partials,
-    int n_partials, uint64_t seed, EdgeTiles e) {
-  __shared__ float red[8];
-  const int64_t tk = (int64_t)blockIdx.x + (EDGE ? e.a0 : 0);
-  const int64_t tr = (int64_t)blockIdx.y + (EDGE ? e.b0 : 0);
-  const int64_t k0 = tk * 128, r0 = tr * 128;
-  uint4 v[8];
-  load_tile_rowwise<EDGE>(x, ld, r0, k0, R, K, v);
-  const float s_enc = tile_encode_scale<FMT>(v, ts, tr * (EDGE ? e.n_a : gridDim.x) + tk,
-                                             tk == 0 && tr == 0, partials, n_partials, red);
-  rowwise_tile<FMT, RND, EDGE>(v, r0, k0, R, K, payload, scales, s_enc, seed);
+__device__ __forceinline__ void row_pass(const uint16_t *tile, const Params &p, int tt, int tc,
+                                         float s_enc, const float *tab) {
+  const int w = threadIdx.x >> 5, l = threadIdx.x & 31, c = l & 15;
+  const int base = 2 * w + (l >> 4);  // row within the tile, minus 16 s
+  const int64_t K = p.C;
+  const int64_t r0 = (int64_t)tt * 128 + base, kc = (int64_t)tc * 128 + 8 * c;
+  const int64_t kb = is_mx<FMT>() ? (K >> 5) : (K >> 4);  // blocks per row
+  const int64_t kbt = (kb + 3) & ~int64_t(3);              // per atom row
+  uint8_t *pay = p.rp + r0 * (K >> 1) + (kc >> 1);
+  // this lane's scale byte (the first lane of its block) for s = 0; row
+  // 16 s + base of the tile sits at (s & 1) * 256 + (s >> 1) * 4 further
+  const int64_t bidx = is_mx<FMT>() ? (kc >> 5) : (kc >> 4);  // block index
+  uint8_t *sb0 = p.rs + ((int64_t)tt * (kbt >> 2) + (bidx >> 2)) * 512 + base * 16 + (bidx & 3);
+  const bool lead = is_mx<FMT>() ? (c & 3) == 0 : (c & 1) == 0;
+#pragma unroll
+  for (int s = 0; s < 8; ++s) {
+    const int rr = 16 * s + base;
+    const uint4 v = lds128(tile + rr * 128 + 8 * c);
+    uint32_t m = absmax8_bf16(v);
+    m = hmax_abs2(m, __shfl_xor_sync(0xFFFFFFFFu, m, 1));
+    uint32_t sbyte;
+    float mult;
+    if constexpr (is_mx<FMT>()) {
+      m = hmax_abs2(m, __shfl_xor_sync(0xFFFFFFFFu, m, 2));
+      sbyte = mx_byte_bf16<FMT>(m);
+      mult = mx_multiplier(sbyte);
+    } else {
+      sbyte = nv_code(__uint_as_float((m & 0x7FFFu) << 16), s_enc);
+      mult = tab[sbyte];
+    }
+    float f[8];
+    unpack_scale8(v, mult, f);
+    uint32_t codes;
+    if constexpr (RND == kSR)
+      codes = e2m1x8_sr_not(f, sr_bits_not(p.rkey0, p.rkey1, (uint64_t)((r0 + 16 * s) * K + kc) >> 3));
+    else
+      codes = e2m1x8_rne(f);
+    const bool inside = !EDGE || (r0 + 16 * s < p.T && kc < K);
+    if (inside) *reinterpret_cast<uint32_t *>(pay + (int64_t)16 * s * (K >> 1)) = codes;
+    if (lead && (!EDGE || bidx < kbt))
+      sb0[(s & 1) * 256 + (s >> 1) * 4] = (EDGE && !inside) ? (uint8_t)0 : (uint8_t)sbyte;
+  }
 }
 
-// --------------------------------------------------------------------------
-// Column-wise quantizer: Q = x^T, x[T, C] row-major; Q[R = C, K = T].
-// The 128(tokens) x 128(channels) tile is staged in shared memory; each
-// thread then owns two adjacent channels and one 32-token block, reading
-// down the columns (a warp reads 128 contiguous bytes per token: no bank
-// conflicts) and keeping all 64 values in registers, so the optional
-// Hadamard-32 is an in-register butterfly.
-// --------------------------------------------------------------------------
+// ------------------------------------------------------- column-wise pass
+// Q = x^T: rows c0.. (channels), K range t0.. (tokens); R = C, K = T.
 // In-place butterfly with strides 1, 2, 4, 8, 16, (a, b) -> (a + b, a - b),
-// on packed pairs: lane lo and lane hi are two independent 32-value blocks
-// (two channels) taking the same steps.
+// on packed pairs (two channels' blocks taking the same steps).
 __device__ __forceinline__ void fwht32x2(uint64_t *v) {
 #pragma unroll
   for (int h = 1; h < 32; h <<= 1) {
@@ -265,181 +317,220 @@ __device__ __forceinline__ void fwht32x2(uint64_t *v) {
     }
   }
 }
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
 
-// Column-wise quantization of the 128 (tokens) x 128 (channels) tile staged
-// in shared memory (tile[token][channel]; complete before the call): Q = x^T,
-// rows c0 .. c0+127 of Q, K range t0 .. t0+127.  sbuf holds 128 x 8 scale
-// bytes.  Ends with the tile's scale words written.  EDGE: Q has C rows and
-// T (a multiple of 32) columns; outside them the staged tile holds zeros.
 template <int FMT, int RND, bool HAD, bool EDGE>
-__device__ __forceinline__ void colwise_tile(const uint16_t *tile, uint8_t *sbuf, int64_t c0,
-                                             int64_t t0, int64_t C, int64_t T,
-                                             uint8_t *__restrict__ payload,
-                                             uint8_t *__restrict__ scales, float s_enc,
-                                             uint64_t seed, uint32_t sign_mask) {
+__device__ __forceinline__ void col_pass(const uint16_t *tile, const Params &p, int tt, int tc,
+                                         float s_enc, const float *tab) {
   const int w = threadIdx.x >> 5, l = threadIdx.x & 31;
-  const int p = (w & 1) * 32 + l;  // channel pair within the tile: 2p, 2p+1
-  const int j = w >> 1;            // 32-token block within the tile
-  float v0[32], v1[32];  // channels 2p and 2p+1
-  if constexpr (HAD) {
-    // the two channels' blocks take the same signs and butterfly: run them
-    // as packed pairs; a sign is the bf16 sign bit, flipped before widening
-    uint64_t w2[32];
+  const int pr = (w & 1) * 32 + l;  // channel pair within the tile: 2 pr, 2 pr + 1
+  const int j = w >> 1;             // 32-token block within the tile
+  const int64_t T = p.T;
+  const int64_t kb = is_mx<FMT>() ? (T >> 5) : (T >> 4);  // blocks per row of Q
+  const int64_t kbt = (kb + 3) & ~int64_t(3);
+  const int64_t kfirst = (int64_t)tt * 128 + 32 * j;  // first K index of the 32-block
+  const uint16_t *src = tile + (32 * j) * 128 + 2 * pr;
+
+  uint64_t v2[32];  // token t: (channel 2 pr, channel 2 pr + 1)
 #pragma unroll
-    for (int t = 0; t < 32; ++t) {
-      uint32_t pair = *reinterpret_cast<const uint32_t *>(&tile[(32 * j + t) * 128 + 2 * p]);
-      if ((sign_mask >> t) & 1u) pair ^= 0x80008000u;
-      w2[t] = f2_pack(bf16lo(pair), bf16hi(pair));
-    }
-    fwht32x2(w2);
-#pragma unroll
-    for (int t = 0; t < 32; ++t) f2_unpack(w2[t], v0[t], v1[t]);
-  } else {
-#pragma unroll
-    for (int t = 0; t < 32; ++t) {
-      const uint32_t pair = *reinterpret_cast<const uint32_t *>(&tile[(32 * j + t) * 128 + 2 * p]);
-      v0[t] = bf16lo(pair);
-      v1[t] = bf16hi(pair);
+  for (int t = 0; t < 32; ++t) {
+    const uint32_t wd = lds32(src + t * 128);
+    if constexpr (HAD) {
+      // the sign flip rides on the unpack: + 0x80000000 flips bit 31 of
+      // (wd << 16), XOR flips it of the high half
+      v2[t] = f2_pack_bits(wd * 65536u + p.sgn[t], (wd & 0xFFFF0000u) ^ p.sgn[t]);
+    } else {
+      v2[t] = f2_pack_bits(wd << 16, wd & 0xFFFF0000u);
     }
   }
-  const int64_t kb = is_mx<FMT>() ? (T >> 5) : (T >> 4);  // blocks per row of Q
-  // blocks per atom row: padded to a multiple of 4 (already one unless EDGE)
-  const int64_t kbt = EDGE ? ((kb + 3) & ~int64_t(3)) : kb;
+  if constexpr (HAD) fwht32x2(v2);
+  float v0[32], v1[32];
+#pragma unroll
+  for (int t = 0; t < 32; ++t) f2_unpack(v2[t], v0[t], v1[t]);
 
-  // block scales of both channels (MX: one 32-block each; NV: two 16-blocks
-  // each, multiplier mult[half][hb])
-  const int64_t kfirst = t0 + 32 * j;  // first K index of this 32-block
+  // block scales of both channels (MX: one 32-block each; NV: two 16-blocks)
   float mult[2][2];
+  uint32_t sbyte[2][2];
 #pragma unroll
   for (int half = 0; half < 2; ++half) {
     const float *v = half ? v1 : v0;
-    const int cl = 2 * p + half;  // channel within the tile
-    // the thread's 32-token block is wholly inside or outside (T % 32 == 0)
-    const bool inside = !EDGE || (c0 + cl < C && kfirst < T);
     if constexpr (is_mx<FMT>()) {
-      float amax = 0.0f;
+      float a = fabsf(v[0]);
 #pragma unroll
-      for (int t = 0; t < 32; ++t) amax = fmaxf(amax, fabsf(v[t]));
-      const uint32_t sbyte = mx_byte<FMT>(amax);
-      mult[half][0] = mult[half][1] = mx_multiplier(sbyte);
-      sbuf[cl * 8 + j] = (EDGE && !inside) ? (uint8_t)0 : (uint8_t)sbyte;
+      for (int t = 1; t < 31; t += 2) a = fmax3(a, fabsf(v[t]), fabsf(v[t + 1]));
+      a = fmaxf(a, fabsf(v[31]));
+      sbyte[half][0] = mx_byte<FMT>(a);
+      mult[half][0] = mult[half][1] = mx_multiplier(sbyte[half][0]);
     } else {
 #pragma unroll
       for (int hb = 0; hb < 2; ++hb) {
-        float amax = 0.0f;
+        float a = fabsf(v[16 * hb]);
 #pragma unroll
-        for (int t = 0; t < 16; ++t) amax = fmaxf(amax, fabsf(v[16 * hb + t]));
-        const uint32_t sbyte = nv_block_scale(amax, s_enc, &mult[half][hb]);
-        sbuf[cl * 8 + 2 * j + hb] = (EDGE && !inside) ? (uint8_t)0 : (uint8_t)sbyte;
+        for (int t = 1; t < 15; t += 2) a = fmax3(a, fabsf(v[16 * hb + t]), fabsf(v[16 * hb + t + 1]));
+        a = fmaxf(a, fabsf(v[16 * hb + 15]));
+        sbyte[half][hb] = nv_code(a, s_enc);
+        mult[half][hb] = tab[sbyte[half][hb]];
       }
     }
   }
   // y = x * multiplier, both channels at once
 #pragma unroll
   for (int t = 0; t < 32; ++t)
-    f2_unpack(f2_mul(f2_pack(v0[t], v1[t]), f2_pack(mult[0][t >> 4], mult[1][t >> 4])), v0[t],
-              v1[t]);
+    f2_unpack(f2_mul(f2_pack(v0[t], v1[t]), f2_pack(mult[0][t >> 4], mult[1][t >> 4])), v0[t], v1[t]);
 
 #pragma unroll
   for (int half = 0; half < 2; ++half) {
     float *v = half ? v1 : v0;
-    const int cl = 2 * p + half;  // channel within the tile
-    const int64_t r = c0 + cl;
-    const bool inside = !EDGE || (r < C && kfirst < T);
+    const int cl = 2 * pr + half;  // channel within the tile
+    const int64_t r = (int64_t)tc * 128 + cl;
+    const bool inside = !EDGE || (r < p.C && kfirst < T);
     uint32_t codes[4];
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
-      if constexpr (RND == kSR) {
-        codes[q] = e2m1x8_sr(&v[8 * q], sr_block_bits(seed, (uint64_t)(r * T + kfirst + 8 * q) >> 3));
-      } else {
+      if constexpr (RND == kSR)
+        codes[q] = e2m1x8_sr_not(&v[8 * q], sr_bits_not(p.ckey0, p.ckey1, (uint64_t)(r * T + kfirst + 8 * q) >> 3));
+      else
         codes[q] = e2m1x8_rne(&v[8 * q]);
-      }
     }
     if (inside)
-      *reinterpret_cast<uint4 *>(payload + r * (T >> 1) + (kfirst >> 1)) =
+      *reinterpret_cast<uint4 *>(p.cp + r * (T >> 1) + (kfirst >> 1)) =
           make_uint4(codes[0], codes[1], codes[2], codes[3]);
-  }
-  __syncthreads();
-  // scale words: MX 4 blocks (one word) per channel, NV 8 blocks (two words)
-  if constexpr (is_mx<FMT>()) {
-    if (threadIdx.x < 128) {
-      const int cl = threadIdx.x;
-      const uint32_t word = *reinterpret_cast<const uint32_t *>(&sbuf[cl * 8]);
-      *reinterpret_cast<uint32_t *>(scales + sf_offset(c0 + cl, t0 >> 5, kbt)) = word;
+    // scale bytes at their atom slots: row r = channel, block kfirst / bs
+    const int64_t bidx = is_mx<FMT>() ? (kfirst >> 5) : (kfirst >> 4);
+    uint8_t *dst = p.cs + ((int64_t)tc * (kbt >> 2) + (bidx >> 2)) * 512 + (cl & 31) * 16 +
+                   ((cl >> 5) & 3) * 4 + (bidx & 3);
+    if constexpr (is_mx<FMT>()) {
+      *dst = (EDGE && !inside) ? (uint8_t)0 : (uint8_t)sbyte[half][0];
+    } else {
+      // the block pair 2j, 2j+1 is adjacent in its atom word
+      if (!EDGE || bidx < kbt)
+        *reinterpret_cast<uint16_t *>(dst) =
+            (EDGE && !inside) ? (uint16_t)0 : (uint16_t)(sbyte[half][0] | (sbyte[half][1] << 8));
     }
-  } else {
-    const int cl = threadIdx.x >> 1, h = threadIdx.x & 1;
-    const uint32_t word = *reinterpret_cast<const uint32_t *>(&sbuf[cl * 8 + 4 * h]);
-    if (!EDGE || (t0 >> 4) + 4 * h < kb)  // else past the padded atoms
-      *reinterpret_cast<uint32_t *>(scales + sf_offset(c0 + cl, (t0 >> 4) + 4 * h, kbt)) = word;
   }
 }
 
-// tiles: x along channels (rows of Q), y along tokens (K of Q); the
-// CTA-local ts index is [channel tile][token tile]
-template <int FMT, int RND, bool HAD, bool EDGE>
-__global__ void __launch_bounds__(256) quant_colwise_kernel(
-    const uint16_t *__restrict__ x, int64_t T, int64_t C, int64_t ld, uint8_t *__restrict__ payload,
-    uint8_t *__restrict__ scales, float *__restrict__ ts, const float *__restrict__ partials,
-    int n_partials, uint64_t seed, uint32_t sign_mask, EdgeTiles e, int n_t) {
-  __shared__ __align__(16) uint16_t tile[128 * 128];  // [token][channel]
-  __shared__ __align__(16) uint8_t sbuf[128 * 8];     // [channel][block in tile]
-  __shared__ float red[8];
-  const int w = threadIdx.x >> 5, l = threadIdx.x & 31;
-  const int64_t tc = (int64_t)blockIdx.x + (EDGE ? e.a0 : 0);
-  const int64_t tt = (int64_t)blockIdx.y + (EDGE ? e.b0 : 0);
-  const int64_t c0 = tc * 128;  // channel = row of Q
-  const int64_t t0 = tt * 128;  // token = K of Q
-  // stage the tile: half-warp per token row, 16 bytes per lane
-  uint4 v[8];
-  load_tile_rowwise<EDGE>(x, ld, t0, c0, T, C, v);
-#pragma unroll
-  for (int s = 0; s < 8; ++s)
-    *reinterpret_cast<uint4 *>(&tile[(16 * s + 2 * w + (l >> 4)) * 128 + 8 * (l & 15)]) = v[s];
-  // the CTA-local tile of Q = x^T is this tile transposed: same maximum;
-  // its ts entry is [c0 / 128][t0 / 128]
-  const float s_enc = tile_encode_scale<FMT>(v, ts, tc * (EDGE ? n_t : gridDim.y) + tt,
-                                             tc == 0 && tt == 0, partials, n_partials, red);
+// --------------------------------------------------------------- kernel
+template <int RF, int RR, int CF, int CR, bool HAD>
+__global__ void __launch_bounds__(kThreads, 2)
+    quant_kernel(const __grid_constant__ CUtensorMap xmap, const Params p) {
+  extern __shared__ uint8_t qsmem_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(qsmem_raw) + 127) &
+                                              ~uintptr_t(127));
+  Ctrl *cb = reinterpret_cast<Ctrl *>(smem + kStages * kTileBytes);
+  const int tid = threadIdx.x;
+  if (tid == 0) {
+    for (int s = 0; s < kStages; ++s)
+      asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(smem_u32(&cb->full[s])) : "memory");
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
   __syncthreads();
-  colwise_tile<FMT, RND, HAD, EDGE>(tile, sbuf, c0, t0, C, T, payload, scales, s_enc, seed,
-                                    sign_mask);
+  // thread 0: per stage, the parity of the loads issued into it so far (bit
+  // k flips with every load into stage k) and whether one is not yet
+  // consumed
+  uint32_t nload_par = 0, pending = 0;
+  if (tid == 0)
+    for (int s = 0; s < kStages; ++s) {
+      const int t = (int)blockIdx.x + s * (int)gridDim.x;
+      if (t < p.ntiles) {
+        issue_tile(smem, cb, &xmap, p, t, s);
+        nload_par ^= 1u << s;
+        pending |= 1u << s;
+      }
+    }
+
+  // NVFP4-global: the encode scale from the amax partials, once per CTA
+  float senc_g = 1.0f;
+  if constexpr (RF == kNVG || CF == kNVG) {
+    float m = 0.0f;
+    for (int i = tid; i < p.np; i += kThreads) m = fmaxf(m, p.partials[i]);
+    senc_g = nv_encode_scale(cta_max256(m, cb->red));
+    if (blockIdx.x == 0 && tid == 0) {
+      if (RF == kNVG) p.rts[0] = nv_decode_scale(senc_g);
+      if (CF == kNVG) p.cts[0] = nv_decode_scale(senc_g);
+    }
+    if (RF == kNVG) build_tab(cb->tab_r, senc_g);
+    if (CF == kNVG) build_tab(cb->tab_c, senc_g);
+    __syncthreads();
+  }
+
+  int it = 0;
+  bool failed = false;
+  for (int t = (int)blockIdx.x; t < p.ntiles; t += (int)gridDim.x, ++it) {
+    const int s = it % kStages;
+    const bool ok = wait_bounded(smem_u32(&cb->full[s]), (uint32_t)((it / kStages) & 1), p.timeout_ns);
+    if (__syncthreads_or(!ok)) {
+      failed = true;
+      if (tid == 0 && p.status && atomicCAS(p.status, 0u, kStatusTimeout) == 0u)
+        atomicExch(p.status + 1, 0x600u | (uint32_t)s);
+      break;
+    }
+    if (tid == 0) pending &= ~(1u << s);
+    const uint16_t *tile = reinterpret_cast<const uint16_t *>(smem + s * kTileBytes);
+    const int tc = t % p.tiles_c, tt = t / p.tiles_c;
+    float senc_r = senc_g, senc_c = senc_g;
+    if constexpr (RF == kNVC || CF == kNVC) {
+      // CTA-local: the tile's amax (Q's tile in either orientation holds the
+      // same values), its decode scale and multiplier table
+      const int w = tid >> 5, l = tid & 31;
+      float m = 0.0f;
+#pragma unroll
+      for (int k = 0; k < 8; ++k)
+        m = fmaxf(m, absmax8(lds128(tile + (16 * k + 2 * w + (l >> 4)) * 128 + 8 * (l & 15))));
+      const float se = nv_encode_scale(cta_max256(m, cb->red));
+      if constexpr (RF == kNVC) {
+        senc_r = se;
+        if (tid == 0) p.rts[(int64_t)tt * p.tiles_c + tc] = nv_decode_scale(se);
+        build_tab(cb->tab_r, se);
+      }
+      if constexpr (CF == kNVC) {
+        senc_c = se;
+        if (tid == 0) p.cts[(int64_t)tc * p.tiles_t + tt] = nv_decode_scale(se);
+        build_tab(cb->tab_c, se);
+      }
+      __syncthreads();
+    }
+    const bool edge = ((int64_t)tt * 128 + 128 > p.T) || ((int64_t)tc * 128 + 128 > p.C);
+    if constexpr (RF != kNone) {
+      if (edge)
+        row_pass<RF, RR, true>(tile, p, tt, tc, senc_r, cb->tab_r);
+      else
+        row_pass<RF, RR, false>(tile, p, tt, tc, senc_r, cb->tab_r);
+    }
+    if constexpr (CF != kNone) {
+      if (edge)
+        col_pass<CF, CR, HAD, true>(tile, p, tt, tc, senc_c, cb->tab_c);
+      else
+        col_pass<CF, CR, HAD, false>(tile, p, tt, tc, senc_c, cb->tab_c);
+    }
+    __syncthreads();  // every read of stage s is done
+    if (tid == 0) {
+      const int tn = t + kStages * (int)gridDim.x;
+      if (tn < p.ntiles) {
+        issue_tile(smem, cb, &xmap, p, tn, s);
+        nload_par ^= 1u << s;
+        pending |= 1u << s;
+      }
+    }
+  }
+  if (failed && tid == 0) {
+    // loads still in flight write this CTA's shared memory: let them land
+    // (the n-th load into a stage completes the phase of parity (n - 1) & 1,
+    // the complement of bit k of nload_par)
+    for (int k = 0; k < kStages; ++k) {
+      if (!((pending >> k) & 1u)) continue;
+      const uint64_t t0 = globaltimer();
+      while (!mbar_try_wait(smem_u32(&cb->full[k]), ((nload_par >> k) & 1u) ^ 1u))
+        if (globaltimer() - t0 > p.timeout_ns) break;
+    }
+  }
 }
 
-// --------------------------------------------------------------------------
-// Dual-orientation producer: one read of x[T, C] emits the row-wise operand
-// (Q = x, any format) and the column-wise MXFP4 operand (Q = x^T, optionally
-// with the fixed-sign Hadamard), e.g. the forward operand and the saved
-// weight-gradient operand of an activation, or the data-gradient and
-// weight-gradient operands of dY.  Bytes equal those of the two single-
-// orientation kernels.
-// --------------------------------------------------------------------------
-// tiles: x along channels, y along tokens; the row-wise operand's CTA-local
-// ts index is [token tile][channel tile].  EDGE launches cover every tile
-// (either orientation's atom stride along K may be the padded one).
-template <int RFMT, int RRND, int CRND, bool HAD, bool EDGE>
-__global__ void __launch_bounds__(256) quant_dual_kernel(
-    const uint16_t *__restrict__ x, int64_t T, int64_t C, int64_t ld, uint8_t *__restrict__ row_payload,
-    uint8_t *__restrict__ row_scales, float *__restrict__ row_ts, uint8_t *__restrict__ col_payload,
-    uint8_t *__restrict__ col_scales, const float *__restrict__ partials, int n_partials,
-    uint64_t row_seed, uint64_t col_seed, uint32_t sign_mask) {
-  __shared__ __align__(16) uint16_t tile[128 * 128];  // [token][channel]
-  __shared__ __align__(16) uint8_t sbuf[128 * 8];
-  __shared__ float red[8];
-  const int w = threadIdx.x >> 5, l = threadIdx.x & 31;
-  const int64_t c0 = (int64_t)blockIdx.x * 128, t0 = (int64_t)blockIdx.y * 128;
-  uint4 v[8];
-  load_tile_rowwise<EDGE>(x, ld, t0, c0, T, C, v);
-#pragma unroll
-  for (int s = 0; s < 8; ++s)
-    *reinterpret_cast<uint4 *>(&tile[(16 * s + 2 * w + (l >> 4)) * 128 + 8 * (l & 15)]) = v[s];
-  const float s_enc = tile_encode_scale<RFMT>(v, row_ts, (int64_t)blockIdx.y * gridDim.x + blockIdx.x,
-                                              blockIdx.x == 0 && blockIdx.y == 0, partials,
-                                              n_partials, red);
-  rowwise_tile<RFMT, RRND, EDGE>(v, t0, c0, T, C, row_payload, row_scales, s_enc, row_seed);
-  __syncthreads();
-  colwise_tile<kMX, CRND, HAD, EDGE>(tile, sbuf, c0, t0, C, T, col_payload, col_scales, 1.0f,
-                                     col_seed, sign_mask);
-}
+}  // namespace qk
 
 // --------------------------------------------------------------------------
 // Diagnostics kernels (element conversions and SR bits, as the quantizers
@@ -482,117 +573,90 @@ cudaError_t launch_tensor_amax(const uint16_t *x, int64_t rows, int64_t cols, in
   return cudaGetLastError();
 }
 
-static unsigned tiles_of(int64_t n) { return (unsigned)((n + 127) / 128); }
+namespace {
 
-// Row-wise: K ragged -> every tile EDGE; else R ragged -> the last row of
-// tiles EDGE, the rest unmasked.
-template <int FMT, int RND>
-static void launch_row(cudaStream_t st, const uint16_t *x, int64_t R, int64_t K, int64_t ld,
-                       uint8_t *p, uint8_t *s, float *ts, const float *part, int np, uint64_t seed) {
-  const unsigned na = tiles_of(K), nb = tiles_of(R);
-  EdgeTiles e = {0, 0, (int)na};
-  if (K % 128) {
-    quant_rowwise_kernel<FMT, RND, true><<<dim3(na, nb), 256, 0, st>>>(x, R, K, ld, p, s, ts, part,
-                                                                       np, seed, e);
-    return;
-  }
-  const unsigned inner = (R % 128) ? nb - 1 : nb;
-  if (inner)
-    quant_rowwise_kernel<FMT, RND, false><<<dim3(na, inner), 256, 0, st>>>(x, R, K, ld, p, s, ts,
-                                                                           part, np, seed, e);
-  if (inner < nb) {
-    e.b0 = (int)inner;
-    quant_rowwise_kernel<FMT, RND, true><<<dim3(na, 1), 256, 0, st>>>(x, R, K, ld, p, s, ts, part,
-                                                                      np, seed, e);
+// Philox4x32-10 key schedule (the Weyl sequence of the two key words),
+// round 9's words complemented so that the kernel's last XOR yields the
+// complemented bits directly.
+void philox_round_keys(uint64_t seed, uint32_t *k0, uint32_t *k1) {
+  uint32_t a = (uint32_t)seed, b = (uint32_t)(seed >> 32);
+  for (int r = 0; r < 10; ++r) {
+    k0[r] = r == 9 ? ~a : a;
+    k1[r] = r == 9 ? ~b : b;
+    a += 0x9E3779B9u;
+    b += 0xBB67AE85u;
   }
 }
 
-cudaError_t launch_quant_rowwise(int fmt, int rnd, const uint16_t *x, int64_t R, int64_t K,
-                                 int64_t ld, uint8_t *payload, uint8_t *scales, float *ts,
-                                 const float *partials, int n_partials, uint64_t seed,
-                                 cudaStream_t st) {
-#define FA4_ROW(F, Q) \
-  if (fmt == F && rnd == Q) launch_row<F, Q>(st, x, R, K, ld, payload, scales, ts, partials, n_partials, seed);
-  FA4_ROW(kMX, kRNE) FA4_ROW(kMX, kSR) FA4_ROW(kNVG, kRNE) FA4_ROW(kNVG, kSR) FA4_ROW(kNVC, kRNE)
-  FA4_ROW(kMXN, kRNE) FA4_ROW(kMXN, kSR)
-  FA4_ROW(kNVC, kSR)
-#undef FA4_ROW
+template <int RF, int RR, int CF, int CR, bool H>
+cudaError_t launch_q(const CUtensorMap &map, const qk::Params &p, cudaStream_t st) {
+  auto kern = qk::quant_kernel<RF, RR, CF, CR, H>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, qk::kSmemBytes);
+  if (e != cudaSuccess) return e;
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int grid = p.ntiles < 2 * sms ? p.ntiles : 2 * sms;
+  kern<<<grid, qk::kThreads, qk::kSmemBytes, st>>>(map, p);
   return cudaGetLastError();
 }
 
-// Column-wise (Q = x^T): T (K of Q) ragged -> every tile EDGE; else C (rows
-// of Q) ragged -> the last column of tiles EDGE, the rest unmasked.
-template <int FMT, int RND, bool HAD>
-static void launch_col(cudaStream_t st, const uint16_t *x, int64_t T, int64_t C, int64_t ld,
-                       uint8_t *p, uint8_t *s, float *ts, const float *part, int np, uint64_t seed,
-                       uint32_t mask) {
-  const unsigned na = tiles_of(C), nb = tiles_of(T);
-  EdgeTiles e = {0, 0, (int)na};
-  if (T % 128) {
-    quant_colwise_kernel<FMT, RND, HAD, true><<<dim3(na, nb), 256, 0, st>>>(
-        x, T, C, ld, p, s, ts, part, np, seed, mask, e, (int)nb);
-    return;
+// Dispatch on (row format, row rounding): the column-wise side fixed.
+template <int CF, int CR, bool H>
+cudaError_t dispatch_row(int rf, int rr, const CUtensorMap &map, const qk::Params &p, cudaStream_t st) {
+#define FA4_Q_ROW(F)                                                              \
+  if (rf == F) return rr == kSR ? launch_q<F, kSR, CF, CR, H>(map, p, st)       \
+                                : launch_q<F, kRNE, CF, CR, H>(map, p, st);
+  FA4_Q_ROW(kMX) FA4_Q_ROW(kNVG) FA4_Q_ROW(kNVC) FA4_Q_ROW(kMXN)
+#undef FA4_Q_ROW
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace
+
+cudaError_t launch_quantize(const QuantArgs &a, cudaStream_t st) {
+  qk::Params p = {};
+  p.T = a.T;
+  p.C = a.C;
+  p.tiles_c = (int)((a.C + 127) / 128);
+  p.tiles_t = (int)((a.T + 127) / 128);
+  p.ntiles = p.tiles_c * p.tiles_t;
+  p.rp = a.row_payload;
+  p.rs = a.row_scales;
+  p.rts = a.row_ts;
+  p.cp = a.col_payload;
+  p.cs = a.col_scales;
+  p.cts = a.col_ts;
+  philox_round_keys(a.row_seed, p.rkey0, p.rkey1);
+  philox_round_keys(a.col_seed, p.ckey0, p.ckey1);
+  for (int t = 0; t < 32; ++t) p.sgn[t] = ((a.sign_mask >> t) & 1u) ? 0x80000000u : 0u;
+  p.partials = a.partials;
+  p.np = a.n_partials;
+  p.status = a.status;
+  p.timeout_ns = a.timeout_ns;
+  CUtensorMap map;
+  if (!make_bf16_tile_map(&map, a.x, a.T, a.C, a.ld)) return cudaErrorInvalidValue;
+  const int rf = a.row_fmt, rr = a.row_rnd, cf = a.col_fmt, cr = a.col_rnd;
+  using namespace qk;
+  if (cf == kNone) return dispatch_row<kNone, kRNE, false>(rf, rr, map, p, st);
+  if (rf == kNone) {
+    // column-wise only
+#define FA4_Q_COL(F, H)                                                              \
+  if (cf == F && a.hadamard == H)                                                    \
+    return cr == kSR ? launch_q<kNone, kRNE, F, kSR, H>(map, p, st)                  \
+                     : launch_q<kNone, kRNE, F, kRNE, H>(map, p, st);
+    FA4_Q_COL(kMX, false) FA4_Q_COL(kMX, true) FA4_Q_COL(kNVG, false) FA4_Q_COL(kNVC, false)
+    FA4_Q_COL(kMXN, false)
+#undef FA4_Q_COL
+    return cudaErrorInvalidValue;
   }
-  const unsigned inner = (C % 128) ? na - 1 : na;
-  if (inner)
-    quant_colwise_kernel<FMT, RND, HAD, false><<<dim3(inner, nb), 256, 0, st>>>(
-        x, T, C, ld, p, s, ts, part, np, seed, mask, e, (int)nb);
-  if (inner < na) {
-    e.a0 = (int)inner;
-    quant_colwise_kernel<FMT, RND, HAD, true><<<dim3(1, nb), 256, 0, st>>>(
-        x, T, C, ld, p, s, ts, part, np, seed, mask, e, (int)nb);
-  }
-}
-
-cudaError_t launch_quant_colwise(int fmt, int rnd, bool hadamard, uint32_t sign_mask,
-                                 const uint16_t *x, int64_t T, int64_t C, int64_t ld,
-                                 uint8_t *payload, uint8_t *scales, float *ts,
-                                 const float *partials, int n_partials, uint64_t seed,
-                                 cudaStream_t st) {
-#define FA4_COL(F, Q, H)                                                                   \
-  if (fmt == F && rnd == Q && hadamard == H)                                               \
-    launch_col<F, Q, H>(st, x, T, C, ld, payload, scales, ts, partials, n_partials, seed, \
-                        sign_mask);
-  FA4_COL(kMX, kRNE, false) FA4_COL(kMX, kSR, false) FA4_COL(kMX, kRNE, true)
-  FA4_COL(kMX, kSR, true) FA4_COL(kNVG, kRNE, false) FA4_COL(kNVG, kSR, false)
-  FA4_COL(kMXN, kRNE, false) FA4_COL(kMXN, kSR, false)
-  FA4_COL(kNVC, kRNE, false) FA4_COL(kNVC, kSR, false)
-#undef FA4_COL
-  return cudaGetLastError();
-}
-
-// Both orientations: either extent ragged -> every tile EDGE.
-template <int RF, int RR, int CR, bool H>
-static void launch_dual_t(cudaStream_t st, const uint16_t *x, int64_t T, int64_t C, int64_t ld,
-                          uint8_t *rp, uint8_t *rs, float *rts, uint8_t *cp, uint8_t *cs,
-                          const float *part, int np, uint64_t rseed, uint64_t cseed, uint32_t mask) {
-  const dim3 g(tiles_of(C), tiles_of(T));
-  if ((T % 128) || (C % 128))
-    quant_dual_kernel<RF, RR, CR, H, true><<<g, 256, 0, st>>>(x, T, C, ld, rp, rs, rts, cp, cs, part,
-                                                              np, rseed, cseed, mask);
-  else
-    quant_dual_kernel<RF, RR, CR, H, false><<<g, 256, 0, st>>>(x, T, C, ld, rp, rs, rts, cp, cs,
-                                                               part, np, rseed, cseed, mask);
-}
-
-cudaError_t launch_quant_dual(int row_fmt, int row_rnd, int col_rnd, bool hadamard,
-                              uint32_t sign_mask, const uint16_t *x, int64_t T, int64_t C,
-                              int64_t ld, uint8_t *row_payload, uint8_t *row_scales, float *row_ts,
-                              uint8_t *col_payload, uint8_t *col_scales, const float *partials,
-                              int n_partials, uint64_t row_seed, uint64_t col_seed,
-                              cudaStream_t st) {
-#define FA4_DUAL(F, RR, CR, H)                                                               \
-  if (row_fmt == F && row_rnd == RR && col_rnd == CR && hadamard == H)                       \
-    launch_dual_t<F, RR, CR, H>(st, x, T, C, ld, row_payload, row_scales, row_ts, col_payload, \
-                                col_scales, partials, n_partials, row_seed, col_seed, sign_mask);
-#define FA4_DUAL_F(F)                                                                 \
-  FA4_DUAL(F, kRNE, kRNE, false) FA4_DUAL(F, kRNE, kRNE, true) FA4_DUAL(F, kRNE, kSR, false) \
-  FA4_DUAL(F, kRNE, kSR, true) FA4_DUAL(F, kSR, kRNE, false) FA4_DUAL(F, kSR, kRNE, true)    \
-  FA4_DUAL(F, kSR, kSR, false) FA4_DUAL(F, kSR, kSR, true)
-  FA4_DUAL_F(kMX) FA4_DUAL_F(kNVG) FA4_DUAL_F(kNVC) FA4_DUAL_F(kMXN)
-#undef FA4_DUAL_F
-#undef FA4_DUAL
-  return cudaGetLastError();
+  // both orientations: the column-wise operand is MXFP4 (optionally Hadamard)
+  if (cf != kMX) return cudaErrorInvalidValue;
+  if (a.hadamard)
+    return cr == kSR ? dispatch_row<kMX, kSR, true>(rf, rr, map, p, st)
+                     : dispatch_row<kMX, kRNE, true>(rf, rr, map, p, st);
+  return cr == kSR ? dispatch_row<kMX, kSR, false>(rf, rr, map, p, st)
+                   : dispatch_row<kMX, kRNE, false>(rf, rr, map, p, st);
 }
 
 cudaError_t launch_debug_convert(const float *y, const uint32_t *u16, int64_t n, uint8_t *rne,
