@@ -117,6 +117,24 @@ def _stream(device: torch.device):
     return ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
 
 
+def _on_tensor_device(fn):
+    """Run a binding with the device of its first CUDA tensor argument (a
+    QTensor's payload counts) current: the library picks the device's SM
+    count and scratch from the current device, and launches on that
+    device's current stream."""
+    import functools
+
+    @functools.wraps(fn)
+    def wrapped(*args, **kwargs):
+        for a in list(args) + list(kwargs.values()):
+            t = a.payload if isinstance(a, QTensor) else a
+            if isinstance(t, torch.Tensor) and t.is_cuda:
+                with torch.cuda.device(t.device):
+                    return fn(*args, **kwargs)
+        return fn(*args, **kwargs)
+    return wrapped
+
+
 @dataclass
 class QTensor:
     """Quantized operand Q[R, K]: ``payload`` uint8 [R, K/2] (K-major, element
@@ -181,10 +199,51 @@ def _rowmajor_bf16(x: torch.Tensor, name: str) -> torch.Tensor:
     return x if x.is_contiguous() else x.contiguous()
 
 
+def _check_qt(q: QTensor, R: int, K: int, fmt: int, device, name: str):
+    """A quantized operand of Q[R, K] in `fmt` whose buffers are large enough
+    for the C calls (which take no buffer sizes) and live on `device`."""
+    if not isinstance(q, QTensor):
+        raise ValueError(f"{name} must be a QTensor")
+    if (q.R, q.K) != (R, K):
+        raise ValueError(f"{name} is [{q.R}, {q.K}], the call needs [{R}, {K}]")
+    same = {fmt} | ({MXFP4, MXFP4_NOCLIP} if fmt in (MXFP4, MXFP4_NOCLIP) else set())
+    if q.fmt not in same:
+        raise ValueError(f"{name} has format {q.fmt}, the call needs {fmt}")
+    _, sb, tc, _ = quant_sizes(R, K, fmt, ROWWISE)
+    for t, n, what in ((q.payload, R * (K // 2), "payload"), (q.scales, sb, "scales")):
+        if t.dtype != torch.uint8 or t.device != device or not t.is_contiguous() or t.numel() < n:
+            raise ValueError(f"{name}.{what} must be a contiguous uint8 tensor of >= {n} bytes on {device}")
+    if tc:
+        t = q.ts
+        if t is None or t.dtype != torch.float32 or t.device != device or not t.is_contiguous() \
+                or t.numel() < tc:
+            raise ValueError(f"{name}.ts must be a contiguous float32 tensor of >= {tc} values on {device}")
+
+
+def _check_out(t: torch.Tensor, shape: tuple, dtypes: tuple, device, name: str, row_stride=False):
+    """A caller-supplied output: `shape`, one of `dtypes`, on `device`,
+    contiguous (or, with row_stride, unit column stride and a row stride the
+    C call can take)."""
+    if t.dtype not in dtypes:
+        raise ValueError(f"{name} must have dtype {' or '.join(str(d) for d in dtypes)}, not {t.dtype}")
+    if tuple(t.shape) != tuple(shape) or t.device != device:
+        raise ValueError(f"{name} must be a {list(shape)} tensor on {device}, "
+                         f"not {list(t.shape)} on {t.device}")
+    if row_stride:
+        if t.dim() != 2 or t.stride(1) != 1 or t.stride(0) < shape[1] or t.stride(0) % 8:
+            raise ValueError(f"{name} needs unit column stride and a row stride >= {shape[1]}, "
+                             "a multiple of 8")
+    elif not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+@_on_tensor_device
 def quantize(x: torch.Tensor, fmt: int, rnd: int = RNE, orient: int = ROWWISE, seed: int = 0,
              out: QTensor | None = None, ws: torch.Tensor | None = None) -> QTensor:
     ld = _as_bf16_2d(x, "x")
     rows, cols = x.shape
+    if out is not None:
+        _check_qt(out, *((rows, cols) if orient == ROWWISE else (cols, rows)), fmt, x.device, "out")
     out = out or empty_qtensor(rows, cols, fmt, orient, x.device)
     need = quant_sizes(rows, cols, fmt, orient)[3]
     ws = _ws(ws, need, x.device)
@@ -193,12 +252,16 @@ def quantize(x: torch.Tensor, fmt: int, rnd: int = RNE, orient: int = ROWWISE, s
     return out
 
 
+@_on_tensor_device
 def quantize_nvfp4_global_noalloc(x: torch.Tensor, rnd: int = RNE, orient: int = ROWWISE,
                                   seed: int = 0, out: QTensor | None = None) -> QTensor:
     """NVFP4-global quantization without a workspace: the amax scratch lives
     in a fixed array inside the library (see include/fa4.h)."""
     ld = _as_bf16_2d(x, "x")
     rows, cols = x.shape
+    if out is not None:
+        _check_qt(out, *((rows, cols) if orient == ROWWISE else (cols, rows)), NVFP4_GLOBAL,
+                  x.device, "out")
     out = out or empty_qtensor(rows, cols, NVFP4_GLOBAL, orient, x.device)
     _check(lib().fa4_quantize_nvfp4_global_noalloc(_ptr(x), rows, cols, ld, rnd, orient, seed,
                                                    out.c(), _stream(x.device)),
@@ -206,10 +269,13 @@ def quantize_nvfp4_global_noalloc(x: torch.Tensor, rnd: int = RNE, orient: int =
     return out
 
 
+@_on_tensor_device
 def hadamard32_quantize(x: torch.Tensor, sign_mask: int, rnd: int = RNE, seed: int = 0,
                         out: QTensor | None = None, ws: torch.Tensor | None = None) -> QTensor:
     ld = _as_bf16_2d(x, "x")
     rows, cols = x.shape
+    if out is not None:
+        _check_qt(out, cols, rows, MXFP4, x.device, "out")
     out = out or empty_qtensor(rows, cols, MXFP4, COLWISE, x.device)
     ws = _ws(ws, WS_HEADER_BYTES, x.device)
     _check(lib().fa4_hadamard32_quantize(_ptr(x), rows, cols, ld, sign_mask & 0xFFFFFFFF, rnd, seed,
@@ -218,6 +284,7 @@ def hadamard32_quantize(x: torch.Tensor, sign_mask: int, rnd: int = RNE, seed: i
     return out
 
 
+@_on_tensor_device
 def quantize_dual(x: torch.Tensor, row_fmt: int, row_rnd: int = RNE, row_seed: int = 0,
                   col_hadamard: bool = True, sign_mask: int = 0, col_rnd: int = RNE,
                   col_seed: int = 0, row_out: QTensor | None = None,
@@ -227,6 +294,10 @@ def quantize_dual(x: torch.Tensor, row_fmt: int, row_rnd: int = RNE, row_seed: i
     MXFP4 operand (with the fixed-sign Hadamard when col_hadamard)."""
     ld = _as_bf16_2d(x, "x")
     rows, cols = x.shape
+    if row_out is not None:
+        _check_qt(row_out, rows, cols, row_fmt, x.device, "row_out")
+    if col_out is not None:
+        _check_qt(col_out, cols, rows, MXFP4, x.device, "col_out")
     row_out = row_out or empty_qtensor(rows, cols, row_fmt, ROWWISE, x.device)
     col_out = col_out or empty_qtensor(rows, cols, MXFP4, COLWISE, x.device)
     need = quant_sizes(rows, cols, row_fmt, ROWWISE)[3]
@@ -238,6 +309,7 @@ def quantize_dual(x: torch.Tensor, row_fmt: int, row_rnd: int = RNE, row_seed: i
     return row_out, col_out
 
 
+@_on_tensor_device
 def gemm(A: QTensor, B: QTensor, alpha: float = 1.0, out_dtype=torch.float32,
          out: torch.Tensor | None = None, ws: torch.Tensor | None = None) -> torch.Tensor:
     """D[M, N] = alpha * A B^T on the block-scaled FP4 tensor cores."""
@@ -248,6 +320,9 @@ def gemm(A: QTensor, B: QTensor, alpha: float = 1.0, out_dtype=torch.float32,
         # leading dimension a multiple of 8 elements (the ABI's row alignment)
         ldd = -(-B.R // 8) * 8
         out = torch.empty((A.R, ldd), dtype=out_dtype, device=dev)[:, :B.R]
+    _check_qt(B, B.R, A.K, A.fmt, dev, "B")
+    _check_qt(A, A.R, A.K, A.fmt, dev, "A")
+    _check_out(out, (A.R, B.R), (torch.bfloat16, torch.float32), dev, "out", row_stride=True)
     od = OUT_FP32 if out.dtype == torch.float32 else OUT_BF16
     ws = _ws(ws, WS_HEADER_BYTES, dev)
     _check(lib().fa4_gemm_blockscaled(A.c(), B.c(), A.R, B.R, A.K, A.fmt, float(alpha), _ptr(out),
@@ -262,12 +337,16 @@ def linear_ws_bytes(kind: int, T: int, Cin: int, Cout: int, fmt: int) -> int:
     return n.value
 
 
+@_on_tensor_device
 def linear_fwd(X: torch.Tensor, Wq: QTensor, fmt: int, out: torch.Tensor | None = None,
                ws: torch.Tensor | None = None) -> torch.Tensor:
     """Y = X W^T; Wq is W[Cout, Cin] quantized row-wise."""
     X = _rowmajor_bf16(X, "X")
     T, Cin = X.shape
     Cout = Wq.R
+    _check_qt(Wq, Cout, Cin, fmt, X.device, "Wq")
+    if out is not None:
+        _check_out(out, (T, Cout), (torch.bfloat16,), X.device, "out")
     out = out if out is not None else torch.empty((T, Cout), dtype=torch.bfloat16, device=X.device)
     ws = _ws(ws, linear_ws_bytes(0, T, Cin, Cout, fmt), X.device)
     _check(lib().fa4_linear_fwd(_ptr(X), Wq.c(), T, Cin, Cout, fmt, _ptr(out), _ptr(ws),
@@ -275,12 +354,16 @@ def linear_fwd(X: torch.Tensor, Wq: QTensor, fmt: int, out: torch.Tensor | None 
     return out
 
 
+@_on_tensor_device
 def linear_dgrad(dY: torch.Tensor, Wq_col: QTensor, fmt: int, rnd: int = SR, seed: int = 0,
                  out: torch.Tensor | None = None, ws: torch.Tensor | None = None) -> torch.Tensor:
     """dX = dY W; Wq_col is W[Cout, Cin] quantized column-wise ([Cin, Cout])."""
     dY = _rowmajor_bf16(dY, "dY")
     T, Cout = dY.shape
     Cin = Wq_col.R
+    _check_qt(Wq_col, Cin, Cout, fmt, dY.device, "Wq_col")
+    if out is not None:
+        _check_out(out, (T, Cin), (torch.bfloat16,), dY.device, "out")
     out = out if out is not None else torch.empty((T, Cin), dtype=torch.bfloat16, device=dY.device)
     ws = _ws(ws, linear_ws_bytes(1, T, Cin, Cout, fmt), dY.device)
     _check(lib().fa4_linear_dgrad(_ptr(dY), Wq_col.c(), T, Cin, Cout, fmt, rnd, seed,
@@ -289,6 +372,7 @@ def linear_dgrad(dY: torch.Tensor, Wq_col: QTensor, fmt: int, rnd: int = SR, see
     return out
 
 
+@_on_tensor_device
 def linear_wgrad(dY: torch.Tensor, X: torch.Tensor, sign_mask: int, rnd: int = RNE, seed: int = 0,
                  out_dtype=torch.float32, out: torch.Tensor | None = None,
                  ws: torch.Tensor | None = None) -> torch.Tensor:
@@ -296,9 +380,14 @@ def linear_wgrad(dY: torch.Tensor, X: torch.Tensor, sign_mask: int, rnd: int = R
     dY = _rowmajor_bf16(dY, "dY")
     X = _rowmajor_bf16(X, "X")
     T, Cout = dY.shape
-    _, Cin = X.shape
+    TX, Cin = X.shape
+    if TX != T or X.device != dY.device:
+        raise ValueError(f"X must have dY's {T} rows and device")
     if out is None:
+        if out_dtype not in (torch.bfloat16, torch.float32):
+            raise ValueError("out_dtype must be torch.bfloat16 or torch.float32")
         out = torch.empty((Cout, Cin), dtype=out_dtype, device=dY.device)
+    _check_out(out, (Cout, Cin), (torch.bfloat16, torch.float32), dY.device, "out")
     od = OUT_FP32 if out.dtype == torch.float32 else OUT_BF16
     ws = _ws(ws, linear_ws_bytes(2, T, Cin, Cout, MXFP4), dY.device)
     _check(lib().fa4_linear_wgrad(_ptr(dY), _ptr(X), T, Cin, Cout,
@@ -307,6 +396,7 @@ def linear_wgrad(dY: torch.Tensor, X: torch.Tensor, sign_mask: int, rnd: int = R
     return out
 
 
+@_on_tensor_device
 def check_device_status(ws: torch.Tensor) -> int:
     """Synchronize and return (and clear) the workspace's device status."""
     return lib().fa4_check_device_status(_ptr(ws), _stream(ws.device))
@@ -343,6 +433,7 @@ def debug_gemm_timeout(A: QTensor, B: QTensor, skip_k_tile: int, timeout_ns: int
     return out
 
 
+@_on_tensor_device
 def linear_fwd_save(X: torch.Tensor, Wq: QTensor, fmt: int, sign_mask: int,
                     out: torch.Tensor | None = None, xcol: QTensor | None = None,
                     ws: torch.Tensor | None = None) -> tuple[torch.Tensor, QTensor]:
@@ -351,6 +442,11 @@ def linear_fwd_save(X: torch.Tensor, Wq: QTensor, fmt: int, sign_mask: int,
     X = _rowmajor_bf16(X, "X")
     T, Cin = X.shape
     Cout = Wq.R
+    _check_qt(Wq, Cout, Cin, fmt, X.device, "Wq")
+    if out is not None:
+        _check_out(out, (T, Cout), (torch.bfloat16,), X.device, "out")
+    if xcol is not None:
+        _check_qt(xcol, Cin, T, MXFP4, X.device, "xcol")
     Y = out if out is not None else torch.empty(T, Cout, dtype=torch.bfloat16, device=X.device)
     xcol = xcol or empty_qtensor(T, Cin, MXFP4, COLWISE, X.device)
     ws = _ws(ws, linear_ws_bytes(3, T, Cin, Cout, fmt), X.device)
@@ -360,6 +456,7 @@ def linear_fwd_save(X: torch.Tensor, Wq: QTensor, fmt: int, sign_mask: int,
     return Y, xcol
 
 
+@_on_tensor_device
 def linear_bwd(dY: torch.Tensor, Wq_col: QTensor, xcol: QTensor, fmt: int, rnd: int = SR,
                seed: int = 0, sign_mask: int = 0, dw_dtype=torch.float32,
                dx: torch.Tensor | None = None, dw: torch.Tensor | None = None,
@@ -369,6 +466,14 @@ def linear_bwd(dY: torch.Tensor, Wq_col: QTensor, xcol: QTensor, fmt: int, rnd: 
     dY = _rowmajor_bf16(dY, "dY")
     T, Cout = dY.shape
     Cin = Wq_col.R
+    _check_qt(Wq_col, Cin, Cout, fmt, dY.device, "Wq_col")
+    _check_qt(xcol, Cin, T, MXFP4, dY.device, "xcol")
+    if dx is not None:
+        _check_out(dx, (T, Cin), (torch.bfloat16,), dY.device, "dx")
+    if dw is not None:
+        _check_out(dw, (Cout, Cin), (torch.bfloat16, torch.float32), dY.device, "dw")
+    elif dw_dtype not in (torch.bfloat16, torch.float32):
+        raise ValueError("dw_dtype must be torch.bfloat16 or torch.float32")
     dX = dx if dx is not None else torch.empty(T, Cin, dtype=torch.bfloat16, device=dY.device)
     dW = dw if dw is not None else torch.empty(Cout, Cin, dtype=dw_dtype, device=dY.device)
     od = OUT_FP32 if dW.dtype == torch.float32 else OUT_BF16
@@ -379,6 +484,7 @@ def linear_bwd(dY: torch.Tensor, Wq_col: QTensor, xcol: QTensor, fmt: int, rnd: 
     return dX, dW
 
 
+@_on_tensor_device
 def gemm_mxout(A: QTensor, B: QTensor, alpha: float = 1.0, store_d: bool = True,
                out: torch.Tensor | None = None, qout: QTensor | None = None,
                ws: torch.Tensor | None = None) -> tuple[torch.Tensor | None, QTensor]:
@@ -387,6 +493,12 @@ def gemm_mxout(A: QTensor, B: QTensor, alpha: float = 1.0, store_d: bool = True,
     if A.K != B.K or A.fmt != B.fmt:
         raise ValueError("A and B must share K and format")
     dev = A.payload.device
+    _check_qt(A, A.R, A.K, A.fmt, dev, "A")
+    _check_qt(B, B.R, A.K, A.fmt, dev, "B")
+    if store_d and out is not None:
+        _check_out(out, (A.R, B.R), (torch.bfloat16,), dev, "out", row_stride=True)
+    if qout is not None:
+        _check_qt(qout, A.R, B.R, MXFP4, dev, "qout")
     if store_d and out is None:
         out = torch.empty((A.R, B.R), dtype=torch.bfloat16, device=dev)
     qout = qout or empty_qtensor(A.R, B.R, MXFP4, ROWWISE, dev)

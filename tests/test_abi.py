@@ -291,3 +291,62 @@ def test_linear_bindings_validate_inputs_before_any_call():
                  lambda: fa.linear_fwd(x.to(torch.bfloat16), q, fa.MXFP4)):
         with pytest.raises(ValueError):
             call()
+
+
+def _qt_cpu(R, K, fmt):
+    import torch
+    _, sb, tc, _ = fa.quant_sizes(R, K, fmt)
+    return fa.QTensor(torch.zeros(R, K // 2, dtype=torch.uint8), torch.zeros(sb, dtype=torch.uint8),
+                      torch.zeros(tc, dtype=torch.float32) if tc else None, R, K, fmt)
+
+
+def test_operand_validation_rejects_mismatched_operands_and_outputs():
+    """The bindings check every operand and caller-supplied output against the
+    call's sizes before reaching the library, whose C calls take no buffer
+    sizes: a quantized operand with the wrong [R, K] or format, short or
+    non-contiguous buffers, a missing second-level scale, an output of the
+    wrong shape, dtype (fp16 is not bf16) or layout.  The checks take the
+    device to compare with, so they run here on CPU tensors."""
+    import torch
+    dev = torch.device("cpu")
+    good = _qt_cpu(256, 512, fa.NVFP4_GLOBAL)
+    fa._check_qt(good, 256, 512, fa.NVFP4_GLOBAL, dev, "q")
+    bad = [
+        (good, 256, 256, fa.NVFP4_GLOBAL),                     # K differs (Wq.K != Cin)
+        (good, 128, 512, fa.NVFP4_GLOBAL),                     # R differs
+        (good, 256, 512, fa.MXFP4),                            # format differs
+        (fa.QTensor(good.payload[:100], good.scales, good.ts, 256, 512, fa.NVFP4_GLOBAL),
+         256, 512, fa.NVFP4_GLOBAL),                           # short payload
+        (fa.QTensor(good.payload, good.scales[:10], good.ts, 256, 512, fa.NVFP4_GLOBAL),
+         256, 512, fa.NVFP4_GLOBAL),                           # short scales
+        (fa.QTensor(good.payload, good.scales, None, 256, 512, fa.NVFP4_GLOBAL),
+         256, 512, fa.NVFP4_GLOBAL),                           # no tensor scale
+        (fa.QTensor(good.payload.t(), good.scales, good.ts, 256, 512, fa.NVFP4_GLOBAL),
+         256, 512, fa.NVFP4_GLOBAL),                           # strided payload
+    ]
+    for q, R, K, fmt in bad:
+        with pytest.raises(ValueError):
+            fa._check_qt(q, R, K, fmt, dev, "q")
+    # MXFP4 and its no-clip variant share layout and scale type
+    fa._check_qt(_qt_cpu(256, 512, fa.MXFP4_NOCLIP), 256, 512, fa.MXFP4, dev, "q")
+    # CTA-local: one decode scale per 128x128 tile
+    nvc = _qt_cpu(256, 512, fa.NVFP4_CTA)
+    assert nvc.ts.numel() == 8
+    with pytest.raises(ValueError):
+        fa._check_qt(fa.QTensor(nvc.payload, nvc.scales, nvc.ts[:4], 256, 512, fa.NVFP4_CTA),
+                     256, 512, fa.NVFP4_CTA, dev, "q")
+    # outputs
+    bf, f32 = (torch.bfloat16,), (torch.bfloat16, torch.float32)
+    fa._check_out(torch.zeros(64, 32, dtype=torch.float32), (64, 32), f32, dev, "out")
+    for t, shape, dt, rs in [
+        (torch.zeros(64, 32, dtype=torch.float16), (64, 32), f32, False),   # fp16 is not bf16
+        (torch.zeros(64, 32, dtype=torch.float32), (64, 32), bf, False),    # dtype not allowed here
+        (torch.zeros(64, 16, dtype=torch.bfloat16), (64, 32), bf, False),   # shape
+        (torch.zeros(32, 64, dtype=torch.bfloat16).t(), (64, 32), bf, False),  # not contiguous
+        (torch.zeros(64, 36, dtype=torch.bfloat16)[:, :32], (64, 32), bf, True),  # row stride % 8
+    ]:
+        with pytest.raises(ValueError):
+            fa._check_out(t, shape, dt, dev, "out", row_stride=rs)
+    # a row stride that is a multiple of 8 is a valid GEMM output
+    fa._check_out(torch.zeros(64, 40, dtype=torch.bfloat16)[:, :32], (64, 32), bf, dev, "out",
+                  row_stride=True)
