@@ -66,10 +66,47 @@ def bf16_half_ulp(v: np.ndarray) -> np.ndarray:
     return np.where(a > 0, np.exp2(e - 8), 0.0)
 
 
-def assert_gemm_close(d_gpu: np.ndarray, d_orc: np.ndarray, tol: float, bf16: bool = False):
+U32 = 2.0 ** -24  # unit roundoff of binary32
+
+
+def accumulation_bound(A: O.QTensor, B: O.QTensor, alpha: float = 1.0, m_idx=None, n_idx=None):
+    """Per-output bound on |D_gpu - D_exact| from binary32 accumulation:
+    (gamma_K + 8u) * |alpha| * sum_k |a_k| |b_k|, with gamma_K = K u / (1 - K u)
+    the recursive-summation bound and a_k, b_k the dequantized operands
+    (second-level scales included; u = 2^-24).  The 8u covers the few
+    roundings outside the sum: alpha and the tensor-scale product, the
+    CTA-local chunk factor and its fused fold.  Far tighter than the
+    configuration's tolerance: a wrong scale on one block row or tile fails
+    it."""
+    a = np.abs(O.dequantize(A, m_idx))
+    b = np.abs(O.dequantize(B, n_idx))
+    K = A.K
+    gamma = K * U32 / (1.0 - K * U32)
+    return (gamma + 8 * U32) * abs(alpha) * (a @ b.T)
+
+
+def assert_gemm_close(d_gpu: np.ndarray, d_orc: np.ndarray, tol: float, bf16: bool = False,
+                      tight=None):
+    """max |D_gpu - D_oracle| <= tol (plus half a bf16 ulp of the exact value
+    for bf16 output) and, when `tight` (accumulation_bound) is given, every
+    element within its accumulation bound too.  Prints the observed worst
+    ratios to both bounds."""
     d_gpu = d_gpu.astype(np.float64)
     err = np.abs(d_gpu - d_orc)
-    allow = tol + (bf16_half_ulp(d_orc) if bf16 else 0.0)
+    half = bf16_half_ulp(d_orc) if bf16 else 0.0
+    allow = tol + half
     worst = float((err - allow).max())
     assert np.all(err <= allow), f"max|err| {err.max():.3e} exceeds the bound by {worst:.3e} (tol {tol:.3e})"
+    msg = f"{'bf16' if bf16 else 'fp32'} out: max|err| {err.max():.3e} = {err.max() / tol:.2e} of tol"
+    if tight is not None:
+        t_allow = tight + half
+        ratio = float((err / np.where(t_allow > 0, t_allow, np.inf)).max())
+        msg += f", {ratio:.3f} of the accumulation bound"
+        bad = err > t_allow
+        if np.any(bad):
+            i = np.argwhere(bad)[0]
+            raise AssertionError(f"{int(bad.sum())} outputs exceed the accumulation bound; first "
+                                 f"{tuple(int(v) for v in i)}: err {err[tuple(i)]:.3e} > "
+                                 f"{t_allow[tuple(i)]:.3e}")
+    print(msg)
     return float(err.max())

@@ -9,7 +9,7 @@ import torch
 import fp4_quantization_block_b200 as fa
 import oracle as O
 import workloads
-from gpu_util import (FMT_IDS, FMTS, assert_gemm_close, assert_qt_equal, need_gpu, to_cpu_qt,
+from gpu_util import (FMT_IDS, FMTS, accumulation_bound, assert_gemm_close, assert_qt_equal, need_gpu, to_cpu_qt,
                       to_gpu_qt)
 
 pytestmark = pytest.mark.gpu
@@ -118,10 +118,13 @@ def test_training_linear_against_the_oracle():
     y, xcol = fa.linear_fwd_save(x.cuda(), to_gpu_qt(Wq), fa.NVFP4_GLOBAL, MASK)
     dx, dw = fa.linear_bwd(dy.cuda(), to_gpu_qt(Wc), xcol, fa.NVFP4_GLOBAL, fa.SR, 5, MASK)
     Xq = O.quantize(x, O.NVFP4_GLOBAL)
-    assert_gemm_close(y.float().cpu().numpy(), O.gemm(Xq, Wq), O.gemm_tolerance(Xq, Wq), bf16=True)
+    assert_gemm_close(y.float().cpu().numpy(), O.gemm(Xq, Wq), O.gemm_tolerance(Xq, Wq), bf16=True,
+                      tight=accumulation_bound(Xq, Wq))
     Gq = O.quantize(dy, O.NVFP4_GLOBAL, O.SR, O.ROWWISE, 5)
-    assert_gemm_close(dx.float().cpu().numpy(), O.gemm(Gq, Wc), O.gemm_tolerance(Gq, Wc), bf16=True)
+    assert_gemm_close(dx.float().cpu().numpy(), O.gemm(Gq, Wc), O.gemm_tolerance(Gq, Wc), bf16=True,
+                      tight=accumulation_bound(Gq, Wc))
     Gc = O.quantize(dy, O.MXFP4, O.RNE, O.COLWISE, hadamard_mask=MASK)
     Xc = O.quantize(x, O.MXFP4, O.RNE, O.COLWISE, hadamard_mask=MASK)
     assert_qt_equal(to_cpu_qt(xcol), Xc)
-    assert_gemm_close(dw.cpu().numpy(), O.gemm(Gc, Xc, 1.0 / 32), O.gemm_tolerance(Gc, Xc, 1.0 / 32))
+    assert_gemm_close(dw.cpu().numpy(), O.gemm(Gc, Xc, 1.0 / 32), O.gemm_tolerance(Gc, Xc, 1.0 / 32),
+                      tight=accumulation_bound(Gc, Xc, 1.0 / 32))

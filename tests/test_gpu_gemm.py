@@ -12,7 +12,7 @@ import torch
 import fp4_quantization_block_b200 as fa
 import oracle as O
 import workloads
-from gpu_util import FMT_IDS, FMTS, assert_gemm_close, need_gpu, to_gpu_qt
+from gpu_util import FMT_IDS, FMTS, accumulation_bound, assert_gemm_close, need_gpu, to_gpu_qt
 
 pytestmark = pytest.mark.gpu
 
@@ -32,7 +32,8 @@ def _run(xa, xb, fmt, alpha=1.0, out=torch.float32, rows=None, cols=None):
     else:
         want = O.gemm_sampled(A, B, alpha) if A.R * B.R * A.K > (1 << 24) else O.gemm(A, B, alpha)
     tol = O.gemm_tolerance(A, B, alpha)
-    return assert_gemm_close(dg, want, tol, bf16=(out == torch.bfloat16)), tol
+    tight = accumulation_bound(A, B, alpha, rows, cols)
+    return assert_gemm_close(dg, want, tol, bf16=(out == torch.bfloat16), tight=tight), tol
 
 
 @pytest.mark.parametrize("fmt", FMTS, ids=[FMT_IDS[f] for f in FMTS])
@@ -89,10 +90,11 @@ def test_persistent_many_tiles(fmt):
     _run(xa, xb, fmt, rows=rows)
 
 
+@pytest.mark.parametrize("fmt", [fa.NVFP4_GLOBAL, fa.NVFP4_CTA, fa.MXFP4], ids=["nvg", "nvc", "mx"])
 @pytest.mark.parametrize("layer", list(workloads.LLAMA8B_LINEARS), ids=str)
-def test_llama8b_forward_shapes_sampled(layer):
-    """The 8B-shaped forward GEMMs at full size (M = 8192 tokens), NVFP4-global:
-    sampled 64 rows and 64 columns of D against the oracle."""
+def test_llama8b_forward_shapes_sampled(layer, fmt):
+    """The 8B-shaped forward GEMMs at full size (M = 8192 tokens) in each scale
+    domain: sampled 64 rows and 64 columns of D against the oracle."""
     need_gpu()
     cin, cout = workloads.LLAMA8B_LINEARS[layer]
     x = workloads.act(workloads.LLAMA8B_TOKENS, cin, seed=1)
@@ -100,11 +102,13 @@ def test_llama8b_forward_shapes_sampled(layer):
     rng = np.random.default_rng(5)
     rows = np.sort(rng.choice(x.shape[0], 64, replace=False))
     cols = np.sort(rng.choice(cout, 64, replace=False))
-    A = O.quantize(x, fa.NVFP4_GLOBAL)
-    B = O.quantize(w, fa.NVFP4_GLOBAL)
+    A = O.quantize(x, fmt)
+    B = O.quantize(w, fmt)
     d = fa.gemm(to_gpu_qt(A), to_gpu_qt(B), 1.0, out_dtype=torch.float32)
     torch.cuda.synchronize()
     dg = d.cpu().numpy().astype(np.float64)
     tol = O.gemm_tolerance(A, B)
-    assert_gemm_close(dg[rows, :], O.gemm_sampled(A, B, 1.0, rows, None), tol)
-    assert_gemm_close(dg[:, cols], O.gemm_sampled(A, B, 1.0, None, cols), tol)
+    assert_gemm_close(dg[rows, :], O.gemm_sampled(A, B, 1.0, rows, None), tol,
+                      tight=accumulation_bound(A, B, 1.0, rows, None))
+    assert_gemm_close(dg[:, cols], O.gemm_sampled(A, B, 1.0, None, cols), tol,
+                      tight=accumulation_bound(A, B, 1.0, None, cols))

@@ -16,7 +16,7 @@ import torch
 import fp4_quantization_block_b200 as fa
 import oracle as O
 import workloads
-from gpu_util import (FMT_IDS, FMTS, assert_gemm_close, assert_qt_equal, need_gpu, to_cpu_qt,
+from gpu_util import (FMT_IDS, FMTS, accumulation_bound, assert_gemm_close, assert_qt_equal, need_gpu, to_cpu_qt,
                       to_gpu_qt)
 
 pytestmark = pytest.mark.gpu
@@ -108,7 +108,7 @@ def test_gemm(fmt, out, mnk):
     torch.cuda.synchronize()
     assert d.shape == (M, N)
     assert_gemm_close(d.float().cpu().numpy(), O.gemm(A, B, 0.5), O.gemm_tolerance(A, B, 0.5),
-                      bf16=(out == torch.bfloat16))
+                      bf16=(out == torch.bfloat16), tight=accumulation_bound(A, B, 0.5))
 
 
 def test_gemm_writes_nothing_outside_d():
