@@ -289,7 +289,14 @@ FA4_API fa4_status fa4_linear_bwd(const void *dY, fa4_qtensor Wq_col, fa4_qtenso
  * the library holds until the process exits.  A call needing more partials
  * than that returns FA4_ERR_WORKSPACE (the launch configuration never does).
  * The first call on a device looks up that array's device address (once per
- * device); make that first call before any stream capture.  Every call
+ * device ordinal, in the context current at that call); make that first
+ * call before any stream capture.  The address is kept for the process: it
+ * does not survive cudaDeviceReset, and it is only valid in the device's
+ * primary context (the CUDA runtime's), so after a reset, or under a
+ * driver-API context of the caller's own, this entry point must not be used
+ * on that device.  A timed-out wait inside the quantize kernel has no status
+ * word to report to here (it leaves the output incomplete); the kernel's
+ * only wait is on its own tile loads.  Every call
  * shares the one array per device: calls that may run at the same time on
  * the GPU (different streams, no ordering between them) race on it and must
  * be serialized by the caller.  Errors: SHAPE, ALIGN, INVALID_ARG, WORKSPACE,

@@ -54,3 +54,22 @@ def test_noalloc_matches_workspace_quantize_twice(rnd, orient):
     b = _noalloc(xs[1], rnd, orient, seed=6)
     _same(a, b)
     _same(a, fa.quantize(xs[1], fa.NVFP4_GLOBAL, rnd, orient, seed=6))
+
+
+@pytest.mark.parametrize("rnd", [fa.RNE, fa.SR], ids=["rne", "sr"])
+def test_noalloc_matches_the_oracle(rnd):
+    """The no-alloc call on its own against the CPU oracle (not only against
+    fa4_quantize): one row-wise and one column-wise tensor, bytes and the
+    FP32 decode scale exact."""
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    import numpy as np
+    import oracle as O
+    x = workloads.act(384, 640, seed=23)
+    for orient in (fa.ROWWISE, fa.COLWISE):
+        got = _noalloc(x.cuda(), rnd, orient, seed=9)
+        torch.cuda.synchronize()
+        want = O.quantize(x, O.NVFP4_GLOBAL, rnd, orient, seed=9)
+        assert np.array_equal(got.payload.cpu().numpy(), want.payload)
+        assert np.array_equal(got.scales.cpu().numpy(), want.scales)
+        assert got.ts.cpu().numpy().view(np.uint32)[0] == want.ts.view(np.uint32)[0]
