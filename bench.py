@@ -827,7 +827,7 @@ def fa4_arm(args, rank, world, device) -> dict | None:
 def profile_arm(args, device) -> dict:
     """Run one call kind on one layer only (warm-up + steps launches), for a
     profiler capture of a single kernel: --profile KIND:LAYER, KIND one of
-    gemm_fwd, gemm_dgrad, gemm_wgrad, quant_fwd_nvg, quant_dgrad_mx_sr,
+    gemm_fwd, gemm_fwd_nvc, gemm_dgrad, gemm_wgrad, quant_fwd_nvg, quant_dgrad_mx_sr,
     quant_wgrad_had, quant_fwd_dual, quant_bwd_dual."""
     import fp4_quantization_block_b200 as fa
     kind, layer = args.profile.split(":")
@@ -838,6 +838,10 @@ def profile_arm(args, device) -> dict:
     ws = fa.workspace(1 << 16, device)
     if kind == "gemm_fwd":
         a, b = fa.quantize(x, fa.NVFP4_GLOBAL, ws=ws), fa.quantize(w, fa.NVFP4_GLOBAL, ws=ws)
+        out = torch.empty(T, cout, dtype=torch.bfloat16, device=device)
+        call = lambda: fa.gemm(a, b, 1.0, out=out, ws=ws)
+    elif kind == "gemm_fwd_nvc":
+        a, b = fa.quantize(x, fa.NVFP4_CTA, ws=ws), fa.quantize(w, fa.NVFP4_CTA, ws=ws)
         out = torch.empty(T, cout, dtype=torch.bfloat16, device=device)
         call = lambda: fa.gemm(a, b, 1.0, out=out, ws=ws)
     elif kind == "gemm_dgrad":
