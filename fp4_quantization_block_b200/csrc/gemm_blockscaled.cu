@@ -453,10 +453,19 @@ __device__ __forceinline__ void sts128(uint32_t addr, uint32_t a, uint32_t b, ui
 __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
-__device__ __forceinline__ void tma_store_2d(const CUtensorMap *map, uint32_t src, int x, int y) {
+// The stores carry an L2 evict-first policy: the output streams out to DRAM
+// while the GEMM computes, instead of lingering dirty in L2 and being
+// written back during whatever memory-bound kernel runs next.
+__device__ __forceinline__ uint64_t l2_evict_first_policy() {
+  uint64_t pol;
+  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
+  return pol;
+}
+__device__ __forceinline__ void tma_store_2d(const CUtensorMap *map, uint32_t src, int x, int y,
+                                             uint64_t policy) {
   asm volatile(
-      "cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%1, %2}], [%3];" ::"l"(map),
-      "r"(x), "r"(y), "r"(src)
+      "cp.async.bulk.tensor.2d.global.shared::cta.bulk_group.L2::cache_hint [%0, {%1, %2}], [%3], %4;" ::"l"(map),
+      "r"(x), "r"(y), "r"(src), "l"(policy)
       : "memory");
 }
 __device__ __forceinline__ void bulk_commit() {
@@ -759,6 +768,7 @@ __global__ void __launch_bounds__(NUM_THREADS_ST, 1)
     constexpr int NCH = COLS / 32;
     float alpha_g = p.alpha;
     if constexpr (KIND == kNVG) alpha_g = p.alpha * p.a_ts[0] * p.b_ts[0];
+    const uint64_t store_policy = l2_evict_first_policy();
     const uint32_t acc_empty_l = leader_addr(&sm->acc_empty);
 
     // stage the scales of k-tile g into tensor-memory buffer g % NBUF_ST
@@ -851,7 +861,7 @@ __global__ void __launch_bounds__(NUM_THREADS_ST, 1)
           fence_proxy_async_smem();
           __syncwarp();
           if (lane == 0) {
-            tma_store_2d(&map_d, ebuf, x0 + 16 * ch, y0);
+            tma_store_2d(&map_d, ebuf, x0 + 16 * ch, y0, store_policy);
             bulk_commit();
           }
         }
@@ -901,7 +911,7 @@ __global__ void __launch_bounds__(NUM_THREADS_ST, 1)
             fence_proxy_async_smem();
             __syncwarp();
             if (lane == 0) {
-              tma_store_2d(&map_d, ebuf, x0 + 32 * ch, y0);
+              tma_store_2d(&map_d, ebuf, x0 + 32 * ch, y0, store_policy);
               bulk_commit();
             }
           }

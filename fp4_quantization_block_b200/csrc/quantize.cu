@@ -137,6 +137,8 @@ struct Params {
 
 struct Ctrl {
   uint64_t full[kStages];
+  uint32_t done[kStages];     // warps finished with the stage's current tile
+  uint32_t nissued[kStages];  // loads issued into the stage so far
   float red[8];
   float tab_r[128];  // NVFP4 row-wise element multipliers s_enc / decode(code)
   float tab_c[128];  // column-wise
@@ -424,22 +426,20 @@ __global__ void __launch_bounds__(kThreads, 2)
   Ctrl *cb = reinterpret_cast<Ctrl *>(smem + kStages * kTileBytes);
   const int tid = threadIdx.x;
   if (tid == 0) {
-    for (int s = 0; s < kStages; ++s)
+    for (int s = 0; s < kStages; ++s) {
       asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(smem_u32(&cb->full[s])) : "memory");
+      cb->done[s] = 0;
+      cb->nissued[s] = 0;
+    }
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   __syncthreads();
-  // thread 0: per stage, the parity of the loads issued into it so far (bit
-  // k flips with every load into stage k) and whether one is not yet
-  // consumed
-  uint32_t nload_par = 0, pending = 0;
   if (tid == 0)
-    for (int s = 0; s < kStages; ++s) {
-      const int t = (int)blockIdx.x + s * (int)gridDim.x;
+    for (int k = 0; k < kStages; ++k) {
+      const int t = (int)blockIdx.x + k * (int)gridDim.x;
       if (t < p.ntiles) {
-        issue_tile(smem, cb, &xmap, p, t, s);
-        nload_par ^= 1u << s;
-        pending |= 1u << s;
+        issue_tile(smem, cb, &xmap, p, t, k);
+        cb->nissued[k] = 1;
       }
     }
 
@@ -458,29 +458,36 @@ __global__ void __launch_bounds__(kThreads, 2)
     __syncthreads();
   }
 
+  // Warps run through the tiles without CTA barriers: a warp releases a
+  // stage when it is done with the tile, and the last warp to release it
+  // loads the tile kStages ahead into it.  (CTA-local NVFP4 needs the
+  // tile's amax from every warp, so it synchronizes the CTA per tile.)
+  constexpr bool kLocal = RF == kNVC || CF == kNVC;
+  const int lane = tid & 31;
   int it = 0;
   bool failed = false;
   for (int t = (int)blockIdx.x; t < p.ntiles; t += (int)gridDim.x, ++it) {
     const int s = it % kStages;
     const bool ok = wait_bounded(smem_u32(&cb->full[s]), (uint32_t)((it / kStages) & 1), p.timeout_ns);
-    if (__syncthreads_or(!ok)) {
+    // the decision to stop is uniform over the CTA (CTA-local) or the warp
+    // (a lane that saw the load land still stops with a lane that gave up)
+    if (kLocal ? __syncthreads_or(!ok) : !__all_sync(0xFFFFFFFFu, ok)) {
       failed = true;
-      if (tid == 0 && p.status && atomicCAS(p.status, 0u, kStatusTimeout) == 0u)
+      if (p.status && atomicCAS(p.status, 0u, kStatusTimeout) == 0u)
         atomicExch(p.status + 1, 0x600u | (uint32_t)s);
       break;
     }
-    if (tid == 0) pending &= ~(1u << s);
     const uint16_t *tile = reinterpret_cast<const uint16_t *>(smem + s * kTileBytes);
     const int tc = t % p.tiles_c, tt = t / p.tiles_c;
     float senc_r = senc_g, senc_c = senc_g;
-    if constexpr (RF == kNVC || CF == kNVC) {
+    if constexpr (kLocal) {
       // CTA-local: the tile's amax (Q's tile in either orientation holds the
       // same values), its decode scale and multiplier table
-      const int w = tid >> 5, l = tid & 31;
+      const int w = tid >> 5;
       float m = 0.0f;
 #pragma unroll
       for (int k = 0; k < 8; ++k)
-        m = fmaxf(m, absmax8(lds128(tile + (16 * k + 2 * w + (l >> 4)) * 128 + 8 * (l & 15))));
+        m = fmaxf(m, absmax8(lds128(tile + (16 * k + 2 * w + (lane >> 4)) * 128 + 8 * (lane & 15))));
       const float se = nv_encode_scale(cta_max256(m, cb->red));
       if constexpr (RF == kNVC) {
         senc_r = se;
@@ -507,24 +514,32 @@ __global__ void __launch_bounds__(kThreads, 2)
       else
         col_pass<CF, CR, HAD, false>(tile, p, tt, tc, senc_c, cb->tab_c);
     }
-    __syncthreads();  // every read of stage s is done
-    if (tid == 0) {
-      const int tn = t + kStages * (int)gridDim.x;
-      if (tn < p.ntiles) {
-        issue_tile(smem, cb, &xmap, p, tn, s);
-        nload_par ^= 1u << s;
-        pending |= 1u << s;
+    if constexpr (kLocal) __syncthreads();  // the multiplier tables are rewritten next tile
+    // release stage s; the last warp out refills it (its reads, and every
+    // other warp's, are ordered before the load by the fence and the
+    // counter's read-modify-write)
+    __syncwarp();
+    if (lane == 0) {
+      __threadfence_block();
+      if (atomicAdd(&cb->done[s], 1u) == kThreads / 32 - 1) {
+        atomicExch(&cb->done[s], 0u);
+        const int tn = t + kStages * (int)gridDim.x;
+        if (tn < p.ntiles) {
+          issue_tile(smem, cb, &xmap, p, tn, s);
+          atomicAdd(&cb->nissued[s], 1u);
+        }
       }
     }
   }
-  if (failed && tid == 0) {
+  if (failed && lane == 0) {
     // loads still in flight write this CTA's shared memory: let them land
-    // (the n-th load into a stage completes the phase of parity (n - 1) & 1,
-    // the complement of bit k of nload_par)
+    // before the warp leaves (the n-th load into a stage completes the
+    // phase of parity (n - 1) & 1)
     for (int k = 0; k < kStages; ++k) {
-      if (!((pending >> k) & 1u)) continue;
+      const uint32_t n = *(volatile uint32_t *)&cb->nissued[k];
+      if (n == 0) continue;
       const uint64_t t0 = globaltimer();
-      while (!mbar_try_wait(smem_u32(&cb->full[k]), ((nload_par >> k) & 1u) ^ 1u))
+      while (!mbar_try_wait(smem_u32(&cb->full[k]), (n - 1) & 1u))
         if (globaltimer() - t0 > p.timeout_ns) break;
     }
   }
