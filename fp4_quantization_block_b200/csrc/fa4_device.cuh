@@ -197,18 +197,22 @@ __device__ __forceinline__ uint32_t nv_block_scale(float amax_b, float s_enc, fl
 }
 
 // ------------------------------------------------------------- Philox ---
-// Philox4x32 with 10 rounds (Salmon, Moraes, Dror, Shaw, "Parallel random
-// numbers: as easy as 1, 2, 3", SC'11).  Each round multiplies words 0 and 2
-// by the two round constants, XORs the high halves with the other words and
-// the key; the key advances by the Weyl increments between rounds.
+// Philox4x32 (Salmon, Moraes, Dror, Shaw, "Parallel random numbers: as easy
+// as 1, 2, 3", SC'11).  Each round multiplies words 0 and 2 by the two round
+// constants, XORs the high halves with the other words and the key; the key
+// advances by the Weyl increments between rounds.  The stochastic-rounding
+// bits use kSrRounds = 7 rounds: the pages fix no generator, only unbiased
+// rounding; the generator's authors report 7 rounds already passing their
+// full statistical test batteries (10 is their default with a margin).
+constexpr int kSrRounds = 7;
 struct u32x4 {
   uint32_t x, y, z, w;
 };
 
-__device__ __forceinline__ u32x4 philox10(uint32_t c0, uint32_t c1, uint32_t c2, uint32_t c3,
-                                          uint32_t k0, uint32_t k1) {
+__device__ __forceinline__ u32x4 philox(uint32_t c0, uint32_t c1, uint32_t c2, uint32_t c3,
+                                        uint32_t k0, uint32_t k1) {
 #pragma unroll
-  for (int r = 0; r < 10; ++r) {
+  for (int r = 0; r < kSrRounds; ++r) {
     // one 32x32 -> 64-bit product per multiplier gives both halves
     const uint64_t p0 = (uint64_t)0xD2511F53u * c0;
     const uint64_t p1 = (uint64_t)0xCD9E8D57u * c2;
@@ -227,7 +231,7 @@ __device__ __forceinline__ u32x4 philox10(uint32_t c0, uint32_t c1, uint32_t c2,
 // operand whose linear index is i = 8j: counter j (64-bit, words 0-1), key =
 // the 64-bit seed.  Element 8j+e uses 16-bit half (e & 1) of word e >> 1.
 __device__ __forceinline__ u32x4 sr_block_bits(uint64_t seed, uint64_t i8) {
-  return philox10((uint32_t)i8, (uint32_t)(i8 >> 32), 0u, 0u, (uint32_t)seed,
+  return philox((uint32_t)i8, (uint32_t)(i8 >> 32), 0u, 0u, (uint32_t)seed,
                   (uint32_t)(seed >> 32));
 }
 __device__ __forceinline__ uint32_t sr_half(const u32x4 &b, int e) {

@@ -124,9 +124,9 @@ struct Params {
   // column-wise operand Q = x^T [C, T]
   uint8_t *cp, *cs;
   float *cts;
-  // Philox4x32-10 round keys of the two seeds (round 9's complemented, see
-  // sr_bits_not)
-  uint32_t rkey0[10], rkey1[10], ckey0[10], ckey1[10];
+  // Philox4x32 round keys of the two seeds (the last round's complemented,
+  // see sr_bits_not)
+  uint32_t rkey0[kSrRounds], rkey1[kSrRounds], ckey0[kSrRounds], ckey1[kSrRounds];
   // fixed-sign Hadamard: 0x80000000 where token t of a 32-block is negated
   uint32_t sgn[32];
   const float *partials;  // NVFP4-global amax partials
@@ -201,11 +201,11 @@ __device__ __forceinline__ uint32_t lds32(const void *p) {
 // The complement of sr_block_bits(seed, i8) (65535 - u in every 16-bit
 // half, the form e2m1x8_sr_not takes), with the round keys in
 // kernel parameters.
-__device__ __forceinline__ u32x4 sr_bits_not(const uint32_t (&k0)[10], const uint32_t (&k1)[10],
-                                             uint64_t i8) {
+__device__ __forceinline__ u32x4 sr_bits_not(const uint32_t (&k0)[kSrRounds],
+                                             const uint32_t (&k1)[kSrRounds], uint64_t i8) {
   uint32_t c0 = (uint32_t)i8, c1 = (uint32_t)(i8 >> 32), c2 = 0u, c3 = 0u;
 #pragma unroll
-  for (int r = 0; r < 10; ++r) {
+  for (int r = 0; r < kSrRounds; ++r) {
     const uint64_t p0 = (uint64_t)0xD2511F53u * c0;
     const uint64_t p1 = (uint64_t)0xCD9E8D57u * c2;
     const uint32_t n0 = (uint32_t)(p1 >> 32) ^ c1 ^ k0[r], n2 = (uint32_t)(p0 >> 32) ^ c3 ^ k1[r];
@@ -590,14 +590,14 @@ cudaError_t launch_tensor_amax(const uint16_t *x, int64_t rows, int64_t cols, in
 
 namespace {
 
-// Philox4x32-10 key schedule (the Weyl sequence of the two key words),
-// round 9's words complemented so that the kernel's last XOR yields the
+// Philox4x32 key schedule (the Weyl sequence of the two key words), the last
+// round's words complemented so that the kernel's last XOR yields the
 // complemented bits directly.
 void philox_round_keys(uint64_t seed, uint32_t *k0, uint32_t *k1) {
   uint32_t a = (uint32_t)seed, b = (uint32_t)(seed >> 32);
-  for (int r = 0; r < 10; ++r) {
-    k0[r] = r == 9 ? ~a : a;
-    k1[r] = r == 9 ? ~b : b;
+  for (int r = 0; r < kSrRounds; ++r) {
+    k0[r] = r == kSrRounds - 1 ? ~a : a;
+    k1[r] = r == kSrRounds - 1 ? ~b : b;
     a += 0x9E3779B9u;
     b += 0xBB67AE85u;
   }

@@ -84,7 +84,7 @@ typedef enum {
 } fa4_format;
 
 /* E2M1 rounding: round-to-nearest-even, or stochastic rounding with 16
- * Philox4x32-10 bits u per element keyed by `seed` ("Format-Aware Fusion...",
+ * Philox4x32-7 bits u per element keyed by `seed` ("Format-Aware Fusion...",
  * section "Two Key Numerical Techniques": row-gradient stochastic rounding):
  * between the neighbouring grid values lo <= |y| < hi, with
  * t = (|y| - lo) / (hi - lo) * 65536, the value rounds up iff u < floor(t). */
@@ -150,7 +150,7 @@ FA4_API fa4_status fa4_quant_sizes(int64_t rows, int64_t cols, fa4_format fmt, f
  *         E4M3 value).  amax_t is the tensor amax (GLOBAL) or the 128x128
  *         tile amax of Q (CTA).  All binary32, round-to-nearest-even.
  * Then y -> E2M1 by RNE (|y| >= 6 gives 6, the sign is kept) or SR.  SR bits
- * for element Q[r][k] come from counter (r*K + k) >> 3 of Philox4x32-10 keyed
+ * for element Q[r][k] come from counter (r*K + k) >> 3 of Philox4x32-7 keyed
  * by `seed`.  Errors: SHAPE, ALIGN, INVALID_ARG, WORKSPACE, CUDA. */
 FA4_API fa4_status fa4_quantize(const void *x, int64_t rows, int64_t cols, int64_t ld, fa4_format fmt,
                         fa4_round rnd, fa4_orient orient, uint64_t seed, fa4_qtensor out,

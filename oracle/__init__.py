@@ -14,7 +14,7 @@ blocks.
 Parity status per function (pins in ``tests/test_oracle_*.py``):
   e2m1_decode, e2m1_rne, e2m1_sr, e4m3_rne/decode, mx_exponent, nv scales,
   hadamard32, sf_offset, quantize, gemm: pinned.
-  sr_bits (Philox4x32-10 stream): pinned by structure (one-round closed form,
+  sr_bits (Philox4x32-7 stream, sr_rounds()): pinned by structure (one-round closed form,
   key-schedule and counter properties) and statistics only; the published
   known-answer vectors are not available, so the exact bit stream is
   "parity unpinned".
@@ -82,6 +82,7 @@ def _setup(lib: ctypes.CDLL) -> ctypes.CDLL:
         "orc_nv_block_scale": (ci, [f32, f32, P]),
         "orc_philox4x32": (None, [P, P, ci, P]),
         "orc_sr_bits": (u32, [u64, u64]),
+        "orc_sr_rounds": (ci, []),
         "orc_sf_offset": (i64, [i64, i64, i64]),
         "orc_sf_bytes": (i64, [i64, i64]),
         "orc_hadamard32": (None, [P, u32, P]),
@@ -167,6 +168,11 @@ def philox4x32(ctr, key, rounds: int = 10) -> np.ndarray:
     out = np.empty(4, dtype=np.uint32)
     load().orc_philox4x32(_ptr(c), _ptr(k), int(rounds), _ptr(out))
     return out
+
+
+def sr_rounds() -> int:
+    """Rounds of the Philox block behind the stochastic-rounding bits."""
+    return int(load().orc_sr_rounds())
 
 
 def sr_bits(seed: int, idx) -> np.ndarray:

@@ -297,15 +297,24 @@ void orc_philox4x32(const uint32_t ctr_in[4], const uint32_t key_in[2], int roun
   out[0] = c0; out[1] = c1; out[2] = c2; out[3] = c3;
 }
 
+/* Rounds of the Philox block behind the stochastic-rounding bits.  The
+ * pages fix no generator, only that the rounding is unbiased; Philox4x32 is
+ * the published counter-based family, and its authors report 7 rounds
+ * already passing their full statistical test batteries (10 is their
+ * default with a safety margin).  7 rounds: the bits are uniform, so the
+ * rounding stays unbiased, at 70% of the ten-round cost. */
+#define ORC_SR_ROUNDS 7
+int orc_sr_rounds(void) { return ORC_SR_ROUNDS; }
+
 /* 16 random bits for element i (linear index in the quantized orientation):
- * one 10-round Philox block per 8 elements, counter = (i>>3) as a 64-bit
- * value in words 0-1, key = the 64-bit seed; word (i>>1)&3, low half for
- * even i and high half for odd i. */
+ * one Philox4x32 block (ORC_SR_ROUNDS rounds) per 8 elements, counter =
+ * (i>>3) as a 64-bit value in words 0-1, key = the 64-bit seed; word
+ * (i>>1)&3, low half for even i and high half for odd i. */
 uint32_t orc_sr_bits(uint64_t seed, uint64_t i) {
   uint32_t ctr[4] = {(uint32_t)(i >> 3), (uint32_t)(i >> 35), 0u, 0u};
   uint32_t key[2] = {(uint32_t)seed, (uint32_t)(seed >> 32)};
   uint32_t out[4];
-  orc_philox4x32(ctr, key, 10, out);
+  orc_philox4x32(ctr, key, ORC_SR_ROUNDS, out);
   uint32_t w = out[(i >> 1) & 3];
   return (i & 1) ? (w >> 16) : (w & 0xFFFFu);
 }

@@ -625,13 +625,15 @@ def pin_philox_structure():
     assert abs(ones - 0.5) < 0.005
     other = O.sr_bits(12346, np.arange(1 << 12, dtype=np.uint64))
     assert np.mean(other == bits[: 1 << 12]) < 0.01
-    # eight elements per Philox block: indices 8j..8j+7 use the four words
+    # eight elements per Philox block of sr_rounds() (= 7) rounds: indices
+    # 8j..8j+7 use the four words
+    assert O.sr_rounds() == 7
     b = O.sr_bits(1, np.arange(16, dtype=np.uint64))
-    w = O.philox4x32([0, 0, 0, 0], [1, 0], 10)
+    w = O.philox4x32([0, 0, 0, 0], [1, 0], O.sr_rounds())
     assert [int(v) for v in b[:8]] == [int(w[i // 2] >> (16 * (i % 2))) & 0xFFFF for i in range(8)]
     # 64-bit counter: the high word comes from index bits 35..
     hi = O.sr_bits(1, np.array([1 << 35], dtype=np.uint64))
-    w2 = O.philox4x32([0, 1, 0, 0], [1, 0], 10)
+    w2 = O.philox4x32([0, 1, 0, 0], [1, 0], O.sr_rounds())
     assert int(hi[0]) == int(w2[0]) & 0xFFFF
 
 
