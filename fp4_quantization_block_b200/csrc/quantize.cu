@@ -153,11 +153,13 @@ __device__ __forceinline__ uint64_t globaltimer() {
   asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
   return t;
 }
+// One bounded probe of a barrier phase; the suspend-time hint (1 ms) lets
+// the hardware park a waiting warp until the tile lands.
 __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   uint32_t ok;
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, 1000000;\n\t"
       "selp.u32 %0, 1, 0, p;\n\t}"
       : "=r"(ok)
       : "r"(bar), "r"(parity)
@@ -171,6 +173,8 @@ __device__ __forceinline__ bool wait_bounded(uint32_t bar, uint32_t parity, uint
     if (globaltimer() - t0 > timeout_ns) return false;
   return true;
 }
+// Every element of x is read once here: the tile loads are evict-first in
+// L2, leaving L2 to the quantized outputs (which the GEMM reads next).
 __device__ __forceinline__ void issue_tile(uint8_t *smem, Ctrl *cb, const CUtensorMap *map,
                                            const Params &p, int t, int s) {
   const uint32_t bar = smem_u32(&cb->full[s]);
@@ -178,10 +182,12 @@ __device__ __forceinline__ void issue_tile(uint8_t *smem, Ctrl *cb, const CUtens
                "r"(kTileBytes)
                : "memory");
   const int x = (t % p.tiles_c) * 128, y = (t / p.tiles_c) * 128;
+  uint64_t pol;
+  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
   asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
-      " [%0], [%1, {%2, %3}], [%4];" ::"r"(smem_u32(smem + s * kTileBytes)),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar)
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes.L2::cache_hint"
+      " [%0], [%1, {%2, %3}], [%4], %5;" ::"r"(smem_u32(smem + s * kTileBytes)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar), "l"(pol)
       : "memory");
 }
 
