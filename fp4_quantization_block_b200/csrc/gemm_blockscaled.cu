@@ -16,11 +16,11 @@
 // (cta_group::2) tiles, output through shared memory and bulk-tensor
 // stores, optionally the output's MXFP4 operand from the epilogue.
 // NVFP4-CTA-local: the second-level scale differs per 128-wide K chunk, so
-// each chunk accumulates into one of three tensor-memory partials (the MMAs
-// may run two chunks ahead) that the epilogue warps fold,
+// each chunk accumulates into one of two tensor-memory partials (the MMAs
+// may run one chunk ahead) that the epilogue warps fold,
 // tsA[m/128][kc] * tsB[n/128][kc] * partial, into FP32 registers as soon as
-// the chunk's MMAs complete; 128-wide tiles, as 2-SM pairs (256 x 128) when
-// M allows.
+// the chunk's MMAs complete; 128-wide 1-SM tiles (a 2-SM 256 x 128 pair
+// form is kept in the template but not dispatched: measured slower).
 //
 // Ragged shapes (M, N any; K a multiple of 32): the grid covers whole tiles;
 // TMA reads zeros for payload outside A and B, scale atoms that the operands
@@ -71,20 +71,31 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t byt
 __device__ __forceinline__ void mbar_arrive(uint32_t bar) {
   asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
 }
-// One bounded probe of a barrier phase.  The suspend-time hint (1 ms) lets
-// the hardware park the waiting warp until the phase completes instead of
-// returning at once, so waiting warps take no issue slots from the working
-// ones (measured: MXFP4 GEMM 4-5% faster on the 8B shapes); callers still
-// loop on it against their own time limit.
+// One bounded probe of a barrier phase.  With HINT, a suspend-time hint
+// (1 ms) lets the hardware park the waiting warp until the phase completes
+// instead of returning at once, so waiting warps take no issue slots from
+// the working ones: measured 4-5% faster for the MXFP4 / NVFP4-global GEMM,
+// 6% slower for the CTA-local one, whose fold warps wait on a short chunk
+// hand-off.  Callers still loop on it against their own time limit.
+template <bool HINT = true>
 __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   uint32_t ok;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, 1000000;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}"
-      : "=r"(ok)
-      : "r"(bar), "r"(parity)
-      : "memory");
+  if constexpr (HINT)
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, 1000000;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity)
+        : "memory");
+  else
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity)
+        : "memory");
   return ok != 0;
 }
 __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap *map, int x, int y,
@@ -367,12 +378,13 @@ struct CfgSt {
   static constexpr int COLS_A = C::ATOMS_K * 4;
   static constexpr int COLS_B = C::ATOMS_K * (BN / 32);
   static constexpr int COLS_BUF = COLS_A + COLS_B;
-  // CTA-local NVFP4 keeps three 128-column chunk partials (the MMA may run
-  // two chunks ahead of the fold) and four scale buffers after them; the
-  // other formats one accumulator and five scale buffers
-  static constexpr int NPART = 3;
+  // CTA-local NVFP4 keeps two 128-column chunk partials (the MMA may run one
+  // chunk ahead of the fold) and five scale buffers after them, like the
+  // other formats' one accumulator and five scale buffers (a third partial,
+  // at the cost of a scale buffer, measured 6-10% slower)
+  static constexpr int NPART = 2;
   static constexpr int SF_COL0 = KIND == kNVC ? NPART * 128 : SF_BASE;
-  static constexpr int NBUF_ST = KIND == kNVC ? 4 : NBUF;
+  static constexpr int NBUF_ST = NBUF;
   // warps arriving per k-tile on a scale buffer (one per lane quadrant, in
   // each CTA of a pair) and per tile on the accumulator (two per quadrant)
   static constexpr int SF_ARRIVALS = PAIR ? 8 : 4;
@@ -402,12 +414,13 @@ constexpr int total_smem_st() {
   return CfgSt<KIND, BN, PAIR>::OFF_CTRL + (int)sizeof(SmemSt) + 1024;
 }
 
+template <bool HINT>
 __device__ __forceinline__ bool wait_st(uint32_t bar, uint32_t parity, SmemSt *sm, const Params &p,
                                         uint32_t where) {
-  if (mbar_try_wait(bar, parity)) return true;
+  if (mbar_try_wait<HINT>(bar, parity)) return true;
   const uint64_t t0 = globaltimer();
   while (true) {
-    if (mbar_try_wait(bar, parity)) return true;
+    if (mbar_try_wait<HINT>(bar, parity)) return true;
     if (*(volatile int *)&sm->abort) return false;
     if (globaltimer() - t0 > p.timeout_ns) {
       *(volatile int *)&sm->abort = 1;
@@ -416,10 +429,11 @@ __device__ __forceinline__ bool wait_st(uint32_t bar, uint32_t parity, SmemSt *s
     }
   }
 }
+template <bool HINT>
 __device__ __forceinline__ bool warp_wait_st(uint32_t bar, uint32_t parity, SmemSt *sm,
                                              const Params &p, uint32_t where) {
   int ok = 0;
-  if ((threadIdx.x & 31) == 0) ok = wait_st(bar, parity, sm, p, where) ? 1 : 0;
+  if ((threadIdx.x & 31) == 0) ok = wait_st<HINT>(bar, parity, sm, p, where) ? 1 : 0;
   return __shfl_sync(0xFFFFFFFFu, ok, 0) != 0;
 }
 // wait until the last copy issued into each stage of a ring has landed
@@ -500,6 +514,7 @@ __global__ void __launch_bounds__(NUM_THREADS_ST, 1)
                    const __grid_constant__ CUtensorMap map_b,
                    const __grid_constant__ CUtensorMap map_d, const Params p) {
   using CS = CfgSt<KIND, BN, PAIR>;
+  constexpr bool kHint = KIND != kNVC;  // see mbar_try_wait
   using C = Cfg<KIND>;
   constexpr int ABS = CS::AB_STAGES, SFS = CS::SF_STAGES;
   extern __shared__ uint8_t smem_raw[];
@@ -582,7 +597,7 @@ __global__ void __launch_bounds__(NUM_THREADS_ST, 1)
         for (int kt = 0; kt < KT; ++kt, ++g) {
           const int s = g % ABS;
           const uint32_t ph = (uint32_t)((g / ABS) & 1);
-          if (!wait_st(smem_u32(&sm->ab_empty[s]), ph ^ 1u, sm, p, 0x100u | s)) {
+          if (!wait_st<kHint>(smem_u32(&sm->ab_empty[s]), ph ^ 1u, sm, p, 0x100u | s)) {
             ok = false;
             break;
           }
@@ -627,7 +642,7 @@ __global__ void __launch_bounds__(NUM_THREADS_ST, 1)
         for (int kt = 0; kt < KT; ++kt, ++g) {
           const int s = g % SFS;
           const uint32_t ph = (uint32_t)((g / SFS) & 1);
-          if (!wait_st(smem_u32(&sm->sfs_empty[s]), ph ^ 1u, sm, p, 0x120u | s)) {
+          if (!wait_st<kHint>(smem_u32(&sm->sfs_empty[s]), ph ^ 1u, sm, p, 0x120u | s)) {
             ok = false;
             break;
           }
@@ -677,13 +692,13 @@ __global__ void __launch_bounds__(NUM_THREADS_ST, 1)
       int g = 0;
       for (int tile = unit; tile < num_tiles && ok; tile += nunits) {
         if constexpr (KIND != kNVC) {
-          if (!wait_st(smem_u32(&sm->acc_empty), acc_phase ^ 1u, sm, p, 0x200u)) break;
+          if (!wait_st<kHint>(smem_u32(&sm->acc_empty), acc_phase ^ 1u, sm, p, 0x200u)) break;
           tc_fence_after();
         }
         for (int kt = 0; kt < KT; ++kt, ++g) {
           const int s = g % ABS, b = g % CS::NBUF_ST;
-          if (!wait_st(smem_u32(&sm->sft_full[b]), (uint32_t)((g / CS::NBUF_ST) & 1), sm, p, 0x230u | b) ||
-              !wait_st(smem_u32(&sm->ab_full[s]), (uint32_t)((g / ABS) & 1), sm, p, 0x210u | s)) {
+          if (!wait_st<kHint>(smem_u32(&sm->sft_full[b]), (uint32_t)((g / CS::NBUF_ST) & 1), sm, p, 0x230u | b) ||
+              !wait_st<kHint>(smem_u32(&sm->ab_full[s]), (uint32_t)((g / ABS) & 1), sm, p, 0x210u | s)) {
             ok = false;
             break;
           }
@@ -703,7 +718,7 @@ __global__ void __launch_bounds__(NUM_THREADS_ST, 1)
               // buffer's previous chunk
               const int q = 2 * g + (j >> 1), pb = q % CS::NPART;
               if ((j & 1) == 0) {
-                if (!wait_st(smem_u32(&sm->part_empty[pb]), (uint32_t)(((q / CS::NPART) & 1) ^ 1), sm,
+                if (!wait_st<kHint>(smem_u32(&sm->part_empty[pb]), (uint32_t)(((q / CS::NPART) & 1) ^ 1), sm,
                              p, 0x240u | pb)) {
                   ok = false;
                   break;
@@ -756,7 +771,7 @@ __global__ void __launch_bounds__(NUM_THREADS_ST, 1)
       else
         tc_commit(smem_u32(&sm->mma_done));
       const uint64_t t0 = globaltimer();
-      while (!mbar_try_wait(smem_u32(&sm->mma_done), 0)) {
+      while (!mbar_try_wait<kHint>(smem_u32(&sm->mma_done), 0)) {
         if (globaltimer() - t0 > p.timeout_ns) {
           if (atomicCAS(p.status, 0u, kStatusTimeout) == 0u) atomicExch(p.status + 1, 0x500u);
           break;
@@ -779,10 +794,10 @@ __global__ void __launch_bounds__(NUM_THREADS_ST, 1)
     // stage the scales of k-tile g into tensor-memory buffer g % NBUF_ST
     auto stage_scales = [&](int g) -> bool {
       const int s = g % SFS, b = g % CS::NBUF_ST;
-      if (!warp_wait_st(smem_u32(&sm->sfs_full[s]), (uint32_t)((g / SFS) & 1), sm, p, 0x320u | s))
+      if (!warp_wait_st<kHint>(smem_u32(&sm->sfs_full[s]), (uint32_t)((g / SFS) & 1), sm, p, 0x320u | s))
         return false;
       if (g >= CS::NBUF_ST &&
-          !warp_wait_st(smem_u32(&sm->sft_empty[b]), (uint32_t)(((g / CS::NBUF_ST) & 1) ^ 1), sm, p,
+          !warp_wait_st<kHint>(smem_u32(&sm->sft_empty[b]), (uint32_t)(((g / CS::NBUF_ST) & 1) ^ 1), sm, p,
                         0x330u | b))
         return false;
       tc_fence_after();
@@ -965,11 +980,12 @@ __global__ void __launch_bounds__(NUM_THREADS_ST, 1)
       for (int tile = unit; tile < num_tiles && ok; tile += nunits) {
         int mt, nt;
         tile_coords(tile, num_m, num_n, p.n_fastest, mt, nt);
-        // packed pairs of accumulator columns (2i, 2i+1): one fma.rn.f32x2
-        // folds both, the same rounding as fmaf on each
-        uint64_t acc2[COLS / 2];
+        // (a packed fma.rn.f32x2 fold, same rounding, measured 5% slower:
+        // the partial's registers from the tensor-memory load are not
+        // paired as its 64-bit operands need)
+        float acc[COLS];
 #pragma unroll
-        for (int i = 0; i < COLS / 2; ++i) acc2[i] = 0ull;
+        for (int i = 0; i < COLS; ++i) acc[i] = 0.0f;
         for (int kt = 0; kt < KT && ok; ++kt, ++g) {
           float fk[2];
 #pragma unroll
@@ -990,7 +1006,7 @@ __global__ void __launch_bounds__(NUM_THREADS_ST, 1)
 #pragma unroll
           for (int c = 0; c < 2; ++c) {
             const int q = 2 * g + c, pb = q % CS::NPART;  // chunk q's partial buffer
-            if (!warp_wait_st(smem_u32(&sm->part_full[pb]), (uint32_t)((q / CS::NPART) & 1), sm, p,
+            if (!warp_wait_st<kHint>(smem_u32(&sm->part_full[pb]), (uint32_t)((q / CS::NPART) & 1), sm, p,
                               0x340u | pb)) {
               ok = false;
               break;
@@ -1009,16 +1025,14 @@ __global__ void __launch_bounds__(NUM_THREADS_ST, 1)
               else
                 mbar_arrive(smem_u32(&sm->part_empty[pb]));
             }
-            const uint64_t f2 = f2_pack(fk[c], fk[c]);
 #pragma unroll
-            for (int i = 0; i < COLS / 2; ++i)
-              acc2[i] = f2_fma(f2, f2_pack_bits(r[2 * i], r[2 * i + 1]), acc2[i]);
+            for (int i = 0; i < COLS; ++i) acc[i] = fmaf(fk[c], __uint_as_float(r[i]), acc[i]);
           }
         }
         if (!ok) break;
         uint32_t r[COLS];
 #pragma unroll
-        for (int i = 0; i < COLS / 2; ++i) f2_unpack_bits(acc2[i], r[2 * i], r[2 * i + 1]);
+        for (int i = 0; i < COLS; ++i) r[i] = __float_as_uint(acc[i]);
         store_tile(r, mt, nt);
       }
     } else {
@@ -1039,7 +1053,7 @@ __global__ void __launch_bounds__(NUM_THREADS_ST, 1)
       if (!ok) break;
       int mt, nt;
       tile_coords(tile, num_m, num_n, p.n_fastest, mt, nt);
-      if (!warp_wait_st(smem_u32(&sm->acc_full), acc_phase, sm, p, 0x310u)) break;
+      if (!warp_wait_st<kHint>(smem_u32(&sm->acc_full), acc_phase, sm, p, 0x310u)) break;
       tc_fence_after();
       uint32_t r[COLS];
 #pragma unroll
