@@ -93,6 +93,10 @@ def _setup(lib: ctypes.CDLL) -> ctypes.CDLL:
         "orc_e2m1_sr_batch": (None, [P, P, i64, P]),
         "orc_e4m3_rne_batch": (None, [P, i64, P]),
         "orc_sr_bits_batch": (None, [u64, P, i64, P]),
+        "orc_exp_f32": (f32, [f32]),
+        "orc_silu_f32": (f32, [f32]),
+        "orc_exp_f32_batch": (None, [P, i64, P]),
+        "orc_swiglu_bf16": (None, [P, i64, i64, i64, P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -180,6 +184,29 @@ def sr_bits(seed: int, idx) -> np.ndarray:
     out = np.empty(i.size, dtype=np.uint32)
     load().orc_sr_bits_batch(int(seed), _ptr(i), i.size, _ptr(out))
     return out
+
+
+def exp_f32(x) -> np.ndarray:
+    """The oracle's binary32 exp (the SwiGLU producer's step-by-step definition)."""
+    a = np.ascontiguousarray(np.asarray(x, dtype=np.float32).ravel())
+    out = np.empty_like(a)
+    load().orc_exp_f32_batch(_ptr(a), a.size, _ptr(out))
+    return out
+
+
+def silu_f32(g: float) -> float:
+    return float(load().orc_silu_f32(float(g)))
+
+
+def swiglu_bf16(z) -> np.ndarray:
+    """h[T, F] = bf16(silu(gate) * up) as bf16 bits (uint16), from z[T, 2F]
+    (torch bf16 or uint16 bf16 bits): gate = z[:, :F], up = z[:, F:]."""
+    bits = _bf16_bits(z)
+    T, F2 = bits.shape
+    assert F2 % 2 == 0
+    h = np.empty((T, F2 // 2), dtype=np.uint16)
+    load().orc_swiglu_bf16(_ptr(bits), T, F2 // 2, F2, _ptr(h))
+    return h
 
 
 def sf_offset(r: int, kb: int, kb_total: int) -> int:

@@ -588,6 +588,74 @@ int orc_gemm(const uint8_t *pa, const uint8_t *sa, const float *tsa, const uint8
 }
 
 /* ------------------------------------------------------------------------ */
+/* SwiGLU producer of the down projection's input.  [FAF] "The Design        */
+/* Philosophy of Format-Aware Fusion" binds each quantization producer to    */
+/* its consumer; the activation h = silu(g) * u of a gated MLP is the        */
+/* producer of the down projection's input.  The pages give no numerics for  */
+/* it.  Reading: binary32 arithmetic, one rounding to bf16 at the end (the   */
+/* activation an unfused pipeline stores), silu(g) = g / (1 + exp(-g)), and  */
+/* exp written out step by step so that every implementation of the path     */
+/* computes the same bits:                                                    */
+/*   clamp x to [-87, 88] (so 2^n below stays a normal scale);              */
+/*   n = rint(x * RN(log2 e));                                                */
+/*   r = x - n ln2 in two fused steps with ln2 = LN2_HI + LN2_LO, LN2_HI     */
+/*       having 15 significant bits (Cody and Waite, "Software Manual for    */
+/*       the Elementary Functions", 1980: the additive range reduction);    */
+/*   p = the degree-6 Taylor polynomial of e^r (|r| <= ln2 / 2), Horner      */
+/*       with fused multiply-adds from 1/720 down;                            */
+/*   exp(x) = p * 2^n.                                                         */
+/* Every step is one IEEE binary32 operation (fmaf: one rounding).           */
+/* ------------------------------------------------------------------------ */
+
+float orc_exp_f32(float x) {
+  if (x < -87.0f) x = -87.0f;
+  if (x > 88.0f) x = 88.0f;
+  const float n = rintf(x * 1.44269502162933349609375f); /* RN(log2 e) */
+  float r = fmaf(-n, 0.693145751953125f, x);             /* LN2_HI */
+  r = fmaf(-n, 1.42860677e-6f, r);                       /* LN2_LO = RN(ln2 - LN2_HI) */
+  float p = 1.38888892e-3f;                              /* RN(1/720) */
+  p = fmaf(p, r, 8.33333377e-3f);                        /* RN(1/120) */
+  p = fmaf(p, r, 4.16666679e-2f);                        /* RN(1/24) */
+  p = fmaf(p, r, 1.66666672e-1f);                        /* RN(1/6) */
+  p = fmaf(p, r, 0.5f);
+  p = fmaf(p, r, 1.0f);
+  p = fmaf(p, r, 1.0f);
+  const uint32_t sbits = (uint32_t)((int)n + 127) << 23;
+  float scale;
+  memcpy(&scale, &sbits, sizeof(scale));
+  return p * scale;
+}
+
+float orc_silu_f32(float g) { return g / (1.0f + orc_exp_f32(-g)); }
+
+/* binary32 -> bf16, round to nearest even (finite values) */
+static uint16_t float_to_bf16_rne(float v) {
+  uint32_t b;
+  memcpy(&b, &v, sizeof(b));
+  b += 0x7FFFu + ((b >> 16) & 1u);
+  return (uint16_t)(b >> 16);
+}
+
+/* h[T, F] (bf16 bits) from z[T, 2F] (bf16 bits, row stride ld): gate =
+ * z[t][f], up = z[t][F + f]; h = bf16(silu(gate) * up). */
+#ifdef PLANT_SWIGLU_SWAP
+#define ORC_GATE(z, t, f) bf16_to_float(z[(t) * ld + F + (f)])
+#define ORC_UP(z, t, f) bf16_to_float(z[(t) * ld + (f)])
+#else
+#define ORC_GATE(z, t, f) bf16_to_float(z[(t) * ld + (f)])
+#define ORC_UP(z, t, f) bf16_to_float(z[(t) * ld + F + (f)])
+#endif
+void orc_swiglu_bf16(const uint16_t *z, int64_t T, int64_t F, int64_t ld, uint16_t *h) {
+  for (int64_t t = 0; t < T; ++t)
+    for (int64_t f = 0; f < F; ++f)
+      h[t * F + f] = float_to_bf16_rne(orc_silu_f32(ORC_GATE(z, t, f)) * ORC_UP(z, t, f));
+}
+
+void orc_exp_f32_batch(const float *x, int64_t n, float *y) {
+  for (int64_t i = 0; i < n; ++i) y[i] = orc_exp_f32(x[i]);
+}
+
+/* ------------------------------------------------------------------------ */
 /* Batch helpers for the tests (plain loops over the scalar rules above).    */
 /* ------------------------------------------------------------------------ */
 

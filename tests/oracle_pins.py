@@ -637,9 +637,60 @@ def pin_philox_structure():
     assert int(hi[0]) == int(w2[0]) & 0xFFFF
 
 
+# ------------------------------------------------------------ SwiGLU ---
+
+def pin_exp_f32():
+    """The producer's binary32 exp against binary64 exp: within 3 units in the
+    last place over the whole clamped range, exact at 0, monotone, and the
+    clamp ends."""
+    x = np.linspace(-87.0, 88.0, 400001).astype(np.float32)
+    e = O.exp_f32(x).astype(np.float64)
+    ref = np.exp(x.astype(np.float64))
+    rel = np.abs(e - ref) / ref
+    assert rel.max() <= 3 * 2.0 ** -23, rel.max()
+    assert float(O.exp_f32([0.0])[0]) == 1.0
+    assert np.all(np.diff(e) >= 0)
+    assert O.exp_f32([-100.0])[0] == O.exp_f32([-87.0])[0]
+    assert O.exp_f32([100.0])[0] == O.exp_f32([88.0])[0]
+
+
+def pin_swiglu():
+    """silu(g) = g / (1 + e^-g) against binary64; h = silu(gate) * up rounded
+    to bf16 against the binary64 product (the nearest bf16, or a neighbour only
+    where the exact value lies within a few binary32 units of a bf16
+    rounding boundary); gate and up taken from the two halves of z."""
+    assert O.silu_f32(0.0) == 0.0
+    for g in (20.0, 30.0, 87.5):
+        assert O.silu_f32(g) == g
+    gs = np.linspace(-80.0, 80.0, 20001).astype(np.float32)
+    got = np.array([O.silu_f32(float(g)) for g in gs])
+    g64 = gs.astype(np.float64)
+    ref = g64 / (1.0 + np.exp(-g64))
+    nz = np.abs(ref) > 1e-30
+    assert np.max(np.abs(got[nz] - ref[nz]) / np.abs(ref[nz])) <= 6 * 2.0 ** -24
+    gen = torch.Generator().manual_seed(7)
+    T, F = 64, 96
+    gate = torch.randn(T, F, generator=gen) * 3.0
+    up = torch.randn(T, F, generator=gen) * 0.25 + 0.1
+    z = torch.cat([gate, up], dim=1).to(torch.bfloat16)
+    h = O.swiglu_bf16(z).astype(np.uint32) << 16
+    hv = h.view(np.float32).astype(np.float64)
+    g64 = z[:, :F].float().double().numpy()
+    u64 = z[:, F:].float().double().numpy()
+    exact = g64 / (1.0 + np.exp(-g64)) * u64
+    want = torch.from_numpy(exact).to(torch.bfloat16).float().double().numpy()  # RNE to bf16
+    ulp_bf16 = np.exp2(np.floor(np.log2(np.maximum(np.abs(exact), 1e-38))) - 7)
+    frac = np.abs(exact) / ulp_bf16 - np.floor(np.abs(exact) / ulp_bf16)
+    near_tie = np.abs(frac - 0.5) < 2.0 ** -12  # within a few binary32 units of a midpoint
+    same = hv == want
+    assert np.all(same | (near_tie & (np.abs(hv - want) <= ulp_bf16 * 1.0001))), \
+        int((~same & ~near_tie).sum())
+    assert same.mean() > 0.999
+
+
 ALL_PINS = [pin_e2m1_decode, pin_e2m1_rne, pin_e2m1_sr, pin_e4m3, pin_mx_exponent,
             pin_mx_exponent_noclip, pin_nv_scales,
             pin_hadamard, pin_swizzle, pin_quantize_rne, pin_quantize_sr, pin_quantize_orientation,
             pin_quantize_hadamard, pin_packing, pin_quantize_ragged, pin_gemm_bruteforce,
             pin_gemm_ragged, pin_gemm_approximates_matmul,
-            pin_philox_structure]
+            pin_philox_structure, pin_exp_f32, pin_swiglu]

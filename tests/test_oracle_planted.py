@@ -23,6 +23,7 @@ PLANTS = {
     "PLANT_CTA_TILE_INDEX": [P.pin_gemm_bruteforce],
     "PLANT_GEMM_DROP_TS": [P.pin_gemm_bruteforce, P.pin_gemm_approximates_matmul],
     "PLANT_NV_NO_SENC": [P.pin_nv_scales, P.pin_quantize_rne],
+    "PLANT_SWIGLU_SWAP": [P.pin_swiglu],
 }
 
 
