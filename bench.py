@@ -410,6 +410,44 @@ def epilogue_quant_run(fa, device, reps: int = 10) -> dict:
     return res
 
 
+def swiglu_quant_run(fa, device, reps: int = 10) -> dict:
+    """The down projection's input from the gate+up output z[8192, 2 x 14336]:
+    the SwiGLU producer fused with its quantizer (row-wise CTA-local NVFP4 and
+    column-wise MXFP4 with the Hadamard, h never written) against the
+    unfused route (torch's bf16 silu(gate) * up writing h, then the dual
+    quantizer reading it).  GB/s over the fused producer's algorithmic bytes:
+    z read (4 B per element of h) + both operands written."""
+    F = LAYERS["down"][0]
+    z = workloads.act(T, 2 * F, seed=9, device=device)
+    rq = fa.empty_qtensor(T, F, fa.NVFP4_CTA, fa.ROWWISE, device)
+    cq = fa.empty_qtensor(T, F, fa.MXFP4, fa.COLWISE, device)
+    h = torch.empty(T, F, dtype=torch.bfloat16, device=device)
+    ws = fa.workspace(1 << 16, device)
+
+    def unfused():
+        torch.mul(torch.nn.functional.silu(z[:, :F]), z[:, F:], out=h)
+        fa.quantize_dual(h, fa.NVFP4_CTA, fa.RNE, 0, True, SIGN_MASK, row_out=rq, col_out=cq, ws=ws)
+
+    runs = {"fused": lambda: fa.swiglu_quantize(z, fa.NVFP4_CTA, fa.RNE, 0, col=True,
+                                                sign_mask=SIGN_MASK, row_out=rq, col_out=cq),
+            "unfused": unfused}
+    res = {"shape": [T, F], "row": "NVFP4-CTA-local RNE", "col": "MXFP4 Hadamard RNE"}
+    for name, fn in runs.items():
+        for _ in range(3):
+            fn()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(reps):
+            fn()
+        e1.record()
+        torch.cuda.synchronize()
+        res[name + "_us"] = round(e0.elapsed_time(e1) * 1000.0 / reps, 1)
+    nbytes = T * F * (4.0 + (0.5 + 1.0 / 16) + (0.5 + 1.0 / 32)) + 4.0 * (T // 128) * (F // 128)
+    res["fused_GBps"] = round(nbytes / (res["fused_us"] * 1e-6) / 1e9, 1)
+    return res
+
+
 STACK_LAYERS = 32
 STACK_BF16_LAYERS = 4          # the last four blocks keep bf16 linears
 STACK_TOKENS = 2 * T           # sequence 8192 x batch 2
@@ -761,6 +799,7 @@ def fa4_arm(args, rank, world, device) -> dict | None:
         sweep = quantize_sweep(fa, device) if solo else []
         gsweep = gemm_sweep(fa, device) if solo else []
         epiq = epilogue_quant_run(fa, device) if solo else {}
+        swq = swiglu_quant_run(fa, device) if solo else {}
         ragged = []
         if solo:
             try:
@@ -798,6 +837,7 @@ def fa4_arm(args, rank, world, device) -> dict | None:
                         "quantize_sweep": sweep,
                         "gemm_sweep": gsweep,
                         "gemm_epilogue_mxfp4": epiq,
+                        "swiglu_quantize": swq,
                         "ragged_sweep": ragged,
                         "linear_stack": stack},
             "roofline": {"bound": "tensor", "achieved": round(dom_tflops, 1),

@@ -24,6 +24,7 @@ import torch
 __all__ = [
     "MXFP4", "NVFP4_GLOBAL", "NVFP4_CTA", "MXFP4_NOCLIP", "RNE", "SR", "ROWWISE", "COLWISE",
     "QTensor", "FA4Error", "lib", "library_path", "quant_sizes", "empty_qtensor", "quantize",
+    "swiglu_quantize",
     "hadamard32_quantize", "quantize_dual", "gemm", "gemm_mxout", "linear_ws_bytes", "linear_fwd", "linear_dgrad",
     "linear_wgrad", "linear_fwd_save", "linear_bwd", "workspace", "check_device_status",
 ]
@@ -90,8 +91,10 @@ def _declare(L: ctypes.CDLL) -> ctypes.CDLL:
         "fa4_check_device_status": [P, P],
         "fa4_debug_convert": [P, P, i64, P, P, P, P],
         "fa4_debug_sr_bits": [u64, P, i64, P, P],
+        "fa4_debug_nv_block_scale": [P, f32, i64, P, P, P],
         "fa4_debug_gemm_timeout": [_QT, _QT, i64, i64, i64, ci, P, i64, ci, u64, P, sz, P],
         "fa4_quantize_nvfp4_global_noalloc": [P, i64, i64, i64, ci, ci, u64, _QT, P],
+        "fa4_swiglu_quantize": [P, i64, i64, i64, ci, ci, u64, _QT, ci, ci, u32, ci, u64, _QT, P],
     }
     for name, args in sig.items():
         fn = getattr(L, name)
@@ -310,6 +313,35 @@ def quantize_dual(x: torch.Tensor, row_fmt: int, row_rnd: int = RNE, row_seed: i
 
 
 @_on_tensor_device
+def swiglu_quantize(z: torch.Tensor, row_fmt: int, row_rnd: int = RNE, row_seed: int = 0,
+                    col: bool = False, col_hadamard: bool = True, sign_mask: int = 0,
+                    col_rnd: int = RNE, col_seed: int = 0, row_out: QTensor | None = None,
+                    col_out: QTensor | None = None) -> tuple[QTensor, QTensor | None]:
+    """The down projection's input h = bf16(silu(gate) * up), gate and up the
+    two halves of z[T, 2F], quantized row-wise (row_fmt MXFP4, MXFP4_NOCLIP
+    or NVFP4_CTA) and, with col, column-wise MXFP4 (optionally through the
+    fixed-sign Hadamard) in one kernel; h is never written."""
+    ld = _as_bf16_2d(z, "z")
+    T, F2 = z.shape
+    if F2 % 2:
+        raise ValueError("z must hold gate and up halves (an even number of columns)")
+    F = F2 // 2
+    if row_out is not None:
+        _check_qt(row_out, T, F, row_fmt, z.device, "row_out")
+    if col and col_out is not None:
+        _check_qt(col_out, F, T, MXFP4, z.device, "col_out")
+    row_out = row_out or empty_qtensor(T, F, row_fmt, ROWWISE, z.device)
+    if col:
+        col_out = col_out or empty_qtensor(T, F, MXFP4, COLWISE, z.device)
+    cq = col_out.c() if col else _QT(None, None, None)
+    _check(lib().fa4_swiglu_quantize(_ptr(z), T, F, ld, row_fmt, row_rnd, row_seed, row_out.c(),
+                                     1 if col else 0, 1 if col_hadamard else 0,
+                                     sign_mask & 0xFFFFFFFF, col_rnd, col_seed, cq,
+                                     _stream(z.device)), "fa4_swiglu_quantize")
+    return row_out, (col_out if col else None)
+
+
+@_on_tensor_device
 def gemm(A: QTensor, B: QTensor, alpha: float = 1.0, out_dtype=torch.float32,
          out: torch.Tensor | None = None, ws: torch.Tensor | None = None) -> torch.Tensor:
     """D[M, N] = alpha * A B^T on the block-scaled FP4 tensor cores."""
@@ -414,6 +446,18 @@ def debug_convert(y: torch.Tensor, u16: torch.Tensor | None = None, e4m3: bool =
     _check(lib().fa4_debug_convert(_ptr(y), _ptr(u16), n, _ptr(rne), _ptr(sr), _ptr(e4),
                                    _stream(y.device)), "fa4_debug_convert")
     return rne, sr, e4
+
+
+def debug_nv_block_scale(amax: torch.Tensor, s_enc: float):
+    """Device NVFP4 block scale of each amax (float32 CUDA tensor) under the
+    encode scale s_enc, as the quantizers compute it: (E4M3 codes uint8,
+    element multipliers float32)."""
+    n = amax.numel()
+    codes = torch.empty(n, dtype=torch.uint8, device=amax.device)
+    mults = torch.empty(n, dtype=torch.float32, device=amax.device)
+    _check(lib().fa4_debug_nv_block_scale(_ptr(amax), float(s_enc), n, _ptr(codes), _ptr(mults),
+                                          _stream(amax.device)), "fa4_debug_nv_block_scale")
+    return codes, mults
 
 
 def debug_sr_bits(seed: int, idx: torch.Tensor) -> torch.Tensor:

@@ -287,6 +287,40 @@ fa4_status fa4_quantize_dual(const void *x, int64_t rows, int64_t cols, int64_t 
                           S(stream));
 }
 
+fa4_status fa4_swiglu_quantize(const void *z, int64_t T, int64_t F, int64_t ld, fa4_format row_fmt,
+                               fa4_round row_rnd, uint64_t row_seed, fa4_qtensor row_out, int col,
+                               int col_hadamard, uint32_t sign_mask, fa4_round col_rnd,
+                               uint64_t col_seed, fa4_qtensor col_out, void *stream) {
+  if (!z || !fmt_ok(row_fmt) || (row_rnd != FA4_RNE && row_rnd != FA4_SR) ||
+      (col && col_rnd != FA4_RNE && col_rnd != FA4_SR))
+    return FA4_ERR_INVALID_ARG;
+  if (row_fmt == FA4_NVFP4_GLOBAL) return FA4_ERR_UNSUPPORTED;
+  if (T <= 0 || F <= 0 || F % 32 || (col && T % 32) || ld < 2 * F || ld % 8) return FA4_ERR_SHAPE;
+  if (!aligned16(z)) return FA4_ERR_ALIGN;
+  fa4_status s = check_qt(row_out, row_fmt);
+  if (s != FA4_OK) return s;
+  if (col && (s = check_qt(col_out, FA4_MXFP4)) != FA4_OK) return s;
+  fa4::SwigluArgs a;
+  a.z = static_cast<const uint16_t *>(z);
+  a.T = T;
+  a.F = F;
+  a.ld = ld;
+  a.row_fmt = row_fmt;
+  a.row_rnd = row_rnd;
+  a.row_payload = static_cast<uint8_t *>(row_out.payload);
+  a.row_scales = static_cast<uint8_t *>(row_out.scales);
+  a.row_ts = row_out.tensor_scale;
+  a.row_seed = row_seed;
+  a.col = col != 0;
+  a.hadamard = col_hadamard != 0;
+  a.sign_mask = sign_mask;
+  a.col_rnd = col_rnd;
+  a.col_payload = col ? static_cast<uint8_t *>(col_out.payload) : nullptr;
+  a.col_scales = col ? static_cast<uint8_t *>(col_out.scales) : nullptr;
+  a.col_seed = col_seed;
+  return cuda_status(fa4::launch_swiglu_quantize(a, S(stream)));
+}
+
 fa4_status fa4_gemm_blockscaled(fa4_qtensor A, fa4_qtensor B, int64_t M, int64_t N, int64_t K,
                                 fa4_format fmt, float alpha, void *D, int64_t ldd,
                                 fa4_out_dtype out_dtype, void *workspace, size_t workspace_bytes,
@@ -471,6 +505,12 @@ fa4_status fa4_debug_convert(const float *y, const uint32_t *u16, int64_t n, uin
   if (n < 0 || (n > 0 && (!y || !rne_codes))) return FA4_ERR_INVALID_ARG;
   if (sr_codes && !u16) return FA4_ERR_INVALID_ARG;
   return cuda_status(fa4::launch_debug_convert(y, u16, n, rne_codes, sr_codes, e4m3_codes, S(stream)));
+}
+
+fa4_status fa4_debug_nv_block_scale(const float *amax, float s_enc, int64_t n, uint8_t *codes,
+                                    float *mults, void *stream) {
+  if (n < 0 || (n > 0 && (!amax || !codes || !mults))) return FA4_ERR_INVALID_ARG;
+  return cuda_status(fa4::launch_debug_nv_block_scale(amax, s_enc, n, codes, mults, S(stream)));
 }
 
 fa4_status fa4_debug_sr_bits(uint64_t seed, const uint64_t *idx, int64_t n, uint32_t *bits,

@@ -37,11 +37,31 @@ struct QuantArgs {
   uint64_t timeout_ns = 2000000000ull;
 };
 cudaError_t launch_quantize(const QuantArgs &a, cudaStream_t st);
+// The SwiGLU producer fused with its quantizer: z[T, 2F] (gate | up, row
+// stride ld) -> h = bf16(silu(gate) * up) quantized row-wise (row_fmt MXFP4,
+// MXFP4 without clipping or CTA-local NVFP4) and, with col, column-wise MXFP4
+// (hadamard: with the fixed-sign Hadamard).
+struct SwigluArgs {
+  const uint16_t *z;
+  int64_t T, F, ld;
+  int row_fmt, row_rnd;
+  uint8_t *row_payload, *row_scales;
+  float *row_ts;
+  uint64_t row_seed;
+  bool col, hadamard;
+  uint32_t sign_mask;
+  int col_rnd;
+  uint8_t *col_payload, *col_scales;
+  uint64_t col_seed;
+};
+cudaError_t launch_swiglu_quantize(const SwigluArgs &a, cudaStream_t st);
 // Tensor map of a bf16 matrix [rows, cols] (row stride ld elements) in
 // 128 x 128 boxes, no swizzle, zero fill past the edges.
 bool make_bf16_tile_map(CUtensorMap *m, const void *base, int64_t rows, int64_t cols, int64_t ld);
 cudaError_t launch_debug_convert(const float *y, const uint32_t *u16, int64_t n, uint8_t *rne,
                                  uint8_t *sr, uint8_t *e4m3, cudaStream_t st);
+cudaError_t launch_debug_nv_block_scale(const float *amax, float s_enc, int64_t n, uint8_t *codes,
+                                        float *mults, cudaStream_t st);
 cudaError_t launch_debug_sr_bits(uint64_t seed, const uint64_t *idx, int64_t n, uint32_t *bits,
                                  cudaStream_t st);
 

@@ -551,6 +551,96 @@ __global__ void __launch_bounds__(kThreads, 2)
   }
 }
 
+// ------------------------------------------------ SwiGLU producer, fused
+// The producer of the down projection's input, fused with its quantizer:
+// z[T, 2F] (the gate+up output: gate = z[:, :F], up = z[:, F:]) ->
+// h = bf16(silu(gate) * up), quantized row-wise (MXFP4, MXFP4 without
+// clipping, or CTA-local NVFP4) and optionally column-wise MXFP4 (with the
+// fixed-sign Hadamard: the down projection's saved weight-gradient operand).
+// h never leaves the chip.  The arithmetic is fixed step by step (binary32,
+// one bf16 rounding at the end): silu(g) = g / (1 + exp(-g)) with
+//   exp(x): clamp x to [-87, 88]; n = rint(x * RN(log2 e));
+//           r = x - n * ln2 in two fused steps (ln2 = a 15-bit head + tail,
+//           the Cody-Waite additive reduction); p = degree-6 Taylor
+//           polynomial of e^r by fused multiply-adds from 1/720; p * 2^n.
+// One CTA of 256 threads per 128 x 128 tile of h: each thread loads its
+// gate and up chunks (16-byte loads, all issued before any arithmetic),
+// computes its 64 values of h into the shared-memory tile, and the row-wise
+// and column-wise passes of the quantizer run on the tile.
+__device__ __forceinline__ float exp_f32(float x) {
+  x = fminf(fmaxf(x, -87.0f), 88.0f);
+  const float n = rintf(__fmul_rn(x, 1.44269502162933349609375f));
+  float r = __fmaf_rn(-n, 0.693145751953125f, x);
+  r = __fmaf_rn(-n, 1.42860677e-6f, r);
+  float q = 1.38888892e-3f;
+  q = __fmaf_rn(q, r, 8.33333377e-3f);
+  q = __fmaf_rn(q, r, 4.16666679e-2f);
+  q = __fmaf_rn(q, r, 1.66666672e-1f);
+  q = __fmaf_rn(q, r, 0.5f);
+  q = __fmaf_rn(q, r, 1.0f);
+  q = __fmaf_rn(q, r, 1.0f);
+  return __fmul_rn(q, __int_as_float(((int)n + 127) << 23));
+}
+// bf16 bits of silu(g) * u for the bf16 values in the halves of gw, uw
+__device__ __forceinline__ uint32_t swiglu2(uint32_t gw, uint32_t uw) {
+  const float g0 = bf16lo(gw), g1 = bf16hi(gw), u0 = bf16lo(uw), u1 = bf16hi(uw);
+  const float h0 = __fmul_rn(__fdiv_rn(g0, __fadd_rn(1.0f, exp_f32(-g0))), u0);
+  const float h1 = __fmul_rn(__fdiv_rn(g1, __fadd_rn(1.0f, exp_f32(-g1))), u1);
+  const __nv_bfloat162 b = __floats2bfloat162_rn(h0, h1);
+  return *reinterpret_cast<const uint32_t *>(&b);
+}
+
+template <int RF, int RR, int CF, int CR, bool HAD>
+__global__ void __launch_bounds__(kThreads, 2)
+    swiglu_quant_kernel(const Params p, const uint16_t *__restrict__ z, int64_t ld) {
+  __shared__ __align__(16) uint16_t tile[128 * 128];
+  __shared__ float red[8];
+  __shared__ float tab[128];
+  const int tid = threadIdx.x, w = tid >> 5, l = tid & 31;
+  const int tc = (int)blockIdx.x, tt = (int)blockIdx.y;
+  const int64_t F = p.C, r0 = (int64_t)tt * 128, c0 = (int64_t)tc * 128;
+  uint4 g[8], u[8];
+#pragma unroll
+  for (int s = 0; s < 8; ++s) {
+    const int64_t r = r0 + 16 * s + 2 * w + (l >> 4), c = c0 + 8 * (l & 15);
+    if (r < p.T && c < F) {
+      g[s] = ld_stream(z + r * ld + c);
+      u[s] = ld_stream(z + r * ld + F + c);
+    } else {
+      g[s] = u[s] = make_uint4(0u, 0u, 0u, 0u);  // h = silu(0) * 0 = 0 outside
+    }
+  }
+#pragma unroll
+  for (int s = 0; s < 8; ++s) {
+    const uint4 h = make_uint4(swiglu2(g[s].x, u[s].x), swiglu2(g[s].y, u[s].y),
+                               swiglu2(g[s].z, u[s].z), swiglu2(g[s].w, u[s].w));
+    *reinterpret_cast<uint4 *>(&tile[(16 * s + 2 * w + (l >> 4)) * 128 + 8 * (l & 15)]) = h;
+  }
+  __syncthreads();
+  float senc = 1.0f;
+  if constexpr (RF == kNVC) {
+    float m = 0.0f;
+#pragma unroll
+    for (int k = 0; k < 8; ++k)
+      m = fmaxf(m, absmax8(lds128(tile + (16 * k + 2 * w + (l >> 4)) * 128 + 8 * (l & 15))));
+    senc = nv_encode_scale(cta_max256(m, red));
+    if (tid == 0) p.rts[(int64_t)tt * p.tiles_c + tc] = nv_decode_scale(senc);
+    build_tab(tab, senc);
+    __syncthreads();
+  }
+  const bool edge = (r0 + 128 > p.T) || (c0 + 128 > F);
+  if (edge)
+    row_pass<RF, RR, true>(tile, p, tt, tc, senc, tab);
+  else
+    row_pass<RF, RR, false>(tile, p, tt, tc, senc, tab);
+  if constexpr (CF != kNone) {
+    if (edge)
+      col_pass<CF, CR, HAD, true>(tile, p, tt, tc, 1.0f, nullptr);
+    else
+      col_pass<CF, CR, HAD, false>(tile, p, tt, tc, 1.0f, nullptr);
+  }
+}
+
 }  // namespace qk
 
 // --------------------------------------------------------------------------
@@ -568,6 +658,20 @@ __global__ void debug_convert_kernel(const float *y, const uint32_t *u16, int64_
     const float sb = fminf(fmaxf(v, 0.001953125f), 448.0f);
     e4m3[i] = (uint8_t)e4m3_rne(sb);
   }
+}
+
+// The NVFP4 block-scale step exactly as the quantizers run it (qk::nv_code
+// and the multiplier table).
+__global__ void debug_nv_block_scale_kernel(const float *amax, float s_enc, int64_t n, uint8_t *codes,
+                                            float *mults) {
+  __shared__ float tab[128];
+  qk::build_tab(tab, s_enc);
+  __syncthreads();
+  const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= n) return;
+  const uint32_t code = qk::nv_code(amax[i], s_enc);
+  codes[i] = (uint8_t)code;
+  mults[i] = tab[code];
 }
 
 __global__ void debug_sr_bits_kernel(uint64_t seed, const uint64_t *idx, int64_t n, uint32_t *bits) {
@@ -680,10 +784,61 @@ cudaError_t launch_quantize(const QuantArgs &a, cudaStream_t st) {
                    : dispatch_row<kMX, kRNE, false>(rf, rr, map, p, st);
 }
 
+namespace {
+template <int RF, int RR, int CF, int CR, bool H>
+cudaError_t launch_sw(const qk::Params &p, const uint16_t *z, int64_t ld, cudaStream_t st) {
+  qk::swiglu_quant_kernel<RF, RR, CF, CR, H>
+      <<<dim3((unsigned)p.tiles_c, (unsigned)p.tiles_t), qk::kThreads, 0, st>>>(p, z, ld);
+  return cudaGetLastError();
+}
+template <int CF, int CR, bool H>
+cudaError_t dispatch_sw(int rf, int rr, const qk::Params &p, const uint16_t *z, int64_t ld,
+                        cudaStream_t st) {
+#define FA4_SW_ROW(F)                                                              \
+  if (rf == F) return rr == kSR ? launch_sw<F, kSR, CF, CR, H>(p, z, ld, st)      \
+                                : launch_sw<F, kRNE, CF, CR, H>(p, z, ld, st);
+  FA4_SW_ROW(kMX) FA4_SW_ROW(kMXN) FA4_SW_ROW(kNVC)
+#undef FA4_SW_ROW
+  return cudaErrorInvalidValue;
+}
+}  // namespace
+
+cudaError_t launch_swiglu_quantize(const SwigluArgs &a, cudaStream_t st) {
+  qk::Params p = {};
+  p.T = a.T;
+  p.C = a.F;
+  p.tiles_c = (int)((a.F + 127) / 128);
+  p.tiles_t = (int)((a.T + 127) / 128);
+  p.ntiles = p.tiles_c * p.tiles_t;
+  p.rp = a.row_payload;
+  p.rs = a.row_scales;
+  p.rts = a.row_ts;
+  p.cp = a.col_payload;
+  p.cs = a.col_scales;
+  philox_round_keys(a.row_seed, p.rkey0, p.rkey1);
+  philox_round_keys(a.col_seed, p.ckey0, p.ckey1);
+  for (int t = 0; t < 32; ++t) p.sgn[t] = ((a.sign_mask >> t) & 1u) ? 0x80000000u : 0u;
+  const int rf = a.row_fmt, rr = a.row_rnd, cr = a.col_rnd;
+  using qk::kNone;
+  if (!a.col) return dispatch_sw<kNone, kRNE, false>(rf, rr, p, a.z, a.ld, st);
+  if (a.hadamard)
+    return cr == kSR ? dispatch_sw<kMX, kSR, true>(rf, rr, p, a.z, a.ld, st)
+                     : dispatch_sw<kMX, kRNE, true>(rf, rr, p, a.z, a.ld, st);
+  return cr == kSR ? dispatch_sw<kMX, kSR, false>(rf, rr, p, a.z, a.ld, st)
+                   : dispatch_sw<kMX, kRNE, false>(rf, rr, p, a.z, a.ld, st);
+}
+
 cudaError_t launch_debug_convert(const float *y, const uint32_t *u16, int64_t n, uint8_t *rne,
                                  uint8_t *sr, uint8_t *e4m3, cudaStream_t st) {
   const unsigned blocks = (unsigned)((n + 255) / 256);
   if (n > 0) debug_convert_kernel<<<blocks, 256, 0, st>>>(y, u16, n, rne, sr, e4m3);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_debug_nv_block_scale(const float *amax, float s_enc, int64_t n, uint8_t *codes,
+                                        float *mults, cudaStream_t st) {
+  const unsigned blocks = (unsigned)((n + 255) / 256);
+  if (n > 0) debug_nv_block_scale_kernel<<<blocks, 256, 0, st>>>(amax, s_enc, n, codes, mults);
   return cudaGetLastError();
 }
 

@@ -188,6 +188,32 @@ FA4_API fa4_status fa4_quantize_dual(const void *x, int64_t rows, int64_t cols, 
                              fa4_round col_rnd, uint64_t col_seed, fa4_qtensor col_out,
                              void *workspace, size_t workspace_bytes, void *stream);
 
+/* The SwiGLU producer of a down projection, fused with its quantizer
+ * ("Format-Aware Fusion...", section "The Design Philosophy of Format-Aware
+ * Fusion": each quantization producer co-designed with its consumer; the
+ * gated-MLP activation is the producer of the down projection's input).
+ * z[T, 2F] is the bf16 gate+up output (row-major, leading dimension ld):
+ * gate = z[:, 0:F], up = z[:, F:2F].  h = bf16(silu(gate) * up) with
+ * silu(g) = g / (1 + exp(-g)) in binary32, rounded once to bf16, where exp is
+ * computed step by step: x clamped to [-87, 88], n = rint(x * RN(log2 e)),
+ * r = x - n ln2 by two fused multiply-adds (ln2 = 0.693145751953125 +
+ * 1.42860677e-6), p = 1 + r(1 + r(1/2 + r(1/6 + r(1/24 + r(1/120 + r/720)))))
+ * by fused multiply-adds with the binary32 coefficients, exp = p * 2^n.
+ * h is quantized row-wise into row_out (Q = h [T, F]; row_fmt FA4_MXFP4,
+ * FA4_MXFP4_NOCLIP or FA4_NVFP4_CTA, rounding row_rnd with row_seed) and,
+ * when col != 0, column-wise into col_out (Q = h^T [F, T], MXFP4, with the
+ * fixed-sign Hadamard when col_hadamard != 0, rounding col_rnd with
+ * col_seed).  Bytes equal fa4_quantize / fa4_quantize_dual applied to h; h
+ * itself is never written.  Requirements: F a multiple of 32, T >= 1 (a
+ * multiple of 32 when col), ld >= 2F and a multiple of 8, pointers 16-byte
+ * aligned.  Errors: INVALID_ARG, SHAPE, ALIGN, UNSUPPORTED (NVFP4-global:
+ * its tensor amax would need h twice), CUDA.  No workspace. */
+FA4_API fa4_status fa4_swiglu_quantize(const void *z, int64_t T, int64_t F, int64_t ld,
+                                       fa4_format row_fmt, fa4_round row_rnd, uint64_t row_seed,
+                                       fa4_qtensor row_out, int col, int col_hadamard,
+                                       uint32_t sign_mask, fa4_round col_rnd, uint64_t col_seed,
+                                       fa4_qtensor col_out, void *stream);
+
 /* Block-scaled FP4 GEMM on the tcgen05 tensor cores:
  *   D[m][n] = alpha * sum_k A[m][k] * B[n][k]       (D = alpha A B^T)
  * with A[M, K] and B[N, K] quantized operands in the same format (both
@@ -330,6 +356,18 @@ FA4_API fa4_status fa4_debug_convert(const float *y, const uint32_t *u16, int64_
                              uint8_t *sr_codes, uint8_t *e4m3_codes, void *stream);
 FA4_API fa4_status fa4_debug_sr_bits(uint64_t seed, const uint64_t *idx, int64_t n, uint32_t *bits,
                              void *stream);
+
+/* Diagnostics: the NVFP4 block-scale step of the quantizers, on n block
+ * amaxes (device pointers, non-negative and finite) under one encode scale
+ * s_enc ("FP4 Is No Longer Just a Hardware Feature...", section "NVFP4 is
+ * more than a 4-bit value": E4M3 block scale under the FP32 tensor scale;
+ * section "The third change": the clamp).  codes[i] = E4M3 code of
+ * (amax[i] / 6) * s_enc clamped to [2^-9, 448]; mults[i] = the element
+ * multiplier s_enc / decode(codes[i]) the quantizers apply.  Computed by
+ * the same device code as fa4_quantize (an exactly rounded division by 6 and
+ * a table of multipliers).  Errors: INVALID_ARG, CUDA. */
+FA4_API fa4_status fa4_debug_nv_block_scale(const float *amax, float s_enc, int64_t n, uint8_t *codes,
+                                            float *mults, void *stream);
 
 /* Diagnostics for the bounded waits: fa4_gemm_blockscaled (fp32 output,
  * alpha 1) with every wait limited to timeout_ns (0 < timeout_ns <= 2 s)

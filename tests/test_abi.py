@@ -149,6 +149,8 @@ def test_debug_entry_points_reject_bad_arguments():
     assert L.fa4_debug_convert(None, None, 10, DEV, None, None, None) == 1
     assert L.fa4_debug_convert(DEV, None, 10, DEV, DEV, None, None) == 1
     assert L.fa4_debug_sr_bits(0, None, 10, DEV, None) == 1
+    assert L.fa4_debug_nv_block_scale(None, 1.0, 10, DEV, DEV, None) == 1
+    assert L.fa4_debug_nv_block_scale(DEV, 1.0, -1, DEV, DEV, None) == 1
     assert L.fa4_debug_gemm_timeout(_qt(), _qt(), 256, 256, 512, 0, DEV, 256, 0, 0, DEV, 4096,
                                     None) == 1
     assert L.fa4_check_device_status(None, None) == 5
@@ -350,3 +352,24 @@ def test_operand_validation_rejects_mismatched_operands_and_outputs():
     # a row stride that is a multiple of 8 is a valid GEMM output
     fa._check_out(torch.zeros(64, 40, dtype=torch.bfloat16)[:, :32], (64, 32), bf, dev, "out",
                   row_stride=True)
+
+
+def test_swiglu_quantize_rejects_bad_arguments():
+    L = fa.lib()
+    q, none = _qt(), fa._QT(None, None, None)
+
+    def call(z=DEV, T=256, F=256, ld=512, fmt=fa.MXFP4, rnd=0, col=0, crnd=0, out=q, cout=none):
+        return L.fa4_swiglu_quantize(z, T, F, ld, fmt, rnd, 0, out, col, 1, 1, crnd, 0, cout, None)
+
+    assert call(z=None) == 1
+    assert call(fmt=9) == 1
+    assert call(rnd=4) == 1
+    assert call(fmt=fa.NVFP4_GLOBAL) == 4
+    assert call(F=100) == 2          # F a multiple of 32
+    assert call(T=0) == 2
+    assert call(ld=400) == 2         # ld >= 2F
+    assert call(ld=516) == 2         # ld a multiple of 8
+    assert call(col=1, T=200) == 2   # column-wise: T a multiple of 32
+    assert call(z=DEV + 8) == 3
+    assert call(out=fa._QT(0, 0x20000, 0x30000)) == 1
+    assert call(col=1, cout=fa._QT(0x10008, 0x20000, 0)) == 3

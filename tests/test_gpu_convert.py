@@ -80,3 +80,24 @@ def test_sr_bits_match_oracle():
         got = fa.debug_sr_bits(seed, torch.from_numpy(idx.view(np.int64)).cuda()).cpu().numpy()
         want = O.sr_bits(seed, idx)
         assert np.array_equal(got.view(np.uint32), want)
+
+
+def test_nv_block_scale_all_bf16_amax():
+    """The quantizers' NVFP4 block-scale step (exactly rounded amax / 6, clamp
+    to [2^-9, 448], E4M3 code, element multiplier s_enc / decode(code) from a
+    table) against the oracle's one-IEEE-operation-at-a-time rule, for every
+    non-negative finite bf16 block amax (subnormals and zero included) under
+    encode scales from tensor amaxes across the range."""
+    need_gpu()
+    bits = np.arange(0x7F80, dtype=np.uint32)  # +0 .. largest finite bf16
+    amax = (bits << 16).view(np.float32)
+    ag = torch.from_numpy(amax.copy()).cuda()
+    for amax_t in (1.0, 6.0, 2688.0, 3.5e-3, 1e-30, 3.0e38, float(amax[1])):
+        s_enc = O.nv_encode_scale(amax_t)
+        codes, mults = fa.debug_nv_block_scale(ag, s_enc)
+        codes, mults = codes.cpu().numpy(), mults.cpu().numpy()
+        want = [O.nv_block_scale(float(a), s_enc) for a in amax]
+        wc = np.array([c for c, _ in want], dtype=np.uint8)
+        wm = np.array([m for _, m in want], dtype=np.float32)
+        bad = np.nonzero((codes != wc) | (mults.view(np.uint32) != wm.view(np.uint32)))[0]
+        assert bad.size == 0, (amax_t, int(bad.size), float(amax[bad[0]]), int(codes[bad[0]]), int(wc[bad[0]]))
