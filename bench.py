@@ -47,7 +47,10 @@ BYTES_PER_ELEM = {"mx": 2.0 + 0.5 + 1.0 / 32, "nvg": 2.0 + 2.0 + 0.5 + 1.0 / 16,
                   "mxnc": 2.0 + 0.5 + 1.0 / 32,
                   # dual producers: one read, both operands written (+ the NVFP4-global amax read)
                   "nvg_dual": 2.0 + 2.0 + (0.5 + 1.0 / 16) + (0.5 + 1.0 / 32),
-                  "mx_dual": 2.0 + (0.5 + 1.0 / 32) + (0.5 + 1.0 / 32)}
+                  "mx_dual": 2.0 + (0.5 + 1.0 / 32) + (0.5 + 1.0 / 32),
+                  # SwiGLU producer, per element of h: gate + up read, NVFP4-CTA-local row
+                  # (+ its tile scale) and MXFP4 column operands written
+                  "swiglu_nvc_dual": 4.0 + (0.5 + 1.0 / 16 + 4.0 / (128 * 128)) + (0.5 + 1.0 / 32)}
 
 
 # DRAM bytes (read + write) per launch of the dominant kernel, the MXFP4
@@ -56,8 +59,8 @@ BYTES_PER_ELEM = {"mx": 2.0 + 0.5 + 1.0 / 32, "nvg": 2.0 + 2.0 + 0.5 + 1.0 / 16,
 # They hold only for the kernel source they were taken on, identified by its
 # SHA-256; after any change the traffic is reported as null until re-taken.
 GEMM_SOURCE = os.path.join(ROOT, "fp4_quantization_block_b200", "csrc", "gemm_blockscaled.cu")
-DOMINANT_TRAFFIC = {"source_sha256": "d160ded496ec1703076f78eb827b753479f388ac755672dd99b705e7ea99c5d1",
-                    "bytes_per_launch": 241203328}
+DOMINANT_TRAFFIC = {"source_sha256": "ff2bfc17e541c379b4a858b70eb94563a7581ad85d1c7ac917f30d62373e43d4",
+                    "bytes_per_launch": 239789152}
 
 
 def dominant_traffic():
@@ -220,6 +223,8 @@ def kernel_work(kind: str, cin: int, cout: int) -> tuple[float, str]:
         return BYTES_PER_ELEM["nvg_dual"] * T * cin, "byte"
     if kind == "quant_bwd_dual":
         return BYTES_PER_ELEM["mx_dual"] * T * cout, "byte"
+    if kind == "swiglu":  # z read (gate + up) + both operands of h[T, cin] written
+        return BYTES_PER_ELEM["swiglu_nvc_dual"] * T * cin, "byte"
     if kind == "quant_fwd_nvg":
         return BYTES_PER_ELEM["nvg"] * T * cin, "byte"
     if kind == "quant_dgrad_mx_sr":
@@ -443,7 +448,7 @@ def swiglu_quant_run(fa, device, reps: int = 10) -> dict:
         e1.record()
         torch.cuda.synchronize()
         res[name + "_us"] = round(e0.elapsed_time(e1) * 1000.0 / reps, 1)
-    nbytes = T * F * (4.0 + (0.5 + 1.0 / 16) + (0.5 + 1.0 / 32)) + 4.0 * (T // 128) * (F // 128)
+    nbytes = BYTES_PER_ELEM["swiglu_nvc_dual"] * T * F
     res["fused_GBps"] = round(nbytes / (res["fused_us"] * 1e-6) / 1e9, 1)
     return res
 
@@ -868,7 +873,9 @@ def profile_arm(args, device) -> dict:
     """Run one call kind on one layer only (warm-up + steps launches), for a
     profiler capture of a single kernel: --profile KIND:LAYER, KIND one of
     gemm_fwd, gemm_fwd_nvc, gemm_dgrad, gemm_wgrad, quant_fwd_nvg, quant_dgrad_mx_sr,
-    quant_wgrad_had, quant_fwd_dual, quant_bwd_dual."""
+    quant_wgrad_had, quant_fwd_dual, quant_bwd_dual, swiglu (LAYER = down: the
+    SwiGLU producer of the down projection's input, NVFP4-CTA-local row +
+    MXFP4 Hadamard column)."""
     import fp4_quantization_block_b200 as fa
     kind, layer = args.profile.split(":")
     cin, cout = LAYERS[layer]
@@ -913,6 +920,12 @@ def profile_arm(args, device) -> dict:
         qc = fa.empty_qtensor(T, cout, fa.MXFP4, fa.COLWISE, device)
         call = lambda: fa.quantize_dual(dy, fa.MXFP4, fa.SR, 1, True, SIGN_MASK,
                                         row_out=qr, col_out=qc, ws=ws)
+    elif kind == "swiglu":
+        z = workloads.act(T, 2 * cin, seed=9, device=device)
+        qr = fa.empty_qtensor(T, cin, fa.NVFP4_CTA, fa.ROWWISE, device)
+        qc = fa.empty_qtensor(T, cin, fa.MXFP4, fa.COLWISE, device)
+        call = lambda: fa.swiglu_quantize(z, fa.NVFP4_CTA, fa.RNE, 0, col=True, sign_mask=SIGN_MASK,
+                                          row_out=qr, col_out=qc)
     else:
         raise SystemExit(f"unknown kind {kind}")
     for _ in range(args.warmup):

@@ -127,3 +127,23 @@ def test_bounded_wait_times_out_in_the_two_sm_kernel():
     assert fa.check_device_status(ws) == 0
     Ao, Bo = O.quantize(a, O.NVFP4_GLOBAL), O.quantize(b, O.NVFP4_GLOBAL)
     assert np.abs(d.cpu().numpy() - O.gemm(Ao, Bo)).max() <= O.gemm_tolerance(Ao, Bo)
+
+
+def test_linear_bindings_copy_strided_inputs():
+    """The linear calls take no leading dimension, so the binding copies a
+    strided input (here a column slice of a wider tensor) to a contiguous
+    one: outputs are byte-identical to the same calls on contiguous copies."""
+    need_gpu()
+    T, Cin, Cout = 256, 384, 512
+    wide_x = workloads.act(T, Cin + 64, seed=31).cuda()
+    wide_dy = workloads.grad(T, Cout + 32, seed=32).cuda()
+    x, dy = wide_x[:, 16:16 + Cin], wide_dy[:, 8:8 + Cout]
+    assert not x.is_contiguous() and not dy.is_contiguous()
+    w = workloads.weight(Cout, Cin, seed=33)
+    wq = to_gpu_qt(O.quantize(w, O.NVFP4_GLOBAL))
+    y1, y2 = fa.linear_fwd(x, wq, fa.NVFP4_GLOBAL), fa.linear_fwd(x.contiguous(), wq, fa.NVFP4_GLOBAL)
+    dw1 = fa.linear_wgrad(dy, x, SIGN_MASK, fa.RNE, 0)
+    dw2 = fa.linear_wgrad(dy.contiguous(), x.contiguous(), SIGN_MASK, fa.RNE, 0)
+    torch.cuda.synchronize()
+    assert torch.equal(y1.view(torch.int16), y2.view(torch.int16))
+    assert torch.equal(dw1.view(torch.int32), dw2.view(torch.int32))
