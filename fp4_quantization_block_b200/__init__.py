@@ -92,6 +92,7 @@ def _declare(L: ctypes.CDLL) -> ctypes.CDLL:
         "fa4_debug_convert": [P, P, i64, P, P, P, P],
         "fa4_debug_sr_bits": [u64, P, i64, P, P],
         "fa4_debug_nv_block_scale": [P, f32, i64, P, P, P],
+        "fa4_debug_silu": [P, i64, P, P],
         "fa4_debug_gemm_timeout": [_QT, _QT, i64, i64, i64, ci, P, i64, ci, u64, P, sz, P],
         "fa4_quantize_nvfp4_global_noalloc": [P, i64, i64, i64, ci, ci, u64, _QT, P],
         "fa4_swiglu_quantize": [P, i64, i64, i64, ci, ci, u64, _QT, ci, ci, u32, ci, u64, _QT, P],
@@ -458,6 +459,16 @@ def debug_nv_block_scale(amax: torch.Tensor, s_enc: float):
     _check(lib().fa4_debug_nv_block_scale(_ptr(amax), float(s_enc), n, _ptr(codes), _ptr(mults),
                                           _stream(amax.device)), "fa4_debug_nv_block_scale")
     return codes, mults
+
+
+def debug_silu(g: torch.Tensor) -> torch.Tensor:
+    """silu(g) in binary32 exactly as the SwiGLU producer computes it, for a
+    contiguous bf16 CUDA tensor g (finite values); float32 result."""
+    if g.dtype != torch.bfloat16 or not g.is_cuda or not g.is_contiguous():
+        raise ValueError("g must be a contiguous bf16 CUDA tensor")
+    out = torch.empty(g.shape, dtype=torch.float32, device=g.device)
+    _check(lib().fa4_debug_silu(_ptr(g), g.numel(), _ptr(out), _stream(g.device)), "fa4_debug_silu")
+    return out
 
 
 def debug_sr_bits(seed: int, idx: torch.Tensor) -> torch.Tensor:

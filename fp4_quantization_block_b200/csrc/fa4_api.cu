@@ -513,6 +513,11 @@ fa4_status fa4_debug_nv_block_scale(const float *amax, float s_enc, int64_t n, u
   return cuda_status(fa4::launch_debug_nv_block_scale(amax, s_enc, n, codes, mults, S(stream)));
 }
 
+fa4_status fa4_debug_silu(const void *g, int64_t n, float *out, void *stream) {
+  if (n < 0 || (n > 0 && (!g || !out))) return FA4_ERR_INVALID_ARG;
+  return cuda_status(fa4::launch_debug_silu(static_cast<const uint16_t *>(g), n, out, S(stream)));
+}
+
 fa4_status fa4_debug_sr_bits(uint64_t seed, const uint64_t *idx, int64_t n, uint32_t *bits,
                              void *stream) {
   if (n < 0 || (n > 0 && (!idx || !bits))) return FA4_ERR_INVALID_ARG;

@@ -62,6 +62,7 @@ cudaError_t launch_debug_convert(const float *y, const uint32_t *u16, int64_t n,
                                  uint8_t *sr, uint8_t *e4m3, cudaStream_t st);
 cudaError_t launch_debug_nv_block_scale(const float *amax, float s_enc, int64_t n, uint8_t *codes,
                                         float *mults, cudaStream_t st);
+cudaError_t launch_debug_silu(const uint16_t *g, int64_t n, float *out, cudaStream_t st);
 cudaError_t launch_debug_sr_bits(uint64_t seed, const uint64_t *idx, int64_t n, uint32_t *bits,
                                  cudaStream_t st);
 

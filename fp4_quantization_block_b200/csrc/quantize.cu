@@ -81,28 +81,59 @@ __device__ __forceinline__ float cta_max256(float v, float *red) {
 
 // --------------------------------------------------------------------------
 // Tensor amax (NVFP4-global, pass 1): grid-stride over x[rows, cols] in
-// 8-element chunks; one partial maximum per CTA.
+// 8-element chunks; one partial maximum per CTA.  Each thread tracks the
+// (row, chunk) of its position and advances it by the grid stride without
+// dividing.  The loads mark a fraction keep_frac of the lines L2 evict-last: the
+// quantizing pass that follows re-reads x (with evict-first loads), and the
+// part of x kept in the 126 MB L2 is then read from L2 instead of HBM.
 // --------------------------------------------------------------------------
+__device__ __forceinline__ uint4 ld_keep(const void *p, uint64_t pol) {
+  uint4 v;
+  asm volatile("ld.global.nc.L1::no_allocate.L2::cache_hint.v4.u32 {%0,%1,%2,%3}, [%4], %5;"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "l"(p), "l"(pol));
+  return v;
+}
+
 __global__ void __launch_bounds__(256) tensor_amax_kernel(const uint16_t *__restrict__ x,
                                                           int64_t rows, int64_t cols, int64_t ld,
+                                                          float keep_frac,
                                                           float *__restrict__ partials) {
   __shared__ float red[8];
+  uint64_t pol;
+  asm volatile("createpolicy.fractional.L2::evict_last.L2::evict_unchanged.b64 %0, %1;"
+               : "=l"(pol) : "f"(keep_frac));
   const int64_t cpr = cols >> 3;  // chunks per row
   const int64_t n = rows * cpr;
-  float m = 0.0f;
-  int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
   const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+  const int64_t sr = stride / cpr, sc = stride - sr * cpr;  // the stride in rows + chunks
+  int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  int64_t r = i / cpr, c = i - r * cpr;
+  float m = 0.0f;
   for (; i + 3 * stride < n; i += 4 * stride) {
     uint4 v[4];
 #pragma unroll
     for (int u = 0; u < 4; ++u) {
-      const int64_t c = i + u * stride;
-      v[u] = ld_stream(x + (c / cpr) * ld + (c % cpr) * 8);
+      v[u] = ld_keep(x + r * ld + c * 8, pol);
+      r += sr;
+      c += sc;
+      if (c >= cpr) {
+        c -= cpr;
+        ++r;
+      }
     }
 #pragma unroll
     for (int u = 0; u < 4; ++u) m = fmaxf(m, absmax8(v[u]));
   }
-  for (; i < n; i += stride) m = fmaxf(m, absmax8(ld_stream(x + (i / cpr) * ld + (i % cpr) * 8)));
+  for (; i < n; i += stride) {
+    m = fmaxf(m, absmax8(ld_keep(x + r * ld + c * 8, pol)));
+    r += sr;
+    c += sc;
+    if (c >= cpr) {
+      c -= cpr;
+      ++r;
+    }
+  }
   m = cta_max256(m, red);
   if (threadIdx.x == 0) partials[blockIdx.x] = m;
 }
@@ -563,35 +594,77 @@ __global__ void __launch_bounds__(kThreads, 2)
 //           r = x - n * ln2 in two fused steps (ln2 = a 15-bit head + tail,
 //           the Cody-Waite additive reduction); p = degree-6 Taylor
 //           polynomial of e^r by fused multiply-adds from 1/720; p * 2^n.
+// Two values at a time on packed binary32 pairs (each lane rounds exactly as
+// the scalar step).  rint(y) for |y| < 2^22 is RN(y + 1.5 * 2^23) - 1.5 *
+// 2^23 (the sum has unit spacing and an even offset, so ties go to even as
+// rint's), and the sum's low bits are n itself, which gives 2^n as an
+// integer.  The quotient g / d (d = 1 + exp(-g) >= 1) is the correctly
+// rounded one through Markstein's correction ("Computation of elementary
+// functions on the IBM RISC System/6000 processor", IBM J. Res. Dev. 34(1),
+// 1990): a hardware reciprocal estimate y0, one Newton step y1 = y0 + y0 (1
+// - d y0), q0 = g y1, the exact remainder r = g - d q0 (one fused
+// multiply-add), q = q0 + r y1.  Both g and d are first scaled by 2^-k, k =
+// min(max(n, 0), 126), which is exact and keeps d in [0.7, 2.9] (1/d would
+// be subnormal for d >= 2^126).  Checked bit for bit against the IEEE quotient for every
+// finite bf16 gate value (fa4_debug_silu).
 // One CTA of 256 threads per 128 x 128 tile of h: each thread loads its
 // gate and up chunks (16-byte loads, all issued before any arithmetic),
 // computes its 64 values of h into the shared-memory tile, and the row-wise
 // and column-wise passes of the quantizer run on the tile.
-__device__ __forceinline__ float exp_f32(float x) {
-  x = fminf(fmaxf(x, -87.0f), 88.0f);
-  const float n = rintf(__fmul_rn(x, 1.44269502162933349609375f));
-  float r = __fmaf_rn(-n, 0.693145751953125f, x);
-  r = __fmaf_rn(-n, 1.42860677e-6f, r);
-  float q = 1.38888892e-3f;
-  q = __fmaf_rn(q, r, 8.33333377e-3f);
-  q = __fmaf_rn(q, r, 4.16666679e-2f);
-  q = __fmaf_rn(q, r, 1.66666672e-1f);
-  q = __fmaf_rn(q, r, 0.5f);
-  q = __fmaf_rn(q, r, 1.0f);
-  q = __fmaf_rn(q, r, 1.0f);
-  return __fmul_rn(q, __int_as_float(((int)n + 127) << 23));
+__device__ __forceinline__ uint64_t f2_splat(float v) { return f2_pack(v, v); }
+__device__ __forceinline__ float rcp_estimate(float d) {
+  float y;
+  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(d));
+  return y;
+}
+// silu of the two bf16 values in the halves of gw, as a packed binary32 pair
+__device__ __forceinline__ uint64_t silu2(uint32_t gw) {
+  const float g0 = bf16lo(gw), g1 = bf16hi(gw);
+  const uint64_t x = f2_pack(fminf(fmaxf(-g0, -87.0f), 88.0f), fminf(fmaxf(-g1, -87.0f), 88.0f));
+  const uint64_t shift = f2_splat(12582912.0f);  // 1.5 * 2^23
+  const uint64_t t = f2_add(f2_mul(x, f2_splat(1.44269502162933349609375f)), shift);
+  const uint64_t nn = f2_sub(shift, t);  // -n, exactly
+  uint64_t r = f2_fma(nn, f2_splat(0.693145751953125f), x);
+  r = f2_fma(nn, f2_splat(1.42860677e-6f), r);
+  uint64_t p = f2_fma(f2_splat(1.38888892e-3f), r, f2_splat(8.33333377e-3f));
+  p = f2_fma(p, r, f2_splat(4.16666679e-2f));
+  p = f2_fma(p, r, f2_splat(1.66666672e-1f));
+  p = f2_fma(p, r, f2_splat(0.5f));
+  p = f2_fma(p, r, f2_splat(1.0f));
+  p = f2_fma(p, r, f2_splat(1.0f));
+  uint32_t t0, t1;
+  f2_unpack_bits(t, t0, t1);
+  // n << 23 (two's complement) from the low bits of t; 2^n and 2^-max(n, 0)
+  const int a0 = (int)(t0 << 23), a1 = (int)(t1 << 23);
+  const uint64_t e = f2_mul(p, f2_pack_bits((uint32_t)a0 + 0x3F800000u, (uint32_t)a1 + 0x3F800000u));
+  const uint64_t d = f2_add(f2_splat(1.0f), e);
+  // 2^-k, k = max(n, 0) capped at 126 (2^-127 is not a normal number):
+  // 0x3F800000 - (n << 23) clamped to [2^-126, 1]
+  const uint32_t s0 = (uint32_t)min(max(0x3F800000 - a0, 0x00800000), 0x3F800000);
+  const uint32_t s1 = (uint32_t)min(max(0x3F800000 - a1, 0x00800000), 0x3F800000);
+  // with negated numerator and reciprocal, so that q keeps the sign of a
+  // zero g: -gs, -y0, -y1, q0 = (-gs)(-y1), -r = ds q0 - gs, q = q0 + (-r)(-y1)
+  const uint64_t ds = f2_mul(d, f2_pack_bits(s0, s1));
+  const uint64_t dn = f2_mul(d, f2_pack_bits(s0 | 0x80000000u, s1 | 0x80000000u));  // -ds
+  const uint64_t gn = f2_mul(f2_pack(g0, g1), f2_pack_bits(s0 | 0x80000000u, s1 | 0x80000000u));
+  float d0, d1;
+  f2_unpack(dn, d0, d1);
+  const uint64_t y0n = f2_pack(rcp_estimate(d0), rcp_estimate(d1));
+  const uint64_t y1n = f2_fma(y0n, f2_fma(ds, y0n, f2_splat(1.0f)), y0n);
+  const uint64_t q0 = f2_mul(gn, y1n);
+  return f2_fma(f2_fma(ds, q0, gn), y1n, q0);
 }
 // bf16 bits of silu(g) * u for the bf16 values in the halves of gw, uw
 __device__ __forceinline__ uint32_t swiglu2(uint32_t gw, uint32_t uw) {
-  const float g0 = bf16lo(gw), g1 = bf16hi(gw), u0 = bf16lo(uw), u1 = bf16hi(uw);
-  const float h0 = __fmul_rn(__fdiv_rn(g0, __fadd_rn(1.0f, exp_f32(-g0))), u0);
-  const float h1 = __fmul_rn(__fdiv_rn(g1, __fadd_rn(1.0f, exp_f32(-g1))), u1);
+  float h0, h1;
+  f2_unpack(f2_mul(silu2(gw), f2_pack(bf16lo(uw), bf16hi(uw))), h0, h1);
   const __nv_bfloat162 b = __floats2bfloat162_rn(h0, h1);
   return *reinterpret_cast<const uint32_t *>(&b);
 }
 
+constexpr int kSwigluCtasPerSm = 2;
 template <int RF, int RR, int CF, int CR, bool HAD>
-__global__ void __launch_bounds__(kThreads, 2)
+__global__ void __launch_bounds__(kThreads, kSwigluCtasPerSm)
     swiglu_quant_kernel(const Params p, const uint16_t *__restrict__ z, int64_t ld) {
   __shared__ __align__(16) uint16_t tile[128 * 128];
   __shared__ float red[8];
@@ -610,24 +683,23 @@ __global__ void __launch_bounds__(kThreads, 2)
       g[s] = u[s] = make_uint4(0u, 0u, 0u, 0u);  // h = silu(0) * 0 = 0 outside
     }
   }
+  uint32_t mb = 0u;  // largest |h| of this thread's values (bf16 bits), for the tile amax
 #pragma unroll
   for (int s = 0; s < 8; ++s) {
     const uint4 h = make_uint4(swiglu2(g[s].x, u[s].x), swiglu2(g[s].y, u[s].y),
                                swiglu2(g[s].z, u[s].z), swiglu2(g[s].w, u[s].w));
     *reinterpret_cast<uint4 *>(&tile[(16 * s + 2 * w + (l >> 4)) * 128 + 8 * (l & 15)]) = h;
+    if constexpr (RF == kNVC) mb = hmax_abs2(mb, absmax8_bf16(h));
   }
-  __syncthreads();
   float senc = 1.0f;
   if constexpr (RF == kNVC) {
-    float m = 0.0f;
-#pragma unroll
-    for (int k = 0; k < 8; ++k)
-      m = fmaxf(m, absmax8(lds128(tile + (16 * k + 2 * w + (l >> 4)) * 128 + 8 * (l & 15))));
-    senc = nv_encode_scale(cta_max256(m, red));
+    // (cta_max256 synchronizes the CTA before its exchange, which also
+    // orders the tile stores above before the passes below)
+    senc = nv_encode_scale(cta_max256(__uint_as_float((mb & 0x7FFFu) << 16), red));
     if (tid == 0) p.rts[(int64_t)tt * p.tiles_c + tc] = nv_decode_scale(senc);
     build_tab(tab, senc);
-    __syncthreads();
   }
+  __syncthreads();
   const bool edge = (r0 + 128 > p.T) || (c0 + 128 > F);
   if (edge)
     row_pass<RF, RR, true>(tile, p, tt, tc, senc, tab);
@@ -674,6 +746,18 @@ __global__ void debug_nv_block_scale_kernel(const float *amax, float s_enc, int6
   mults[i] = tab[code];
 }
 
+// silu(g) exactly as the SwiGLU producer computes it, for n bf16 values
+// (pairs; an odd tail value is paired with zero).
+__global__ void debug_silu_kernel(const uint16_t *g, int64_t n, float *out) {
+  const int64_t i = 2 * ((int64_t)blockIdx.x * blockDim.x + threadIdx.x);
+  if (i >= n) return;
+  const uint32_t gw = (uint32_t)g[i] | (i + 1 < n ? (uint32_t)g[i + 1] << 16 : 0u);
+  float s0, s1;
+  f2_unpack(qk::silu2(gw), s0, s1);
+  out[i] = s0;
+  if (i + 1 < n) out[i + 1] = s1;
+}
+
 __global__ void debug_sr_bits_kernel(uint64_t seed, const uint64_t *idx, int64_t n, uint32_t *bits) {
   const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
   if (i >= n) return;
@@ -694,7 +778,10 @@ int amax_partials_count(int64_t rows, int64_t cols) {
 
 cudaError_t launch_tensor_amax(const uint16_t *x, int64_t rows, int64_t cols, int64_t ld,
                                float *partials, int n_partials, cudaStream_t st) {
-  tensor_amax_kernel<<<n_partials, 256, 0, st>>>(x, rows, cols, ld, partials);
+  // keep at most ~80 MB of x (of the 126 MB L2) for the quantizing pass
+  const double bytes = 2.0 * (double)rows * (double)cols;
+  const float keep = bytes <= 80.0e6 ? 1.0f : (float)(80.0e6 / bytes);
+  tensor_amax_kernel<<<n_partials, 256, 0, st>>>(x, rows, cols, ld, keep, partials);
   return cudaGetLastError();
 }
 
@@ -839,6 +926,12 @@ cudaError_t launch_debug_nv_block_scale(const float *amax, float s_enc, int64_t 
                                         float *mults, cudaStream_t st) {
   const unsigned blocks = (unsigned)((n + 255) / 256);
   if (n > 0) debug_nv_block_scale_kernel<<<blocks, 256, 0, st>>>(amax, s_enc, n, codes, mults);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_debug_silu(const uint16_t *g, int64_t n, float *out, cudaStream_t st) {
+  const unsigned blocks = (unsigned)(((n + 1) / 2 + 255) / 256);
+  if (n > 0) debug_silu_kernel<<<blocks, 256, 0, st>>>(g, n, out);
   return cudaGetLastError();
 }
 

@@ -369,6 +369,16 @@ FA4_API fa4_status fa4_debug_sr_bits(uint64_t seed, const uint64_t *idx, int64_t
 FA4_API fa4_status fa4_debug_nv_block_scale(const float *amax, float s_enc, int64_t n, uint8_t *codes,
                                             float *mults, void *stream);
 
+/* Diagnostics: silu(g) = g / (1 + exp(-g)) in binary32 exactly as
+ * fa4_swiglu_quantize computes it (the exp defined step by step, the
+ * correctly rounded quotient), for n bf16 gate values g (device pointer, bf16
+ * bits, finite) into out[n] (device, binary32).  The gated-MLP activation is
+ * the producer of the down projection's input ("Format-Aware Fusion: The
+ * Engineering Practice That Doubles FP4 Pretraining Throughput", section
+ * "The Design Philosophy of Format-Aware Fusion").  Errors: INVALID_ARG,
+ * CUDA. */
+FA4_API fa4_status fa4_debug_silu(const void *g, int64_t n, float *out, void *stream);
+
 /* Diagnostics for the bounded waits: fa4_gemm_blockscaled (fp32 output,
  * alpha 1) with every wait limited to timeout_ns (0 < timeout_ns <= 2 s)
  * and, when skip_k_tile >= 0, a producer that never loads the skip_k_tile-th

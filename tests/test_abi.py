@@ -151,6 +151,8 @@ def test_debug_entry_points_reject_bad_arguments():
     assert L.fa4_debug_sr_bits(0, None, 10, DEV, None) == 1
     assert L.fa4_debug_nv_block_scale(None, 1.0, 10, DEV, DEV, None) == 1
     assert L.fa4_debug_nv_block_scale(DEV, 1.0, -1, DEV, DEV, None) == 1
+    assert L.fa4_debug_silu(None, 10, DEV, None) == 1
+    assert L.fa4_debug_silu(DEV, -1, DEV, None) == 1
     assert L.fa4_debug_gemm_timeout(_qt(), _qt(), 256, 256, 512, 0, DEV, 256, 0, 0, DEV, 4096,
                                     None) == 1
     assert L.fa4_check_device_status(None, None) == 5

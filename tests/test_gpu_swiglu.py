@@ -84,3 +84,18 @@ def test_swiglu_8b_down_input_sampled():
     c0 = 128 * int(rng.integers(F // 128))
     _check(z, fa.NVFP4_CTA, fa.RNE, (fa.RNE, True), row_range=(r0, r0 + 128),
            col_range=(c0, c0 + 128))
+
+
+def test_silu_every_finite_bf16_gate():
+    """silu in binary32 as the producer computes it (packed exp steps, the
+    quotient through a reciprocal estimate and Markstein's correction)
+    against the oracle's IEEE steps, for every finite bf16 gate value."""
+    need_gpu()
+    bits = np.arange(1 << 16, dtype=np.uint32)
+    finite = ((bits >> 7) & 0xFF) != 0xFF
+    g16 = bits[finite].astype(np.uint16)
+    g = torch.from_numpy(g16.view(np.int16).copy()).view(torch.bfloat16)
+    got = fa.debug_silu(g.cuda()).cpu().numpy()
+    want = np.array([O.silu_f32(v) for v in g.float().numpy()], dtype=np.float32)
+    bad = np.nonzero(got.view(np.uint32) != want.view(np.uint32))[0]
+    assert bad.size == 0, (int(bad.size), float(g.float()[bad[0]]), float(got[bad[0]]), float(want[bad[0]]))
