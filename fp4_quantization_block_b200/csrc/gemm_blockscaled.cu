@@ -42,6 +42,7 @@
 
 #include "fa4_device.cuh"
 #include "fa4_kernels.h"
+#include "launch.cuh"
 
 namespace fa4 {
 namespace gemm {
@@ -579,6 +580,10 @@ __global__ void __launch_bounds__(NUM_THREADS_ST, 1)
     cluster_sync();  // the peer's barriers exist before any remote arrive
   }
   tc_fence_after();
+  // the prologue above touches no global memory; the previous kernel in the
+  // stream may still be running until here
+  grid_dependency_wait();
+  grid_dependents_launch();
   const uint32_t tmem = sm->tmem_base;
   // barriers the pair's MMA waits on live in the leader (rank 0)
   auto leader_addr = [&](const void *local) -> uint32_t {
@@ -1215,13 +1220,14 @@ static cudaError_t launch_st(const GemmArgs &a, cudaStream_t st) {
   cfg.blockDim = dim3(gemm_st::NUM_THREADS_ST);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = st;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = PAIR ? 2 : 1;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
+  cudaLaunchAttribute attr[2];
+  attr[0] = pdl_attribute();
+  attr[1].id = cudaLaunchAttributeClusterDimension;
+  attr[1].val.clusterDim.x = PAIR ? 2 : 1;
+  attr[1].val.clusterDim.y = 1;
+  attr[1].val.clusterDim.z = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = PAIR ? 1 : 0;
+  cfg.numAttrs = PAIR ? 2 : 1;
   // persistent grid: no more units than can be resident at once (pairs must
   // sit in one GPC, so fewer than SMs/2 pairs may fit)
   int units = PAIR ? sms / 2 : sms;

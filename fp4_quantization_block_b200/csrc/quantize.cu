@@ -51,6 +51,7 @@
 
 #include "fa4_device.cuh"
 #include "fa4_kernels.h"
+#include "launch.cuh"
 
 namespace fa4 {
 
@@ -103,6 +104,8 @@ __global__ void __launch_bounds__(256) tensor_amax_kernel(const uint16_t *__rest
   uint64_t pol;
   asm volatile("createpolicy.fractional.L2::evict_last.L2::evict_unchanged.b64 %0, %1;"
                : "=l"(pol) : "f"(keep_frac));
+  grid_dependency_wait();
+  grid_dependents_launch();
   const int64_t cpr = cols >> 3;  // chunks per row
   const int64_t n = rows * cpr;
   const int64_t stride = (int64_t)gridDim.x * blockDim.x;
@@ -470,6 +473,8 @@ __global__ void __launch_bounds__(kThreads, 2)
     }
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
+  grid_dependency_wait();
+  grid_dependents_launch();
   __syncthreads();
   if (tid == 0)
     for (int k = 0; k < kStages; ++k) {
@@ -672,6 +677,8 @@ __global__ void __launch_bounds__(kThreads, kSwigluCtasPerSm)
   const int tid = threadIdx.x, w = tid >> 5, l = tid & 31;
   const int tc = (int)blockIdx.x, tt = (int)blockIdx.y;
   const int64_t F = p.C, r0 = (int64_t)tt * 128, c0 = (int64_t)tc * 128;
+  grid_dependency_wait();
+  grid_dependents_launch();
   uint4 g[8], u[8];
 #pragma unroll
   for (int s = 0; s < 8; ++s) {
@@ -781,8 +788,9 @@ cudaError_t launch_tensor_amax(const uint16_t *x, int64_t rows, int64_t cols, in
   // keep at most ~80 MB of x (of the 126 MB L2) for the quantizing pass
   const double bytes = 2.0 * (double)rows * (double)cols;
   const float keep = bytes <= 80.0e6 ? 1.0f : (float)(80.0e6 / bytes);
-  tensor_amax_kernel<<<n_partials, 256, 0, st>>>(x, rows, cols, ld, keep, partials);
-  return cudaGetLastError();
+  const cudaError_t e = launch_pdl(tensor_amax_kernel, dim3((unsigned)n_partials), dim3(256), 0, st, x,
+                                   rows, cols, ld, keep, partials);
+  return e != cudaSuccess ? e : cudaGetLastError();
 }
 
 namespace {
@@ -809,8 +817,8 @@ cudaError_t launch_q(const CUtensorMap &map, const qk::Params &p, cudaStream_t s
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   const int grid = p.ntiles < 2 * sms ? p.ntiles : 2 * sms;
-  kern<<<grid, qk::kThreads, qk::kSmemBytes, st>>>(map, p);
-  return cudaGetLastError();
+  e = launch_pdl(kern, dim3((unsigned)grid), dim3(qk::kThreads), qk::kSmemBytes, st, map, p);
+  return e != cudaSuccess ? e : cudaGetLastError();
 }
 
 // Dispatch on (row format, row rounding): the column-wise side fixed.
@@ -874,9 +882,10 @@ cudaError_t launch_quantize(const QuantArgs &a, cudaStream_t st) {
 namespace {
 template <int RF, int RR, int CF, int CR, bool H>
 cudaError_t launch_sw(const qk::Params &p, const uint16_t *z, int64_t ld, cudaStream_t st) {
-  qk::swiglu_quant_kernel<RF, RR, CF, CR, H>
-      <<<dim3((unsigned)p.tiles_c, (unsigned)p.tiles_t), qk::kThreads, 0, st>>>(p, z, ld);
-  return cudaGetLastError();
+  const cudaError_t e = launch_pdl(qk::swiglu_quant_kernel<RF, RR, CF, CR, H>,
+                                   dim3((unsigned)p.tiles_c, (unsigned)p.tiles_t), dim3(qk::kThreads),
+                                   0, st, p, z, ld);
+  return e != cudaSuccess ? e : cudaGetLastError();
 }
 template <int CF, int CR, bool H>
 cudaError_t dispatch_sw(int rf, int rr, const qk::Params &p, const uint16_t *z, int64_t ld,
