@@ -361,8 +361,11 @@ struct CfgSt {
   static constexpr int AB_BYTES = A_BYTES + B_BYTES;
   static constexpr int SF_BYTES = SFA_BYTES + SFB_BYTES;
   static constexpr int SF_STAGES = BN == 256 ? 5 : 8;
-  // epilogue staging: one 32-row x 64-byte output chunk per epilogue warp
-  static constexpr int EPI_WARP_BYTES = 2048;
+  // epilogue staging: EPI_BUFS buffers of one 32-row x 64-byte output chunk
+  // per epilogue warp (a warp fills one while the bulk-tensor engine reads
+  // the other)
+  static constexpr int EPI_BUFS = 2;
+  static constexpr int EPI_WARP_BYTES = 2048 * EPI_BUFS;
   static constexpr int EPI_BYTES = 8 * EPI_WARP_BYTES;
   static constexpr int SMEM_LIMIT = 232448;  // 227 KB per block (opt-in)
   static constexpr int RESERVE = 2048;       // control block + alignment slack
@@ -491,9 +494,11 @@ __device__ __forceinline__ void tma_store_2d(const CUtensorMap *map, uint32_t sr
 __device__ __forceinline__ void bulk_commit() {
   asm volatile("cp.async.bulk.commit_group;" ::: "memory");
 }
-// the shared-memory source of every committed store has been read
-__device__ __forceinline__ void bulk_wait_read_all() {
-  asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+// the shared-memory source of all but the N most recent committed stores
+// has been read
+template <int N>
+__device__ __forceinline__ void bulk_wait_read() {
+  asm volatile("cp.async.bulk.wait_group.read %0;" ::"n"(N) : "memory");
 }
 // every committed store has completed
 __device__ __forceinline__ void bulk_wait_all() {
@@ -789,6 +794,7 @@ __global__ void __launch_bounds__(NUM_THREADS_ST, 1)
     const int h = (warp - 2) >> 2;  // which of the quadrant's two warps
     const uint32_t lane_base = tmem + ((uint32_t)(32 * q) << 16);
     const uint32_t ebuf = smem_u32(smem + CS::OFF_EPI + (warp - 2) * CS::EPI_WARP_BYTES);
+    int epi_next = 0;  // the staging buffer the next output chunk goes through
     constexpr int COLS = BN / 2;
     constexpr int NCH = COLS / 32;
     float alpha_g = p.alpha;
@@ -864,7 +870,7 @@ __global__ void __launch_bounds__(NUM_THREADS_ST, 1)
       // has read it
       const int y0 = mt * CS::TILE_M + (int)rank * 128 + 32 * q;
       const int x0 = nt * BN + h * COLS;
-      const uint32_t row_base = ebuf + lane * 64;
+      const uint32_t row_off = lane * 64;
       const int sw = (lane >> 1) & 3;
       // ragged shapes: these 32 rows may lie wholly below D (the bulk-tensor
       // store clips a box that only reaches past M or N)
@@ -873,12 +879,14 @@ __global__ void __launch_bounds__(NUM_THREADS_ST, 1)
 #pragma unroll
         for (int ch = 0; ch < COLS / 16; ++ch) {
           if (p.ragged && (!rows_in || (int64_t)(x0 + 16 * ch) >= p.N)) continue;
-          if (lane == 0) bulk_wait_read_all();
+          const uint32_t buf = ebuf + 2048u * (uint32_t)epi_next;
+          epi_next = epi_next + 1 == CS::EPI_BUFS ? 0 : epi_next + 1;
+          if (lane == 0) bulk_wait_read<CS::EPI_BUFS - 1>();
           __syncwarp();
 #pragma unroll
           for (int j = 0; j < 4; ++j) {
             const uint32_t *v = &r[16 * ch + 4 * j];
-            sts128(row_base + 16 * (j ^ sw), __float_as_uint(__uint_as_float(v[0]) * alpha_g),
+            sts128(buf + row_off + 16 * (j ^ sw), __float_as_uint(__uint_as_float(v[0]) * alpha_g),
                    __float_as_uint(__uint_as_float(v[1]) * alpha_g),
                    __float_as_uint(__uint_as_float(v[2]) * alpha_g),
                    __float_as_uint(__uint_as_float(v[3]) * alpha_g));
@@ -886,7 +894,7 @@ __global__ void __launch_bounds__(NUM_THREADS_ST, 1)
           fence_proxy_async_smem();
           __syncwarp();
           if (lane == 0) {
-            tma_store_2d(&map_d, ebuf, x0 + 16 * ch, y0, store_policy);
+            tma_store_2d(&map_d, buf, x0 + 16 * ch, y0, store_policy);
             bulk_commit();
           }
         }
@@ -928,15 +936,17 @@ __global__ void __launch_bounds__(NUM_THREADS_ST, 1)
             sword |= sbyte << (8 * ch);
           }
           if (p.store_d && chunk_in) {
-            if (lane == 0) bulk_wait_read_all();
+            const uint32_t buf = ebuf + 2048u * (uint32_t)epi_next;
+            epi_next = epi_next + 1 == CS::EPI_BUFS ? 0 : epi_next + 1;
+            if (lane == 0) bulk_wait_read<CS::EPI_BUFS - 1>();
             __syncwarp();
 #pragma unroll
             for (int j = 0; j < 4; ++j)
-              sts128(row_base + 16 * (j ^ sw), w[4 * j], w[4 * j + 1], w[4 * j + 2], w[4 * j + 3]);
+              sts128(buf + row_off + 16 * (j ^ sw), w[4 * j], w[4 * j + 1], w[4 * j + 2], w[4 * j + 3]);
             fence_proxy_async_smem();
             __syncwarp();
             if (lane == 0) {
-              tma_store_2d(&map_d, ebuf, x0 + 32 * ch, y0, store_policy);
+              tma_store_2d(&map_d, buf, x0 + 32 * ch, y0, store_policy);
               bulk_commit();
             }
           }
