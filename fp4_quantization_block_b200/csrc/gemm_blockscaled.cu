@@ -514,6 +514,32 @@ __device__ __forceinline__ void tmem_st4(uint32_t taddr, const uint4 &v) {
                : "memory");
 }
 
+// N consecutive columns (N = 8, 16 or 32) of this warp's 32 lanes, one
+// word per lane and column
+__device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t *v) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"r"(taddr),
+               "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7])
+               : "memory");
+}
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t *v) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
+      "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(taddr),
+      "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]), "r"(v[8]),
+      "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15])
+      : "memory");
+}
+template <int N>
+__device__ __forceinline__ void tmem_st_cols(uint32_t taddr, const uint32_t *v) {
+  static_assert(N == 8 || N == 16 || N == 32, "column count");
+  if constexpr (N == 8) {
+    tmem_st8(taddr, v);
+  } else {
+    tmem_st16(taddr, v);
+    if constexpr (N == 32) tmem_st16(taddr + 16, v + 16);
+  }
+}
+
 template <int KIND, int BN, bool PAIR, bool QOUT>
 __global__ void __launch_bounds__(NUM_THREADS_ST, 1)
     gemm_st_kernel(const __grid_constant__ CUtensorMap map_a,
@@ -837,16 +863,26 @@ __global__ void __launch_bounds__(NUM_THREADS_ST, 1)
                  (a_in && a < na)
                      ? *reinterpret_cast<const uint32_t *>(sfa_s + a * 512 + lane * 16 + 4 * q)
                      : 0u);
-      // B: atom a of each 128-row block: row 32w + lane is word w of atom row `lane`
+      // B: atom a of each 128-row block: row 32w + lane is word w of atom row
+      // `lane`, in columns 4 (a * BN/128 + nb) + w: the k-tile's B words are
+      // COLS_B consecutive columns, written by one or two wide stores
+      constexpr int NBK = BN / 128;
+      uint32_t bw[CS::COLS_B];
 #pragma unroll
       for (int a = 0; a < C::ATOMS_K; ++a) {
 #pragma unroll
-        for (int nb = 0; nb < BN / 128; ++nb)
-          tmem_st4(col + CS::COLS_A + (BN / 32) * a + 4 * nb,
-                   (b_in[nb] && a < na)
-                       ? *reinterpret_cast<const uint4 *>(sfb_s + nb * C::SFA_BYTES + a * 512 + lane * 16)
-                       : make_uint4(0u, 0u, 0u, 0u));
+        for (int nb = 0; nb < NBK; ++nb) {
+          const uint4 v = (b_in[nb] && a < na)
+                              ? *reinterpret_cast<const uint4 *>(sfb_s + nb * C::SFA_BYTES + a * 512 + lane * 16)
+                              : make_uint4(0u, 0u, 0u, 0u);
+          uint32_t *d = &bw[4 * (a * NBK + nb)];
+          d[0] = v.x;
+          d[1] = v.y;
+          d[2] = v.z;
+          d[3] = v.w;
+        }
       }
+      tmem_st_cols<CS::COLS_B>(col + CS::COLS_A, bw);
       asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
       tc_fence_before();
       __syncwarp();
