@@ -540,7 +540,9 @@ __device__ __forceinline__ void tmem_st_cols(uint32_t taddr, const uint32_t *v) 
   }
 }
 
-template <int KIND, int BN, bool PAIR, bool QOUT>
+// RAG: some tile reaches past M, N or K (Params::ragged); aligned shapes run
+// an instantiation without the edge checks
+template <int KIND, int BN, bool PAIR, bool QOUT, bool RAG>
 __global__ void __launch_bounds__(NUM_THREADS_ST, 1)
     gemm_st_kernel(const __grid_constant__ CUtensorMap map_a,
                    const __grid_constant__ CUtensorMap map_b,
@@ -684,7 +686,7 @@ __global__ void __launch_bounds__(NUM_THREADS_ST, 1)
           }
           const uint32_t fb = smem_u32(&sm->sfs_full[s]);
           const uint32_t dst = smem_u32(smem + CS::OFF_SF + s * CS::SF_BYTES);
-          if (!p.ragged) {
+          if (!RAG) {
             mbar_arrive_expect_tx(fb, CS::SF_BYTES);
             bulk_load(dst, p.a_scales + ((int64_t)rb_a * kbt4 + (int64_t)kt * C::ATOMS_K) * 512,
                       CS::SFA_BYTES, fb);
@@ -846,7 +848,7 @@ __global__ void __launch_bounds__(NUM_THREADS_ST, 1)
       bool a_in = true, b_in[BN / 128];
 #pragma unroll
       for (int nb = 0; nb < BN / 128; ++nb) b_in[nb] = true;
-      if (p.ragged) {
+      if (RAG) {
         const int kt = g % KT;
         int mt, nt;
         tile_coords(unit + (g / KT) * nunits, num_m, num_n, p.n_fastest, mt, nt);
@@ -910,11 +912,11 @@ __global__ void __launch_bounds__(NUM_THREADS_ST, 1)
       const int sw = (lane >> 1) & 3;
       // ragged shapes: these 32 rows may lie wholly below D (the bulk-tensor
       // store clips a box that only reaches past M or N)
-      const bool rows_in = !p.ragged || (int64_t)y0 < p.M;
+      const bool rows_in = !RAG || (int64_t)y0 < p.M;
       if (p.out_fp32) {
 #pragma unroll
         for (int ch = 0; ch < COLS / 16; ++ch) {
-          if (p.ragged && (!rows_in || (int64_t)(x0 + 16 * ch) >= p.N)) continue;
+          if (RAG && (!rows_in || (int64_t)(x0 + 16 * ch) >= p.N)) continue;
           const uint32_t buf = ebuf + 2048u * (uint32_t)epi_next;
           epi_next = epi_next + 1 == CS::EPI_BUFS ? 0 : epi_next + 1;
           if (lane == 0) bulk_wait_read<CS::EPI_BUFS - 1>();
@@ -939,7 +941,7 @@ __global__ void __launch_bounds__(NUM_THREADS_ST, 1)
         uint32_t sword = 0;  // this row's MXFP4 scale bytes, one per 32-column chunk
 #pragma unroll
         for (int ch = 0; ch < COLS / 32; ++ch) {
-          const bool chunk_in = !p.ragged || (rows_in && (int64_t)(x0 + 32 * ch) < p.N);
+          const bool chunk_in = !RAG || (rows_in && (int64_t)(x0 + 32 * ch) < p.N);
           uint32_t w[16];  // the chunk's 32 bf16 values of D, packed in pairs
 #pragma unroll
           for (int u = 0; u < 16; ++u) {
@@ -966,7 +968,7 @@ __global__ void __launch_bounds__(NUM_THREADS_ST, 1)
             const uint4 codes = make_uint4(e2m1x8_rne(&f[0]), e2m1x8_rne(&f[8]),
                                            e2m1x8_rne(&f[16]), e2m1x8_rne(&f[24]));
             // rows and blocks outside D hold zero accumulators: scale byte 0
-            if (!p.ragged || (row < p.M && (int64_t)(x0 + 32 * ch) < p.N))
+            if (!RAG || (row < p.M && (int64_t)(x0 + 32 * ch) < p.N))
               *reinterpret_cast<uint4 *>(p.q_payload + row * (p.N >> 1) + ((x0 + 32 * ch) >> 1)) =
                   codes;
             sword |= sbyte << (8 * ch);
@@ -993,7 +995,7 @@ __global__ void __launch_bounds__(NUM_THREADS_ST, 1)
           // ragged: rows up to the next multiple of 128 and blocks up to the
           // next multiple of 4 are the operand's padding (written, zero)
           const int64_t nbk = p.N >> 5;
-          if (!p.ragged || (row < p.rb_a * 128 && (int64_t)(x0 >> 5) < nbk)) {
+          if (!RAG || (row < p.rb_a * 128 && (int64_t)(x0 >> 5) < nbk)) {
             uint8_t *sdst = p.q_scales + sf_offset(row, x0 >> 5, (nbk + 3) & ~int64_t(3));
             if constexpr (COLS == 128)
               *reinterpret_cast<uint32_t *>(sdst) = sword;
@@ -1255,7 +1257,8 @@ static cudaError_t launch_st(const GemmArgs &a, cudaStream_t st) {
   gemm::Params p = make_params(a);
   constexpr int TILE_M = PAIR ? 256 : gemm::BM;
   p.ragged = (a.M % TILE_M) || (a.N % BN) || (a.K % gemm::BK);
-  auto kern = gemm_st::gemm_st_kernel<KIND, BN, PAIR, QOUT>;
+  auto kern = p.ragged ? gemm_st::gemm_st_kernel<KIND, BN, PAIR, QOUT, true>
+                       : gemm_st::gemm_st_kernel<KIND, BN, PAIR, QOUT, false>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
   int dev = 0, sms = 148;
