@@ -827,6 +827,7 @@ __global__ void __launch_bounds__(NUM_THREADS_ST, 1)
     constexpr int NCH = COLS / 32;
     float alpha_g = p.alpha;
     if constexpr (KIND == kNVG) alpha_g = p.alpha * p.a_ts[0] * p.b_ts[0];
+    const uint64_t alpha2 = f2_pack(alpha_g, alpha_g);
     const uint64_t store_policy = l2_evict_first_policy();
     const uint32_t acc_empty_l = leader_addr(&sm->acc_empty);
 
@@ -924,10 +925,10 @@ __global__ void __launch_bounds__(NUM_THREADS_ST, 1)
 #pragma unroll
           for (int j = 0; j < 4; ++j) {
             const uint32_t *v = &r[16 * ch + 4 * j];
-            sts128(buf + row_off + 16 * (j ^ sw), __float_as_uint(__uint_as_float(v[0]) * alpha_g),
-                   __float_as_uint(__uint_as_float(v[1]) * alpha_g),
-                   __float_as_uint(__uint_as_float(v[2]) * alpha_g),
-                   __float_as_uint(__uint_as_float(v[3]) * alpha_g));
+            uint32_t o0, o1, o2, o3;
+            f2_unpack_bits(f2_mul(f2_pack_bits(v[0], v[1]), alpha2), o0, o1);
+            f2_unpack_bits(f2_mul(f2_pack_bits(v[2], v[3]), alpha2), o2, o3);
+            sts128(buf + row_off + 16 * (j ^ sw), o0, o1, o2, o3);
           }
           fence_proxy_async_smem();
           __syncwarp();
@@ -946,8 +947,9 @@ __global__ void __launch_bounds__(NUM_THREADS_ST, 1)
 #pragma unroll
           for (int u = 0; u < 16; ++u) {
             const int i = 32 * ch + 2 * u;
-            __nv_bfloat162 b2 = __floats2bfloat162_rn(__uint_as_float(r[i]) * alpha_g,
-                                                      __uint_as_float(r[i + 1]) * alpha_g);
+            float lo, hi;  // alpha * the pair, one packed multiply (each lane rounded)
+            f2_unpack(f2_mul(f2_pack_bits(r[i], r[i + 1]), alpha2), lo, hi);
+            __nv_bfloat162 b2 = __floats2bfloat162_rn(lo, hi);
             w[u] = *reinterpret_cast<uint32_t *>(&b2);
           }
           if constexpr (QOUT) {
