@@ -161,6 +161,8 @@ struct Params {
   // Philox4x32 round keys of the two seeds (the last round's complemented,
   // see sr_bits_not)
   uint32_t rkey0[kSrRounds], rkey1[kSrRounds], ckey0[kSrRounds], ckey1[kSrRounds];
+  // round-1 constants of each seed for counters below 2^32 (sr_bits_not32)
+  uint32_t rpre_hi, rpre_lo, cpre_hi, cpre_lo;
   // fixed-sign Hadamard: 0x80000000 where token t of a 32-block is negated
   uint32_t sgn[32];
   const float *partials;  // NVFP4-global amax partials
@@ -256,6 +258,29 @@ __device__ __forceinline__ u32x4 sr_bits_not(const uint32_t (&k0)[kSrRounds],
   }
   return {c0, ~c1, c2, ~c3};
 }
+// The same for a counter below 2^32 (its high word zero): in round 0 three
+// of the four words are zero, and round 1 multiplies the constant k0[0], so
+// pre_hi = hi(0xD2511F53 * k0[0]) ^ k1[1] and pre_lo = lo(0xD2511F53 * k0[0])
+// come from the host and the first two rounds cost one product each.
+__device__ __forceinline__ u32x4 sr_bits_not32(const uint32_t (&k0)[kSrRounds],
+                                               const uint32_t (&k1)[kSrRounds], uint32_t pre_hi,
+                                               uint32_t pre_lo, uint32_t i8) {
+  const uint64_t q0 = (uint64_t)0xD2511F53u * i8;  // round 0: c = (i8, 0, 0, 0)
+  const uint64_t q1 = (uint64_t)0xCD9E8D57u * ((uint32_t)(q0 >> 32) ^ k1[0]);  // round 1
+  uint32_t c0 = (uint32_t)(q1 >> 32) ^ k0[1], c1 = (uint32_t)q1;
+  uint32_t c2 = (uint32_t)q0 ^ pre_hi, c3 = pre_lo;
+#pragma unroll
+  for (int r = 2; r < kSrRounds; ++r) {
+    const uint64_t p0 = (uint64_t)0xD2511F53u * c0;
+    const uint64_t p1 = (uint64_t)0xCD9E8D57u * c2;
+    const uint32_t n0 = (uint32_t)(p1 >> 32) ^ c1 ^ k0[r], n2 = (uint32_t)(p0 >> 32) ^ c3 ^ k1[r];
+    c1 = (uint32_t)p1;
+    c3 = (uint32_t)p0;
+    c0 = n0;
+    c2 = n2;
+  }
+  return {c0, ~c1, c2, ~c3};
+}
 
 // MX scale byte from the bf16 bits of a block amax (either half of m): the
 // binary32 exponent field of a bf16 value is its own exponent field, so
@@ -297,7 +322,8 @@ __device__ __forceinline__ void unpack_scale8(const uint4 &w, float mult, float 
 
 // ---------------------------------------------------------- row-wise pass
 // Q = x: rows t0.., K range c0..; R = T, K = C.
-template <int FMT, int RND, bool EDGE>
+// C32: every linear index of the operand is below 2^32 (32-bit SR counters)
+template <int FMT, int RND, bool EDGE, bool C32>
 __device__ __forceinline__ void row_pass(const uint16_t *tile, const Params &p, int tt, int tc,
                                          float s_enc, const float *tab) {
   const int w = threadIdx.x >> 5, l = threadIdx.x & 31, c = l & 15;
@@ -312,6 +338,8 @@ __device__ __forceinline__ void row_pass(const uint16_t *tile, const Params &p, 
   const int64_t bidx = is_mx<FMT>() ? (kc >> 5) : (kc >> 4);  // block index
   uint8_t *sb0 = p.rs + ((int64_t)tt * (kbt >> 2) + (bidx >> 2)) * 512 + base * 16 + (bidx & 3);
   const bool lead = is_mx<FMT>() ? (c & 3) == 0 : (c & 1) == 0;
+  // (C32) linear index of this lane's first element, and the step to row 16 s
+  const uint32_t idx32 = (uint32_t)(r0 * K + kc), step32 = (uint32_t)(16 * K);
 #pragma unroll
   for (int s = 0; s < 8; ++s) {
     const int rr = 16 * s + base;
@@ -331,7 +359,10 @@ __device__ __forceinline__ void row_pass(const uint16_t *tile, const Params &p, 
     float f[8];
     unpack_scale8(v, mult, f);
     uint32_t codes;
-    if constexpr (RND == kSR)
+    if constexpr (RND == kSR && C32)
+      codes = e2m1x8_sr_not(f, sr_bits_not32(p.rkey0, p.rkey1, p.rpre_hi, p.rpre_lo,
+                                             (idx32 + (uint32_t)s * step32) >> 3));
+    else if constexpr (RND == kSR)
       codes = e2m1x8_sr_not(f, sr_bits_not(p.rkey0, p.rkey1, (uint64_t)((r0 + 16 * s) * K + kc) >> 3));
     else
       codes = e2m1x8_rne(f);
@@ -365,7 +396,7 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
   return r;
 }
 
-template <int FMT, int RND, bool HAD, bool EDGE>
+template <int FMT, int RND, bool HAD, bool EDGE, bool C32>
 __device__ __forceinline__ void col_pass(const uint16_t *tile, const Params &p, int tt, int tc,
                                          float s_enc, const float *tab) {
   const int w = threadIdx.x >> 5, l = threadIdx.x & 31;
@@ -433,7 +464,10 @@ __device__ __forceinline__ void col_pass(const uint16_t *tile, const Params &p, 
     uint32_t codes[4];
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
-      if constexpr (RND == kSR)
+      if constexpr (RND == kSR && C32)
+        codes[q] = e2m1x8_sr_not(&v[8 * q], sr_bits_not32(p.ckey0, p.ckey1, p.cpre_hi, p.cpre_lo,
+                                                          ((uint32_t)(r * T + kfirst) + 8u * q) >> 3));
+      else if constexpr (RND == kSR)
         codes[q] = e2m1x8_sr_not(&v[8 * q], sr_bits_not(p.ckey0, p.ckey1, (uint64_t)(r * T + kfirst + 8 * q) >> 3));
       else
         codes[q] = e2m1x8_rne(&v[8 * q]);
@@ -457,7 +491,7 @@ __device__ __forceinline__ void col_pass(const uint16_t *tile, const Params &p, 
 }
 
 // --------------------------------------------------------------- kernel
-template <int RF, int RR, int CF, int CR, bool HAD>
+template <int RF, int RR, int CF, int CR, bool HAD, bool C32>
 __global__ void __launch_bounds__(kThreads, 2)
     quant_kernel(const __grid_constant__ CUtensorMap xmap, const Params p) {
   extern __shared__ uint8_t qsmem_raw[];
@@ -546,15 +580,15 @@ __global__ void __launch_bounds__(kThreads, 2)
     const bool edge = ((int64_t)tt * 128 + 128 > p.T) || ((int64_t)tc * 128 + 128 > p.C);
     if constexpr (RF != kNone) {
       if (edge)
-        row_pass<RF, RR, true>(tile, p, tt, tc, senc_r, cb->tab_r);
+        row_pass<RF, RR, true, C32>(tile, p, tt, tc, senc_r, cb->tab_r);
       else
-        row_pass<RF, RR, false>(tile, p, tt, tc, senc_r, cb->tab_r);
+        row_pass<RF, RR, false, C32>(tile, p, tt, tc, senc_r, cb->tab_r);
     }
     if constexpr (CF != kNone) {
       if (edge)
-        col_pass<CF, CR, HAD, true>(tile, p, tt, tc, senc_c, cb->tab_c);
+        col_pass<CF, CR, HAD, true, C32>(tile, p, tt, tc, senc_c, cb->tab_c);
       else
-        col_pass<CF, CR, HAD, false>(tile, p, tt, tc, senc_c, cb->tab_c);
+        col_pass<CF, CR, HAD, false, C32>(tile, p, tt, tc, senc_c, cb->tab_c);
     }
     if constexpr (kLocal) __syncthreads();  // the multiplier tables are rewritten next tile
     // release stage s; the last warp out refills it (its reads, and every
@@ -709,14 +743,14 @@ __global__ void __launch_bounds__(kThreads, kSwigluCtasPerSm)
   __syncthreads();
   const bool edge = (r0 + 128 > p.T) || (c0 + 128 > F);
   if (edge)
-    row_pass<RF, RR, true>(tile, p, tt, tc, senc, tab);
+    row_pass<RF, RR, true, false>(tile, p, tt, tc, senc, tab);
   else
-    row_pass<RF, RR, false>(tile, p, tt, tc, senc, tab);
+    row_pass<RF, RR, false, false>(tile, p, tt, tc, senc, tab);
   if constexpr (CF != kNone) {
     if (edge)
-      col_pass<CF, CR, HAD, true>(tile, p, tt, tc, 1.0f, nullptr);
+      col_pass<CF, CR, HAD, true, false>(tile, p, tt, tc, 1.0f, nullptr);
     else
-      col_pass<CF, CR, HAD, false>(tile, p, tt, tc, 1.0f, nullptr);
+      col_pass<CF, CR, HAD, false, false>(tile, p, tt, tc, 1.0f, nullptr);
   }
 }
 
@@ -808,9 +842,19 @@ void philox_round_keys(uint64_t seed, uint32_t *k0, uint32_t *k1) {
   }
 }
 
+// Round-1 constants of sr_bits_not32 from a seed's round keys.
+void philox_round1_consts(const uint32_t *k0, const uint32_t *k1, uint32_t *pre_hi, uint32_t *pre_lo) {
+  const uint64_t prod = (uint64_t)0xD2511F53u * k0[0];
+  *pre_hi = (uint32_t)(prod >> 32) ^ k1[1];
+  *pre_lo = (uint32_t)prod;
+}
+
 template <int RF, int RR, int CF, int CR, bool H>
 cudaError_t launch_q(const CUtensorMap &map, const qk::Params &p, cudaStream_t st) {
-  auto kern = qk::quant_kernel<RF, RR, CF, CR, H>;
+  auto kern = qk::quant_kernel<RF, RR, CF, CR, H, false>;
+  // stochastic rounding with every linear index below 2^32: 32-bit counters
+  if constexpr (RR == kSR || CR == kSR)
+    if ((uint64_t)p.T * (uint64_t)p.C < (uint64_t(1) << 32)) kern = qk::quant_kernel<RF, RR, CF, CR, H, true>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, qk::kSmemBytes);
   if (e != cudaSuccess) return e;
   int dev = 0, sms = 148;
@@ -849,6 +893,8 @@ cudaError_t launch_quantize(const QuantArgs &a, cudaStream_t st) {
   p.cts = a.col_ts;
   philox_round_keys(a.row_seed, p.rkey0, p.rkey1);
   philox_round_keys(a.col_seed, p.ckey0, p.ckey1);
+  philox_round1_consts(p.rkey0, p.rkey1, &p.rpre_hi, &p.rpre_lo);
+  philox_round1_consts(p.ckey0, p.ckey1, &p.cpre_hi, &p.cpre_lo);
   for (int t = 0; t < 32; ++t) p.sgn[t] = ((a.sign_mask >> t) & 1u) ? 0x80000000u : 0u;
   p.partials = a.partials;
   p.np = a.n_partials;

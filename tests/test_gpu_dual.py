@@ -85,6 +85,23 @@ def test_llama8b_full_size_sampled(layer):
     _check(x, fa.NVFP4_GLOBAL, fa.RNE, fa.RNE, True, rows=(r0, r0 + 128), cols=(c0, c0 + 128))
 
 
+def test_sr_counters_of_a_2_32_element_tensor():
+    """A tensor of 2^32 elements takes the quantizers' 64-bit Philox counter
+    path (smaller ones take the 32-bit one): MXFP4 stochastic rounding
+    row-wise and column-wise from one read, bytes of the last 128-row block
+    of each operand (the largest counters) against the oracle."""
+    need_gpu()
+    T, C = 32768, 131072
+    gen = torch.Generator(device="cuda").manual_seed(61)
+    xg = torch.randn(T, C, device="cuda", dtype=torch.bfloat16, generator=gen)
+    try:
+        _check(xg.cpu(), fa.MXFP4, fa.SR, fa.SR, False, x_gpu=xg, rows=(T - 128, T),
+               cols=(C - 128, C), seeds=(71, 73))
+    finally:
+        del xg
+        torch.cuda.empty_cache()
+
+
 @pytest.mark.parametrize("fmt", [fa.MXFP4, fa.NVFP4_GLOBAL], ids=["mx", "nvg"])
 def test_training_linear_equals_the_separate_calls(fmt):
     """linear_fwd_save + linear_bwd (dual producers) give exactly the bytes of
