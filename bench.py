@@ -15,7 +15,7 @@ workloads.py).  Each step reads ~1.1 GB of bf16 inputs, more than the 126 MB
 L2, so no timed iteration finds its inputs in L2.
 
 Prints one JSON line (rank 0).  `value` is whole-job tokens/s; the three
-metrics the FP4 path is judged on (fused-quantize GB/s, block-scaled GEMM
+metrics of the FP4 path (fused-quantize GB/s, block-scaled GEMM
 TFLOP/s, linear tokens/s) are under "metrics".
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl fa4|reference]
