@@ -702,7 +702,7 @@ __device__ __forceinline__ uint32_t swiglu2(uint32_t gw, uint32_t uw) {
 }
 
 constexpr int kSwigluCtasPerSm = 2;
-template <int RF, int RR, int CF, int CR, bool HAD>
+template <int RF, int RR, int CF, int CR, bool HAD, bool C32>
 __global__ void __launch_bounds__(kThreads, kSwigluCtasPerSm)
     swiglu_quant_kernel(const Params p, const uint16_t *__restrict__ z, int64_t ld) {
   __shared__ __align__(16) uint16_t tile[128 * 128];
@@ -743,14 +743,14 @@ __global__ void __launch_bounds__(kThreads, kSwigluCtasPerSm)
   __syncthreads();
   const bool edge = (r0 + 128 > p.T) || (c0 + 128 > F);
   if (edge)
-    row_pass<RF, RR, true, false>(tile, p, tt, tc, senc, tab);
+    row_pass<RF, RR, true, C32>(tile, p, tt, tc, senc, tab);
   else
-    row_pass<RF, RR, false, false>(tile, p, tt, tc, senc, tab);
+    row_pass<RF, RR, false, C32>(tile, p, tt, tc, senc, tab);
   if constexpr (CF != kNone) {
     if (edge)
-      col_pass<CF, CR, HAD, true, false>(tile, p, tt, tc, 1.0f, nullptr);
+      col_pass<CF, CR, HAD, true, C32>(tile, p, tt, tc, 1.0f, nullptr);
     else
-      col_pass<CF, CR, HAD, false, false>(tile, p, tt, tc, 1.0f, nullptr);
+      col_pass<CF, CR, HAD, false, C32>(tile, p, tt, tc, 1.0f, nullptr);
   }
 }
 
@@ -928,8 +928,11 @@ cudaError_t launch_quantize(const QuantArgs &a, cudaStream_t st) {
 namespace {
 template <int RF, int RR, int CF, int CR, bool H>
 cudaError_t launch_sw(const qk::Params &p, const uint16_t *z, int64_t ld, cudaStream_t st) {
-  const cudaError_t e = launch_pdl(qk::swiglu_quant_kernel<RF, RR, CF, CR, H>,
-                                   dim3((unsigned)p.tiles_c, (unsigned)p.tiles_t), dim3(qk::kThreads),
+  auto kern = qk::swiglu_quant_kernel<RF, RR, CF, CR, H, false>;
+  // stochastic rounding with every linear index below 2^32: 32-bit counters
+  if constexpr (RR == kSR || CR == kSR)
+    if ((uint64_t)p.T * (uint64_t)p.C < (uint64_t(1) << 32)) kern = qk::swiglu_quant_kernel<RF, RR, CF, CR, H, true>;
+  const cudaError_t e = launch_pdl(kern, dim3((unsigned)p.tiles_c, (unsigned)p.tiles_t), dim3(qk::kThreads),
                                    0, st, p, z, ld);
   return e != cudaSuccess ? e : cudaGetLastError();
 }
@@ -959,6 +962,8 @@ cudaError_t launch_swiglu_quantize(const SwigluArgs &a, cudaStream_t st) {
   p.cs = a.col_scales;
   philox_round_keys(a.row_seed, p.rkey0, p.rkey1);
   philox_round_keys(a.col_seed, p.ckey0, p.ckey1);
+  philox_round1_consts(p.rkey0, p.rkey1, &p.rpre_hi, &p.rpre_lo);
+  philox_round1_consts(p.ckey0, p.ckey1, &p.cpre_hi, &p.cpre_lo);
   for (int t = 0; t < 32; ++t) p.sgn[t] = ((a.sign_mask >> t) & 1u) ? 0x80000000u : 0u;
   const int rf = a.row_fmt, rr = a.row_rnd, cr = a.col_rnd;
   using qk::kNone;
