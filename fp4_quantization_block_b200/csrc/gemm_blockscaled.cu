@@ -433,12 +433,12 @@ __device__ __forceinline__ bool wait_st(uint32_t bar, uint32_t parity, SmemSt *s
     }
   }
 }
+// every lane of the warp probes the barrier; the vote keeps the outcome
+// uniform even if a lane's wait ran out while another's phase completed
 template <bool HINT>
 __device__ __forceinline__ bool warp_wait_st(uint32_t bar, uint32_t parity, SmemSt *sm,
                                              const Params &p, uint32_t where) {
-  int ok = 0;
-  if ((threadIdx.x & 31) == 0) ok = wait_st<HINT>(bar, parity, sm, p, where) ? 1 : 0;
-  return __shfl_sync(0xFFFFFFFFu, ok, 0) != 0;
+  return __all_sync(0xFFFFFFFFu, wait_st<HINT>(bar, parity, sm, p, where));
 }
 // wait until the last copy issued into each stage of a ring has landed
 __device__ __forceinline__ void drain_ring(uint64_t *full, int n, uint32_t issued,
@@ -859,13 +859,21 @@ __global__ void __launch_bounds__(NUM_THREADS_ST, 1)
 #pragma unroll
         for (int nb = 0; nb < BN / 128; ++nb) b_in[nb] = nt * (BN / 128) + nb < p.rb_b;
       }
-      // A: row 32q + lane is word q of atom row `lane`
+      // A: the MMA reads row 32q + lane's word (word q of atom row `lane`) in
+      // column 4a + q of this quadrant; the whole atom row goes into columns
+      // 4a .. 4a + 3 (the other three words are not read here), so all of
+      // the k-tile's A words are COLS_A consecutive columns and one store
+      uint32_t aw[CS::COLS_A];
 #pragma unroll
-      for (int a = 0; a < C::ATOMS_K; ++a)
-        tmem_st1(col + 4 * a + q,
-                 (a_in && a < na)
-                     ? *reinterpret_cast<const uint32_t *>(sfa_s + a * 512 + lane * 16 + 4 * q)
-                     : 0u);
+      for (int a = 0; a < C::ATOMS_K; ++a) {
+        const uint4 v = (a_in && a < na) ? *reinterpret_cast<const uint4 *>(sfa_s + a * 512 + lane * 16)
+                                         : make_uint4(0u, 0u, 0u, 0u);
+        aw[4 * a] = v.x;
+        aw[4 * a + 1] = v.y;
+        aw[4 * a + 2] = v.z;
+        aw[4 * a + 3] = v.w;
+      }
+      tmem_st_cols<CS::COLS_A>(col, aw);
       // B: atom a of each 128-row block: row 32w + lane is word w of atom row
       // `lane`, in columns 4 (a * BN/128 + nb) + w: the k-tile's B words are
       // COLS_B consecutive columns, written by one or two wide stores
