@@ -728,6 +728,8 @@ __global__ void __launch_bounds__(NUM_THREADS_ST, 1)
       uint32_t acc_phase = 0;
       bool ok = true;
       int g = 0;
+      const uint64_t a_desc0 = operand_desc(smem_u32(smem + CS::OFF_A));
+      const uint64_t b_desc0 = operand_desc(smem_u32(smem + CS::OFF_B));
       for (int tile = unit; tile < num_tiles && ok; tile += nunits) {
         if constexpr (KIND != kNVC) {
           if (!wait_st<kHint>(smem_u32(&sm->acc_empty), acc_phase ^ 1u, sm, p, 0x200u)) break;
@@ -741,8 +743,11 @@ __global__ void __launch_bounds__(NUM_THREADS_ST, 1)
             break;
           }
           tc_fence_after();
-          const uint32_t a_base = smem_u32(smem + CS::OFF_A + s * CS::A_BYTES);
-          const uint32_t b_base = smem_u32(smem + CS::OFF_B + s * CS::B_BYTES);
+          // operand descriptors of the stage's first K step: the start
+          // address field (address / 16, 14 bits, shared memory stays below
+          // 256 KB) advances by 2 per 32-byte K step
+          const uint64_t a_desc = a_desc0 + (uint64_t)((s * CS::A_BYTES) >> 4);
+          const uint64_t b_desc = b_desc0 + (uint64_t)((s * CS::B_BYTES) >> 4);
           const uint32_t sf_col = tmem + CS::SF_COL0 + b * CS::COLS_BUF;
 #pragma unroll
           for (int j = 0; j < BK / 64; ++j) {
@@ -764,12 +769,12 @@ __global__ void __launch_bounds__(NUM_THREADS_ST, 1)
                 tc_fence_after();
               }
               if constexpr (PAIR)
-                tc_mma_pair<KIND>(tmem + 128 * pb, operand_desc(a_base + j * 32),
-                                  operand_desc(b_base + j * 32), instr_desc_pair<KIND, BN>(sf_id),
+                tc_mma_pair<KIND>(tmem + 128 * pb, a_desc + 2 * j,
+                                  b_desc + 2 * j, instr_desc_pair<KIND, BN>(sf_id),
                                   sfa, sfb, (uint32_t)(j & 1));
               else
-                tc_mma<KIND>(tmem + 128 * pb, operand_desc(a_base + j * 32),
-                             operand_desc(b_base + j * 32), instr_desc<KIND, BN>(sf_id), sfa, sfb,
+                tc_mma<KIND>(tmem + 128 * pb, a_desc + 2 * j,
+                             b_desc + 2 * j, instr_desc<KIND, BN>(sf_id), sfa, sfb,
                              (uint32_t)(j & 1));
               if (j & 1) {
                 if constexpr (PAIR)
@@ -780,10 +785,10 @@ __global__ void __launch_bounds__(NUM_THREADS_ST, 1)
             } else {
               const uint32_t acc = (kt > 0 || j > 0) ? 1u : 0u;
               if constexpr (PAIR)
-                tc_mma_pair<KIND>(tmem, operand_desc(a_base + j * 32), operand_desc(b_base + j * 32),
+                tc_mma_pair<KIND>(tmem, a_desc + 2 * j, b_desc + 2 * j,
                                   instr_desc_pair<KIND>(sf_id), sfa, sfb, acc);
               else
-                tc_mma<KIND>(tmem, operand_desc(a_base + j * 32), operand_desc(b_base + j * 32),
+                tc_mma<KIND>(tmem, a_desc + 2 * j, b_desc + 2 * j,
                              instr_desc<KIND, BN>(sf_id), sfa, sfb, acc);
             }
           }
